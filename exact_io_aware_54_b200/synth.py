@@ -1,0 +1,66 @@
+"""Seeded synthetic inputs shared by the tests, the smoke check and the benchmark.
+
+This module holds random-number generation and nothing of the attention
+arithmetic.  Every tensor is drawn in fp32 from N(0, 1) with a seeded
+``torch.Generator`` and rounded once to bf16 (round-to-nearest-even); the same
+bf16 bits go to the GPU and, widened exactly to fp64, to the CPU oracle.
+
+Prefill tensors are token-major ``[B, N, H, d]``; decode uses ``q [B, H, d]``
+and a packed, ragged KV cache ``k, v [total, H, d]`` addressed by
+``cu_seqlens [B+1]`` (int32, exclusive prefix sum of the lengths).
+"""
+from __future__ import annotations
+
+import torch
+
+# seeds of the five workloads (one per workload, tensors drawn Q, K, V, dO with
+# seed+0 .. seed+3)
+SEEDS = {"tiny": 54001, "gpt2m": 54002, "prefill8k": 54003, "decode": 54004, "long16k": 54005}
+
+
+def _normal(shape, seed: int, device="cpu", mult: float = 1.0) -> torch.Tensor:
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    x = torch.randn(*shape, generator=g, device=device, dtype=torch.float32)
+    if mult != 1.0:
+        x.mul_(mult)
+    return x.to(torch.bfloat16)
+
+
+def prefill_inputs(seed: int, B: int, Nq: int, Nk: int, H: int, d: int, q_mult: float = 1.0,
+                   with_dout: bool = False, device="cpu"):
+    """Q [B, Nq, H, d], K, V [B, Nk, H, d] (and dO [B, Nq, H, d]) as bf16."""
+    q = _normal((B, Nq, H, d), seed + 0, device, q_mult)
+    k = _normal((B, Nk, H, d), seed + 1, device)
+    v = _normal((B, Nk, H, d), seed + 2, device)
+    if not with_dout:
+        return q, k, v
+    do = _normal((B, Nq, H, d), seed + 3, device)
+    return q, k, v, do
+
+
+def ragged_lengths(seed: int, B: int, lo: int, hi: int) -> torch.Tensor:
+    """B integer lengths drawn uniformly from [lo, hi] (both ends inclusive)."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return torch.randint(lo, hi + 1, (B,), generator=g, dtype=torch.int64)
+
+
+def cu_seqlens_of(lengths) -> torch.Tensor:
+    """Exclusive prefix sum [B+1] as int32 (cu[0] = 0)."""
+    lengths = torch.as_tensor(lengths, dtype=torch.int64)
+    cu = torch.zeros(len(lengths) + 1, dtype=torch.int64)
+    cu[1:] = torch.cumsum(lengths, 0)
+    return cu.to(torch.int32)
+
+
+def decode_inputs(seed: int, lengths, H: int, d: int, device="cpu"):
+    """q [B, H, d], packed k, v [sum(lengths), H, d] (bf16) and cu_seqlens [B+1] (int32, CPU)."""
+    lengths = torch.as_tensor(lengths, dtype=torch.int64)
+    B = len(lengths)
+    total = int(lengths.sum())
+    cu = cu_seqlens_of(lengths)
+    q = _normal((B, H, d), seed + 0, device)
+    k = _normal((total, H, d), seed + 1, device)
+    v = _normal((total, H, d), seed + 2, device)
+    return q, k, v, cu
