@@ -1,0 +1,227 @@
+"""Exact, IO-aware multi-head attention for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libfa.so`` (declared in ``include/fa.h``):
+argument marshalling only.  Every step of the computation runs in the library's
+CUDA kernels; PyTorch only provides device memory and the current stream.  There
+is no CPU or library fallback: when ``libfa.so`` is missing or cannot be loaded,
+every call raises.
+
+Entry points (same names as the C ABI):
+
+* :func:`fa_fwd` -- forward pass, returns ``(o, lse)``;
+* :func:`fa_bwd` -- recompute backward pass, returns ``(dq, dk, dv)``;
+* :func:`fa_decode_splitkv` -- split-KV decode over a ragged packed KV cache,
+  returns ``(o, lse)``;
+* :func:`fa_check` -- synchronise and read the kernels' status word.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "FAError", "lib_path", "load", "fa_fwd", "fa_bwd", "fa_decode_splitkv", "fa_check",
+    "fa_fwd_workspace_size", "fa_bwd_workspace_size", "fa_decode_workspace_size", "fa_decode_num_splits",
+    "fa_version", "STATUS",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+STATUS = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_ALIGNMENT",
+          4: "FA_ERR_WORKSPACE", 5: "FA_ERR_CUDA", 6: "FA_ERR_TIMEOUT"}
+
+
+class FAError(RuntimeError):
+    """A non-zero fa_status returned by the library."""
+
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+def lib_path() -> str:
+    return os.environ.get("FA_LIB", os.path.join(_HERE, "libfa.so"))
+
+
+_lib = None
+_lock = threading.Lock()
+_vp = ctypes.c_void_p
+_i = ctypes.c_int
+_f = ctypes.c_float
+_sz = ctypes.c_size_t
+
+
+def load():
+    """Load libfa.so (raises if it is absent: there is no fallback path)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        path = lib_path()
+        if not os.path.exists(path):
+            raise ImportError(f"libfa.so not found at {path}; build it with "
+                              f"`python -m exact_io_aware_54_b200.build`")
+        lib = ctypes.CDLL(path)
+        lib.fa_fwd.argtypes = [_vp] * 5 + [_i] * 6 + [_f, _vp, _sz, _vp]
+        lib.fa_bwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _vp, _sz, _vp]
+        lib.fa_decode_splitkv.argtypes = [_vp] * 4 + [_i] * 6 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
+        for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_decode_splitkv):
+            fn.restype = _i
+        lib.fa_fwd_workspace_size.argtypes = [_i] * 5
+        lib.fa_fwd_workspace_size.restype = _sz
+        lib.fa_bwd_workspace_size.argtypes = [_i] * 5
+        lib.fa_bwd_workspace_size.restype = _sz
+        lib.fa_decode_workspace_size.argtypes = [_i] * 5
+        lib.fa_decode_workspace_size.restype = _sz
+        lib.fa_decode_num_splits.argtypes = [_i] * 5
+        lib.fa_decode_num_splits.restype = _i
+        lib.fa_check.argtypes = [_vp, _vp]
+        lib.fa_check.restype = _i
+        lib.fa_status_string.argtypes = [_i]
+        lib.fa_status_string.restype = ctypes.c_char_p
+        lib.fa_version.argtypes = []
+        lib.fa_version.restype = ctypes.c_char_p
+        _lib = lib
+        return lib
+
+
+def fa_version() -> str:
+    return load().fa_version().decode()
+
+
+def fa_fwd_workspace_size(B, H, Nq, Nk, d) -> int:
+    return int(load().fa_fwd_workspace_size(B, H, Nq, Nk, d))
+
+
+def fa_bwd_workspace_size(B, H, Nq, Nk, d) -> int:
+    return int(load().fa_bwd_workspace_size(B, H, Nq, Nk, d))
+
+
+def fa_decode_workspace_size(B, H, max_seqlen_k, d, num_splits=0) -> int:
+    return int(load().fa_decode_workspace_size(B, H, max_seqlen_k, d, num_splits))
+
+
+def fa_decode_num_splits(B, H, max_seqlen_k, d, num_splits=0) -> int:
+    return int(load().fa_decode_num_splits(B, H, max_seqlen_k, d, num_splits))
+
+
+# --------------------------------------------------------------------------- workspaces
+
+_ws_cache: dict = {}
+
+
+def workspace(nbytes: int, device, tag: str = "default") -> torch.Tensor:
+    """A zero-initialised workspace of at least `nbytes`, reused per (device, tag).
+
+    The library keeps a workspace consistent between calls (tickets reset
+    themselves, fa_check clears the status word), so it is zeroed only once."""
+    dev = torch.device(device)
+    key = (dev.type, dev.index if dev.index is not None else torch.cuda.current_device(), tag)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
+        _ws_cache[key] = ws
+    return ws
+
+
+def _stream_ptr(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check_tensor(name, t, dtype, shape=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _raise(fn, status):
+    if status != 0:
+        raise FAError(fn, status)
+
+
+def _scale(softmax_scale):
+    return 0.0 if softmax_scale is None else float(softmax_scale)
+
+
+# --------------------------------------------------------------------------- entry points
+
+
+def fa_fwd(q, k, v, causal: bool = False, softmax_scale=None, out=None, lse=None, ws=None):
+    """Forward pass.  q [B, Nq, H, d], k/v [B, Nk, H, d] bf16 -> (o [B, Nq, H, d], lse [B, H, Nq] fp32)."""
+    lib = load()
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    _check_tensor("q", q, torch.bfloat16)
+    _check_tensor("k", k, torch.bfloat16, (B, Nk, H, d))
+    _check_tensor("v", v, torch.bfloat16, (B, Nk, H, d))
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check_tensor("out", out, torch.bfloat16, q.shape)
+    _check_tensor("lse", lse, torch.float32, (B, H, Nq))
+    need = lib.fa_fwd_workspace_size(B, H, Nq, Nk, d)
+    if ws is None:
+        ws = workspace(need, q.device, "fwd")
+    st = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Nq, Nk, d,
+                    int(bool(causal)), _scale(softmax_scale), ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
+    _raise("fa_fwd", st)
+    return out, lse
+
+
+def fa_bwd(q, k, v, o, dout, lse, causal: bool = False, softmax_scale=None, dq=None, dk=None, dv=None, ws=None):
+    """Backward pass.  Returns (dq, dk, dv) in bf16, gradients of sum(O * dout)."""
+    lib = load()
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    for name, t, shp in (("q", q, None), ("k", k, (B, Nk, H, d)), ("v", v, (B, Nk, H, d)), ("o", o, q.shape),
+                         ("dout", dout, q.shape)):
+        _check_tensor(name, t, torch.bfloat16, shp)
+    _check_tensor("lse", lse, torch.float32, (B, H, Nq))
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = lib.fa_bwd_workspace_size(B, H, Nq, Nk, d)
+    if ws is None:
+        ws = workspace(need, q.device, "bwd")
+    st = lib.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                    dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, Nq, Nk, d, int(bool(causal)),
+                    _scale(softmax_scale), ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
+    _raise("fa_bwd", st)
+    return dq, dk, dv
+
+
+def fa_decode_splitkv(q, k, v, cu_seqlens_k, max_seqlen_k: int, causal: bool = False, softmax_scale=None,
+                      num_splits: int = 0, out=None, lse=None, ws=None):
+    """Split-KV decode.  q [B, H, d]; k/v [total, H, d] bf16; cu_seqlens_k int32 [B+1] on the device.
+    Returns (o [B, H, d] bf16, lse [B, H] fp32)."""
+    lib = load()
+    B, H, d = q.shape
+    _check_tensor("q", q, torch.bfloat16)
+    _check_tensor("k", k, torch.bfloat16)
+    _check_tensor("v", v, torch.bfloat16, k.shape)
+    _check_tensor("cu_seqlens_k", cu_seqlens_k, torch.int32, (B + 1,))
+    if k.dim() != 3 or k.shape[1] != H or k.shape[2] != d:
+        raise ValueError("k/v must be [total, H, d]")
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    need = lib.fa_decode_workspace_size(B, H, int(max_seqlen_k), d, int(num_splits))
+    if ws is None:
+        ws = workspace(need, q.device, "decode")
+    st = lib.fa_decode_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens_k.data_ptr(), B, H, 1,
+                               int(max_seqlen_k), d, int(bool(causal)), _scale(softmax_scale), int(num_splits),
+                               out.data_ptr(), lse.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
+    _raise("fa_decode_splitkv", st)
+    return out, lse
+
+
+def fa_check(ws: torch.Tensor) -> int:
+    """Synchronise the current stream and return the kernels' status (0 = FA_OK)."""
+    return int(load().fa_check(ws.data_ptr(), _stream_ptr(ws.device)))

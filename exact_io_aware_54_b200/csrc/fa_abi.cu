@@ -1,0 +1,257 @@
+// fa_abi.cu -- the C ABI of libfa.so: argument checks, workspace carving, TMA
+// descriptor encoding and kernel launches.  No device memory is allocated here.
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "fa_internal.h"
+
+namespace fa {
+
+int num_sms() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev >= 0 && dev < 64) {
+    if (cached[dev] == 0) {
+      int n = 0;
+      if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+      cached[dev] = n;
+    }
+    return cached[dev];
+  }
+  return 148;
+}
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool encode_bshd_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int D) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)N * H * D * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+static unsigned long long wait_timeout_ns() {
+  static unsigned long long v = [] {
+    unsigned long long ms = 2000;
+    if (const char* env = getenv("FA_WAIT_TIMEOUT_MS")) {
+      const unsigned long long x = strtoull(env, nullptr, 10);
+      if (x > 0) ms = x;
+    }
+    return ms * 1000000ull;
+  }();
+  return v;
+}
+
+static bool checks_enabled() {
+  const char* env = getenv("FA_CHECKS");
+  return env && env[0] == '1';
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+static bool dims_ok(int B, int H, int Nq, int Nk, int d) {
+  if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0) return false;
+  // TMA coordinates and the row arithmetic use 32-bit ints
+  const long long rows_q = (long long)B * Nq * H, rows_k = (long long)B * Nk * H;
+  return rows_q < (1LL << 31) && rows_k < (1LL << 31) && (long long)d * H < (1LL << 20);
+}
+
+static float resolve_scale(float s, int d) { return s > 0.f ? s : 1.0f / sqrtf((float)d); }
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_version(void) { return "0.1.0"; }
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_ALIGNMENT: return "FA_ERR_ALIGNMENT";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+size_t fa_fwd_workspace_size(int B, int H, int Nq, int Nk, int d) {
+  if (!dims_ok(B, H, Nq, Nk, d) || (d != 64 && d != 128)) return 0;
+  return kStatusBytes;
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int Nq, int Nk, int d) {
+  if (!dims_ok(B, H, Nq, Nk, d) || (d != 64 && d != 128)) return 0;
+  return kStatusBytes + up256(sizeof(float) * (size_t)B * Nq * H * d) + up256(sizeof(float) * (size_t)B * H * Nq);
+}
+
+int fa_decode_num_splits(int B, int H, int max_seqlen_k, int d, int num_splits) {
+  if (B <= 0 || H <= 0 || max_seqlen_k < 0 || (d != 64 && d != 128) || num_splits < 0) return 0;
+  return decode_plan(B, H, max_seqlen_k, d, num_splits).splits;
+}
+
+size_t fa_decode_workspace_size(int B, int H, int max_seqlen_k, int d, int num_splits) {
+  if (B <= 0 || H <= 0 || max_seqlen_k < 0 || (d != 64 && d != 128) || num_splits < 0) return 0;
+  return decode_workspace_bytes(B, H, d, decode_plan(B, H, max_seqlen_k, d, num_splits));
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                 int d, int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
+                 cudaStream_t stream) {
+  if (!q || !k || !v || !o || !lse || !dims_ok(B, H, Nq, Nk, d)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < fa_fwd_workspace_size(B, H, Nq, Nk, d))
+    return FA_ERR_WORKSPACE;
+  FwdLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.status = static_cast<int*>(workspace);
+  a.B = B;
+  a.H = H;
+  a.Nq = Nq;
+  a.Nk = Nk;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.scale = resolve_scale(softmax_scale, d);
+  a.timeout_ns = wait_timeout_ns();
+  return launch_fwd(a, stream);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d, int causal,
+                 float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !do_ || !lse || !dq || !dk || !dv || !dims_ok(B, H, Nq, Nk, d))
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(do_) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return FA_ERR_ALIGNMENT;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, Nq, Nk, d))
+    return FA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  BwdLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.dout = do_;
+  a.lse = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.status = reinterpret_cast<int*>(ws);
+  a.dq_acc = reinterpret_cast<float*>(ws + kStatusBytes);
+  a.delta = reinterpret_cast<float*>(ws + kStatusBytes + up256(sizeof(float) * (size_t)B * Nq * H * d));
+  a.B = B;
+  a.H = H;
+  a.Nq = Nq;
+  a.Nk = Nk;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.scale = resolve_scale(softmax_scale, d);
+  a.timeout_ns = wait_timeout_ns();
+  return launch_bwd(a, stream);
+}
+
+fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_k, int B, int H,
+                            int Nq, int max_seqlen_k, int d, int causal, float softmax_scale, int num_splits, void* o,
+                            float* lse, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  (void)causal;  // one query row: the bottom-right aligned mask admits every key
+  if (!q || !k || !v || !cu_seqlens_k || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || Nq != 1 || max_seqlen_k < 0 || num_splits < 0) return FA_ERR_INVALID_ARG;
+  if ((long long)B * H >= (1LL << 31)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return FA_ERR_ALIGNMENT;
+  const DecodePlan plan = decode_plan(B, H, max_seqlen_k, d, num_splits);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < decode_workspace_bytes(B, H, d, plan))
+    return FA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DecodeLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.cu_seqlens = cu_seqlens_k;
+  a.o = o;
+  a.lse = lse;
+  a.status = reinterpret_cast<int*>(ws);
+  size_t off = kStatusBytes;
+  a.tickets = reinterpret_cast<int*>(ws + off);
+  off += up256(sizeof(int) * (size_t)B * H);
+  a.part_ml = reinterpret_cast<float*>(ws + off);
+  off += up256(sizeof(float) * 2 * (size_t)B * H * plan.splits);
+  a.part_u = reinterpret_cast<float*>(ws + off);
+  a.B = B;
+  a.H = H;
+  a.max_seqlen_k = max_seqlen_k;
+  a.d = d;
+  a.scale = resolve_scale(softmax_scale, d);
+  a.plan = plan;
+  a.check_args = checks_enabled() ? 1 : 0;
+  a.timeout_ns = wait_timeout_ns();
+  return launch_decode(a, stream);
+}
+
+fa_status fa_check(void* workspace, cudaStream_t stream) {
+  if (!workspace) return FA_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(stream) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  int status = 0;
+  if (cudaMemcpy(&status, workspace, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  if (status != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(workspace, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+  }
+  switch (status) {
+    case 0: return FA_OK;
+    case kStatusTimeout: return FA_ERR_TIMEOUT;
+    case kStatusBadArg: return FA_ERR_INVALID_ARG;
+    default: return FA_ERR_CUDA;
+  }
+}
+
+}  // extern "C"

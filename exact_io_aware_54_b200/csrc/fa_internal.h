@@ -1,0 +1,91 @@
+// fa_internal.h -- declarations shared by the C ABI layer and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "../../include/fa.h"
+
+namespace fa {
+
+// Workspace: the first kStatusBytes hold the status word (int32) and padding.
+constexpr size_t kStatusBytes = 256;
+
+// Status codes recorded by kernels in the workspace status word (fa_status values).
+constexpr int kStatusTimeout = 6;
+constexpr int kStatusBadArg = 1;
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+// Encode a TMA descriptor for a bf16 tensor [B, N, H, D] (D innermost), with a
+// box of 128 rows x 64 columns and 128-byte swizzle.  Returns false on failure.
+bool encode_bshd_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int D);
+
+struct FwdLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  void* o;
+  float* lse;
+  int* status;
+  int B, H, Nq, Nk, d, causal;
+  float scale;
+  unsigned long long timeout_ns;
+};
+fa_status launch_fwd(const FwdLaunch& a, cudaStream_t stream);
+
+struct BwdLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* o;
+  const void* dout;
+  const float* lse;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* dq_acc;  // [B, Nq, H, d] fp32
+  float* delta;   // [B, H, Nq] fp32
+  int* status;
+  int B, H, Nq, Nk, d, causal;
+  float scale;
+  unsigned long long timeout_ns;
+};
+fa_status launch_bwd(const BwdLaunch& a, cudaStream_t stream);
+
+// Split-KV decode plan: keys per chunk and chunks per sequence.
+struct DecodePlan {
+  int chunk;       // keys per split (multiple of 8)
+  int splits;      // splits for a sequence of max_seqlen_k keys
+  int groups;      // head groups per sequence
+  int heads_per_group;
+};
+DecodePlan decode_plan(int B, int H, int max_seqlen_k, int d, int num_splits);
+
+struct DecodeLaunch {
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* cu_seqlens;
+  void* o;
+  float* lse;
+  int* status;
+  int* tickets;        // [B * H], zero between calls (self-resetting)
+  float* part_ml;      // [B, H, splits, 2]  (m in log2 units, l)
+  float* part_u;       // [B, H, splits, d]
+  int B, H, max_seqlen_k, d;
+  float scale;
+  DecodePlan plan;
+  int check_args;      // validate cu_seqlens on the device first
+  unsigned long long timeout_ns;
+};
+fa_status launch_decode(const DecodeLaunch& a, cudaStream_t stream);
+
+size_t decode_workspace_bytes(int B, int H, int d, const DecodePlan& plan);
+
+}  // namespace fa

@@ -1,0 +1,509 @@
+// fwd_sm100.cu -- exact attention forward pass for B200 (sm_100a).
+//
+// What it computes ("FlashAttention saves IO, not N^2 work", sections 1-3; Flash
+// Attention wiki note, "Online Softmax", "Tiling" and "Flash Attention V2 的改进"):
+// for every (batch b, head h, query row i)
+//     o_i   = sum_j softmax_j(scale * q_i . k_j) v_j
+//     lse_i = ln sum_j exp(scale * q_i . k_j)
+// visiting the keys one 128-row tile at a time with the running (m, l, u) row
+// state, so the score and probability tiles only ever live in tensor memory.
+//
+// B200 design
+//  * Work item = (b, h, pair of 128-row query tiles).  Persistent grid, one CTA
+//    per SM; items are taken round-robin, heaviest (latest causal rows) first.
+//  * Warp roles (320 threads):
+//      warp 0      TMA producer: Q tiles, then K/V tiles through a ring of smem
+//                  slots (mbarrier full/empty pairs).
+//      warp 1      TMEM allocator and tcgen05.mma issuer (one thread).
+//      warps 2-5   softmax group for query tile 0, warps 6-9 for tile 1; thread
+//                  = query row = TMEM lane.
+//  * Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
+//    O1 [384,384+d).  P (bf16) is written over the first 64 columns of its S
+//    tile and fed to the P.V MMA directly from tensor memory.
+//  * The two query tiles ping-pong: while one softmax group works on its scores
+//    the tensor core runs the other tile's MMAs.
+//  * Online softmax in the log2 domain (x = s * scale * log2 e).  The running
+//    max is only moved when a tile raises it by more than 8 (a factor 256), so
+//    the O rescale (a TMEM round trip) is rare; the result is unchanged because
+//    numerator and denominator use the same reference.  The 1/l normalisation
+//    happens once, in the epilogue.
+//  * Causal (bottom-right aligned): KV tiles entirely above the diagonal are
+//    never loaded or multiplied; only tiles that cross it are masked.
+//  * Epilogue: O/l -> bf16 -> swizzled smem (the Q tile's slot) -> TMA store;
+//    lse as coalesced fp32 stores.
+#include "fa_internal.h"
+#include "ptx.cuh"
+
+namespace fa {
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+// tensor-memory column of the score tile / O accumulator of query tile t
+__host__ __device__ constexpr uint32_t tm_s(int t) { return t * 128u; }
+__host__ __device__ constexpr uint32_t tm_o(int t) { return 256u + t * 128u; }
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kTileBytes = 128 * D * 2;   // one 128-row bf16 tile of Q, K or V
+  static constexpr int kBoxes = D / 64;            // 64-column (128-byte) TMA boxes per tile
+  static constexpr int kBoxBytes = 128 * 128;      // 16 KB
+  static constexpr int kStages = (D == 64) ? 8 : 4;
+  static constexpr int kOffQ = 0;                  // Q tile 0, Q tile 1
+  static constexpr int kOffRing = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
+  // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], epi[2]
+  static constexpr int kNumBars = 2 + 2 * kStages + 8;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
+};
+
+struct FwdArgs {
+  float* lse;
+  int* status;
+  int B, H, Nq, Nk;
+  int causal;
+  float scale_log2;
+  int n_pairs;
+  int n_items;
+  unsigned long long timeout_ns;
+};
+
+__device__ __forceinline__ void item_coords(const FwdArgs& a, int w, int& b, int& h, int& pair) {
+  const int bh_count = a.B * a.H;
+  const int pr = w / bh_count;
+  const int bh = w - pr * bh_count;
+  pair = a.causal ? (a.n_pairs - 1 - pr) : pr;
+  b = bh / a.H;
+  h = bh - b * a.H;
+}
+
+// Number of KV tiles query tile starting at row0 needs; -1 when the tile is empty.
+__device__ __forceinline__ int tile_kv_count(const FwdArgs& a, int row0) {
+  if (row0 >= a.Nq) return -1;
+  if (!a.causal) return (a.Nk + 127) >> 7;
+  const int last = min(row0 + 127, a.Nq - 1);
+  long long kend = (long long)last + 1 + a.Nk - a.Nq;
+  if (kend <= 0) return 0;
+  if (kend > a.Nk) kend = a.Nk;
+  return (int)((kend + 127) >> 7);
+}
+
+__device__ __forceinline__ void record_timeout(int* status, volatile int* abort_flag) {
+  *abort_flag = 1;
+  atomicCAS(status, 0, kStatusTimeout);
+}
+
+// Warp-uniform bounded wait: lane 0 waits, the verdict is broadcast.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long timeout_ns) {
+  bool ok = true;
+  if (lane_id() == 0) ok = mbar_wait(bar, parity, timeout_ns);
+  return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+}
+
+template <int D>
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+    umma_ss(d_tmem, sdesc_sw128(q_smem + off, 16, 1024), sdesc_sw128(k_smem + off, 16, 1024), idesc,
+            kk > 0 ? 1u : 0u);
+  }
+}
+
+template <int D>
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    umma_ts(o_tmem, p_tmem + kk * 8, sdesc_sw128(v_smem + kk * 2048, 16384, 1024), idesc,
+            (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+               const FwdArgs a) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* bar_q_full = bars + 0;
+  uint64_t* bar_q_empty = bars + 1;
+  uint64_t* bar_kv_full = bars + 2;
+  uint64_t* bar_kv_empty = bars + 2 + L::kStages;
+  uint64_t* bar_s_full = bars + 2 + 2 * L::kStages;
+  uint64_t* bar_p_full = bar_s_full + 2;
+  uint64_t* bar_o_done = bar_s_full + 4;
+  uint64_t* bar_epi = bar_s_full + 6;
+  uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);
+
+  const uint32_t warp = warp_id();
+  const uint32_t lane = lane_id();
+  const uint32_t smem_base = smem_u32(smem);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q_full, 1);
+    mbar_init(bar_q_empty, 2);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(bar_kv_full + s, 1);
+      mbar_init(bar_kv_empty + s, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar_s_full + t, 1);
+      mbar_init(bar_p_full + t, 128);
+      mbar_init(bar_o_done + t, 1);
+      mbar_init(bar_epi + t, 128);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_base_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      uint32_t item_iter = 0, g = 0;
+      for (int w = blockIdx.x; w < a.n_items && !*abort_flag; w += gridDim.x, ++item_iter) {
+        int b, h, pair;
+        item_coords(a, w, b, h, pair);
+        const int row0 = pair * 256;
+        const int n0 = tile_kv_count(a, row0), n1 = tile_kv_count(a, row0 + 128);
+        const int nkv = max(n0, n1);
+        if (!mbar_wait(bar_q_empty, (item_iter & 1) ^ 1, a.timeout_ns)) {
+          record_timeout(a.status, abort_flag);
+          break;
+        }
+        mbar_arrive_expect_tx(bar_q_full, 2 * L::kTileBytes);
+        for (int t = 0; t < 2; ++t)
+          for (int bx = 0; bx < L::kBoxes; ++bx)
+            tma_load_4d(smem + L::kOffQ + t * L::kTileBytes + bx * L::kBoxBytes, &tmQ, bar_q_full, bx * 64, h,
+                        row0 + t * 128, b);
+        for (int j = 0; j < nkv; ++j) {
+          for (int kv = 0; kv < 2; ++kv, ++g) {
+            const uint32_t slot = g % L::kStages, phase = (g / L::kStages) & 1;
+            if (!mbar_wait(bar_kv_empty + slot, phase ^ 1, a.timeout_ns)) {
+              record_timeout(a.status, abort_flag);
+              j = nkv;
+              break;
+            }
+            mbar_arrive_expect_tx(bar_kv_full + slot, L::kTileBytes);
+            uint8_t* dst = smem + L::kOffRing + slot * L::kTileBytes;
+            for (int bx = 0; bx < L::kBoxes; ++bx)
+              tma_load_4d(dst + bx * L::kBoxBytes, kv == 0 ? &tmK : &tmV, bar_kv_full + slot, bx * 64, h, j * 128,
+                          b);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t item_iter = 0, g = 0;
+      uint32_t s_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
+      const uint32_t q_smem[2] = {smem_base + L::kOffQ, smem_base + L::kOffQ + L::kTileBytes};
+      bool ok = true;
+      auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) {
+        if (!ok) return false;
+        if (!mbar_wait(bar, parity, a.timeout_ns) || *abort_flag) {
+          record_timeout(a.status, abort_flag);
+          ok = false;
+        }
+        return ok;
+      };
+      for (int w = blockIdx.x; w < a.n_items && ok; w += gridDim.x, ++item_iter) {
+        int b, h, pair;
+        item_coords(a, w, b, h, pair);
+        const int row0 = pair * 256;
+        const int nt[2] = {tile_kv_count(a, row0), tile_kv_count(a, row0 + 128)};
+        const int nkv = max(nt[0], nt[1]);
+        if (!wait_or_abort(bar_q_full, item_iter & 1)) break;
+        tc_fence_after();
+        // K_0 : first scores of both tiles
+        uint32_t slot_k = 0;
+        if (nkv > 0) {
+          slot_k = g % L::kStages;
+          if (!wait_or_abort(bar_kv_full + slot_k, (g / L::kStages) & 1)) break;
+          tc_fence_after();
+          ++g;
+          const uint32_t k_smem = smem_base + L::kOffRing + slot_k * L::kTileBytes;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (nt[t] > 0) {
+              issue_qk<D>(tmem_base + tm_s(t), q_smem[t], k_smem);
+              umma_commit(bar_s_full + t);
+            }
+          }
+          umma_commit(bar_kv_empty + slot_k);
+        }
+        for (int j = 0; j < nkv && ok; ++j) {
+          const uint32_t slot_v = g % L::kStages;
+          if (!wait_or_abort(bar_kv_full + slot_v, (g / L::kStages) & 1)) break;
+          tc_fence_after();
+          ++g;
+          const uint32_t v_smem = smem_base + L::kOffRing + slot_v * L::kTileBytes;
+          const bool more = (j + 1 < nkv);
+          uint32_t k_smem = 0;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (j < nt[t]) {
+              if (!wait_or_abort(bar_p_full + t, p_cnt[t] & 1)) break;
+              tc_fence_after();
+              ++p_cnt[t];
+              issue_pv<D>(tmem_base + tm_o(t), tmem_base + tm_s(t), v_smem, j > 0);
+            }
+            if (t == 0 && more) {
+              slot_k = g % L::kStages;
+              if (!wait_or_abort(bar_kv_full + slot_k, (g / L::kStages) & 1)) break;
+              tc_fence_after();
+              ++g;
+              k_smem = smem_base + L::kOffRing + slot_k * L::kTileBytes;
+            }
+            if (more && j + 1 < nt[t]) {
+              issue_qk<D>(tmem_base + tm_s(t), q_smem[t], k_smem);
+              umma_commit(bar_s_full + t);
+            }
+          }
+          if (!ok) break;
+          umma_commit(bar_kv_empty + slot_v);
+          if (more) umma_commit(bar_kv_empty + slot_k);
+        }
+        if (!ok) break;
+        // one completion per present tile and item: all of this tile's MMAs are done
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+          if (nt[t] >= 0) umma_commit(bar_o_done + t);
+        (void)s_cnt;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax groups
+    const int t = (warp - 2) >> 2;               // query tile of this group
+    const uint32_t quarter = warp & 3;           // TMEM lane quarter this warp may access
+    const int r = quarter * 32 + lane;           // row within the tile
+    const uint32_t lane_field = (quarter * 32) << 16;
+    const uint32_t tS = tmem_base + lane_field + tm_s(t);
+    const uint32_t tO = tmem_base + lane_field + tm_o(t);
+    const int tid_in_group = threadIdx.x - 64 - t * 128;
+    uint32_t s_cnt = 0, tile_iter = 0;  // tile_iter counts items in which this tile is present
+    uint8_t* q_tile = smem + L::kOffQ + t * L::kTileBytes;
+    const uint32_t q_tile_u32 = smem_u32(q_tile);
+
+    for (int w = blockIdx.x; w < a.n_items; w += gridDim.x) {
+      if (*abort_flag) break;
+      int b, h, pair;
+      item_coords(a, w, b, h, pair);
+      const int row0 = pair * 256 + t * 128;
+      const int nkv = tile_kv_count(a, row0);
+      if (nkv < 0) {  // this query tile lies past Nq: nothing to compute or store
+        if (tid_in_group == 0) mbar_arrive(bar_q_empty);
+        __syncwarp();
+        continue;
+      }
+      const int row = row0 + r;
+      // visible keys of this row: [0, lim)
+      int lim = a.Nk;
+      if (a.causal) lim = max(0, min(a.Nk, row + 1 + a.Nk - a.Nq));
+      const int group_first_lim = a.causal ? (row0 + 1 + a.Nk - a.Nq) : a.Nk;  // smallest lim in the tile
+
+      float m2 = -INFINITY;  // running reference max (log2 domain)
+      float l = 0.f;         // running sum of the bf16-rounded probabilities
+      bool ok = true;
+      for (int j = 0; j < nkv; ++j, ++s_cnt) {
+        if (!warp_wait(bar_s_full + t, s_cnt & 1, a.timeout_ns) || *abort_flag) {
+          if (lane == 0) record_timeout(a.status, abort_flag);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t s[4][32];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tmem_ld32(tS + i * 32, s[i]);
+        tmem_ld_wait(s[0]);
+        reg_pin(s[1]);
+        reg_pin(s[2]);
+        reg_pin(s[3]);
+
+        // mask (only tiles that cross the diagonal or the key tail)
+        const int kbase = j * 128;
+        if (kbase + 128 > min(group_first_lim, a.Nk) || kbase + 128 > a.Nk) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (kbase + i * 32 + c >= lim) s[i][c] = __float_as_uint(-INFINITY);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int c = 0; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(s[i][c]));
+        const float m_tile = mx * a.scale_log2;  // scale > 0, so max commutes with the scaling
+        const bool need = (m2 == -INFINITY) || (m_tile > m2 + kRescaleThreshold);
+        const float m_use = need ? fmaxf(m2, m_tile) : m2;
+        const float alpha = (m2 == -INFINITY) ? 0.f : ex2(m2 - m_use);
+        const float m_ref = (m_use == -INFINITY) ? 0.f : m_use;
+        // probabilities, rounded to bf16 exactly as the P.V MMA will see them
+        float rs0 = 0.f, rs1 = 0.f;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int ii = 0; ii < 2; ++ii) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const float p0 = ex2(fmaf(__uint_as_float(s[hf * 2 + ii][c]), a.scale_log2, -m_ref));
+              const float p1 = ex2(fmaf(__uint_as_float(s[hf * 2 + ii][c + 1]), a.scale_log2, -m_ref));
+              const uint32_t packed = pack_bf16x2(p0, p1);
+              pk[ii * 16 + (c >> 1)] = packed;
+              rs0 += __uint_as_float(packed << 16);
+              rs1 += __uint_as_float(packed & 0xFFFF0000u);
+            }
+          }
+          tmem_st32(tS + hf * 32, pk);
+        }
+        l = l * alpha + (rs0 + rs1);
+        m2 = m_use;
+        // rescale the O accumulator when some row of this warp moved its reference.
+        // The previous P.V of this tile has completed: the scores just read were
+        // issued after it and tcgen05 operations complete in order.
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc * 32, o);
+            tmem_ld_wait(o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(tO + cc * 32, o);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar_p_full + t);
+      }
+      if (!ok) break;
+
+      // ---------------------------------------------------------------- epilogue
+      if (!warp_wait(bar_o_done + t, tile_iter & 1, a.timeout_ns) || *abort_flag) {
+        if (lane == 0) record_timeout(a.status, abort_flag);
+        break;
+      }
+      tc_fence_after();
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        if (nkv > 0) {
+          tmem_ld32(tO + cc * 32, o);
+          tmem_ld_wait(o);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = 0u;
+        }
+        const int box = cc >> 1;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int chunk = (cc & 1) * 4 + q4;  // 16-byte chunk within the 128-byte row
+          const uint32_t addr = q_tile_u32 + box * L::kBoxBytes + r * 128 + ((chunk ^ (r & 7)) << 4);
+          const float* f = reinterpret_cast<const float*>(o) + q4 * 8;
+          st_shared_v4(addr, pack_bf16x2(f[0] * inv_l, f[1] * inv_l), pack_bf16x2(f[2] * inv_l, f[3] * inv_l),
+                       pack_bf16x2(f[4] * inv_l, f[5] * inv_l), pack_bf16x2(f[6] * inv_l, f[7] * inv_l));
+        }
+      }
+      if (row < a.Nq) {
+        const float lse = (l > 0.f) ? (m2 + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        a.lse[((size_t)b * a.H + h) * a.Nq + row] = lse;
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar_epi + t);
+      bool epi_ok = true;
+      if (tid_in_group == 0) {
+        if (!mbar_wait(bar_epi + t, tile_iter & 1, a.timeout_ns)) {
+          record_timeout(a.status, abort_flag);
+          epi_ok = false;
+        } else {
+          for (int bx = 0; bx < L::kBoxes; ++bx)
+            tma_store_4d(&tmO, q_tile + bx * L::kBoxBytes, bx * 64, h, row0, b);
+          bulk_commit_group();
+          bulk_wait_group_read0();
+          mbar_arrive(bar_q_empty);
+        }
+      }
+      // keep the warp converged before its next tcgen05 instruction
+      if (__shfl_sync(0xffffffffu, epi_ok ? 1 : 0, 0) == 0) break;
+      ++tile_iter;
+    }
+    if (tid_in_group == 0) bulk_wait_group0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace
+
+template <int D>
+static fa_status launch_fwd_impl(const FwdLaunch& L0, cudaStream_t stream) {
+  using L = FwdLayout<D>;
+  static bool attr_done[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  if (dev < 64 && !attr_done[dev]) {
+    if (cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes) !=
+        cudaSuccess)
+      return FA_ERR_CUDA;
+    attr_done[dev] = true;
+  }
+  CUtensorMap tq, tk, tv, to;
+  if (!encode_bshd_map(&tq, L0.q, L0.B, L0.Nq, L0.H, D) || !encode_bshd_map(&tk, L0.k, L0.B, L0.Nk, L0.H, D) ||
+      !encode_bshd_map(&tv, L0.v, L0.B, L0.Nk, L0.H, D) || !encode_bshd_map(&to, L0.o, L0.B, L0.Nq, L0.H, D))
+    return FA_ERR_CUDA;
+  FwdArgs a;
+  a.lse = L0.lse;
+  a.status = L0.status;
+  a.B = L0.B;
+  a.H = L0.H;
+  a.Nq = L0.Nq;
+  a.Nk = L0.Nk;
+  a.causal = L0.causal;
+  a.scale_log2 = L0.scale * 1.4426950408889634f;
+  a.n_pairs = (L0.Nq + 255) / 256;
+  a.n_items = a.n_pairs * L0.B * L0.H;
+  a.timeout_ns = L0.timeout_ns;
+  const int grid = std::min(a.n_items, num_sms() * 1);
+  fwd_kernel<D><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status launch_fwd(const FwdLaunch& L0, cudaStream_t stream) {
+  if (L0.d == 64) return launch_fwd_impl<64>(L0, stream);
+  if (L0.d == 128) return launch_fwd_impl<128>(L0, stream);
+  return FA_ERR_UNSUPPORTED;
+}
+
+}  // namespace fa

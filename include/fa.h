@@ -1,0 +1,151 @@
+/*
+ * fa.h -- C ABI of libfa.so: exact, IO-aware multi-head attention on B200 (sm_100a).
+ *
+ * The operation is exact attention, O = softmax(scale * Q K^T) V, per batch
+ * element and head ("FlashAttention saves IO, not N^2 work", section 1:
+ * S = QK^T / sqrt(d), P = softmax(S), O = PV).  It is computed tile by tile
+ * with an online softmax so that the N x N score and probability matrices never
+ * reach device memory (same page, sections 2-3; Flash Attention wiki note,
+ * "Online Softmax" and "Tiling").  The backward pass recomputes S and P from the
+ * saved per-row log-sum-exp ("AI Bible 13", section 03, second axe: keep only O
+ * and the row statistics).  Decode splits each row's KV history into chunks and
+ * merges the chunks' (m, l, u) states (first page, sections 3 and 7; section 6
+ * for the decode shapes).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers, 16-byte aligned, contiguous, in the
+ *    layouts stated per call.  bf16 means IEEE bfloat16 (2 bytes).
+ *  - The caller owns every buffer, including `workspace`.  The library never
+ *    allocates device memory, never keeps a pointer after returning, and never
+ *    synchronises the device (except fa_check).
+ *  - Work is enqueued asynchronously on `stream` (0 = legacy default stream).
+ *    Launch failures are returned as FA_ERR_CUDA; the CUDA error is consumed.
+ *  - Supported head dimensions: d in {64, 128}.  Only bf16 inputs/outputs.
+ *  - softmax_scale <= 0 selects 1/sqrt(d).
+ *  - causal != 0 applies a bottom-right aligned mask: query row i (of Nq) sees
+ *    key j (of Nk) iff j <= i + (Nk - Nq).  A query row that sees no key gets
+ *    O = 0 and LSE = -inf (and zero gradients).  For decode (one query row) the
+ *    mask admits every key and is a no-op.
+ *  - LSE is the natural-log log-sum-exp of the scaled scores of a row:
+ *    lse_i = m_i + ln(l_i), with m_i the row max and l_i = sum_j exp(s_ij - m_i).
+ *  - A workspace must be zero-filled (cudaMemset) before its first use.  After
+ *    that the library keeps it consistent by itself: decode merge tickets reset
+ *    themselves and fa_check clears the status word.  Two calls that may run at
+ *    the same time on the GPU must not share a workspace.
+ *  - Every wait inside a kernel is bounded (default about 2 s; environment
+ *    variable FA_WAIT_TIMEOUT_MS overrides it).  A wait that runs out makes the
+ *    kernel record FA_ERR_TIMEOUT in the workspace's status word and return
+ *    without further work; fa_check reports it.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null pointer, non-positive size, Nq != 1 for decode, ... */
+  FA_ERR_UNSUPPORTED = 2, /* head dimension or configuration this build does not implement */
+  FA_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned */
+  FA_ERR_WORKSPACE = 4,   /* workspace null or smaller than the *_workspace_size query */
+  FA_ERR_CUDA = 5,        /* a CUDA runtime/driver call or kernel launch failed */
+  FA_ERR_TIMEOUT = 6      /* a kernel's bounded wait ran out (reported by fa_check) */
+} fa_status;
+
+/*
+ * Forward pass.
+ *   q   : [B, Nq, H, d] bf16 (token-major, d innermost)
+ *   k, v: [B, Nk, H, d] bf16
+ *   o   : [B, Nq, H, d] bf16 (written)
+ *   lse : [B, H, Nq]    fp32 (written) -- saved for the backward pass
+ *   workspace: at least fa_fwd_workspace_size(...) bytes of device memory,
+ *              16-byte aligned; holds the kernel status word.
+ * Sizes: B, H, Nq, Nk >= 1; d in {64, 128}.  q/k/v must not alias o/lse.
+ * Returns FA_OK when the work was enqueued.
+ */
+FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int Nq, int Nk, int d, int causal, float softmax_scale, void* workspace,
+                 size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Backward pass (recompute form).
+ *   q, o, do_ : [B, Nq, H, d] bf16 ; k, v : [B, Nk, H, d] bf16
+ *   lse       : [B, H, Nq] fp32 as written by fa_fwd with the same arguments
+ *   dq        : [B, Nq, H, d] bf16 (written)
+ *   dk, dv    : [B, Nk, H, d] bf16 (written)
+ *   workspace : at least fa_bwd_workspace_size(...) bytes; holds an fp32 dQ
+ *               accumulator [B, Nq, H, d], the row terms D_i = dO_i . O_i
+ *               [B, H, Nq] fp32, and the status word.  The call clears the dQ
+ *               accumulator itself.
+ * Gradients are of the scalar sum(O * dO) with respect to q, k and v.  The dq
+ * accumulation uses fp32 atomics, so dq is reproducible only up to summation
+ * order.
+ */
+FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* do_,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d,
+                 int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
+                 cudaStream_t stream);
+
+/*
+ * Split-KV decode over a ragged, packed KV cache.
+ *   q           : [B, H, d] bf16 (one query row per sequence: Nq must be 1)
+ *   k, v        : [total_kv, H, d] bf16; sequence b owns rows
+ *                 cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1
+ *   cu_seqlens_k: device int32 [B+1], non-decreasing, cu_seqlens_k[0] = 0
+ *                 (validated on the device only when FA_CHECKS=1)
+ *   max_seqlen_k: an upper bound of every sequence length (plays the role of Nk)
+ *   num_splits  : chunks per sequence; 0 picks a value from the shape
+ *   o           : [B, H, d] bf16 (written);  lse : [B, H] fp32 (written)
+ *   workspace   : at least fa_decode_workspace_size(B, H, max_seqlen_k, d, num_splits)
+ *                 bytes; holds the per-chunk (m, l, u) partial states, the merge
+ *                 tickets and the status word.
+ * A sequence of length 0 gets O = 0 and LSE = -inf.
+ */
+FA_API fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_k,
+                            int B, int H, int Nq, int max_seqlen_k, int d, int causal,
+                            float softmax_scale, int num_splits, void* o, float* lse, void* workspace,
+                            size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace sizes in bytes for the calls above (0 when the arguments are invalid). */
+FA_API size_t fa_fwd_workspace_size(int B, int H, int Nq, int Nk, int d);
+FA_API size_t fa_bwd_workspace_size(int B, int H, int Nq, int Nk, int d);
+FA_API size_t fa_decode_workspace_size(int B, int H, int max_seqlen_k, int d, int num_splits);
+
+/*
+ * Number of KV chunks per sequence that fa_decode_splitkv uses for these
+ * arguments (num_splits = 0 resolves to the automatic choice).
+ */
+FA_API int fa_decode_num_splits(int B, int H, int max_seqlen_k, int d, int num_splits);
+
+/*
+ * Synchronises `stream` and reads the status word that the kernels of the
+ * previous call(s) with this workspace recorded.  Returns FA_OK, FA_ERR_TIMEOUT
+ * (a bounded wait ran out), FA_ERR_INVALID_ARG (FA_CHECKS=1 found malformed
+ * cu_seqlens) or FA_ERR_CUDA.
+ */
+FA_API fa_status fa_check(void* workspace, cudaStream_t stream);
+
+/* Human-readable name of a status code (static string). */
+FA_API const char* fa_status_string(fa_status status);
+
+/* Library version as "major.minor.patch" (static string). */
+FA_API const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

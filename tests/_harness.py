@@ -1,0 +1,68 @@
+"""Shared helpers for the GPU parity tests: tolerances and comparisons.
+
+Tolerances (bf16 inputs, fp32 accumulation, N(0,1) data):
+  O    : max |o_gpu - o_oracle| <= 1e-2 and mean |.| <= 1e-3
+  LSE  : |lse_gpu - lse_oracle| <= 1e-4 * max(1, |lse_oracle|)
+  dQ/dK/dV : max |g_gpu - g_oracle| / max |g_oracle| <= 2e-2 (per tensor)
+"""
+import math
+
+import numpy as np
+import torch
+
+O_MAX_ABS = 1e-2
+O_MEAN_ABS = 1e-3
+LSE_REL = 1e-4
+GRAD_REL = 2e-2
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def compare_o(o_gpu, o_ref, what="O", mean_tol=O_MEAN_ABS, max_tol=O_MAX_ABS):
+    o_gpu = np.asarray(o_gpu, dtype=np.float64)
+    o_ref = np.asarray(o_ref, dtype=np.float64)
+    assert o_gpu.shape == o_ref.shape, (o_gpu.shape, o_ref.shape)
+    assert np.all(np.isfinite(o_gpu)), f"{what}: non-finite values"
+    err = np.abs(o_gpu - o_ref)
+    mx, mean = float(err.max(initial=0.0)), float(err.mean()) if err.size else 0.0
+    assert mx <= max_tol, f"{what}: max abs err {mx:.3e} > {max_tol}"
+    assert mean <= mean_tol, f"{what}: mean abs err {mean:.3e} > {mean_tol}"
+    return mx, mean
+
+
+def compare_lse(lse_gpu, lse_ref, what="LSE"):
+    lse_gpu = np.asarray(lse_gpu, dtype=np.float64)
+    lse_ref = np.asarray(lse_ref, dtype=np.float64)
+    assert lse_gpu.shape == lse_ref.shape
+    inf_ref = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lse_gpu), inf_ref), f"{what}: -inf rows differ"
+    fin = ~inf_ref
+    if fin.any():
+        err = np.abs(lse_gpu[fin] - lse_ref[fin]) / np.maximum(1.0, np.abs(lse_ref[fin]))
+        assert np.all(np.isfinite(lse_gpu[fin])), f"{what}: non-finite"
+        assert float(err.max()) <= LSE_REL, f"{what}: rel err {float(err.max()):.3e} > {LSE_REL}"
+
+
+def compare_grad(g_gpu, g_ref, what):
+    g_gpu = np.asarray(g_gpu, dtype=np.float64)
+    g_ref = np.asarray(g_ref, dtype=np.float64)
+    assert np.all(np.isfinite(g_gpu)), f"{what}: non-finite values"
+    scale = float(np.abs(g_ref).max(initial=0.0))
+    err = float(np.abs(g_gpu - g_ref).max(initial=0.0))
+    if scale == 0.0:
+        assert err == 0.0, f"{what}: expected zeros, max {err}"
+        return 0.0
+    assert err / scale <= GRAD_REL, f"{what}: normalised max err {err / scale:.3e} > {GRAD_REL}"
+    return err / scale
+
+
+def rounding_floor(o_ref):
+    """mean |bf16(o) - o|: the error that storing the exact output in bf16 alone makes."""
+    t = torch.from_numpy(np.asarray(o_ref, dtype=np.float64))
+    return float((t.to(torch.bfloat16).to(torch.float64) - t).abs().mean())
+
+
+def default_scale(d):
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,97 @@
+"""GPU parity of fa_fwd against the fp64 oracle (through the C ABI binding)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_io_aware_54_b200 import fa_check, fa_fwd, synth, workspace
+from tests._harness import compare_lse, compare_o, default_scale, f64, rounding_floor
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(q, k, v, causal, scale=None):
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o, lse = fa_fwd(qd, kd, vd, causal=causal, softmax_scale=scale)
+    torch.cuda.synchronize()
+    assert fa_check(workspace(256, qd.device, "fwd")) == 0
+    return o, lse
+
+
+def _full_check(B, Nq, Nk, H, d, causal, seed, q_mult=1.0, scale=None):
+    q, k, v = synth.prefill_inputs(seed, B, Nq, Nk, H, d, q_mult=q_mult)
+    sc = default_scale(d) if scale is None else scale
+    o, lse = _run(q, k, v, causal, scale)
+    o_ref, lse_ref = oracle.attn_fwd(f64(q), f64(k), f64(v), causal, sc)
+    mx, mean = compare_o(f64(o), o_ref)
+    compare_lse(f64(lse), lse_ref)
+    return mx, mean, o_ref
+
+
+def test_tiny_config_noncausal():
+    """B=1, H=2, N=256, d=64, non-causal, scale 1/8 (seed 54001)."""
+    _full_check(1, 256, 256, 2, 64, False, synth.SEEDS["tiny"])
+
+
+def test_tiny_config_q_times_40():
+    """Same shape with Q x 40: raw scores span about +-1000, exercising max subtraction."""
+    mx, mean, o_ref = _full_check(1, 256, 256, 2, 64, False, synth.SEEDS["tiny"], q_mult=40.0)
+    floor = rounding_floor(o_ref)
+    assert floor < 1e-3  # the bf16 storage floor itself is inside the bar
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Nq,Nk", [(1, 1), (1, 300), (129, 129), (200, 200), (256, 640), (383, 257), (513, 130),
+                                   (640, 1000)])
+def test_edge_shapes(d, causal, Nq, Nk):
+    _full_check(2, Nq, Nk, 3, d, causal, 1000 + Nq + Nk + d + causal)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_many_items_per_cta(d):
+    """More (b, h, q-tile pair) items than SMs: each persistent CTA loops over several."""
+    _full_check(4, 512, 512, 48, d, True, 777 + d)
+
+
+def test_explicit_scale():
+    _full_check(1, 300, 300, 2, 64, True, 4242, scale=0.37)
+
+
+def _sampled_rows_check(B, N, H, d, causal, seed, n_heads=6, n_rows=48):
+    q, k, v = synth.prefill_inputs(seed, B, N, N, H, d, device="cuda")
+    o, lse = fa_fwd(q, k, v, causal=causal)
+    torch.cuda.synchronize()
+    assert fa_check(workspace(256, q.device, "fwd")) == 0
+    g = np.random.default_rng(seed)
+    heads = [(0, 0), (B - 1, H - 1)] + [(int(g.integers(B)), int(g.integers(H))) for _ in range(n_heads - 2)]
+    for b, h in heads:
+        rows = np.unique(np.concatenate([[0, 1, 127, 128, N - 1], g.integers(0, N, n_rows)]))
+        kk, vv = f64(k[b, :, h]), f64(v[b, :, h])
+        o_ref, lse_ref = oracle.attn_fwd_rows(f64(q[b, rows, h]), rows, kk, vv, N, causal, default_scale(d))
+        compare_o(f64(o[b, rows, h]), o_ref, what=f"O[b={b},h={h}]")
+        compare_lse(f64(lse[b, h, rows]), lse_ref, what=f"LSE[b={b},h={h}]")
+
+
+def test_gpt2_medium_shape_sampled():
+    """B=64, H=16, N=1024, d=64, causal: sampled rows of sampled heads."""
+    _sampled_rows_check(64, 1024, 16, 64, True, synth.SEEDS["gpt2m"])
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_long_prefill_sampled(causal):
+    """B=1, H=32, N=8192, d=128 (causal and non-causal): sampled rows."""
+    _sampled_rows_check(1, 8192, 32, 128, causal, synth.SEEDS["prefill8k"], n_heads=4, n_rows=24)
+
+
+def test_long_sequence_sampled():
+    """B=1, H=16, N=16384, d=64, causal: sampled rows."""
+    _sampled_rows_check(1, 16384, 16, 64, True, synth.SEEDS["long16k"], n_heads=3, n_rows=16)
+
+
+def test_deterministic_and_reentrant():
+    q, k, v = synth.prefill_inputs(5, 2, 333, 333, 4, 64, device="cuda")
+    o1, l1 = fa_fwd(q, k, v, causal=True)
+    o2, l2 = fa_fwd(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
