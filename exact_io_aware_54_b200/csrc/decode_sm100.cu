@@ -22,8 +22,8 @@
 //    shuffle levels, the stage max three; every lane keeps a partial u over the
 //    keys of its slot, summed across slots once at the end.
 //  * The last warp of each (sequence, head) to finish its chunk -- found with an
-//    atomic ticket -- merges the chunk states and writes o and lse; the ticket
-//    is reset for the next call.  A sequence with a single chunk skips the
+//    atomic ticket tagged with the call's epoch -- merges the chunk states and
+//    writes o and lse.  A sequence with a single chunk skips the
 //    partial-state round trip.
 #include "fa_internal.h"
 #include "ptx.cuh"
@@ -55,7 +55,8 @@ struct DecArgs {
   __nv_bfloat16* o;
   float* lse;
   int* status;
-  int* tickets;
+  unsigned long long* tickets;
+  unsigned int epoch;
   float* part_ml;
   float* part_u;
   int B, H, max_seqlen_k;
@@ -74,6 +75,21 @@ __device__ __forceinline__ void bf16x8_to_f32(uint32_t a, uint32_t b, uint32_t c
   f[5] = __uint_as_float(c & 0xFFFF0000u);
   f[6] = __uint_as_float(d << 16);
   f[7] = __uint_as_float(d & 0xFFFF0000u);
+}
+
+// Arrival on a merge ticket.  A ticket holds (call epoch << 32 | arrivals); a
+// ticket whose epoch is not this call's -- stale or never initialised -- counts
+// as zero arrivals, so the workspace needs no clearing between calls.  Returns
+// the number of arrivals of this call including this one.
+__device__ __forceinline__ unsigned ticket_arrive(unsigned long long* t, unsigned epoch) {
+  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(t), assumed;
+  do {
+    assumed = old;
+    const unsigned long long next =
+        ((assumed >> 32) == epoch) ? assumed + 1 : ((static_cast<unsigned long long>(epoch) << 32) | 1ull);
+    old = atomicCAS(t, assumed, next);
+  } while (old != assumed);
+  return ((old >> 32) == epoch) ? static_cast<unsigned>(old & 0xffffffffu) + 1u : 1u;
 }
 
 template <int D>
@@ -292,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
   __threadfence();
   __syncwarp();
   int last = 0;
-  if (lane == 0) last = (atomicAdd(a.tickets + bh, 1) == nsplit - 1) ? 1 : 0;
+  if (lane == 0) last = (ticket_arrive(a.tickets + bh, a.epoch) == nsplit) ? 1 : 0;
   last = __shfl_sync(0xffffffffu, last, 0);
   if (!last) return;
   __threadfence();
@@ -330,10 +346,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
 #pragma unroll
   for (int e = 0; e < kPerLane; e += 2)
     *reinterpret_cast<uint32_t*>(out + e) = pack_bf16x2(U[e] * inv, U[e + 1] * inv);
-  if (lane == 0) {
-    a.lse[bh] = (Lsum > 0.f) ? (M + __log2f(Lsum)) * 0.69314718055994530942f : -INFINITY;
-    a.tickets[bh] = 0;  // ready for the next call
-  }
+  if (lane == 0) a.lse[bh] = (Lsum > 0.f) ? (M + __log2f(Lsum)) * 0.69314718055994530942f : -INFINITY;
 }
 
 // Optional argument check of cu_seqlens (FA_CHECKS=1).
@@ -387,7 +400,7 @@ DecodePlan decode_plan(int B, int H, int max_seqlen_k, int d, int num_splits) {
 size_t decode_workspace_bytes(int B, int H, int d, const DecodePlan& plan) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
   size_t bytes = kStatusBytes;
-  bytes += up(sizeof(int) * (size_t)B * H);
+  bytes += up(sizeof(unsigned long long) * (size_t)B * H);
   bytes += up(sizeof(float) * 2 * (size_t)B * H * plan.splits);
   bytes += up(sizeof(float) * (size_t)d * B * H * plan.splits);
   return bytes;
@@ -414,6 +427,7 @@ static fa_status launch_decode_impl(const DecodeLaunch& L0, cudaStream_t stream)
   a.lse = L0.lse;
   a.status = L0.status;
   a.tickets = L0.tickets;
+  a.epoch = L0.epoch;
   a.part_ml = L0.part_ml;
   a.part_u = L0.part_u;
   a.B = L0.B;

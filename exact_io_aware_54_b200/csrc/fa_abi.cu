@@ -4,6 +4,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
+#include <chrono>
 #include <mutex>
 
 #include "fa_internal.h"
@@ -84,6 +86,19 @@ static bool dims_ok(int B, int H, int Nq, int Nk, int d) {
 }
 
 static float resolve_scale(float s, int d) { return s > 0.f ? s : 1.0f / sqrtf((float)d); }
+
+// Call epochs for the decode merge tickets: distinct for every call in this
+// process, and started from the clock so that a workspace left by an earlier
+// process is unlikely to carry a matching tag.
+static unsigned next_epoch() {
+  static std::atomic<unsigned> counter{static_cast<unsigned>(
+      std::chrono::steady_clock::now().time_since_epoch().count() * 2654435761ull)};
+  unsigned e;
+  do {
+    e = counter.fetch_add(1, std::memory_order_relaxed) + 1;
+  } while (e == 0);
+  return e;
+}
 
 }  // namespace fa
 
@@ -212,8 +227,9 @@ fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, const i
   a.lse = lse;
   a.status = reinterpret_cast<int*>(ws);
   size_t off = kStatusBytes;
-  a.tickets = reinterpret_cast<int*>(ws + off);
-  off += up256(sizeof(int) * (size_t)B * H);
+  a.tickets = reinterpret_cast<unsigned long long*>(ws + off);
+  a.epoch = next_epoch();
+  off += up256(sizeof(unsigned long long) * (size_t)B * H);
   a.part_ml = reinterpret_cast<float*>(ws + off);
   off += up256(sizeof(float) * 2 * (size_t)B * H * plan.splits);
   a.part_u = reinterpret_cast<float*>(ws + off);

@@ -75,7 +75,8 @@ struct DecodeLaunch {
   void* o;
   float* lse;
   int* status;
-  int* tickets;        // [B * H], zero between calls (self-resetting)
+  unsigned long long* tickets;  // [B * H] merge tickets, epoch-tagged (no clearing needed)
+  unsigned int epoch;           // distinct per call
   float* part_ml;      // [B, H, splits, 2]  (m in log2 units, l)
   float* part_u;       // [B, H, splits, d]
   int B, H, max_seqlen_k, d;

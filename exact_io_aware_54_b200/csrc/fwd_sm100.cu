@@ -26,7 +26,9 @@
 //    max is only moved when a tile raises it by more than 8 (a factor 256), so
 //    the O rescale (a TMEM round trip) is rare; the result is unchanged because
 //    numerator and denominator use the same reference.  The 1/l normalisation
-//    happens once, in the epilogue.
+//    happens once, in the epilogue.  Two row sums are kept: the sum of the
+//    bf16-rounded probabilities (exactly the weights the P.V MMA used) divides
+//    O, and the sum of the unrounded ones gives lse.
 //  * Causal (bottom-right aligned): KV tiles entirely above the diagonal are
 //    never loaded or multiplied; only tiles that cross it are masked.
 //  * Epilogue: O/l -> bf16 -> swizzled smem (the Q tile's slot) -> TMA store;
@@ -327,7 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int group_first_lim = a.causal ? (row0 + 1 + a.Nk - a.Nq) : a.Nk;  // smallest lim in the tile
 
       float m2 = -INFINITY;  // running reference max (log2 domain)
-      float l = 0.f;         // running sum of the bf16-rounded probabilities
+      float l = 0.f;         // running sum of the bf16-rounded probabilities (normalises O)
+      float le = 0.f;        // running sum of the unrounded probabilities (gives lse)
       bool ok = true;
       for (int j = 0; j < nkv; ++j, ++s_cnt) {
         if (!warp_wait(bar_s_full + t, s_cnt & 1, a.timeout_ns) || *abort_flag) {
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float alpha = (m2 == -INFINITY) ? 0.f : ex2(m2 - m_use);
         const float m_ref = (m_use == -INFINITY) ? 0.f : m_use;
         // probabilities, rounded to bf16 exactly as the P.V MMA will see them
-        float rs0 = 0.f, rs1 = 0.f;
+        float rs0 = 0.f, rs1 = 0.f, re0 = 0.f, re1 = 0.f;
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           uint32_t pk[32];
@@ -378,11 +381,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               pk[ii * 16 + (c >> 1)] = packed;
               rs0 += __uint_as_float(packed << 16);
               rs1 += __uint_as_float(packed & 0xFFFF0000u);
+              re0 += p0;
+              re1 += p1;
             }
           }
           tmem_st32(tS + hf * 32, pk);
         }
         l = l * alpha + (rs0 + rs1);
+        le = le * alpha + (re0 + re1);
         m2 = m_use;
         // rescale the O accumulator when some row of this warp moved its reference.
         // The previous P.V of this tile has completed: the scores just read were
@@ -432,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (row < a.Nq) {
-        const float lse = (l > 0.f) ? (m2 + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
+        const float lse = (le > 0.f) ? (m2 + __log2f(le)) * 0.69314718055994530942f : -INFINITY;
         a.lse[((size_t)b * a.H + h) * a.Nq + row] = lse;
       }
       fence_proxy_async_smem();

@@ -29,10 +29,12 @@
  *    mask admits every key and is a no-op.
  *  - LSE is the natural-log log-sum-exp of the scaled scores of a row:
  *    lse_i = m_i + ln(l_i), with m_i the row max and l_i = sum_j exp(s_ij - m_i).
- *  - A workspace must be zero-filled (cudaMemset) before its first use.  After
- *    that the library keeps it consistent by itself: decode merge tickets reset
- *    themselves and fa_check clears the status word.  Two calls that may run at
- *    the same time on the GPU must not share a workspace.
+ *  - A workspace must be zero-filled (cudaMemset) before its first use, so that
+ *    its status word starts clear.  After that the library keeps it consistent
+ *    by itself: fa_check clears the status word, and the decode merge tickets
+ *    carry a per-call tag, so a workspace may be reused for any shape without
+ *    clearing.  Two calls that may run at the same time on the GPU must not
+ *    share a workspace.
  *  - Every wait inside a kernel is bounded (default about 2 s; environment
  *    variable FA_WAIT_TIMEOUT_MS overrides it).  A wait that runs out makes the
  *    kernel record FA_ERR_TIMEOUT in the workspace's status word and return

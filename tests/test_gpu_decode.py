@@ -53,6 +53,20 @@ def test_repeated_calls_reuse_workspace():
         _check([777, 3000, 64], 16, 128, 500 + i)
 
 
+def test_workspace_reuse_across_shapes():
+    """One workspace reused by calls whose partial-state layout differs (the merge
+    tickets of a later call land where an earlier call kept partial states)."""
+    ws = torch.zeros(1 << 24, dtype=torch.uint8, device="cuda")
+    for lengths, H in (([900, 50], 12), ([300, 17, 1024], 40), ([64], 3), ([2000, 5, 700, 1], 24)):
+        q, k, v, cu = synth.decode_inputs(len(lengths) + H, lengths, H, 128)
+        o, lse = fa_decode_splitkv(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), max(lengths), ws=ws)
+        torch.cuda.synchronize()
+        assert fa_check(ws) == 0
+        o_ref, lse_ref = oracle.decode(f64(q), f64(k), f64(v), cu.numpy(), default_scale(128))
+        compare_o(f64(o), o_ref)
+        compare_lse(f64(lse), lse_ref)
+
+
 def test_batched_ragged_full_size_sampled():
     """64 sequences, H=32, d=128, lengths uniform in [512, 16384] (seed 54004), packed with
     cu_seqlens; outputs of sampled sequences are checked against the oracle."""
