@@ -1,0 +1,497 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200.
+
+One step = forward + recompute backward of causal multi-head attention at the
+GPT-2-medium attention shape (B=64, H=16, N=1024, d=64, bf16), the workload the
+headline metric is quoted on.  The value is algorithmic TFLOP/s of the whole job:
+(4 + 10) * B * H * d * (causal pairs) per step, summed over ranks, divided by the
+slowest rank's device time.  The other workloads (long prefill, decode, long
+training sequence) are timed once each and reported under "extra".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With --gpus N > 1 it runs under torchrun, one process per GPU; every rank
+processes its own full workload (weak scaling, no data exchange), and only the
+timing is reduced (max over ranks).  ``--impl reference`` times the fp64 CPU
+oracle on a bounded sample of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOPS (% of BF16 tensor peak); decode KV GB/s (% of HBM)"
+WORKLOAD = dict(B=64, H=16, N=1024, d=64, causal=True)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2 ** 20
+
+
+# ----------------------------------------------------------------------------- work counts
+
+def causal_pairs(Nq: int, Nk: int, causal: bool) -> int:
+    if not causal:
+        return Nq * Nk
+    return sum(max(0, min(Nk, i + 1 + Nk - Nq)) for i in range(Nq))
+
+
+def fwd_flops(B, H, Nq, Nk, d, causal):
+    return 4 * B * H * d * causal_pairs(Nq, Nk, causal)
+
+
+def bwd_flops(B, H, Nq, Nk, d, causal):
+    return 10 * B * H * d * causal_pairs(Nq, Nk, causal)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """SM clock, power and clock-event (throttle) reasons sampled through NVML every
+    20 ms while active (the data nvidia-smi's clocks query shows)."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4}
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self._stop = None
+        self._thread = None
+
+    def start(self):
+        import threading
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML unavailable: no clock record
+            return
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                    rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                    self.samples.append((sm, rs, pw))
+                except Exception:
+                    pass
+                time.sleep(0.02)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
+
+    def stop(self):
+        if self._thread is None:
+            return None
+        self._stop.set()
+        self._thread.join(timeout=2)
+        if not self.samples:
+            return None
+        sm = [x[0] for x in self.samples]
+        reasons = sorted({n for _, rs, _ in self.samples for n, bit in self.REASONS.items() if rs & bit})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "power_w_max": round(max(x[2] for x in self.samples), 1), "samples": len(self.samples)}
+
+
+# ----------------------------------------------------------------------------- timing helpers
+
+def device_time_ms(fn, iters, stream=None):
+    stream = stream or torch.cuda.current_stream()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record(stream)
+    for i in range(iters):
+        fn(i)
+    e.record(stream)
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / iters
+
+
+def profile_kernels(fa):
+    """Per-kernel launches and device time recorded by the library's launch profiler."""
+    import ctypes
+    lib = fa.load()
+    lib.fa_profile_get.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(ctypes.c_int),
+                                   ctypes.POINTER(ctypes.c_double)]
+    out = {}
+    for i in range(lib.fa_profile_count()):
+        name = ctypes.c_char_p()
+        n = ctypes.c_int()
+        ms = ctypes.c_double()
+        if lib.fa_profile_get(i, ctypes.byref(name), ctypes.byref(n), ctypes.byref(ms)) == 0 and n.value:
+            out[name.value.decode()] = {"launches": n.value, "total_ms": ms.value}
+    return out
+
+
+def source_sha(fname):
+    with open(os.path.join(ROOT, "exact_io_aware_54_b200", "csrc", fname), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def committed_traffic(kernel):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source is unchanged."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)[kernel]
+        if t["source_sha256_16"] != source_sha(t["source_file"]):
+            return None
+        return float(t["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import exact_io_aware_54_b200 as fa
+    from exact_io_aware_54_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    B, H, N, d, causal = (WORKLOAD[k] for k in ("B", "H", "N", "d", "causal"))
+    q, k, v, do = synth.prefill_inputs(synth.SEEDS["gpt2m"] + 1000 * rank, B, N, N, H, d, with_dout=True,
+                                       device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def step(_i=0):
+        fa.fa_fwd(q, k, v, causal=causal, out=o, lse=lse)
+        fa.fa_bwd(q, k, v, o, do, lse, causal=causal, dq=dq, dk=dk, dv=dv)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert fa.fa_check(fa.workspace(256, dev, "fwd")) == 0 and fa.fa_check(fa.workspace(256, dev, "bwd")) == 0
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    fa.load().fa_profile_start()
+    ms = device_time_ms(step, args.steps)
+    fa.load().fa_profile_stop()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    kernels = profile_kernels(fa)
+
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    ms_max = float(t.item())
+    step_flops = fwd_flops(B, H, N, N, d, causal) + bwd_flops(B, H, N, N, d, causal)
+    value = world * step_flops / (ms_max * 1e-3) / 1e12
+
+    pk, pk_src = peaks()
+    # roofline of the dominant kernel (largest device time in the timed region)
+    work = {"fa_fwd_kernel": ("tensor", fwd_flops(B, H, N, N, d, causal)),
+            "fa_bwd_main_kernel": ("tensor", bwd_flops(B, H, N, N, d, causal)),
+            "fa_bwd_preprocess_kernel": ("hbm", B * N * H * d * (2 + 2 + 4) + B * H * N * 4),
+            "fa_bwd_convert_kernel": ("hbm", B * N * H * d * (4 + 2))}
+    per_kernel = {}
+    for name, kv in kernels.items():
+        avg = kv["total_ms"] / kv["launches"]
+        bound, units = work.get(name, ("hbm", 0))
+        ach = units / (avg * 1e-3) / (1e12 if bound == "tensor" else 1e9)
+        peak = pk["bf16_tflops"] if bound == "tensor" else pk["hbm_gbs"]
+        per_kernel[name] = {"launches": kv["launches"], "avg_ms": round(avg, 5), "bound": bound,
+                            "achieved": round(ach, 1), "unit": "TFLOP/s" if bound == "tensor" else "GB/s",
+                            "frac": round(ach / peak, 4)}
+    dom = max(kernels, key=lambda n: kernels[n]["total_ms"]) if kernels else None
+    roofline = None
+    if dom:
+        pkk = per_kernel[dom]
+        src = {"fa_fwd_kernel": "fwd_sm100.cu"}.get(dom, "bwd_sm100.cu")
+        roofline = {"kernel": dom, "bound": pkk["bound"], "achieved": pkk["achieved"],
+                    "peak": pk["bf16_tflops"] if pkk["bound"] == "tensor" else pk["hbm_gbs"],
+                    "peak_source": pk_src + (" burst bf16 (cuBLAS)" if pkk["bound"] == "tensor" else " copy"),
+                    "unit": pkk["unit"], "frac": pkk["frac"], "traffic": committed_traffic(dom),
+                    "algorithmic_units_per_launch": work[dom][1], "source": src}
+
+    launches = sum(kv["launches"] for kv in kernels.values())
+
+    # end to end through the public API: pinned host inputs in, gradients out, every step
+    e2e = None
+    if True:
+        hq, hk, hv, hdo = (x.cpu().pin_memory() for x in (q, k, v, do))
+        hdq, hdk, hdv = (torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in (dq, dk, dv))
+        dq2, dk2, dv2 = torch.empty_like(dq), torch.empty_like(dk), torch.empty_like(dv)
+        q2, k2, v2, do2 = (torch.empty_like(x) for x in (q, k, v, do))
+
+        def e2e_step(_i=0):
+            q2.copy_(hq, non_blocking=True)
+            k2.copy_(hk, non_blocking=True)
+            v2.copy_(hv, non_blocking=True)
+            do2.copy_(hdo, non_blocking=True)
+            fa.fa_fwd(q2, k2, v2, causal=causal, out=o, lse=lse)
+            fa.fa_bwd(q2, k2, v2, o, do2, lse, causal=causal, dq=dq2, dk=dk2, dv=dv2)
+            hdq.copy_(dq2, non_blocking=True)
+            hdk.copy_(dk2, non_blocking=True)
+            hdv.copy_(dv2, non_blocking=True)
+
+        e2e_step()
+        n_e2e = max(3, min(args.steps, 10))
+        e_ms = device_time_ms(e2e_step, n_e2e)
+        et = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+        if world > 1:
+            torch.distributed.all_reduce(et, op=torch.distributed.ReduceOp.MAX)
+        hin = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
+        hout = sum(x.numel() * x.element_size() for x in (hdq, hdk, hdv))
+        e2e = {"value": round(world * step_flops / (float(et.item()) * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": hin, "d2h_bytes_per_step": hout, "ms_per_step": round(float(et.item()), 4)}
+        del hq, hk, hv, hdo, hdq, hdk, hdv, dq2, dk2, dv2, q2, k2, v2, do2
+
+    extra = run_extra(args, fa, synth, dev, pk) if (rank == 0 and not args.no_extra) else None
+    del q, k, v, do, o, lse, dq, dk, dv
+    torch.cuda.empty_cache()
+
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu_base = cpu_baseline(args.cpu_seconds)
+
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_max, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,1) bf16)",
+        "config": {"workload": "gpt2-medium-shaped attention training step: fwd + recompute bwd, causal",
+                   "B": B, "H": H, "N": N, "d": d, "causal": causal, "flops_per_step": step_flops,
+                   "frac_of_peak": round(value / world / pk["bf16_tflops"], 4),
+                   "l2": "no flush: the inputs of one step (Q, K, V, O, dO: 640 MiB) exceed the 126 MB L2",
+                   "parallelism": f"replicas x{world} (independent shards, no collective)"},
+        "roofline": roofline, "kernels": per_kernel, "cpu_baseline": cpu_base, "e2e": e2e,
+        "gpu_launches": launches, "clocks": clocks, "extra": extra,
+    }
+    return line
+
+
+def _rotating(make, total_bytes_of_one):
+    """Enough input sets that consecutive iterations never find their inputs in L2."""
+    n = max(2, math.ceil(3 * L2_BYTES / max(1, total_bytes_of_one)))
+    return [make(i) for i in range(n)]
+
+
+def run_extra(args, fa, synth, dev, pk):
+    out = {}
+    iters = max(5, min(args.steps, 40))
+    # long prefill forward, B=1 H=32 N=8192 d=128 (causal and not)
+    sets = _rotating(lambda i: synth.prefill_inputs(synth.SEEDS["prefill8k"] + 10 * i, 1, 8192, 8192, 32, 128,
+                                                    device=dev), 3 * 64 * 2 ** 20)
+    o = torch.empty_like(sets[0][0])
+    lse = torch.empty(1, 32, 8192, dtype=torch.float32, device=dev)
+    for causal in (True, False):
+        def f(i, causal=causal):
+            q, k, v = sets[i % len(sets)]
+            fa.fa_fwd(q, k, v, causal=causal, out=o, lse=lse)
+        for i in range(3):
+            f(i)
+        ms = device_time_ms(f, iters)
+        tf = fwd_flops(1, 32, 8192, 8192, 128, causal) / (ms * 1e-3) / 1e12
+        out["prefill8k_fwd_causal" if causal else "prefill8k_fwd_noncausal"] = {
+            "ms": round(ms, 4), "TFLOP/s": round(tf, 1), "frac_of_peak": round(tf / pk["bf16_tflops"], 4),
+            "l2": f"{len(sets)} rotating input sets"}
+    del sets, o, lse
+    torch.cuda.empty_cache()
+
+    # decode: single request, L=8192, H=32, d=128
+    L = 8192
+    sets = _rotating(lambda i: tuple(t.to(dev) for t in synth.decode_inputs(synth.SEEDS["decode"] + 10 * i, [L], 32,
+                                                                            128, device=dev)), 2 * L * 32 * 128 * 2)
+    o = torch.empty_like(sets[0][0])
+    lse = torch.empty(1, 32, dtype=torch.float32, device=dev)
+
+    def g(i):
+        q, k, v, cu = sets[i % len(sets)]
+        fa.fa_decode_splitkv(q, k, v, cu, L, out=o, lse=lse)
+    for i in range(3):
+        g(i)
+    ms = device_time_ms(g, max(20, iters))
+    gbs = 2 * 2 * 32 * 128 * L / (ms * 1e-3) / 1e9
+    out["decode_single_8k"] = {"ms": round(ms, 5), "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4),
+                               "splits": fa.fa_decode_num_splits(1, 32, L, 128, 0),
+                               "l2": f"{len(sets)} rotating KV caches"}
+    del sets, o, lse
+    torch.cuda.empty_cache()
+
+    # decode: 64 ragged sequences, lengths U[512, 16384]
+    lengths = synth.ragged_lengths(synth.SEEDS["decode"], 64, 512, 16384)
+    q, k, v, cu = synth.decode_inputs(synth.SEEDS["decode"], lengths, 32, 128, device=dev)
+    cu = cu.to(dev)
+    maxL = int(lengths.max())
+    o = torch.empty_like(q)
+    lse = torch.empty(64, 32, dtype=torch.float32, device=dev)
+
+    def g2(i):
+        fa.fa_decode_splitkv(q, k, v, cu, maxL, out=o, lse=lse)
+    for i in range(3):
+        g2(i)
+    ms = device_time_ms(g2, iters)
+    kv_bytes = 2 * 2 * 32 * 128 * int(lengths.sum())
+    gbs = kv_bytes / (ms * 1e-3) / 1e9
+    out["decode_batched_ragged"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                                    "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4), "kv_bytes": kv_bytes,
+                                    "splits": fa.fa_decode_num_splits(64, 32, maxL, 128, 0),
+                                    "l2": "no flush: KV cache is 70x the L2"}
+    del q, k, v, cu, o, lse
+    torch.cuda.empty_cache()
+
+    # long training sequence, B=1 H=16 N=16384 d=64 causal: fwd + bwd and peak memory
+    q, k, v, do = synth.prefill_inputs(synth.SEEDS["long16k"], 1, 16384, 16384, 16, 64, with_dout=True, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(1, 16, 16384, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_f = fa.workspace(fa.fa_fwd_workspace_size(1, 16, 16384, 16384, 64), dev, "long16k_fwd")
+    ws_b = fa.workspace(fa.fa_bwd_workspace_size(1, 16, 16384, 16384, 64), dev, "long16k_bwd")
+    torch.cuda.synchronize()
+    base = torch.cuda.memory_allocated(dev)
+    torch.cuda.reset_peak_memory_stats(dev)
+    free0, _ = torch.cuda.mem_get_info(dev)
+
+    def h(i):
+        fa.fa_fwd(q, k, v, causal=True, out=o, lse=lse, ws=ws_f)
+        fa.fa_bwd(q, k, v, o, do, lse, causal=True, dq=dq, dk=dk, dv=dv, ws=ws_b)
+    for i in range(2):
+        h(i)
+    ms = device_time_ms(h, max(3, iters // 2))
+    free1, _ = torch.cuda.mem_get_info(dev)
+    peak_extra = torch.cuda.max_memory_allocated(dev) - base
+    fl = fwd_flops(1, 16, 16384, 16384, 64, True) + bwd_flops(1, 16, 16384, 16384, 64, True)
+    tf = fl / (ms * 1e-3) / 1e12
+    out["long16k_fwd_bwd"] = {
+        "ms": round(ms, 4), "TFLOP/s": round(tf, 1), "frac_of_peak": round(tf / pk["bf16_tflops"], 4),
+        "peak_alloc_increase_bytes_during_calls": int(peak_extra),
+        "device_free_bytes_change": int(free0 - free1),
+        "workspace_bytes": int(ws_f.numel() + ws_b.numel()),
+        "one_NxN_bf16_matrix_bytes": 16384 * 16384 * 2,
+        "o_n_memory_ok": bool(peak_extra < 16384 * 16384 * 2 and (ws_f.numel() + ws_b.numel()) < 16384 * 16384 * 2)}
+    return out
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def _oracle_sample(seconds, step_idx=0, heads=16):
+    """Time the fp64 oracle (fwd + bwd) on `heads` heads of one batch element of the
+    bench workload, repeated until `seconds` of oracle time have passed (at least
+    once); input generation is not timed.  Returns (algorithmic flops, seconds, heads)."""
+    import oracle
+    from exact_io_aware_54_b200 import synth
+    B, H, N, d, causal = (WORKLOAD[k] for k in ("B", "H", "N", "d", "causal"))
+    scale = 1.0 / math.sqrt(d)
+    flops, el, calls = 0, 0.0, 0
+    while True:
+        b = (step_idx * 7 + calls) % B
+        q, k, v, do = synth.prefill_inputs(synth.SEEDS["gpt2m"] + 17 * b, 1, N, N, H, d, with_dout=True)
+        arrs = [x[:, :, :heads].double().numpy() for x in (q, k, v, do)]
+        ts = time.perf_counter()
+        oracle.attn_fwd(arrs[0], arrs[1], arrs[2], causal, scale)
+        oracle.attn_bwd(*arrs, causal, scale)
+        el += time.perf_counter() - ts
+        calls += 1
+        flops += fwd_flops(1, heads, N, N, d, causal) + bwd_flops(1, heads, N, N, d, causal)
+        if el >= seconds:
+            return flops, el, calls * heads
+
+
+def cpu_baseline(seconds):
+    import oracle
+    flops, el, heads = _oracle_sample(seconds)
+    return {"value": round(flops / el / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{heads} whole heads (16 per call) of the B=64 H=16 N=1024 d=64 causal step, "
+                      f"fp64 fwd + bwd, {el:.1f} s of oracle time"}
+
+
+def run_reference(args, rank):
+    """The oracle as it stands, one bounded sample of the workload per step."""
+    if rank != 0:
+        return None
+    import oracle
+    n = args.steps + args.warmup
+    heads = 16 if n <= 60 else (4 if n <= 300 else 1)
+    for i in range(args.warmup):
+        _oracle_sample(0.0, i, heads)
+    t_flops, t_el, done = 0, 0.0, 0
+    for i in range(args.steps):
+        f, el, hd = _oracle_sample(0.0, i, heads)
+        t_flops += f
+        t_el += el
+        done += hd
+    value = t_flops / t_el / 1e12
+    sample = f"{heads} whole head(s) of one batch element per step ({done} heads in total), fp64 fwd + bwd"
+    cpu = {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+           "sample": sample}
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * t_el / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded N(0,1) bf16, widened to fp64)",
+            "config": {"workload": "gpt2-medium-shaped attention training step: fwd + recompute bwd, causal",
+                       **{k: WORKLOAD[k] for k in ("B", "H", "N", "d", "causal")}, "sample": sample},
+            "cpu_baseline": cpu, "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                                         "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        line = run_reference(args, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

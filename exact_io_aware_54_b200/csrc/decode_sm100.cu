@@ -22,8 +22,8 @@
 //    shuffle levels, the stage max three; every lane keeps a partial u over the
 //    keys of its slot, summed across slots once at the end.
 //  * The last warp of each (sequence, head) to finish its chunk -- found with an
-//    atomic ticket tagged with the call's epoch -- merges the chunk states and
-//    writes o and lse.  A sequence with a single chunk skips the
+//    atomic ticket -- merges the chunk states and writes o and lse, then resets
+//    the ticket, so tickets are zero between calls.  A sequence with a single chunk skips the
 //    partial-state round trip.
 #include "fa_internal.h"
 #include "ptx.cuh"
@@ -55,8 +55,7 @@ struct DecArgs {
   __nv_bfloat16* o;
   float* lse;
   int* status;
-  unsigned long long* tickets;
-  unsigned int epoch;
+  unsigned int* tickets;
   float* part_ml;
   float* part_u;
   int B, H, max_seqlen_k;
@@ -75,21 +74,6 @@ __device__ __forceinline__ void bf16x8_to_f32(uint32_t a, uint32_t b, uint32_t c
   f[5] = __uint_as_float(c & 0xFFFF0000u);
   f[6] = __uint_as_float(d << 16);
   f[7] = __uint_as_float(d & 0xFFFF0000u);
-}
-
-// Arrival on a merge ticket.  A ticket holds (call epoch << 32 | arrivals); a
-// ticket whose epoch is not this call's -- stale or never initialised -- counts
-// as zero arrivals, so the workspace needs no clearing between calls.  Returns
-// the number of arrivals of this call including this one.
-__device__ __forceinline__ unsigned ticket_arrive(unsigned long long* t, unsigned epoch) {
-  unsigned long long old = *reinterpret_cast<volatile unsigned long long*>(t), assumed;
-  do {
-    assumed = old;
-    const unsigned long long next =
-        ((assumed >> 32) == epoch) ? assumed + 1 : ((static_cast<unsigned long long>(epoch) << 32) | 1ull);
-    old = atomicCAS(t, assumed, next);
-  } while (old != assumed);
-  return ((old >> 32) == epoch) ? static_cast<unsigned>(old & 0xffffffffu) + 1u : 1u;
 }
 
 template <int D>
@@ -308,13 +292,17 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
   __threadfence();
   __syncwarp();
   int last = 0;
-  if (lane == 0) last = (ticket_arrive(a.tickets + bh, a.epoch) == nsplit) ? 1 : 0;
+  if (lane == 0) last = (atomicAdd(a.tickets + bh, 1u) == (unsigned)(nsplit - 1)) ? 1 : 0;
   last = __shfl_sync(0xffffffffu, last, 0);
   if (!last) return;
   __threadfence();
 
   // ------------------------------------------------------------------ merge (last chunk of b, h)
+  // Pass 1: lanes stride over the chunks for the common reference max.  Pass 2:
+  // batches of 16 chunks issue all their loads before any use, so the chain of
+  // L2 round trips is nsplit / 16 long rather than nsplit.
   constexpr int kPerLane = D / 32;
+  constexpr int kBatch = 16;
   const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + bh * a.splits;
   float M = -INFINITY;
   for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, __ldcg(ml + s).x);
@@ -325,20 +313,32 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
 #pragma unroll
   for (int e = 0; e < kPerLane; ++e) U[e] = 0.f;
   const float* pu = a.part_u + bh * a.splits * D + lane * kPerLane;
-  for (int s = 0; s < nsplit; ++s) {
-    const float2 st = __ldcg(ml + s);
-    const float w = (st.x == -INFINITY) ? 0.f : ex2(st.x - M_ref);
-    Lsum = fmaf(w, st.y, Lsum);
-    if constexpr (kPerLane == 4) {
-      const float4 uu = __ldcg(reinterpret_cast<const float4*>(pu + (size_t)s * D));
-      U[0] = fmaf(w, uu.x, U[0]);
-      U[1] = fmaf(w, uu.y, U[1]);
-      U[2] = fmaf(w, uu.z, U[2]);
-      U[3] = fmaf(w, uu.w, U[3]);
-    } else {
-      const float2 uu = __ldcg(reinterpret_cast<const float2*>(pu + (size_t)s * D));
-      U[0] = fmaf(w, uu.x, U[0]);
-      U[1] = fmaf(w, uu.y, U[1]);
+  for (int s0 = 0; s0 < nsplit; s0 += kBatch) {
+    float2 st[kBatch];
+    float uu[kBatch][kPerLane];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int s = min(s0 + i, nsplit - 1);
+      st[i] = __ldcg(ml + s);
+      if constexpr (kPerLane == 4) {
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(pu + (size_t)s * D));
+        uu[i][0] = x.x;
+        uu[i][1] = x.y;
+        uu[i][2] = x.z;
+        uu[i][3] = x.w;
+      } else {
+        const float2 x = __ldcg(reinterpret_cast<const float2*>(pu + (size_t)s * D));
+        uu[i][0] = x.x;
+        uu[i][1] = x.y;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const bool live = (s0 + i) < nsplit;
+      const float w = (!live || st[i].x == -INFINITY) ? 0.f : ex2(st[i].x - M_ref);
+      Lsum = fmaf(w, st[i].y, Lsum);
+#pragma unroll
+      for (int e = 0; e < kPerLane; ++e) U[e] = fmaf(w, uu[i][e], U[e]);
     }
   }
   const float inv = (Lsum > 0.f) ? 1.f / Lsum : 0.f;
@@ -346,7 +346,10 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
 #pragma unroll
   for (int e = 0; e < kPerLane; e += 2)
     *reinterpret_cast<uint32_t*>(out + e) = pack_bf16x2(U[e] * inv, U[e + 1] * inv);
-  if (lane == 0) a.lse[bh] = (Lsum > 0.f) ? (M + __log2f(Lsum)) * 0.69314718055994530942f : -INFINITY;
+  if (lane == 0) {
+    a.lse[bh] = (Lsum > 0.f) ? (M + __log2f(Lsum)) * 0.69314718055994530942f : -INFINITY;
+    a.tickets[bh] = 0u;  // every chunk of (b, h) has arrived: ready for the next call
+  }
 }
 
 // Optional argument check of cu_seqlens (FA_CHECKS=1).
@@ -399,8 +402,8 @@ DecodePlan decode_plan(int B, int H, int max_seqlen_k, int d, int num_splits) {
 
 size_t decode_workspace_bytes(int B, int H, int d, const DecodePlan& plan) {
   auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-  size_t bytes = kStatusBytes;
-  bytes += up(sizeof(unsigned long long) * (size_t)B * H);
+  size_t bytes = kStatusBytes + kDecodeTicketBytes;
+  if ((size_t)B * H > kDecodeFixedTickets) bytes += up(sizeof(unsigned) * (size_t)B * H);
   bytes += up(sizeof(float) * 2 * (size_t)B * H * plan.splits);
   bytes += up(sizeof(float) * (size_t)d * B * H * plan.splits);
   return bytes;
@@ -427,7 +430,6 @@ static fa_status launch_decode_impl(const DecodeLaunch& L0, cudaStream_t stream)
   a.lse = L0.lse;
   a.status = L0.status;
   a.tickets = L0.tickets;
-  a.epoch = L0.epoch;
   a.part_ml = L0.part_ml;
   a.part_u = L0.part_u;
   a.B = L0.B;
@@ -439,14 +441,24 @@ static fa_status launch_decode_impl(const DecodeLaunch& L0, cudaStream_t stream)
   a.scale_log2 = L0.scale * 1.4426950408889634f;
   a.check_args = L0.check_args;
   a.timeout_ns = L0.timeout_ns;
+  if (L0.clear_tickets) {
+    if (cudaMemsetAsync(L0.tickets, 0, sizeof(unsigned) * (size_t)L0.B * L0.H, stream) != cudaSuccess)
+      return FA_ERR_CUDA;
+  }
   if (L0.check_args) {
+    prof_before(stream, kKDecodeCheck);
     check_cu_seqlens_kernel<<<(L0.B + 256) / 256, 256, 0, stream>>>(L0.cu_seqlens, L0.B, L0.max_seqlen_k,
                                                                       L0.status);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    const cudaError_t err = cudaGetLastError();
+    prof_after(stream, kKDecodeCheck);
+    if (err != cudaSuccess) return FA_ERR_CUDA;
   }
   dim3 grid(L0.plan.splits, L0.plan.groups, L0.B);
+  prof_before(stream, kKDecode);
   decode_kernel<D><<<grid, kThreads, L::kSmemBytes, stream>>>(a);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  const cudaError_t err = cudaGetLastError();
+  prof_after(stream, kKDecode);
+  return err == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status launch_decode(const DecodeLaunch& L0, cudaStream_t stream) {

@@ -5,12 +5,67 @@
 #include <string.h>
 
 #include <atomic>
-#include <chrono>
 #include <mutex>
+#include <vector>
 
 #include "fa_internal.h"
 
 namespace fa {
+
+// ----------------------------------------------------------------------------- launch profiler
+
+namespace {
+const char* const kKernelNames[kKCount] = {"fa_fwd_kernel", "fa_bwd_preprocess_kernel", "fa_bwd_main_kernel",
+                                           "fa_bwd_convert_kernel", "fa_decode_kernel",
+                                           "fa_decode_check_kernel"};
+struct ProfRecord {
+  int kernel;
+  cudaEvent_t start, stop;
+};
+std::mutex g_prof_mu;
+std::atomic<bool> g_prof_on{false};
+std::vector<cudaEvent_t> g_event_pool;
+size_t g_pool_used = 0;
+std::vector<ProfRecord> g_records;
+int g_launches[kKCount] = {};
+double g_total_ms[kKCount] = {};
+bool g_prof_error = false;
+
+cudaEvent_t pool_event() {
+  if (g_pool_used == g_event_pool.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      g_prof_error = true;
+      return nullptr;
+    }
+    g_event_pool.push_back(e);
+  }
+  return g_event_pool[g_pool_used++];
+}
+}  // namespace
+
+void prof_before(cudaStream_t s, int kernel_id) {
+  if (!g_prof_on.load(std::memory_order_relaxed)) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  ProfRecord r;
+  r.kernel = kernel_id;
+  r.start = pool_event();
+  r.stop = pool_event();
+  if (!r.start || !r.stop) return;
+  if (cudaEventRecord(r.start, s) != cudaSuccess) g_prof_error = true;
+  g_records.push_back(r);
+}
+
+void prof_after(cudaStream_t s, int kernel_id) {
+  if (!g_prof_on.load(std::memory_order_relaxed)) return;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto it = g_records.rbegin(); it != g_records.rend(); ++it) {
+    if (it->kernel == kernel_id) {
+      if (cudaEventRecord(it->stop, s) != cudaSuccess) g_prof_error = true;
+      return;
+    }
+  }
+}
 
 int num_sms() {
   static int cached[64] = {};
@@ -86,19 +141,6 @@ static bool dims_ok(int B, int H, int Nq, int Nk, int d) {
 }
 
 static float resolve_scale(float s, int d) { return s > 0.f ? s : 1.0f / sqrtf((float)d); }
-
-// Call epochs for the decode merge tickets: distinct for every call in this
-// process, and started from the clock so that a workspace left by an earlier
-// process is unlikely to carry a matching tag.
-static unsigned next_epoch() {
-  static std::atomic<unsigned> counter{static_cast<unsigned>(
-      std::chrono::steady_clock::now().time_since_epoch().count() * 2654435761ull)};
-  unsigned e;
-  do {
-    e = counter.fetch_add(1, std::memory_order_relaxed) + 1;
-  } while (e == 0);
-  return e;
-}
 
 }  // namespace fa
 
@@ -227,12 +269,17 @@ fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, const i
   a.lse = lse;
   a.status = reinterpret_cast<int*>(ws);
   size_t off = kStatusBytes;
-  a.tickets = reinterpret_cast<unsigned long long*>(ws + off);
-  a.epoch = next_epoch();
-  off += up256(sizeof(unsigned long long) * (size_t)B * H);
+  a.tickets = reinterpret_cast<unsigned*>(ws + off);
+  a.clear_tickets = 0;
+  off += kDecodeTicketBytes;
   a.part_ml = reinterpret_cast<float*>(ws + off);
   off += up256(sizeof(float) * 2 * (size_t)B * H * plan.splits);
   a.part_u = reinterpret_cast<float*>(ws + off);
+  off += up256(sizeof(float) * (size_t)d * B * H * plan.splits);
+  if ((size_t)B * H > kDecodeFixedTickets) {
+    a.tickets = reinterpret_cast<unsigned*>(ws + off);
+    a.clear_tickets = 1;
+  }
   a.B = B;
   a.H = H;
   a.max_seqlen_k = max_seqlen_k;
@@ -242,6 +289,49 @@ fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, const i
   a.check_args = checks_enabled() ? 1 : 0;
   a.timeout_ns = wait_timeout_ns();
   return launch_decode(a, stream);
+}
+
+fa_status fa_profile_start(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_records.clear();
+  g_pool_used = 0;
+  g_prof_error = false;
+  for (int i = 0; i < kKCount; ++i) {
+    g_launches[i] = 0;
+    g_total_ms[i] = 0.0;
+  }
+  g_prof_on.store(true);
+  return FA_OK;
+}
+
+fa_status fa_profile_stop(void) {
+  g_prof_on.store(false);
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  bool bad = g_prof_error;
+  for (const ProfRecord& r : g_records) {
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) {
+      cudaGetLastError();
+      bad = true;
+      continue;
+    }
+    g_launches[r.kernel] += 1;
+    g_total_ms[r.kernel] += ms;
+  }
+  g_records.clear();
+  g_pool_used = 0;
+  return bad ? FA_ERR_CUDA : FA_OK;
+}
+
+int fa_profile_count(void) { return kKCount; }
+
+fa_status fa_profile_get(int id, const char** name, int* launches, double* total_ms) {
+  if (id < 0 || id >= kKCount) return FA_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  if (name) *name = kKernelNames[id];
+  if (launches) *launches = g_launches[id];
+  if (total_ms) *total_ms = g_total_ms[id];
+  return FA_OK;
 }
 
 fa_status fa_check(void* workspace, cudaStream_t stream) {

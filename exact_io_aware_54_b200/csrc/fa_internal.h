@@ -15,9 +15,23 @@ namespace fa {
 // Workspace: the first kStatusBytes hold the status word (int32) and padding.
 constexpr size_t kStatusBytes = 256;
 
+// Decode merge tickets live in a fixed region right after the status word, so
+// they stay at the same place whatever the shape of the call; the last arrival
+// of every (sequence, head) resets its ticket.  Calls with more than
+// kDecodeFixedTickets (sequence, head) pairs use a region after the partial
+// states that is cleared on every call.
+constexpr size_t kDecodeFixedTickets = 65536;
+constexpr size_t kDecodeTicketBytes = kDecodeFixedTickets * 4;
+
 // Status codes recorded by kernels in the workspace status word (fa_status values).
 constexpr int kStatusTimeout = 6;
 constexpr int kStatusBadArg = 1;
+
+// Kernels the library launches (for the optional launch profiler).
+enum KernelId { kKFwd = 0, kKBwdPre, kKBwdMain, kKBwdConvert, kKDecode, kKDecodeCheck, kKCount };
+// Bracket a launch with profiling events when profiling is on (no-ops otherwise).
+void prof_before(cudaStream_t s, int kernel_id);
+void prof_after(cudaStream_t s, int kernel_id);
 
 // Number of SMs of the current device (cached per device).
 int num_sms();
@@ -75,8 +89,8 @@ struct DecodeLaunch {
   void* o;
   float* lse;
   int* status;
-  unsigned long long* tickets;  // [B * H] merge tickets, epoch-tagged (no clearing needed)
-  unsigned int epoch;           // distinct per call
+  unsigned int* tickets;  // [B * H] merge tickets, zero between calls
+  int clear_tickets;      // tickets live outside the fixed region: clear them first
   float* part_ml;      // [B, H, splits, 2]  (m in log2 units, l)
   float* part_u;       // [B, H, splits, d]
   int B, H, max_seqlen_k, d;

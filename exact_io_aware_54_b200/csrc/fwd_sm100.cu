@@ -502,8 +502,11 @@ static fa_status launch_fwd_impl(const FwdLaunch& L0, cudaStream_t stream) {
   a.n_items = a.n_pairs * L0.B * L0.H;
   a.timeout_ns = L0.timeout_ns;
   const int grid = std::min(a.n_items, num_sms() * 1);
+  prof_before(stream, kKFwd);
   fwd_kernel<D><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  const cudaError_t err = cudaGetLastError();
+  prof_after(stream, kKFwd);
+  return err == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status launch_fwd(const FwdLaunch& L0, cudaStream_t stream) {

@@ -29,12 +29,12 @@
  *    mask admits every key and is a no-op.
  *  - LSE is the natural-log log-sum-exp of the scaled scores of a row:
  *    lse_i = m_i + ln(l_i), with m_i the row max and l_i = sum_j exp(s_ij - m_i).
- *  - A workspace must be zero-filled (cudaMemset) before its first use, so that
- *    its status word starts clear.  After that the library keeps it consistent
- *    by itself: fa_check clears the status word, and the decode merge tickets
- *    carry a per-call tag, so a workspace may be reused for any shape without
- *    clearing.  Two calls that may run at the same time on the GPU must not
- *    share a workspace.
+ *  - A workspace must be zero-filled (cudaMemset) before its first use.  After
+ *    that the library keeps it consistent by itself and it may be reused for
+ *    any shape: fa_check clears the status word, and the decode merge tickets
+ *    sit at a fixed place and reset themselves.  After fa_check has reported
+ *    FA_ERR_TIMEOUT, zero the workspace again before reusing it.  Two calls
+ *    that may run at the same time on the GPU must not share a workspace.
  *  - Every wait inside a kernel is bounded (default about 2 s; environment
  *    variable FA_WAIT_TIMEOUT_MS overrides it).  A wait that runs out makes the
  *    kernel record FA_ERR_TIMEOUT in the workspace's status word and return
@@ -145,6 +145,24 @@ FA_API const char* fa_status_string(fa_status status);
 
 /* Library version as "major.minor.patch" (static string). */
 FA_API const char* fa_version(void);
+
+/*
+ * Launch profiling (off by default; the pages ask for evidence of which kernel
+ * actually ran -- "FlashAttention saves IO, not N^2 work", section 8).
+ * Between fa_profile_start and fa_profile_stop every kernel the library
+ * launches is bracketed by a pair of CUDA events on its stream.  fa_profile_stop
+ * waits for those events and totals them per kernel; fa_profile_get then
+ * returns, for kernel index `id` in [0, fa_profile_count()), its name, the number
+ * of launches and their summed device time in milliseconds.  Returns FA_OK, or
+ * FA_ERR_INVALID_ARG for a bad index, FA_ERR_CUDA when an event call failed.
+ * The events are driver objects created on first use and kept for reuse; no
+ * device memory is allocated.  Profiling is process-wide and not meant for
+ * concurrent use from several threads.
+ */
+FA_API fa_status fa_profile_start(void);
+FA_API fa_status fa_profile_stop(void);
+FA_API int fa_profile_count(void);
+FA_API fa_status fa_profile_get(int id, const char** name, int* launches, double* total_ms);
 
 #ifdef __cplusplus
 }

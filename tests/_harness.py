@@ -3,7 +3,9 @@
 Tolerances (bf16 inputs, fp32 accumulation, N(0,1) data):
   O    : max |o_gpu - o_oracle| <= 1e-2 and mean |.| <= 1e-3
   LSE  : |lse_gpu - lse_oracle| <= 1e-4 * max(1, |lse_oracle|)
-  dQ/dK/dV : max |g_gpu - g_oracle| / max |g_oracle| <= 2e-2 (per tensor)
+  dQ/dK/dV : max |g_gpu - g_oracle| / max(max |g_oracle|, 1e-3) <= 2e-2 (per tensor)
+             (the 1e-3 floor only matters when the exact gradient is zero, e.g. a
+             single key, where the GPU result is rounding noise of order 1e-7)
 """
 import math
 
@@ -14,6 +16,7 @@ O_MAX_ABS = 1e-2
 O_MEAN_ABS = 1e-3
 LSE_REL = 1e-4
 GRAD_REL = 2e-2
+GRAD_FLOOR = 1e-3
 
 
 def f64(t: torch.Tensor) -> np.ndarray:
@@ -49,11 +52,8 @@ def compare_grad(g_gpu, g_ref, what):
     g_gpu = np.asarray(g_gpu, dtype=np.float64)
     g_ref = np.asarray(g_ref, dtype=np.float64)
     assert np.all(np.isfinite(g_gpu)), f"{what}: non-finite values"
-    scale = float(np.abs(g_ref).max(initial=0.0))
+    scale = max(float(np.abs(g_ref).max(initial=0.0)), GRAD_FLOOR)
     err = float(np.abs(g_gpu - g_ref).max(initial=0.0))
-    if scale == 0.0:
-        assert err == 0.0, f"{what}: expected zeros, max {err}"
-        return 0.0
     assert err / scale <= GRAD_REL, f"{what}: normalised max err {err / scale:.3e} > {GRAD_REL}"
     return err / scale
 
