@@ -173,6 +173,7 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     B, H, N, d, causal = (WORKLOAD[k] for k in ("B", "H", "N", "d", "causal"))
+    B = args.batch or B
     q, k, v, do = synth.prefill_inputs(synth.SEEDS["gpt2m"] + 1000 * rank, B, N, N, H, d, with_dout=True,
                                        device=dev)
     o = torch.empty_like(q)
@@ -464,6 +465,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override B of the step (small cases for profiler captures; 0 = the workload's B=64)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     args = ap.parse_args()
     if args.warmup < 3:
