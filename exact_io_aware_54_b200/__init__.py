@@ -23,7 +23,7 @@ import threading
 import torch
 
 __all__ = [
-    "FAError", "lib_path", "load", "fa_fwd", "fa_bwd", "fa_decode_splitkv", "fa_check",
+    "FAError", "lib_path", "load", "fa_fwd", "fa_bwd", "fa_decode_splitkv", "fa_decode_splitkv_noalloc", "fa_check",
     "fa_fwd_workspace_size", "fa_bwd_workspace_size", "fa_decode_workspace_size", "fa_decode_num_splits",
     "fa_version", "STATUS",
 ]
@@ -67,7 +67,8 @@ def load():
         lib.fa_fwd.argtypes = [_vp] * 5 + [_i] * 6 + [_f, _vp, _sz, _vp]
         lib.fa_bwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _vp, _sz, _vp]
         lib.fa_decode_splitkv.argtypes = [_vp] * 4 + [_i] * 6 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
-        for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_decode_splitkv):
+        lib.fa_decode_splitkv_noalloc.argtypes = [_vp] * 4 + [_i] * 6 + [_f, _i, _vp, _vp, _vp]
+        for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_decode_splitkv, lib.fa_decode_splitkv_noalloc):
             fn.restype = _i
         lib.fa_fwd_workspace_size.argtypes = [_i] * 5
         lib.fa_fwd_workspace_size.restype = _sz
@@ -219,6 +220,26 @@ def fa_decode_splitkv(q, k, v, cu_seqlens_k, max_seqlen_k: int, causal: bool = F
                                int(max_seqlen_k), d, int(bool(causal)), _scale(softmax_scale), int(num_splits),
                                out.data_ptr(), lse.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
     _raise("fa_decode_splitkv", st)
+    return out, lse
+
+
+def fa_decode_splitkv_noalloc(q, k, v, cu_seqlens_k, max_seqlen_k: int, causal: bool = False, softmax_scale=None,
+                              num_splits: int = 0, out=None, lse=None):
+    """fa_decode_splitkv without a workspace: the library's own fixed 16 MiB device
+    scratch holds the chunk states, for callers that cannot allocate device memory.
+    Only the outputs below are allocated here, by torch, when not given."""
+    lib = load()
+    B, H, d = q.shape
+    _check_tensor("q", q, torch.bfloat16)
+    _check_tensor("k", k, torch.bfloat16)
+    _check_tensor("v", v, torch.bfloat16, k.shape)
+    _check_tensor("cu_seqlens_k", cu_seqlens_k, torch.int32, (B + 1,))
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    st = lib.fa_decode_splitkv_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens_k.data_ptr(), B, H, 1,
+                                       int(max_seqlen_k), d, int(bool(causal)), _scale(softmax_scale),
+                                       int(num_splits), out.data_ptr(), lse.data_ptr(), _stream_ptr(q.device))
+    _raise("fa_decode_splitkv_noalloc", st)
     return out, lse
 
 

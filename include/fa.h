@@ -121,6 +121,33 @@ FA_API fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, 
                             float softmax_scale, int num_splits, void* o, float* lse, void* workspace,
                             size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * fa_decode_splitkv without a workspace, for callers that cannot allocate
+ * device memory -- for example an operator inside a host framework that owns
+ * every device allocation and offers it no allocator, or a serving loop that
+ * must never call cudaMalloc (which may synchronise the device).  The pages
+ * have no counterpart of this call; it exists for such callers only.
+ *
+ * Arguments, layouts and results are those of fa_decode_splitkv.  The chunk
+ * states live instead in a scratch array of 16 MiB compiled into the library,
+ * which every GPU that loads the library holds until the process exits.
+ *  - The call allocates nothing.  Its first call on a device looks up the
+ *    array's device address (cudaGetSymbolAddress, with that device current);
+ *    make that first call before any stream capture.
+ *  - Returns FA_ERR_WORKSPACE when the shape needs more than the 16 MiB of
+ *    scratch (B * H * splits * (d + 2) * 4 bytes plus small overheads); pass a
+ *    smaller num_splits then.
+ *  - All calls share the one array, and each call clears the parts that must
+ *    start at zero.  Calls whose kernels may overlap on the GPU (concurrent
+ *    streams, several host threads) therefore race: serialise them.
+ *  - Bounded waits still end a stuck kernel, but there is no workspace for
+ *    fa_check, so this call does not report FA_ERR_TIMEOUT.
+ */
+FA_API fa_status fa_decode_splitkv_noalloc(const void* q, const void* k, const void* v,
+                                           const int32_t* cu_seqlens_k, int B, int H, int Nq,
+                                           int max_seqlen_k, int d, int causal, float softmax_scale,
+                                           int num_splits, void* o, float* lse, cudaStream_t stream);
+
 /* Workspace sizes in bytes for the calls above (0 when the arguments are invalid). */
 FA_API size_t fa_fwd_workspace_size(int B, int H, int Nq, int Nk, int d);
 FA_API size_t fa_bwd_workspace_size(int B, int H, int Nq, int Nk, int d);
