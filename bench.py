@@ -299,9 +299,25 @@ def _rotating(make, total_bytes_of_one):
     return [make(i) for i in range(n)]
 
 
-def run_extra(args, fa, synth, dev, pk):
+EXTRA_WORKLOADS = ("prefill8k", "decode_single", "decode_batched", "long16k")
+
+
+def run_extra(args, fa, synth, dev, pk, only=None):
     out = {}
     iters = max(5, min(args.steps, 40))
+    want = (lambda name: only is None or only == name)
+    if want("prefill8k"):
+        _extra_prefill(out, iters, fa, synth, dev, pk)
+    if want("decode_single"):
+        _extra_decode_single(out, iters, fa, synth, dev, pk)
+    if want("decode_batched"):
+        _extra_decode_batched(out, iters, fa, synth, dev, pk)
+    if want("long16k"):
+        _extra_long16k(out, iters, fa, synth, dev, pk)
+    return out
+
+
+def _extra_prefill(out, iters, fa, synth, dev, pk):
     # long prefill forward, B=1 H=32 N=8192 d=128 (causal and not)
     sets = _rotating(lambda i: synth.prefill_inputs(synth.SEEDS["prefill8k"] + 10 * i, 1, 8192, 8192, 32, 128,
                                                     device=dev), 3 * 64 * 2 ** 20)
@@ -321,6 +337,8 @@ def run_extra(args, fa, synth, dev, pk):
     del sets, o, lse
     torch.cuda.empty_cache()
 
+
+def _extra_decode_single(out, iters, fa, synth, dev, pk):
     # decode: single request, L=8192, H=32, d=128
     L = 8192
     sets = _rotating(lambda i: tuple(t.to(dev) for t in synth.decode_inputs(synth.SEEDS["decode"] + 10 * i, [L], 32,
@@ -341,6 +359,8 @@ def run_extra(args, fa, synth, dev, pk):
     del sets, o, lse
     torch.cuda.empty_cache()
 
+
+def _extra_decode_batched(out, iters, fa, synth, dev, pk):
     # decode: 64 ragged sequences, lengths U[512, 16384]
     lengths = synth.ragged_lengths(synth.SEEDS["decode"], 64, 512, 16384)
     q, k, v, cu = synth.decode_inputs(synth.SEEDS["decode"], lengths, 32, 128, device=dev)
@@ -363,6 +383,8 @@ def run_extra(args, fa, synth, dev, pk):
     del q, k, v, cu, o, lse
     torch.cuda.empty_cache()
 
+
+def _extra_long16k(out, iters, fa, synth, dev, pk):
     # long training sequence, B=1 H=16 N=16384 d=64 causal: fwd + bwd and peak memory
     q, k, v, do = synth.prefill_inputs(synth.SEEDS["long16k"], 1, 16384, 16384, 16, 64, with_dout=True, device=dev)
     o = torch.empty_like(q)
@@ -392,7 +414,6 @@ def run_extra(args, fa, synth, dev, pk):
         "workspace_bytes": int(ws_f.numel() + ws_b.numel()),
         "one_NxN_bf16_matrix_bytes": 16384 * 16384 * 2,
         "o_n_memory_ok": bool(peak_extra < 16384 * 16384 * 2 and (ws_f.numel() + ws_b.numel()) < 16384 * 16384 * 2)}
-    return out
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -465,6 +486,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=EXTRA_WORKLOADS, default=None,
+                    help="time only this one of the other workloads and print its figures (profiling aid)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override B of the step (small cases for profiler captures; 0 = the workload's B=64)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -475,6 +498,15 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.only:
+        # one of the other workloads alone (used for profiler captures); no contract line
+        import exact_io_aware_54_b200 as fa
+        from exact_io_aware_54_b200 import synth
+        dev = torch.device("cuda", local_rank)
+        torch.cuda.set_device(dev)
+        print(json.dumps(run_extra(args, fa, synth, dev, peaks()[0], only=args.only)), flush=True)
+        return
 
     if args.impl == "reference":
         line = run_reference(args, rank)

@@ -8,7 +8,7 @@
 
 #include <algorithm>
 
-#include "../../include/fa.h"
+#include "fa.h"  // include/ (on the compiler include path)
 
 namespace fa {
 
@@ -39,6 +39,9 @@ int num_sms();
 // Encode a TMA descriptor for a bf16 tensor [B, N, H, D] (D innermost), with a
 // box of 128 rows x 64 columns and 128-byte swizzle.  Returns false on failure.
 bool encode_bshd_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int D);
+
+// The same for an fp32 tensor [B, N, H, D]: box of 128 rows x 32 columns (128 bytes), 128-byte swizzle.
+bool encode_bshd_map_f32(CUtensorMap* map, const void* ptr, int B, int N, int H, int D);
 
 struct FwdLaunch {
   const void* q;

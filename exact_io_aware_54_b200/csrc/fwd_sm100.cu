@@ -11,11 +11,13 @@
 // B200 design
 //  * Work item = (b, h, pair of 128-row query tiles).  Persistent grid, one CTA
 //    per SM; items are taken round-robin, heaviest (latest causal rows) first.
-//  * Warp roles (320 threads):
+//  * Warp roles (384 threads, three warpgroups):
 //      warp 0      TMA producer: Q tiles, then K/V tiles through a ring of smem
 //                  slots (mbarrier full/empty pairs).
 //      warp 1      TMEM allocator and tcgen05.mma issuer (one thread).
-//      warps 2-5   softmax group for query tile 0, warps 6-9 for tile 1; thread
+//      warps 2-3   idle (they complete the first warpgroup, which hands most of
+//                  its registers to the softmax warpgroups).
+//      warps 4-7   softmax group for query tile 0, warps 8-11 for tile 1; thread
 //                  = query row = TMEM lane.
 //  * Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
 //    O1 [384,384+d).  P (bf16) is written over the first 64 columns of its S
@@ -29,6 +31,9 @@
 //    happens once, in the epilogue.  Two row sums are kept: the sum of the
 //    bf16-rounded probabilities (exactly the weights the P.V MMA used) divides
 //    O, and the sum of the unrounded ones gives lse.
+//  * Per score element the softmax issues few instructions: packed fp32x2 FMA
+//    (scale and subtract), MUFU exp2, packed bf16 conversion and packed fp32x2
+//    adds into the two row sums; the row max uses 3-input max.
 //  * Causal (bottom-right aligned): KV tiles entirely above the diagonal are
 //    never loaded or multiplied; only tiles that cross it are masked.
 //  * Epilogue: O/l -> bf16 -> swizzled smem (the Q tile's slot) -> TMA store;
@@ -40,7 +45,12 @@ namespace fa {
 
 namespace {
 
-constexpr int kThreads = 320;
+constexpr int kThreads = 384;
+// Register split: launched at 168 per thread (384 x 168 = 64512); the producer /
+// MMA warpgroup drops to 56 and the two softmax warpgroups rise to 224:
+// 128 x 56 + 256 x 224 = 64512.
+constexpr uint32_t kRegsLow = 80, kRegsHigh = 208;
+static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * 168, "register split exceeds the launch budget");
 constexpr uint32_t kTmemCols = 512;
 // tensor-memory column of the score tile / O accumulator of query tile t
 __host__ __device__ constexpr uint32_t tm_s(int t) { return t * 128u; }
@@ -159,9 +169,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar_s_full + t, 1);
-      mbar_init(bar_p_full + t, 128);
+      mbar_init(bar_p_full + t, 4);  // one arrival per softmax warp
       mbar_init(bar_o_done + t, 1);
-      mbar_init(bar_epi + t, 128);
+      mbar_init(bar_epi + t, 4);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -182,7 +192,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_base_slot;
 
-  if (warp == 0) {
+  if (warp < 4) {
+   regs_dec<kRegsLow>();
+   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t item_iter = 0, g = 0;
@@ -298,15 +310,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         (void)s_cnt;
       }
     }
+   }
   } else {
+    regs_inc<kRegsHigh>();
     // ------------------------------------------------------------------ softmax groups
-    const int t = (warp - 2) >> 2;               // query tile of this group
+    const int t = (warp - 4) >> 2;               // query tile of this group
     const uint32_t quarter = warp & 3;           // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;           // row within the tile
     const uint32_t lane_field = (quarter * 32) << 16;
     const uint32_t tS = tmem_base + lane_field + tm_s(t);
     const uint32_t tO = tmem_base + lane_field + tm_o(t);
-    const int tid_in_group = threadIdx.x - 64 - t * 128;
+    const int tid_in_group = threadIdx.x - 128 - t * 128;
     uint32_t s_cnt = 0, tile_iter = 0;  // tile_iter counts items in which this tile is present
     uint8_t* q_tile = smem + L::kOffQ + t * L::kTileBytes;
     const uint32_t q_tile_u32 = smem_u32(q_tile);
@@ -356,39 +370,48 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < 32; ++c)
               if (kbase + i * 32 + c >= lim) s[i][c] = __float_as_uint(-INFINITY);
         }
-        float mx = -INFINITY;
+        // row max with four independent 3-input max chains
+        float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int i = 0; i < 4; ++i)
 #pragma unroll
-          for (int c = 0; c < 32; ++c) mx = fmaxf(mx, __uint_as_float(s[i][c]));
+          for (int c = 0; c < 32; c += 2)
+            mxv[i] = fmax3(mxv[i], __uint_as_float(s[i][c]), __uint_as_float(s[i][c + 1]));
+        const float mx = fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3]));
         const float m_tile = mx * a.scale_log2;  // scale > 0, so max commutes with the scaling
         const bool need = (m2 == -INFINITY) || (m_tile > m2 + kRescaleThreshold);
         const float m_use = need ? fmaxf(m2, m_tile) : m2;
         const float alpha = (m2 == -INFINITY) ? 0.f : ex2(m2 - m_use);
         const float m_ref = (m_use == -INFINITY) ? 0.f : m_use;
-        // probabilities, rounded to bf16 exactly as the P.V MMA will see them
-        float rs0 = 0.f, rs1 = 0.f, re0 = 0.f, re1 = 0.f;
+        // probabilities p = exp2(s * scale_log2 - m_ref), two lanes of work per packed op
+        const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_ref, -m_ref);
+        float2 ex0 = make_float2(0.f, 0.f), ex1 = make_float2(0.f, 0.f);  // unrounded sums
+        float2 rd0 = make_float2(0.f, 0.f), rd1 = make_float2(0.f, 0.f);  // sums of the bf16 values
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
           uint32_t pk[32];
 #pragma unroll
           for (int ii = 0; ii < 2; ++ii) {
 #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              const float p0 = ex2(fmaf(__uint_as_float(s[hf * 2 + ii][c]), a.scale_log2, -m_ref));
-              const float p1 = ex2(fmaf(__uint_as_float(s[hf * 2 + ii][c + 1]), a.scale_log2, -m_ref));
-              const uint32_t packed = pack_bf16x2(p0, p1);
-              pk[ii * 16 + (c >> 1)] = packed;
-              rs0 += __uint_as_float(packed << 16);
-              rs1 += __uint_as_float(packed & 0xFFFF0000u);
-              re0 += p0;
-              re1 += p1;
+            for (int c = 0; c < 32; c += 4) {
+              const uint32_t* sr = s[hf * 2 + ii];
+              const float2 x0 = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2);
+              const float2 x1 = ffma2(make_float2(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), sc2, nm2);
+              const float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
+              const float2 p1 = make_float2(ex2(x1.x), ex2(x1.y));
+              const uint32_t k0 = pack_bf16x2(p0.x, p0.y), k1 = pack_bf16x2(p1.x, p1.y);
+              pk[ii * 16 + (c >> 1)] = k0;
+              pk[ii * 16 + (c >> 1) + 1] = k1;
+              ex0 = fadd2(ex0, p0);
+              ex1 = fadd2(ex1, p1);
+              rd0 = fadd2(rd0, make_float2(__uint_as_float(k0 << 16), __uint_as_float(k0 & 0xFFFF0000u)));
+              rd1 = fadd2(rd1, make_float2(__uint_as_float(k1 << 16), __uint_as_float(k1 & 0xFFFF0000u)));
             }
           }
           tmem_st32(tS + hf * 32, pk);
         }
-        l = l * alpha + (rs0 + rs1);
-        le = le * alpha + (re0 + re1);
+        l = l * alpha + ((rd0.x + rd0.y) + (rd1.x + rd1.y));
+        le = le * alpha + ((ex0.x + ex0.y) + (ex1.x + ex1.y));
         m2 = m_use;
         // rescale the O accumulator when some row of this warp moved its reference.
         // The previous P.V of this tile has completed: the scores just read were
@@ -406,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar_p_full + t);
+        mbar_arrive_warp(bar_p_full + t);
       }
       if (!ok) break;
 
@@ -442,7 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         a.lse[((size_t)b * a.H + h) * a.Nq + row] = lse;
       }
       fence_proxy_async_smem();
-      mbar_arrive(bar_epi + t);
+      mbar_arrive_warp(bar_epi + t);
       bool epi_ok = true;
       if (tid_in_group == 0) {
         if (!mbar_wait(bar_epi + t, tile_iter & 1, a.timeout_ns)) {
