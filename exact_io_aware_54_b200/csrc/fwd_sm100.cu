@@ -115,25 +115,26 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsign
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
+// S = Q K^T for one 128x128 tile: K-major operands, 16-wide k-steps of 32 bytes
+// inside each 128-byte swizzle row, 64-column boxes 16 KB apart.
 template <int D>
-__device__ __forceinline__ void issue_qk(uint32_t d_tmem, uint32_t q_smem, uint32_t k_smem) {
+__device__ __forceinline__ void issue_qk(uint32_t d_tmem, SDesc q, SDesc k) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-    umma_ss(d_tmem, sdesc_sw128(q_smem + off, 16, 1024), sdesc_sw128(k_smem + off, 16, 1024), idesc,
-            kk > 0 ? 1u : 0u);
+    const uint32_t off = (kk >> 2) * 1024 + (kk & 3) * 2;  // 16-byte units
+    umma_ss(d_tmem, sdesc_at(q, off), sdesc_at(k, off), idesc, kk > 0 ? 1u : 0u);
   }
 }
 
+// O (+)= P V: P bf16 in tensor memory (8 columns per 16 keys), V MN-major in smem
+// (16 keys = 2048 bytes per k-step).
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, uint32_t v_smem, bool accumulate) {
+__device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, SDesc v, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    umma_ts(o_tmem, p_tmem + kk * 8, sdesc_sw128(v_smem + kk * 2048, 16384, 1024), idesc,
-            (accumulate || kk > 0) ? 1u : 0u);
-  }
+  for (int kk = 0; kk < 8; ++kk)
+    umma_ts(o_tmem, p_tmem + kk * 8, sdesc_at(v, kk * 128), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D>
@@ -235,7 +236,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t item_iter = 0, g = 0;
       uint32_t s_cnt[2] = {0, 0}, p_cnt[2] = {0, 0};
-      const uint32_t q_smem[2] = {smem_base + L::kOffQ, smem_base + L::kOffQ + L::kTileBytes};
+      const SDesc q_desc[2] = {sdesc_make(smem_base + L::kOffQ, 16, 1024),
+                               sdesc_make(smem_base + L::kOffQ + L::kTileBytes, 16, 1024)};
+      const SDesc ring_k = sdesc_make(smem_base + L::kOffRing, 16, 1024);      // K tiles, K-major
+      const SDesc ring_v = sdesc_make(smem_base + L::kOffRing, 16384, 1024);   // V tiles, MN-major
+      constexpr uint32_t kSlot16 = L::kTileBytes / 16;
       bool ok = true;
       auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) {
         if (!ok) return false;
@@ -260,11 +265,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!wait_or_abort(bar_kv_full + slot_k, (g / L::kStages) & 1)) break;
           tc_fence_after();
           ++g;
-          const uint32_t k_smem = smem_base + L::kOffRing + slot_k * L::kTileBytes;
+          const SDesc k_desc = SDesc{ring_k.lo + slot_k * kSlot16, ring_k.hi};
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (nt[t] > 0) {
-              issue_qk<D>(tmem_base + tm_s(t), q_smem[t], k_smem);
+              issue_qk<D>(tmem_base + tm_s(t), q_desc[t], k_desc);
               umma_commit(bar_s_full + t);
             }
           }
@@ -275,26 +280,26 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!wait_or_abort(bar_kv_full + slot_v, (g / L::kStages) & 1)) break;
           tc_fence_after();
           ++g;
-          const uint32_t v_smem = smem_base + L::kOffRing + slot_v * L::kTileBytes;
+          const SDesc v_desc = SDesc{ring_v.lo + slot_v * kSlot16, ring_v.hi};
           const bool more = (j + 1 < nkv);
-          uint32_t k_smem = 0;
+          SDesc k_desc = ring_k;
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (j < nt[t]) {
               if (!wait_or_abort(bar_p_full + t, p_cnt[t] & 1)) break;
               tc_fence_after();
               ++p_cnt[t];
-              issue_pv<D>(tmem_base + tm_o(t), tmem_base + tm_s(t), v_smem, j > 0);
+              issue_pv<D>(tmem_base + tm_o(t), tmem_base + tm_s(t), v_desc, j > 0);
             }
             if (t == 0 && more) {
               slot_k = g % L::kStages;
               if (!wait_or_abort(bar_kv_full + slot_k, (g / L::kStages) & 1)) break;
               tc_fence_after();
               ++g;
-              k_smem = smem_base + L::kOffRing + slot_k * L::kTileBytes;
+              k_desc = SDesc{ring_k.lo + slot_k * kSlot16, ring_k.hi};
             }
             if (more && j + 1 < nt[t]) {
-              issue_qk<D>(tmem_base + tm_s(t), q_smem[t], k_smem);
+              issue_qk<D>(tmem_base + tm_s(t), q_desc[t], k_desc);
               umma_commit(bar_s_full + t);
             }
           }

@@ -313,6 +313,22 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
          (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// A matrix descriptor split in halves: the start address lives in the low word
+// (in 16-byte units), so advancing along K or to another tile is one 32-bit add.
+struct SDesc {
+  uint32_t lo, hi;
+};
+
+__device__ __forceinline__ SDesc sdesc_make(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  const uint64_t d = sdesc_sw128(saddr, lbo, sbo);
+  return SDesc{static_cast<uint32_t>(d), static_cast<uint32_t>(d >> 32)};
+}
+
+// Descriptor of the same layout starting `off16` 16-byte units further on.
+__device__ __forceinline__ uint64_t sdesc_at(SDesc d, uint32_t off16) {
+  return (static_cast<uint64_t>(d.hi) << 32) | static_cast<uint64_t>(d.lo + off16);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 accumulate.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
