@@ -11,17 +11,19 @@
 //
 // Three kernels:
 //   1. preprocess: D_i = dO_i . O_i (fp32) and a zeroed fp32 dQ accumulator;
-//   2. main (tcgen05): one CTA per (b, h, 128-key tile); K_j and V_j stay in
-//      shared memory while the CTA walks the 128-row query tiles that can see
-//      them (from the causal diagonal onward).  Each query tile is processed as
-//      two halves of 64 queries so that the dS warps work on one half while the
-//      tensor core computes the other:
-//        S^T = K Q^T and dP^T = V dO^T      (M = 128 keys, N = 64 queries)
-//        P^T -> tensor memory (bf16), dS^T -> shared memory (bf16, swizzled)
-//        dV += P^T dO (A from tensor memory),  dK += dS^T Q
-//        dQ_tile = dS K                      (M = 128 queries, A read MN-major)
-//      dQ tiles leave tensor memory through fp32 vector reductions into the
-//      accumulator; dK and dV leave once, through a TMA store.
+//   2. main (tcgen05): one CTA per (b, h, 128-key tile); K_j and V_j stay on chip
+//      while the CTA walks the 128-row query tiles that can see them (from the
+//      causal diagonal onward).  Per query tile i:
+//        S^T = K Q_i^T, dP^T = V dO_i^T       (M = 128 keys, N = 128 queries)
+//        dS warps: P^T and dS^T (bf16) into tensor memory over S^T / dP^T, dS
+//                  into a swizzled shared-memory tile
+//        dV += P^T dO_i, dK += dS^T Q_i        (A operands from tensor memory)
+//        dQ_i = dS K                           (M = 128 queries, A read MN-major)
+//      The tensor core runs dV/dK(i), then S^T/dP^T(i+1), then dQ(i): the dS warps
+//      compute tile i+1 while dQ(i) runs, and drain dQ(i) (fp32 vector reductions
+//      into the accumulator) once their tile i+1 is done.  Every instruction has
+//      N >= 64; tcgen05.mma has a fixed cost of about 44 cycles per instruction,
+//      so the score MMAs use the full N = 128.  dK and dV leave once, through TMA.
 //   3. convert: dQ = bf16(scale * accumulator).
 #include "fa_internal.h"
 #include "ptx.cuh"
@@ -33,17 +35,12 @@ namespace {
 constexpr int kThreads = 320;  // warp 0 TMA + stats, warp 1 MMA, warps 2-9 dS warps (two column groups)
 constexpr uint32_t kTmemCols = 512;
 
-// A query tile of 128 rows is processed in kSteps steps of kNq queries.  The
-// tensor core computes step t+2's S^T and dP^T into one of two ping-pong buffers
-// while the dS warps work on step t+1 and the MMAs of step t (dV, dK) run.
 template <int D>
 struct BwdLayout {
-  static constexpr int kNq = (D == 64) ? 64 : 32;  // queries per step
-  static constexpr int kSteps = 128 / kNq;
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kBoxes = D / 64;
   static constexpr int kBoxBytes = 16384;
-  static constexpr int kQStages = 2;
+  static constexpr int kQStages = (D == 64) ? 3 : 2;  // query tiles prefetched ahead
   static constexpr int kDsBufs = (D == 64) ? 2 : 1;
   static constexpr int kDsBytes = 2 * 16384;  // [64-query atom][128 keys][64 queries] bf16, 128-byte swizzle
   static constexpr int kOffK = 0;
@@ -51,25 +48,24 @@ struct BwdLayout {
   static constexpr int kOffQ = 2 * kTileBytes;
   static constexpr int kOffDO = kOffQ + kQStages * kTileBytes;
   static constexpr int kOffDS = kOffDO + kQStages * kTileBytes;
-  static constexpr int kOffStat = kOffDS + kDsBufs * kDsBytes;  // per stage: lse2[128], D[128]
-  // d = 64: dQ tiles leave through an fp32 staging tile and a TMA reduce-add
-  // (two 128-row x 32-column boxes, one per dS column group); d = 128 uses
-  // per-thread vector reductions instead (no room for the staging tile).
-  static constexpr bool kDqTma = (D == 64);
-  static constexpr int kOffDQ = kOffStat + kQStages * 2 * 128 * 4;
-  static constexpr int kOffBar = kOffDQ + (kDqTma ? 128 * D * 4 : 0);
-  // kv_full, q_full[QS], q_empty[QS], s_full[2], p_full[2], ds_free[DSB], dq_full, dq_empty, dkv_done, epi,
-  // dq_staged[2], dq_stage_free[2]
-  static constexpr int kNumBars = 1 + 2 * kQStages + 4 + kDsBufs + 4 + 4;
+  static constexpr int kOffStat = kOffDS + kDsBufs * kDsBytes;  // per stage: -lse2[128], -D[128]
+  static constexpr int kOffBar = kOffStat + kQStages * 2 * 128 * 4;
+  // kv_full, q_full[QS], q_empty[QS], s_full, p_full, ds_free[DSB], dq_full, dq_empty, dkv_done, epi, kv_tmem
+  static constexpr int kNumBars = 1 + 2 * kQStages + 2 + kDsBufs + 5;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64;
-  // tensor memory columns
-  __host__ __device__ static constexpr uint32_t tm_st(int b) { return b * kNq; }           // S^T buffers (P^T bf16 over them)
-  __host__ __device__ static constexpr uint32_t tm_dpt(int b) { return 2 * kNq + b * kNq; }  // dP^T buffers
-  static constexpr uint32_t kTmDV = 4 * kNq;
-  static constexpr uint32_t kTmDK = 4 * kNq + D;
-  static constexpr uint32_t kTmDQ = 4 * kNq + 2 * D;
-  static_assert(kTmDQ + D <= kTmemCols, "tensor memory budget");
+  // Tensor memory columns.  d = 64 also keeps K and V there (bf16 pairs) as the A
+  // operands of S^T and dP^T, and writes dS^T over dP^T as the A operand of dK;
+  // d = 128 has no room for that, reads K, V and dS^T from shared memory, and
+  // puts the dQ tile over the dP^T columns (drained before the next dP^T).
+  static constexpr bool kKVInTmem = (D == 64);
+  static constexpr uint32_t kTmSt = 0;     // S^T, P^T bf16 over it
+  static constexpr uint32_t kTmDPt = 128;  // dP^T, (d = 64) dS^T bf16 over it
+  static constexpr uint32_t kTmDV = 256;
+  static constexpr uint32_t kTmDK = 256 + D;
+  static constexpr uint32_t kTmDQ = (D == 64) ? 384 : kTmDPt;
+  static constexpr uint32_t kTmK = 448, kTmV = 480;
+  static_assert(kTmDK + D <= kTmemCols && (!kKVInTmem || kTmV + D / 2 <= kTmemCols), "tensor memory budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -102,50 +98,48 @@ __device__ __forceinline__ bool warp_wait_b(uint64_t* bar, uint32_t parity, unsi
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
-// X^T step = A . B_step^T  (M = 128 keys, N = kNq queries, K = D), both K-major.
-// Used for S^T = K Q^T and dP^T = V dO^T.
-template <int D>
-__device__ __forceinline__ void issue_step_scores(uint32_t d_tmem, uint32_t a_smem, uint32_t b_step_smem) {
-  using L = BwdLayout<D>;
-  constexpr uint32_t idesc = idesc_bf16_f32(128, L::kNq, false, false);
+// X^T = A . B^T for one query tile (M = 128 keys, N = 128 queries, K = D): S^T = K Q^T
+// or dP^T = V dO^T.  A is in tensor memory (bf16 pairs) when kAT, else K-major smem;
+// B is the query-side tile, K-major smem.  Offsets in 16-byte units.
+template <int D, bool kAT>
+__device__ __forceinline__ void issue_scores(uint32_t d_tmem, uint32_t a_tmem, SDesc a_smem, SDesc b) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, false, false);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-    umma_ss(d_tmem, sdesc_sw128(a_smem + off, 16, 1024), sdesc_sw128(b_step_smem + off, 16, 1024), idesc,
-            kk > 0 ? 1u : 0u);
+    const uint32_t off = (kk >> 2) * 1024 + (kk & 3) * 2;
+    if (kAT)
+      umma_ts(d_tmem, a_tmem + kk * 8, sdesc_at(b, off), idesc, kk > 0 ? 1u : 0u);
+    else
+      umma_ss(d_tmem, sdesc_at(a_smem, off), sdesc_at(b, off), idesc, kk > 0 ? 1u : 0u);
   }
 }
 
-// acc (+)= A . B_step where B_step is kNq rows (queries) x D, read MN-major (N = D).
-// A is P^T in tensor memory (kAFromTmem) or dS^T in shared memory, K-major.  In
-// tensor memory each dS column group keeps its P^T over the start of its own S^T
-// columns: queries [g*kNq/2, (g+1)*kNq/2) of the step sit at columns g*kNq/2 ..
-// g*kNq/2 + kNq/4 (two bf16 per column).
-template <int D, bool kAFromTmem>
-__device__ __forceinline__ void issue_step_acc(uint32_t acc_tmem, uint32_t a, uint32_t b_step_smem, bool first) {
-  using L = BwdLayout<D>;
-  constexpr int kHalf = L::kNq / 2, kPerGroup = kHalf / 16;  // 16-query k-steps per column group
+// acc (+)= X^T . B with X^T = P^T or dS^T (M = 128 keys, K = 128 queries) and B the
+// query tile (128 queries x D) read MN-major.  In tensor memory (kAT) the dS warp
+// group g keeps its 64 queries as bf16 pairs over the first 32 of its 64 columns:
+// queries 16kk..16kk+15 sit at column (kk / 4) * 64 + (kk % 4) * 8.  From smem, X^T
+// is the K-major dS^T tile.
+template <int D, bool kAT>
+__device__ __forceinline__ void issue_acc(uint32_t acc_tmem, uint32_t a_tmem, SDesc a_smem, SDesc b, bool first) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
 #pragma unroll
-  for (int kk = 0; kk < L::kNq / 16; ++kk) {
-    const uint64_t bdesc = sdesc_sw128(b_step_smem + kk * 2048, 16384, 1024);
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint64_t bdesc = sdesc_at(b, kk * 128);
     const uint32_t acc = (first && kk == 0) ? 0u : 1u;
-    if (kAFromTmem)
-      umma_ts(acc_tmem, a + (kk / kPerGroup) * kHalf + (kk % kPerGroup) * 8, bdesc, idesc, acc);
+    if (kAT)
+      umma_ts(acc_tmem, a_tmem + (kk >> 2) * 64 + (kk & 3) * 8, bdesc, idesc, acc);
     else
-      umma_ss(acc_tmem, sdesc_sw128(a + kk * 32, 16, 1024), bdesc, idesc, acc);
+      umma_ss(acc_tmem, sdesc_at(a_smem, (kk >> 2) * 1024 + (kk & 3) * 2), bdesc, idesc, acc);
   }
 }
 
 // dQ tile = dS . K  (M = 128 queries, N = D, K = 128 keys); dS and K both MN-major.
 template <int D>
-__device__ __forceinline__ void issue_dq(uint32_t dq_tmem, uint32_t ds_smem, uint32_t k_smem) {
+__device__ __forceinline__ void issue_dq(uint32_t dq_tmem, SDesc ds, SDesc k) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, true, true);
 #pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    umma_ss(dq_tmem, sdesc_sw128(ds_smem + kk * 2048, 16384, 1024), sdesc_sw128(k_smem + kk * 2048, 16384, 1024),
-            idesc, kk > 0 ? 1u : 0u);
-  }
+  for (int kk = 0; kk < 8; ++kk)
+    umma_ss(dq_tmem, sdesc_at(ds, kk * 128), sdesc_at(k, kk * 128), idesc, kk > 0 ? 1u : 0u);
 }
 
 // P and dS for one key row and kN consecutive queries:
@@ -191,23 +185,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
-                    const __grid_constant__ CUtensorMap tmDQacc, const BwdArgs a) {
+                    const BwdArgs a) {
   using L = BwdLayout<D>;
-  constexpr int kNq = L::kNq, kSteps = L::kSteps, kHalf = kNq / 2;  // kHalf: queries per dS warp per step
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* bar_kv_full = bars;
   uint64_t* bar_q_full = bars + 1;
   uint64_t* bar_q_empty = bar_q_full + L::kQStages;
   uint64_t* bar_s_full = bar_q_empty + L::kQStages;
-  uint64_t* bar_p_full = bar_s_full + 2;
-  uint64_t* bar_ds_free = bar_p_full + 2;
+  uint64_t* bar_p_full = bar_s_full + 1;
+  uint64_t* bar_ds_free = bar_p_full + 1;
   uint64_t* bar_dq_full = bar_ds_free + L::kDsBufs;
   uint64_t* bar_dq_empty = bar_dq_full + 1;
   uint64_t* bar_dkv_done = bar_dq_empty + 1;
   uint64_t* bar_epi = bar_dkv_done + 1;
-  uint64_t* bar_dq_staged = bar_epi + 1;
-  uint64_t* bar_dq_stage_free = bar_dq_staged + 2;
+  uint64_t* bar_kv_tmem = bar_epi + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);
 
@@ -223,7 +215,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   int i_first = 0;
   if (a.causal) i_first = max(0, j * 128 - (a.Nk - a.Nq)) >> 7;
   const int n_iters = n_qtiles - i_first;
-  const int n_steps = n_iters * kSteps;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv_full, 1);
@@ -231,19 +222,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_q_full + s, 2);  // TMA bytes + the producer's stats
       mbar_init(bar_q_empty + s, 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(bar_s_full + t, 1);
-      mbar_init(bar_p_full + t, 8);  // one arrival per dS warp
-    }
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_p_full, 8);  // one arrival per dS warp
     for (int s = 0; s < L::kDsBufs; ++s) mbar_init(bar_ds_free + s, 1);
     mbar_init(bar_dq_full, 1);
     mbar_init(bar_dq_empty, 8);
     mbar_init(bar_dkv_done, 1);
     mbar_init(bar_epi, 8);
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(bar_dq_staged + g, 4);
-      mbar_init(bar_dq_stage_free + g, 1);
-    }
+    mbar_init(bar_kv_tmem, 8);
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -275,13 +261,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int it = 0; it < n_iters; ++it) {
       const int st = it % L::kQStages;
+      const int q0 = (i_first + it) * 128;
+      // -lse in log2 units (-inf for rows past Nq or with no visible key: P = 0 there)
+      // and -D, negated so that the dS warps use them as addends.  The global loads
+      // are issued before waiting for the stage so that their latency overlaps it.
+      float nl2[4], nd[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int q = q0 + lane + 32 * e;
+        nl2[e] = -INFINITY;
+        nd[e] = 0.f;
+        if (q < a.Nq) {
+          const float lse = a.lse[stat_row + q];
+          nl2[e] = (lse == -INFINITY) ? -INFINITY : -lse * 1.4426950408889634f;
+          nd[e] = -a.delta[stat_row + q];
+        }
+      }
       bool ok = true;
       if (lane == 0) ok = mbar_wait(bar_q_empty + st, ((it / L::kQStages) & 1) ^ 1, a.timeout_ns) && !*abort_flag;
       if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) {
         if (lane == 0) bwd_timeout(a.status, abort_flag);
         break;
       }
-      const int q0 = (i_first + it) * 128;
       if (lane == 0) {
         mbar_arrive_expect_tx(bar_q_full + st, 2 * L::kTileBytes);
         for (int bx = 0; bx < L::kBoxes; ++bx) {
@@ -291,20 +292,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                       h, q0, b);
         }
       }
-      // -lse in log2 units (-inf for rows past Nq or with no visible key: P = 0 there)
-      // and -D, negated so that the dS warps use them as addends
       float* stat = reinterpret_cast<float*>(smem + L::kOffStat) + st * 256;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int c = lane + 32 * e, q = q0 + c;
-        float nl2 = -INFINITY, nd = 0.f;
-        if (q < a.Nq) {
-          const float lse = a.lse[stat_row + q];
-          nl2 = (lse == -INFINITY) ? -INFINITY : -lse * 1.4426950408889634f;
-          nd = -a.delta[stat_row + q];
-        }
-        stat[c] = nl2;
-        stat[128 + c] = nd;
+        stat[lane + 32 * e] = nl2[e];
+        stat[128 + lane + 32 * e] = nd[e];
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_q_full + st);
@@ -313,40 +305,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(bar_kv_full, 0, a.timeout_ns);
-      const uint32_t k_s = sbase + L::kOffK, v_s = sbase + L::kOffV;
-      auto q_stage = [&](int it) { return sbase + L::kOffQ + (it % L::kQStages) * L::kTileBytes; };
-      auto do_stage = [&](int it) { return sbase + L::kOffDO + (it % L::kQStages) * L::kTileBytes; };
-      // S^T and dP^T of global step t into ping-pong buffer t % 2
-      auto issue_scores = [&](int t) -> bool {
-        const int it = t / kSteps, s = t - (t / kSteps) * kSteps;
-        if (s == 0) {
-          if (!mbar_wait(bar_q_full + (it % L::kQStages), (it / L::kQStages) & 1, a.timeout_ns) || *abort_flag)
-            return false;
-          tc_fence_after();
-        }
-        const int buf = t & 1;
-        issue_step_scores<D>(tmem + L::tm_st(buf), k_s, q_stage(it) + s * kNq * 128);
-        issue_step_scores<D>(tmem + L::tm_dpt(buf), v_s, do_stage(it) + s * kNq * 128);
-        umma_commit(bar_s_full + buf);
+      if (ok && L::kKVInTmem) ok = mbar_wait(bar_kv_tmem, 0, a.timeout_ns);
+      // operand descriptors, built once; tiles are reached by 32-bit adds (16-byte units)
+      const SDesc k_kmaj = sdesc_make(sbase + L::kOffK, 16, 1024), v_kmaj = sdesc_make(sbase + L::kOffV, 16, 1024);
+      const SDesc k_mn = sdesc_make(sbase + L::kOffK, 16384, 1024);
+      const SDesc q_kmaj = sdesc_make(sbase + L::kOffQ, 16, 1024), do_kmaj = sdesc_make(sbase + L::kOffDO, 16, 1024);
+      const SDesc q_mn = sdesc_make(sbase + L::kOffQ, 16384, 1024), do_mn = sdesc_make(sbase + L::kOffDO, 16384, 1024);
+      const SDesc ds_kmaj = sdesc_make(sbase + L::kOffDS, 16, 1024), ds_mn = sdesc_make(sbase + L::kOffDS, 16384, 1024);
+      constexpr uint32_t kTile16 = L::kTileBytes / 16, kDs16 = L::kDsBytes / 16;
+      auto at = [](SDesc d, uint32_t off16) { return SDesc{d.lo + off16, d.hi}; };
+      // S^T and dP^T of query tile `it`
+      auto issue_sdp = [&](int it) -> bool {
+        const int st = it % L::kQStages;
+        if (!mbar_wait(bar_q_full + st, (it / L::kQStages) & 1, a.timeout_ns) || *abort_flag) return false;
+        tc_fence_after();
+        issue_scores<D, L::kKVInTmem>(tmem + L::kTmSt, tmem + L::kTmK, k_kmaj, at(q_kmaj, st * kTile16));
+        issue_scores<D, L::kKVInTmem>(tmem + L::kTmDPt, tmem + L::kTmV, v_kmaj, at(do_kmaj, st * kTile16));
+        umma_commit(bar_s_full);
         return true;
       };
-      if (ok) {
+      // dV and dK of query tile `it` (after the dS warps released it)
+      auto issue_dvdk = [&](int it) -> bool {
+        if (!mbar_wait(bar_p_full, it & 1, a.timeout_ns) || *abort_flag) return false;
         tc_fence_after();
-        for (int t = 0; t < 2 && t < n_steps && ok; ++t) ok = issue_scores(t);
-      }
-      for (int t = 0; t < n_steps && ok; ++t) {
-        const int it = t / kSteps, s = t - (t / kSteps) * kSteps, buf = t & 1;
-        if (!mbar_wait(bar_p_full + buf, (t >> 1) & 1, a.timeout_ns) || *abort_flag) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t ds_s = sbase + L::kOffDS + (it % L::kDsBufs) * L::kDsBytes;
-        // dS^T of this step: atom (s * kNq) / 64, byte offset ((s * kNq) % 64) * 2 inside the 128-byte rows
-        const uint32_t ds_step = ds_s + ((s * kNq) >> 6) * 16384 + ((s * kNq) & 63) * 2;
-        issue_step_acc<D, true>(tmem + L::kTmDV, tmem + L::tm_st(buf), do_stage(it) + s * kNq * 128, t == 0);
-        issue_step_acc<D, false>(tmem + L::kTmDK, ds_step, q_stage(it) + s * kNq * 128, t == 0);
-        if (s == kSteps - 1) {
+        const int st = it % L::kQStages;
+        issue_acc<D, true>(tmem + L::kTmDV, tmem + L::kTmSt, ds_kmaj, at(do_mn, st * kTile16), it == 0);
+        issue_acc<D, L::kKVInTmem>(tmem + L::kTmDK, tmem + L::kTmDPt, at(ds_kmaj, (it % L::kDsBufs) * kDs16),
+                                   at(q_mn, st * kTile16), it == 0);
+        umma_commit(bar_q_empty + st);  // Q and dO of this tile are no longer read
+        return true;
+      };
+      auto issue_dq_tile = [&](int it) {
+        issue_dq<D>(tmem + L::kTmDQ, at(ds_mn, (it % L::kDsBufs) * kDs16), k_mn);
+        umma_commit(bar_dq_full);
+        umma_commit(bar_ds_free + (it % L::kDsBufs));
+      };
+      if (ok) tc_fence_after();
+      if constexpr (D == 64) {
+        // dV/dK(i), S^T/dP^T(i+1), dQ(i): the dS warps work on tile i+1 while dQ(i) runs
+        if (ok && n_iters > 0) ok = issue_sdp(0);
+        for (int it = 0; it < n_iters && ok; ++it) {
+          if (!issue_dvdk(it)) {
+            ok = false;
+            break;
+          }
+          if (it + 1 < n_iters && !issue_sdp(it + 1)) {
+            ok = false;
+            break;
+          }
           if (it > 0) {  // the previous dQ tile must have left tensor memory
             if (!mbar_wait(bar_dq_empty, (it - 1) & 1, a.timeout_ns) || *abort_flag) {
               ok = false;
@@ -354,12 +360,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
           }
-          issue_dq<D>(tmem + L::kTmDQ, ds_s, k_s);
-          umma_commit(bar_dq_full);
-          umma_commit(bar_ds_free + (it % L::kDsBufs));
-          umma_commit(bar_q_empty + (it % L::kQStages));
+          issue_dq_tile(it);
         }
-        if (t + 2 < n_steps) ok = issue_scores(t + 2);
+      } else {
+        // the dQ tile uses the dP^T columns: it is drained before the next dP^T
+        for (int it = 0; it < n_iters && ok; ++it) {
+          if (it > 0) {
+            if (!mbar_wait(bar_dq_empty, (it - 1) & 1, a.timeout_ns) || *abort_flag) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          if (!issue_sdp(it) || !issue_dvdk(it)) {
+            ok = false;
+            break;
+          }
+          issue_dq_tile(it);
+        }
       }
       if (!ok) bwd_timeout(a.status, abort_flag);
       umma_commit(bar_dkv_done);
@@ -367,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------------ dS warps (thread = key)
     const uint32_t quarter = warp & 3;
-    const int grp = (warp - 2) >> 2;  // column group: queries [grp * kHalf, +kHalf) of each step
+    const int grp = (warp - 2) >> 2;  // column group: queries [64 grp, 64 grp + 64) of each tile
     const int r = quarter * 32 + lane;
     const int key = j * 128 + r;
     const uint32_t lane_field = (quarter * 32) << 16;
@@ -377,14 +395,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qmin = a.causal ? key - (a.Nk - a.Nq) : -(1 << 30);
     bool ok = true;
 
-    // dQ tile of query tile `it`: this group's D/2 columns leave tensor memory and
-    // are added into the fp32 accumulator
-    int drains = 0;
-    auto drain_dq = [&](int it) -> bool {
-      if constexpr (L::kDqTma) {
-        // the staging box of this group must have been read by the previous reduce
-        if (!warp_wait_b(bar_dq_stage_free + grp, (drains & 1) ^ 1, a.timeout_ns)) return false;
+    if constexpr (L::kKVInTmem) {
+      // K (group 0) or V (group 1) row of this key into tensor memory as bf16 pairs
+      if (!warp_wait_b(bar_kv_full, 0, a.timeout_ns)) ok = false;
+      if (ok) {
+        const uint32_t src = sbase + (grp == 0 ? L::kOffK : L::kOffV) + r * 128;
+        uint32_t row[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          ld_shared_v4(src + ((c ^ (r & 7)) << 4), row[4 * c], row[4 * c + 1], row[4 * c + 2], row[4 * c + 3]);
+        tmem_st32(tmem + lane_field + (grp == 0 ? L::kTmK : L::kTmV), row);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive_warp(bar_kv_tmem);
       }
+    }
+
+    // dQ tile of query tile `it`: this group's D/2 columns, fp32 vector reductions
+    // into the accumulator
+    auto drain_dq = [&](int it) -> bool {
       if (!warp_wait_b(bar_dq_full, it & 1, a.timeout_ns) || *abort_flag) return false;
       tc_fence_after();
       uint32_t g[D / 64][32];
@@ -395,110 +424,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int cc = 1; cc < D / 64; ++cc) reg_pin(g[cc]);
       tc_fence_before();
       mbar_arrive_warp(bar_dq_empty);
-      const int q0 = (i_first + it) * 128;
-      if constexpr (L::kDqTma) {
-        // row r of box grp, 128-byte swizzle; one elected thread adds the box into global memory
-        const uint32_t box = sbase + L::kOffDQ + grp * 16384 + r * 128;
+      const int q = (i_first + it) * 128 + r;
+      if (q < a.Nq) {
+        float* dst = a.dq_acc + (((size_t)b * a.Nq + q) * a.H + h) * D + grp * (D / 2);
 #pragma unroll
-        for (int c = 0; c < 8; ++c)
-          st_shared_v4(box + ((c ^ (r & 7)) << 4), g[0][4 * c], g[0][4 * c + 1], g[0][4 * c + 2], g[0][4 * c + 3]);
-        fence_proxy_async_smem();
-        mbar_arrive_warp(bar_dq_staged + grp);
-        bool staged = true;
-        if (quarter == 2 && lane == 0) {  // first warp of the group
-          staged = mbar_wait(bar_dq_staged + grp, drains & 1, a.timeout_ns);
-          if (staged) {
-            tma_reduce_add_4d(&tmDQacc, smem + L::kOffDQ + grp * 16384, grp * 32, h, q0, b);
-            bulk_commit_group();
-            bulk_wait_group_read0();
-            mbar_arrive(bar_dq_stage_free + grp);
-          }
-        }
-        if (__shfl_sync(0xffffffffu, staged ? 1 : 0, 0) == 0) return false;
-      } else {
-        const int q = q0 + r;
-        if (q < a.Nq) {
-          float* dst = a.dq_acc + (((size_t)b * a.Nq + q) * a.H + h) * D + grp * (D / 2);
+        for (int cc = 0; cc < D / 64; ++cc)
 #pragma unroll
-          for (int cc = 0; cc < D / 64; ++cc)
-#pragma unroll
-            for (int e = 0; e < 32; e += 4)
-              red_add_v4(dst + cc * 32 + e, __uint_as_float(g[cc][e]), __uint_as_float(g[cc][e + 1]),
-                         __uint_as_float(g[cc][e + 2]), __uint_as_float(g[cc][e + 3]));
-        }
+          for (int e = 0; e < 32; e += 4)
+            red_add_v4(dst + cc * 32 + e, __uint_as_float(g[cc][e]), __uint_as_float(g[cc][e + 1]),
+                       __uint_as_float(g[cc][e + 2]), __uint_as_float(g[cc][e + 3]));
       }
-      ++drains;
       return true;
     };
 
-    for (int t = 0; t < n_steps && ok; ++t) {
-      const int it = t / kSteps, s = t - (t / kSteps) * kSteps, buf = t & 1;
+    for (int it = 0; it < n_iters && ok; ++it) {
       const int st = it % L::kQStages;
       const int q0 = (i_first + it) * 128;
-      if (s == 0) {
-        // stats of this query tile are staged with it; its dS buffer must be free
-        if (!warp_wait_b(bar_q_full + st, (it / L::kQStages) & 1, a.timeout_ns) ||
-            !warp_wait_b(bar_ds_free + (it % L::kDsBufs), ((it / L::kDsBufs) & 1) ^ 1, a.timeout_ns) ||
-            *abort_flag) {
-          ok = false;
-          break;
-        }
-      }
-      if (!warp_wait_b(bar_s_full + buf, (t >> 1) & 1, a.timeout_ns) || *abort_flag) {
+      // the stats of this query tile are staged with it; its dS buffer must be free
+      if (!warp_wait_b(bar_q_full + st, (it / L::kQStages) & 1, a.timeout_ns) ||
+          !warp_wait_b(bar_ds_free + (it % L::kDsBufs), ((it / L::kDsBufs) & 1) ^ 1, a.timeout_ns) ||
+          !warp_wait_b(bar_s_full, it & 1, a.timeout_ns) || *abort_flag) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int qs = q0 + s * kNq + grp * kHalf;  // first query of this warp's columns
-      const uint32_t stat_u32 = sbase + L::kOffStat + st * 1024 + (s * kNq + grp * kHalf) * 4;
-      uint32_t sv[kHalf], dp[kHalf];
-      if constexpr (kHalf == 32) {
-        tmem_ld32(tmem + lane_field + L::tm_st(buf) + grp * kHalf, sv);
-        tmem_ld32(tmem + lane_field + L::tm_dpt(buf) + grp * kHalf, dp);
+      const uint32_t ds_row = sbase + L::kOffDS + (it % L::kDsBufs) * L::kDsBytes + grp * 16384 + r * 128;
+#pragma unroll 1
+      for (int ch = 0; ch < 2; ++ch) {
+        const int col = 64 * grp + 32 * ch;  // first query of this chunk within the tile
+        const int qs = q0 + col;
+        uint32_t sv[32], dp[32];
+        tmem_ld32(tmem + lane_field + L::kTmSt + col, sv);
+        tmem_ld32(tmem + lane_field + L::kTmDPt + col, dp);
         tmem_ld_wait(sv);
         reg_pin(dp);
-      } else {
-        tmem_ld16(tmem + lane_field + L::tm_st(buf) + grp * kHalf, sv);
-        tmem_ld16(tmem + lane_field + L::tm_dpt(buf) + grp * kHalf, dp);
-        tmem_ld_wait16(sv);
-        reg_pin16(dp);
-      }
-      const bool tile_mask = (j * 128 + 128 > a.Nk) || (a.causal && (j * 128 + 127 - (a.Nk - a.Nq) > qs));
-      uint32_t pk[kHalf / 2], dk2[kHalf / 2];
-      if (tile_mask)
-        ds_block<kHalf, true>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2);
-      else
-        ds_block<kHalf, false>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2);
-      // P^T (bf16 pairs) over the start of this group's own S^T columns (the other
-      // group may still be reading its columns)
-      if constexpr (kHalf == 32)
-        tmem_st16(tmem + lane_field + L::tm_st(buf) + grp * kHalf, pk);
-      else
-        tmem_st8(tmem + lane_field + L::tm_st(buf) + grp * kHalf, pk);
-      // dS^T row of this key for these queries: kHalf/8 chunks of 16 bytes, 128-byte swizzle
-      const uint32_t ds_u32 = sbase + L::kOffDS + (it % L::kDsBufs) * L::kDsBytes;
-      const int qt = s * kNq + grp * kHalf;  // query offset within the tile
-      const uint32_t row_base = ds_u32 + (qt >> 6) * 16384 + r * 128;
+        const uint32_t stat_u32 = sbase + L::kOffStat + st * 1024 + col * 4;
+        const bool tile_mask = (j * 128 + 128 > a.Nk) || (a.causal && (j * 128 + 127 - (a.Nk - a.Nq) > qs));
+        uint32_t pk[16], dk2[16];
+        if (tile_mask)
+          ds_block<32, true>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2);
+        else
+          ds_block<32, false>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2);
+        // P^T (and dS^T) as bf16 pairs over the columns of this group already read
+        tmem_st16(tmem + lane_field + L::kTmSt + 64 * grp + 16 * ch, pk);
+        if constexpr (L::kKVInTmem) tmem_st16(tmem + lane_field + L::kTmDPt + 64 * grp + 16 * ch, dk2);
+        // dS^T row of this key: 4 chunks of 16 bytes, 128-byte swizzle
 #pragma unroll
-      for (int c8 = 0; c8 < kHalf / 8; ++c8) {
-        const int chunk = ((qt & 63) >> 3) + c8;
-        st_shared_v4(row_base + ((chunk ^ (r & 7)) << 4), dk2[c8 * 4 + 0], dk2[c8 * 4 + 1], dk2[c8 * 4 + 2],
-                     dk2[c8 * 4 + 3]);
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int chunk = 4 * ch + c4;
+          st_shared_v4(ds_row + ((chunk ^ (r & 7)) << 4), dk2[4 * c4], dk2[4 * c4 + 1], dk2[4 * c4 + 2],
+                       dk2[4 * c4 + 3]);
+        }
       }
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive_warp(bar_p_full + buf);
-      // the previous query tile's dQ is complete by now (it ran before this step's scores)
-      if (s == kSteps - 1 && it > 0) {
-        if (!drain_dq(it - 1)) {
-          ok = false;
-          break;
-        }
-      }
+      mbar_arrive_warp(bar_p_full);
+      // d = 64: the previous tile's dQ ran while this tile was computed;
+      // d = 128: this tile's dQ follows right after dV / dK
+      if (D == 64 && it > 0) ok = drain_dq(it - 1);
+      if (D == 128) ok = drain_dq(it);
     }
-    if (ok && n_iters > 0) ok = drain_dq(n_iters - 1);
-    if (quarter == 2 && lane == 0) bulk_wait_group0();  // reduce-adds of this thread have landed
+    if (D == 64 && ok && n_iters > 0) ok = drain_dq(n_iters - 1);
     // ---------------------------------------------------------------- dK / dV epilogue
     // group 0 stores dK (times scale) through the K tile's smem, group 1 dV through V's
     if (ok && warp_wait_b(bar_dkv_done, 0, a.timeout_ns) && !*abort_flag) {
@@ -529,6 +516,411 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_store_4d(&tmDK, smem + L::kOffK + bx * L::kBoxBytes, bx * 64, h, j * 128, b);
             tma_store_4d(&tmDV, smem + L::kOffV + bx * L::kBoxBytes, bx * 64, h, j * 128, b);
           }
+          bulk_commit_group();
+          bulk_wait_group0();
+        } else {
+          bwd_timeout(a.status, abort_flag);
+        }
+      }
+      __syncwarp();
+    } else if (lane == 0) {
+      bwd_timeout(a.status, abort_flag);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------
+// d = 64: pipelined main kernel.
+//
+// The dS warps copy S^T and dP^T of a query tile into registers and release both
+// tensor-memory tiles at once, so the tensor core computes the next tile's scores
+// while they work.  P^T goes to its own tensor-memory columns and dK reads dS^T
+// from shared memory: no tensor-memory location is written by one MMA while an
+// earlier MMA still reads it, so the tensor core never drains between tiles.  Four
+// drain warps move each dQ tile out of tensor memory and add it to the fp32
+// accumulator with TMA reductions of whole 128-byte rows.
+//
+// Tensor core order per query tile i:   S^T(i+1) dP^T(i+1) | dV(i) dK(i) | dQ(i)
+// dS warps:   load S^T(i), dP^T(i) -> release -> P^T(i) to TMEM, dS(i) to smem
+// drain warps: dQ(i) TMEM -> smem (32 columns at a time) -> TMA reduce-add
+struct PipeLayout {
+  static constexpr int D = 64;
+  static constexpr int kTileBytes = 128 * D * 2;  // 16 KB
+  static constexpr int kQStages = 3;
+  static constexpr int kDsBufs = 2;
+  static constexpr int kDsBytes = 2 * 16384;        // [64-query atom][128 keys][64 queries] bf16
+  static constexpr int kStageBytes = 128 * 32 * 4;  // one fp32 box of dQ: 128 queries x 32 columns
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kTileBytes;
+  static constexpr int kOffQ = 2 * kTileBytes;
+  static constexpr int kOffDO = kOffQ + kQStages * kTileBytes;
+  static constexpr int kOffDS = kOffDO + kQStages * kTileBytes;
+  static constexpr int kOffStage = kOffDS + kDsBufs * kDsBytes;
+  static constexpr int kOffStat = kOffStage + kStageBytes;  // per stage: -lse2[128], -D[128]
+  static constexpr int kOffBar = kOffStat + kQStages * 2 * 128 * 4;
+  // kv_full, q_full[QS], q_empty[QS], s_full, s_free, p_full, pt_free, ds_free[DSB],
+  // dq_full, dq_empty, stage_full, stage_free, dkv_done, epi
+  static constexpr int kNumBars = 1 + 2 * kQStages + 4 + kDsBufs + 6;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 64;
+  static constexpr uint32_t kTmSt = 0, kTmDPt = 128, kTmPt = 256, kTmDV = 320, kTmDK = 384, kTmDQ = 448;
+  static_assert(kTmDQ + D <= kTmemCols, "tensor memory budget");
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+// warps 0-3: TMA producer, MMA issuer, two idle; 4-7: dQ drain; 8-15: dS (two column groups)
+constexpr int kPipeThreads = 512;
+constexpr uint32_t kPipeRegsCtl = 56, kPipeRegsDrain = 72, kPipeRegsDs = 192;
+static_assert(128 * kPipeRegsCtl + 128 * kPipeRegsDrain + 256 * kPipeRegsDs <= kPipeThreads * 128,
+              "register split exceeds the launch budget");
+
+// acc (+)= X^T . B with X^T (M = 128 keys, K = 128 queries) in tensor memory as bf16
+// pairs, query pair p at column p; B the query tile read MN-major.
+template <int D>
+__device__ __forceinline__ void issue_acc_tmem_linear(uint32_t acc_tmem, uint32_t a_tmem, SDesc b, bool first) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk)
+    umma_ts(acc_tmem, a_tmem + kk * 8, sdesc_at(b, kk * 128), idesc, (first && kk == 0) ? 0u : 1u);
+}
+
+__global__ void __launch_bounds__(kPipeThreads, 1)
+    bwd_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                    const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
+                    const __grid_constant__ CUtensorMap tmDQ, const BwdArgs a) {
+  using L = PipeLayout;
+  constexpr int D = L::D;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* bar_kv_full = bars;
+  uint64_t* bar_q_full = bars + 1;
+  uint64_t* bar_q_empty = bar_q_full + L::kQStages;
+  uint64_t* bar_s_full = bar_q_empty + L::kQStages;
+  uint64_t* bar_s_free = bar_s_full + 1;
+  uint64_t* bar_p_full = bar_s_free + 1;
+  uint64_t* bar_pt_free = bar_p_full + 1;
+  uint64_t* bar_ds_free = bar_pt_free + 1;
+  uint64_t* bar_dq_full = bar_ds_free + L::kDsBufs;
+  uint64_t* bar_dq_empty = bar_dq_full + 1;
+  uint64_t* bar_stage_full = bar_dq_empty + 1;
+  uint64_t* bar_stage_free = bar_stage_full + 1;
+  uint64_t* bar_dkv_done = bar_stage_free + 1;
+  uint64_t* bar_epi = bar_dkv_done + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  const uint32_t sbase = smem_u32(smem);
+
+  const int bh_count = a.B * a.H;
+  const int j = blockIdx.x / bh_count;
+  const int bh = blockIdx.x - j * bh_count;
+  const int b = bh / a.H, h = bh - (bh / a.H) * a.H;
+  const int n_qtiles = (a.Nq + 127) >> 7;
+  int i_first = 0;
+  if (a.causal) i_first = max(0, j * 128 - (a.Nk - a.Nq)) >> 7;
+  const int n_iters = n_qtiles - i_first;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_kv_full, 1);
+    for (int s = 0; s < L::kQStages; ++s) {
+      mbar_init(bar_q_full + s, 2);  // TMA bytes + the producer's stats
+      mbar_init(bar_q_empty + s, 1);
+    }
+    mbar_init(bar_s_full, 1);
+    mbar_init(bar_s_free, 8);  // one arrival per dS warp
+    mbar_init(bar_p_full, 8);
+    mbar_init(bar_pt_free, 1);
+    for (int s = 0; s < L::kDsBufs; ++s) mbar_init(bar_ds_free + s, 1);
+    mbar_init(bar_dq_full, 1);
+    mbar_init(bar_dq_empty, 4);  // one arrival per drain warp
+    mbar_init(bar_stage_full, 4);
+    mbar_init(bar_stage_free, 1);
+    mbar_init(bar_dkv_done, 1);
+    mbar_init(bar_epi, 8);
+    *abort_flag = 0;
+    fence_mbar_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmDO);
+    tma_prefetch_desc(&tmDQ);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const size_t stat_row = ((size_t)b * a.H + h) * a.Nq;
+
+  if (warp < 4) {
+    regs_dec<kPipeRegsCtl>();
+    if (warp == 0) {
+      // -------------------------------------------------------------- producer: TMA tiles + lse/D
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar_kv_full, 2 * L::kTileBytes);
+        tma_load_4d(smem + L::kOffK, &tmK, bar_kv_full, 0, h, j * 128, b);
+        tma_load_4d(smem + L::kOffV, &tmV, bar_kv_full, 0, h, j * 128, b);
+      }
+      for (int it = 0; it < n_iters; ++it) {
+        const int st = it % L::kQStages;
+        const int q0 = (i_first + it) * 128;
+        // -lse in log2 units (-inf for rows past Nq or with no visible key: P = 0) and
+        // -D, negated so that the dS warps add them; loads issued before the wait
+        float nl2[4], nd[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int q = q0 + lane + 32 * e;
+          nl2[e] = -INFINITY;
+          nd[e] = 0.f;
+          if (q < a.Nq) {
+            const float lse = a.lse[stat_row + q];
+            nl2[e] = (lse == -INFINITY) ? -INFINITY : -lse * 1.4426950408889634f;
+            nd[e] = -a.delta[stat_row + q];
+          }
+        }
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(bar_q_empty + st, ((it / L::kQStages) & 1) ^ 1, a.timeout_ns) && !*abort_flag;
+        if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) {
+          if (lane == 0) bwd_timeout(a.status, abort_flag);
+          break;
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(bar_q_full + st, 2 * L::kTileBytes);
+          tma_load_4d(smem + L::kOffQ + st * L::kTileBytes, &tmQ, bar_q_full + st, 0, h, q0, b);
+          tma_load_4d(smem + L::kOffDO + st * L::kTileBytes, &tmDO, bar_q_full + st, 0, h, q0, b);
+        }
+        float* stat = reinterpret_cast<float*>(smem + L::kOffStat) + st * 256;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          stat[lane + 32 * e] = nl2[e];
+          stat[128 + lane + 32 * e] = nd[e];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_q_full + st);
+      }
+    } else if (warp == 1 && lane == 0) {
+      // -------------------------------------------------------------- MMA issuer
+      bool ok = mbar_wait(bar_kv_full, 0, a.timeout_ns);
+      const SDesc k_kmaj = sdesc_make(sbase + L::kOffK, 16, 1024), v_kmaj = sdesc_make(sbase + L::kOffV, 16, 1024);
+      const SDesc k_mn = sdesc_make(sbase + L::kOffK, 16384, 1024);
+      const SDesc q_kmaj = sdesc_make(sbase + L::kOffQ, 16, 1024), do_kmaj = sdesc_make(sbase + L::kOffDO, 16, 1024);
+      const SDesc q_mn = sdesc_make(sbase + L::kOffQ, 16384, 1024), do_mn = sdesc_make(sbase + L::kOffDO, 16384, 1024);
+      const SDesc ds_kmaj = sdesc_make(sbase + L::kOffDS, 16, 1024), ds_mn = sdesc_make(sbase + L::kOffDS, 16384, 1024);
+      constexpr uint32_t kTile16 = L::kTileBytes / 16, kDs16 = L::kDsBytes / 16;
+      auto at = [](SDesc d, uint32_t off16) { return SDesc{d.lo + off16, d.hi}; };
+      auto issue_sdp = [&](int it) -> bool {
+        const int st = it % L::kQStages;
+        if (!mbar_wait(bar_q_full + st, (it / L::kQStages) & 1, a.timeout_ns) || *abort_flag) return false;
+        tc_fence_after();
+        issue_scores<D, false>(tmem + L::kTmSt, 0u, k_kmaj, at(q_kmaj, st * kTile16));
+        issue_scores<D, false>(tmem + L::kTmDPt, 0u, v_kmaj, at(do_kmaj, st * kTile16));
+        umma_commit(bar_s_full);
+        return true;
+      };
+      if (ok) {
+        tc_fence_after();
+        if (n_iters > 0) ok = issue_sdp(0);
+      }
+      for (int it = 0; it < n_iters && ok; ++it) {
+        const int st = it % L::kQStages;
+        const int db = it % L::kDsBufs;
+        // the dS warps hold S^T(it) and dP^T(it) in registers: start the next tile's
+        if (!mbar_wait(bar_s_free, it & 1, a.timeout_ns) || *abort_flag) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (it + 1 < n_iters && !issue_sdp(it + 1)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait(bar_p_full, it & 1, a.timeout_ns) || *abort_flag) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_acc_tmem_linear<D>(tmem + L::kTmDV, tmem + L::kTmPt, at(do_mn, st * kTile16), it == 0);
+        issue_acc<D, false>(tmem + L::kTmDK, 0u, at(ds_kmaj, db * kDs16), at(q_mn, st * kTile16), it == 0);
+        umma_commit(bar_q_empty + st);  // Q and dO of this tile are no longer read
+        umma_commit(bar_pt_free);       // nor is P^T
+        if (it > 0) {                   // the previous dQ tile must have left tensor memory
+          if (!mbar_wait(bar_dq_empty, (it - 1) & 1, a.timeout_ns) || *abort_flag) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        issue_dq<D>(tmem + L::kTmDQ, at(ds_mn, db * kDs16), k_mn);
+        umma_commit(bar_dq_full);
+        umma_commit(bar_ds_free + db);
+      }
+      if (!ok) bwd_timeout(a.status, abort_flag);
+      umma_commit(bar_dkv_done);
+    }
+  } else if (warp < 8) {
+    regs_dec<kPipeRegsDrain>();
+    // ---------------------------------------------------------------- dQ drain (thread = query)
+    const uint32_t quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_field = (quarter * 32) << 16;
+    const bool issuer = (warp == 4);
+    const uint32_t stage_row = sbase + L::kOffStage + r * 128;
+    bool ok = true;
+    for (int it = 0; it < n_iters && ok; ++it) {
+      const int q0 = (i_first + it) * 128;
+      if (!warp_wait_b(bar_dq_full, it & 1, a.timeout_ns) || *abort_flag) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll 1
+      for (int half = 0; half < 2 && ok; ++half) {
+        uint32_t g[32];
+        tmem_ld32(tmem + lane_field + L::kTmDQ + half * 32, g);
+        tmem_ld_wait(g);
+        if (half == 1) {  // the whole tile is in registers or already staged
+          tc_fence_before();
+          mbar_arrive_warp(bar_dq_empty);
+        }
+        const int k = 2 * it + half;
+        if (k > 0 && (!warp_wait_b(bar_stage_free, (k - 1) & 1, a.timeout_ns) || *abort_flag)) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(stage_row + ((c ^ (r & 7)) << 4), g[4 * c], g[4 * c + 1], g[4 * c + 2], g[4 * c + 3]);
+        fence_proxy_async_smem();
+        mbar_arrive_warp(bar_stage_full);
+        if (issuer) {
+          bool iss_ok = true;
+          if (lane == 0) {
+            iss_ok = mbar_wait(bar_stage_full, k & 1, a.timeout_ns);
+            if (iss_ok) {
+              tma_reduce_add_4d(&tmDQ, smem + L::kOffStage, half * 32, h, q0, b);
+              bulk_commit_group();
+              bulk_wait_group_read0();
+              mbar_arrive(bar_stage_free);
+            }
+          }
+          if (__shfl_sync(0xffffffffu, iss_ok ? 1 : 0, 0) == 0) ok = false;
+        }
+      }
+    }
+    if (issuer && lane == 0) bulk_wait_group0();
+    if (!ok && lane == 0) bwd_timeout(a.status, abort_flag);
+  } else {
+    regs_inc<kPipeRegsDs>();
+    // ---------------------------------------------------------------- dS warps (thread = key)
+    const uint32_t quarter = warp & 3;
+    const int grp = (warp - 8) >> 2;  // column group: queries [64 grp, 64 grp + 64) of each tile
+    const int r = quarter * 32 + lane;
+    const int key = j * 128 + r;
+    const uint32_t lane_field = (quarter * 32) << 16;
+    const bool key_ok = key < a.Nk;
+    const int qmin = a.causal ? key - (a.Nk - a.Nq) : -(1 << 30);
+    const int col = 64 * grp;
+    bool ok = true;
+    for (int it = 0; it < n_iters && ok; ++it) {
+      const int st = it % L::kQStages;
+      const int db = it % L::kDsBufs;
+      const int q0 = (i_first + it) * 128;
+      if (!warp_wait_b(bar_q_full + st, (it / L::kQStages) & 1, a.timeout_ns) ||
+          !warp_wait_b(bar_s_full, it & 1, a.timeout_ns) || *abort_flag) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sv0[32], sv1[32], dp0[32], dp1[32];
+      tmem_ld32(tmem + lane_field + L::kTmSt + col, sv0);
+      tmem_ld32(tmem + lane_field + L::kTmSt + col + 32, sv1);
+      tmem_ld32(tmem + lane_field + L::kTmDPt + col, dp0);
+      tmem_ld32(tmem + lane_field + L::kTmDPt + col + 32, dp1);
+      tmem_ld_wait(sv0);
+      reg_pin(sv1);
+      reg_pin(dp0);
+      reg_pin(dp1);
+      tc_fence_before();
+      mbar_arrive_warp(bar_s_free);  // S^T / dP^T may be overwritten
+      const uint32_t stat_u32 = sbase + L::kOffStat + st * 1024 + col * 4;
+      const uint32_t ds_row = sbase + L::kOffDS + db * L::kDsBytes + grp * 16384 + r * 128;
+      const int qs0 = q0 + col, qs1 = q0 + col + 32;
+      const bool key_tail = j * 128 + 128 > a.Nk;
+      const int last_key_qmin = j * 128 + 127 - (a.Nk - a.Nq);
+      uint32_t pk[16], dk2[16];
+      if (key_tail || (a.causal && last_key_qmin > qs0))
+        ds_block<32, true>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk, dk2);
+      else
+        ds_block<32, false>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk, dk2);
+      // P^T may be written once the previous tile's dV has read it
+      if (it > 0 && (!warp_wait_b(bar_pt_free, (it - 1) & 1, a.timeout_ns) || *abort_flag)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      tmem_st16(tmem + lane_field + L::kTmPt + 32 * grp, pk);
+      if (!warp_wait_b(bar_ds_free + db, ((it / L::kDsBufs) & 1) ^ 1, a.timeout_ns) || *abort_flag) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4)
+        st_shared_v4(ds_row + ((c4 ^ (r & 7)) << 4), dk2[4 * c4], dk2[4 * c4 + 1], dk2[4 * c4 + 2], dk2[4 * c4 + 3]);
+      if (key_tail || (a.causal && last_key_qmin > qs1))
+        ds_block<32, true>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk, dk2);
+      else
+        ds_block<32, false>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk, dk2);
+      tmem_st16(tmem + lane_field + L::kTmPt + 32 * grp + 16, pk);
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4)
+        st_shared_v4(ds_row + (((4 + c4) ^ (r & 7)) << 4), dk2[4 * c4], dk2[4 * c4 + 1], dk2[4 * c4 + 2],
+                     dk2[4 * c4 + 3]);
+      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive_warp(bar_p_full);
+    }
+    // ---------------------------------------------------------------- dK / dV epilogue
+    // group 0 stores dK (times scale) through the K tile's smem, group 1 dV through V's
+    if (ok && warp_wait_b(bar_dkv_done, 0, a.timeout_ns) && !*abort_flag) {
+      tc_fence_after();
+      const uint32_t src = tmem + lane_field + (grp == 0 ? L::kTmDK : L::kTmDV);
+      const uint32_t dst = sbase + (grp == 0 ? L::kOffK : L::kOffV);
+      const float mul = grp == 0 ? a.scale : 1.f;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(src + cc * 32, o);
+        tmem_ld_wait(o);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int chunk = cc * 4 + q4;
+          const uint32_t addr = dst + r * 128 + ((chunk ^ (r & 7)) << 4);
+          const float* f = reinterpret_cast<const float*>(o) + q4 * 8;
+          st_shared_v4(addr, pack_bf16x2(f[0] * mul, f[1] * mul), pack_bf16x2(f[2] * mul, f[3] * mul),
+                       pack_bf16x2(f[4] * mul, f[5] * mul), pack_bf16x2(f[6] * mul, f[7] * mul));
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive_warp(bar_epi);
+      if (warp == 8 && lane == 0) {
+        if (mbar_wait(bar_epi, 0, a.timeout_ns)) {
+          tma_store_4d(&tmDK, smem + L::kOffK, 0, h, j * 128, b);
+          tma_store_4d(&tmDV, smem + L::kOffV, 0, h, j * 128, b);
           bulk_commit_group();
           bulk_wait_group0();
         } else {
@@ -608,9 +1000,12 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes) !=
-        cudaSuccess)
-      return FA_ERR_CUDA;
+    cudaError_t e;
+    if constexpr (D == 64)
+      e = cudaFuncSetAttribute(bwd_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PipeLayout::kSmemBytes);
+    else
+      e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+    if (e != cudaSuccess) return FA_ERR_CUDA;
     attr_done[dev] = true;
   }
   // 1. D rows and a zeroed dQ accumulator
@@ -627,11 +1022,10 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
     if (err != cudaSuccess) return FA_ERR_CUDA;
   }
   // 2. main kernel
-  CUtensorMap tq, tk, tv, tdo, tdk, tdv, tdq;
+  CUtensorMap tq, tk, tv, tdo, tdk, tdv;
   if (!encode_bshd_map(&tq, L0.q, L0.B, L0.Nq, L0.H, D) || !encode_bshd_map(&tk, L0.k, L0.B, L0.Nk, L0.H, D) ||
       !encode_bshd_map(&tv, L0.v, L0.B, L0.Nk, L0.H, D) || !encode_bshd_map(&tdo, L0.dout, L0.B, L0.Nq, L0.H, D) ||
-      !encode_bshd_map(&tdk, L0.dk, L0.B, L0.Nk, L0.H, D) || !encode_bshd_map(&tdv, L0.dv, L0.B, L0.Nk, L0.H, D) ||
-      !encode_bshd_map_f32(&tdq, L0.dq_acc, L0.B, L0.Nq, L0.H, D))
+      !encode_bshd_map(&tdk, L0.dk, L0.B, L0.Nk, L0.H, D) || !encode_bshd_map(&tdv, L0.dv, L0.B, L0.Nk, L0.H, D))
     return FA_ERR_CUDA;
   BwdArgs a;
   a.lse = L0.lse;
@@ -650,7 +1044,14 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   const long long grid = (long long)a.n_kv_tiles * L0.B * L0.H;
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   prof_before(stream, kKBwdMain);
-  bwd_main_kernel<D><<<(unsigned)grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, tdq, a);
+  if constexpr (D == 64) {
+    CUtensorMap tdq;
+    if (!encode_bshd_map_f32(&tdq, L0.dq_acc, L0.B, L0.Nq, L0.H, D)) return FA_ERR_CUDA;
+    bwd_pipe_kernel<<<(unsigned)grid, kPipeThreads, PipeLayout::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv,
+                                                                                        tdq, a);
+  } else {
+    bwd_main_kernel<D><<<(unsigned)grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
+  }
   const cudaError_t err_main = cudaGetLastError();
   prof_after(stream, kKBwdMain);
   if (err_main != cudaSuccess) return FA_ERR_CUDA;
