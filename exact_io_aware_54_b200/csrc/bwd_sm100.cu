@@ -545,18 +545,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 // from shared memory: no tensor-memory location is written by one MMA while an
 // earlier MMA still reads it, so the tensor core never drains between tiles.  Four
 // drain warps move each dQ tile out of tensor memory and add it to the fp32
-// accumulator with TMA reductions of whole 128-byte rows.
+// accumulator.  A thread holds one query row; each warp turns its 32 rows around
+// in shared memory so that one vector reduction instruction covers four whole
+// 128-byte rows (reductions of partial rows run at half the L2 rate).
 //
 // Tensor core order per query tile i:   S^T(i+1) dP^T(i+1) | dV(i) dK(i) | dQ(i)
-// dS warps:   load S^T(i), dP^T(i) -> release -> P^T(i) to TMEM, dS(i) to smem
-// drain warps: dQ(i) TMEM -> smem (32 columns at a time) -> TMA reduce-add
+// dS warps:    load S^T(i), dP^T(i) -> release -> P^T(i) to TMEM, dS(i) to smem
+// drain warps: dQ(i) TMEM -> registers -> release -> smem transpose -> red.global.add.v4
 struct PipeLayout {
   static constexpr int D = 64;
   static constexpr int kTileBytes = 128 * D * 2;  // 16 KB
   static constexpr int kQStages = 3;
   static constexpr int kDsBufs = 2;
   static constexpr int kDsBytes = 2 * 16384;        // [64-query atom][128 keys][64 queries] bf16
-  static constexpr int kStageBytes = 128 * 32 * 4;  // one fp32 box of dQ: 128 queries x 32 columns
+  static constexpr int kStageBytes = 4 * 32 * 128;  // per drain warp: 32 rows x 32 fp32 columns
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
   static constexpr int kOffQ = 2 * kTileBytes;
@@ -566,8 +568,8 @@ struct PipeLayout {
   static constexpr int kOffStat = kOffStage + kStageBytes;  // per stage: -lse2[128], -D[128]
   static constexpr int kOffBar = kOffStat + kQStages * 2 * 128 * 4;
   // kv_full, q_full[QS], q_empty[QS], s_full, s_free, p_full, pt_free, ds_free[DSB],
-  // dq_full, dq_empty, stage_full, stage_free, dkv_done, epi
-  static constexpr int kNumBars = 1 + 2 * kQStages + 4 + kDsBufs + 6;
+  // dq_full, dq_empty, dkv_done, epi
+  static constexpr int kNumBars = 1 + 2 * kQStages + 4 + kDsBufs + 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64;
   static constexpr uint32_t kTmSt = 0, kTmDPt = 128, kTmPt = 256, kTmDV = 320, kTmDK = 384, kTmDQ = 448;
@@ -576,7 +578,7 @@ struct PipeLayout {
 };
 // warps 0-3: TMA producer, MMA issuer, two idle; 4-7: dQ drain; 8-15: dS (two column groups)
 constexpr int kPipeThreads = 512;
-constexpr uint32_t kPipeRegsCtl = 56, kPipeRegsDrain = 72, kPipeRegsDs = 192;
+constexpr uint32_t kPipeRegsCtl = 56, kPipeRegsDrain = 88, kPipeRegsDs = 184;
 static_assert(128 * kPipeRegsCtl + 128 * kPipeRegsDrain + 256 * kPipeRegsDs <= kPipeThreads * 128,
               "register split exceeds the launch budget");
 
@@ -594,7 +596,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     bwd_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                     const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
-                    const __grid_constant__ CUtensorMap tmDQ, const BwdArgs a) {
+                    const BwdArgs a) {
   using L = PipeLayout;
   constexpr int D = L::D;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -609,9 +611,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   uint64_t* bar_ds_free = bar_pt_free + 1;
   uint64_t* bar_dq_full = bar_ds_free + L::kDsBufs;
   uint64_t* bar_dq_empty = bar_dq_full + 1;
-  uint64_t* bar_stage_full = bar_dq_empty + 1;
-  uint64_t* bar_stage_free = bar_stage_full + 1;
-  uint64_t* bar_dkv_done = bar_stage_free + 1;
+  uint64_t* bar_dkv_done = bar_dq_empty + 1;
   uint64_t* bar_epi = bar_dkv_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);
@@ -641,8 +641,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     for (int s = 0; s < L::kDsBufs; ++s) mbar_init(bar_ds_free + s, 1);
     mbar_init(bar_dq_full, 1);
     mbar_init(bar_dq_empty, 4);  // one arrival per drain warp
-    mbar_init(bar_stage_full, 4);
-    mbar_init(bar_stage_free, 1);
     mbar_init(bar_dkv_done, 1);
     mbar_init(bar_epi, 8);
     *abort_flag = 0;
@@ -654,7 +652,6 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmDO);
-    tma_prefetch_desc(&tmDQ);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -775,53 +772,43 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     regs_dec<kPipeRegsDrain>();
     // ---------------------------------------------------------------- dQ drain (thread = query)
     const uint32_t quarter = warp & 3;
-    const int r = quarter * 32 + lane;
     const uint32_t lane_field = (quarter * 32) << 16;
-    const bool issuer = (warp == 4);
-    const uint32_t stage_row = sbase + L::kOffStage + r * 128;
+    // this warp's 4 KB turn-around buffer: row = lane, 16-byte chunk c at (c ^ (row & 7))
+    const uint32_t scratch = sbase + L::kOffStage + quarter * 4096;
+    const int rr_sub = lane >> 3, cc = lane & 7;  // read side: row 4k + rr_sub, chunk cc
     bool ok = true;
     for (int it = 0; it < n_iters && ok; ++it) {
-      const int q0 = (i_first + it) * 128;
+      const int q0 = (i_first + it) * 128 + quarter * 32;  // first query row of this warp
       if (!warp_wait_b(bar_dq_full, it & 1, a.timeout_ns) || *abort_flag) {
         ok = false;
         break;
       }
       tc_fence_after();
 #pragma unroll 1
-      for (int half = 0; half < 2 && ok; ++half) {
+      for (int half = 0; half < 2; ++half) {
         uint32_t g[32];
         tmem_ld32(tmem + lane_field + L::kTmDQ + half * 32, g);
         tmem_ld_wait(g);
-        if (half == 1) {  // the whole tile is in registers or already staged
+        if (half == 1) {  // the tile is out of tensor memory
           tc_fence_before();
           mbar_arrive_warp(bar_dq_empty);
         }
-        const int k = 2 * it + half;
-        if (k > 0 && (!warp_wait_b(bar_stage_free, (k - 1) & 1, a.timeout_ns) || *abort_flag)) {
-          ok = false;
-          break;
-        }
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-          st_shared_v4(stage_row + ((c ^ (r & 7)) << 4), g[4 * c], g[4 * c + 1], g[4 * c + 2], g[4 * c + 3]);
-        fence_proxy_async_smem();
-        mbar_arrive_warp(bar_stage_full);
-        if (issuer) {
-          bool iss_ok = true;
-          if (lane == 0) {
-            iss_ok = mbar_wait(bar_stage_full, k & 1, a.timeout_ns);
-            if (iss_ok) {
-              tma_reduce_add_4d(&tmDQ, smem + L::kOffStage, half * 32, h, q0, b);
-              bulk_commit_group();
-              bulk_wait_group_read0();
-              mbar_arrive(bar_stage_free);
-            }
-          }
-          if (__shfl_sync(0xffffffffu, iss_ok ? 1 : 0, 0) == 0) ok = false;
+          st_shared_v4(scratch + lane * 128 + ((c ^ (lane & 7)) << 4), g[4 * c], g[4 * c + 1], g[4 * c + 2],
+                       g[4 * c + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int row = 4 * k + rr_sub;
+          const float4 v = ld_shared_f4(scratch + row * 128 + ((cc ^ (row & 7)) << 4));
+          if (q0 + row < a.Nq)
+            red_add_v4(a.dq_acc + (((size_t)b * a.Nq + q0 + row) * a.H + h) * D + half * 32 + cc * 4, v.x, v.y, v.z,
+                       v.w);
         }
+        __syncwarp();
       }
     }
-    if (issuer && lane == 0) bulk_wait_group0();
     if (!ok && lane == 0) bwd_timeout(a.status, abort_flag);
   } else {
     regs_inc<kPipeRegsDs>();
@@ -1045,10 +1032,7 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   prof_before(stream, kKBwdMain);
   if constexpr (D == 64) {
-    CUtensorMap tdq;
-    if (!encode_bshd_map_f32(&tdq, L0.dq_acc, L0.B, L0.Nq, L0.H, D)) return FA_ERR_CUDA;
-    bwd_pipe_kernel<<<(unsigned)grid, kPipeThreads, PipeLayout::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv,
-                                                                                        tdq, a);
+    bwd_pipe_kernel<<<(unsigned)grid, kPipeThreads, PipeLayout::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
   } else {
     bwd_main_kernel<D><<<(unsigned)grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
   }
