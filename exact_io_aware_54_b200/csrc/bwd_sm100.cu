@@ -80,6 +80,8 @@ struct BwdArgs {
   float scale_log2;
   int n_kv_tiles;
   unsigned long long timeout_ns;
+  uint4* dk;  // [B, Nk, H, D] bf16, written directly by the d = 64 kernel
+  uint4* dv;
 };
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
@@ -552,33 +554,42 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Tensor core order per query tile i:   S^T(i+1) dP^T(i+1) | dV(i) dK(i) | dQ(i)
 // dS warps:    load S^T(i), dP^T(i) -> release -> P^T(i) to TMEM, dS(i) to smem
 // drain warps: dQ(i) TMEM -> registers -> release -> smem transpose -> red.global.add.v4
+//
+// The kernel is persistent: one CTA per SM walks the work items (key tile, b, h),
+// heaviest first.  Every role counts query tiles over all its items, so the
+// per-tile barriers run on one stream of phases.  K has two slots and the next
+// item's K is loaded a whole item ahead; V has one slot, released after the item's
+// last dP^T, so the next V loads while the last query tile is finished.  The dS
+// warps write dK and dV straight from registers to global memory.
 struct PipeLayout {
   static constexpr int D = 64;
   static constexpr int kTileBytes = 128 * D * 2;  // 16 KB
   static constexpr int kQStages = 3;
   static constexpr int kDsBufs = 2;
-  static constexpr int kDsBytes = 2 * 16384;        // [64-query atom][128 keys][64 queries] bf16
-  static constexpr int kStageBytes = 4 * 32 * 128;  // per drain warp: 32 rows x 32 fp32 columns
-  static constexpr int kOffK = 0;
-  static constexpr int kOffV = kTileBytes;
-  static constexpr int kOffQ = 2 * kTileBytes;
+  static constexpr int kDsBytes = 2 * 16384;  // [64-query atom][128 keys][64 queries] bf16
+  // the drain warps turn dQ rows around in the first 16 KB of the dS buffer of the
+  // tile they drain (its MMAs have completed; its next writer waits for them)
+  static constexpr int kScratchBytes = 4 * 32 * 128;
+  static constexpr int kOffK = 0;  // two slots
+  static constexpr int kOffV = 2 * kTileBytes;
+  static constexpr int kOffQ = 3 * kTileBytes;
   static constexpr int kOffDO = kOffQ + kQStages * kTileBytes;
   static constexpr int kOffDS = kOffDO + kQStages * kTileBytes;
-  static constexpr int kOffStage = kOffDS + kDsBufs * kDsBytes;
-  static constexpr int kOffStat = kOffStage + kStageBytes;  // per stage: -lse2[128], -D[128]
+  static constexpr int kOffStat = kOffDS + kDsBufs * kDsBytes;  // per stage: -lse2[128], -D[128]
   static constexpr int kOffBar = kOffStat + kQStages * 2 * 128 * 4;
-  // kv_full, q_full[QS], q_empty[QS], s_full, s_free, p_full, pt_free, ds_free[DSB],
-  // dq_full, dq_empty, dkv_done, epi
-  static constexpr int kNumBars = 1 + 2 * kQStages + 4 + kDsBufs + 4;
+  // k_full[2], k_free[2], v_full, v_free, q_full[QS], q_empty[QS], s_full, s_free, p_full,
+  // pt_free, ds_free[DSB], dq_full, dq_empty, dkv_done, acc_free
+  static constexpr int kNumBars = 6 + 2 * kQStages + 4 + kDsBufs + 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64;
   static constexpr uint32_t kTmSt = 0, kTmDPt = 128, kTmPt = 256, kTmDV = 320, kTmDK = 384, kTmDQ = 448;
   static_assert(kTmDQ + D <= kTmemCols, "tensor memory budget");
+  static_assert(kScratchBytes <= kDsBytes, "drain scratch");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 // warps 0-3: TMA producer, MMA issuer, two idle; 4-7: dQ drain; 8-15: dS (two column groups)
 constexpr int kPipeThreads = 512;
-constexpr uint32_t kPipeRegsCtl = 56, kPipeRegsDrain = 88, kPipeRegsDs = 184;
+constexpr uint32_t kPipeRegsCtl = 72, kPipeRegsDrain = 80, kPipeRegsDs = 176;
 static_assert(128 * kPipeRegsCtl + 128 * kPipeRegsDrain + 256 * kPipeRegsDs <= kPipeThreads * 128,
               "register split exceeds the launch budget");
 
@@ -592,17 +603,85 @@ __device__ __forceinline__ void issue_acc_tmem_linear(uint32_t acc_tmem, uint32_
     umma_ts(acc_tmem, a_tmem + kk * 8, sdesc_at(b, kk * 128), idesc, (first && kk == 0) ? 0u : 1u);
 }
 
+// Work item w: key tile j = w / (B H) (small j first: under the causal mask they see
+// the most query tiles), head (b, h) = w % (B H); query tiles i_first .. n_qtiles - 1.
+// CTA c takes the items of its column in a snake order over rounds of gridDim.x
+// items (c, 2G - 1 - c, 2G + c, ...), which pairs heavy rounds with light ones.
+__device__ __forceinline__ int pipe_item_index(int k) {
+  const int g = gridDim.x;
+  return k * g + ((k & 1) ? (g - 1 - (int)blockIdx.x) : (int)blockIdx.x);
+}
+struct PipeItem {
+  int j, b, h, i_first, n;
+};
+__device__ __forceinline__ PipeItem pipe_item(const BwdArgs& a, int w) {
+  PipeItem it;
+  const int bh_count = a.B * a.H;
+  it.j = w / bh_count;
+  const int bh = w - it.j * bh_count;
+  it.b = bh / a.H;
+  it.h = bh - it.b * a.H;
+  const int n_qtiles = (a.Nq + 127) >> 7;
+  it.i_first = a.causal ? (max(0, it.j * 128 - (a.Nk - a.Nq)) >> 7) : 0;
+  it.n = n_qtiles - it.i_first;
+  return it;
+}
+
+// Walks the query tiles of this CTA's items in order.
+struct PipeCursor {
+  int k;  // item counter of this CTA
+  int t;  // query tile within the item
+  bool valid;
+  PipeItem itm;
+  __device__ __forceinline__ void start(const BwdArgs& a, int n_items) {
+    k = 0;
+    t = 0;
+    const int w = pipe_item_index(0);
+    valid = w < n_items;
+    if (valid) itm = pipe_item(a, w);
+  }
+  __device__ __forceinline__ void advance(const BwdArgs& a, int n_items) {
+    if (++t < itm.n) return;
+    t = 0;
+    ++k;
+    const int w = pipe_item_index(k);
+    valid = w < n_items;
+    if (valid) itm = pipe_item(a, w);
+  }
+};
+
+// -lse in log2 units (-inf for rows past Nq or with no visible key: P = 0) and -D of
+// four query rows per lane, negated so that the dS warps add them.
+__device__ __forceinline__ void pipe_load_stats(const BwdArgs& a, const PipeCursor& c, uint32_t lane, float (&nl2)[4],
+                                                float (&nd)[4]) {
+  const size_t stat_row = ((size_t)c.itm.b * a.H + c.itm.h) * a.Nq;
+  const int q0 = (c.itm.i_first + c.t) * 128;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const int q = q0 + lane + 32 * e;
+    nl2[e] = -INFINITY;
+    nd[e] = 0.f;
+    if (q < a.Nq) {
+      const float lse = a.lse[stat_row + q];
+      nl2[e] = (lse == -INFINITY) ? -INFINITY : -lse * 1.4426950408889634f;
+      nd[e] = -a.delta[stat_row + q];
+    }
+  }
+}
+
 __global__ void __launch_bounds__(kPipeThreads, 1)
     bwd_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                    const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDV,
                     const BwdArgs a) {
   using L = PipeLayout;
   constexpr int D = L::D;
   extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
-  uint64_t* bar_kv_full = bars;
-  uint64_t* bar_q_full = bars + 1;
+  uint64_t* bar_k_full = bars;  // [2]
+  uint64_t* bar_k_free = bars + 2;  // [2]
+  uint64_t* bar_v_full = bars + 4;
+  uint64_t* bar_v_free = bars + 5;
+  uint64_t* bar_q_full = bars + 6;
   uint64_t* bar_q_empty = bar_q_full + L::kQStages;
   uint64_t* bar_s_full = bar_q_empty + L::kQStages;
   uint64_t* bar_s_free = bar_s_full + 1;
@@ -612,24 +691,21 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   uint64_t* bar_dq_full = bar_ds_free + L::kDsBufs;
   uint64_t* bar_dq_empty = bar_dq_full + 1;
   uint64_t* bar_dkv_done = bar_dq_empty + 1;
-  uint64_t* bar_epi = bar_dkv_done + 1;
+  uint64_t* bar_acc_free = bar_dkv_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);
 
   const uint32_t warp = warp_id(), lane = lane_id();
   const uint32_t sbase = smem_u32(smem);
-
-  const int bh_count = a.B * a.H;
-  const int j = blockIdx.x / bh_count;
-  const int bh = blockIdx.x - j * bh_count;
-  const int b = bh / a.H, h = bh - (bh / a.H) * a.H;
-  const int n_qtiles = (a.Nq + 127) >> 7;
-  int i_first = 0;
-  if (a.causal) i_first = max(0, j * 128 - (a.Nk - a.Nq)) >> 7;
-  const int n_iters = n_qtiles - i_first;
+  const int n_items = a.n_kv_tiles * a.B * a.H;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar_kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_k_full + s, 1);
+      mbar_init(bar_k_free + s, 1);
+    }
+    mbar_init(bar_v_full, 1);
+    mbar_init(bar_v_free, 1);
     for (int s = 0; s < L::kQStages; ++s) {
       mbar_init(bar_q_full + s, 2);  // TMA bytes + the producer's stats
       mbar_init(bar_q_empty + s, 1);
@@ -638,11 +714,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     mbar_init(bar_s_free, 8);  // one arrival per dS warp
     mbar_init(bar_p_full, 8);
     mbar_init(bar_pt_free, 1);
-    for (int s = 0; s < L::kDsBufs; ++s) mbar_init(bar_ds_free + s, 1);
+    for (int s = 0; s < L::kDsBufs; ++s) mbar_init(bar_ds_free + s, 1 + 4);  // dQ MMA + the drain warps
     mbar_init(bar_dq_full, 1);
     mbar_init(bar_dq_empty, 4);  // one arrival per drain warp
     mbar_init(bar_dkv_done, 1);
-    mbar_init(bar_epi, 8);
+    mbar_init(bar_acc_free, 8);
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -661,44 +737,42 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const size_t stat_row = ((size_t)b * a.H + h) * a.Nq;
 
   if (warp < 4) {
     regs_dec<kPipeRegsCtl>();
     if (warp == 0) {
       // -------------------------------------------------------------- producer: TMA tiles + lse/D
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar_kv_full, 2 * L::kTileBytes);
-        tma_load_4d(smem + L::kOffK, &tmK, bar_kv_full, 0, h, j * 128, b);
-        tma_load_4d(smem + L::kOffV, &tmV, bar_kv_full, 0, h, j * 128, b);
-      }
-      for (int it = 0; it < n_iters; ++it) {
-        const int st = it % L::kQStages;
-        const int q0 = (i_first + it) * 128;
-        // -lse in log2 units (-inf for rows past Nq or with no visible key: P = 0) and
-        // -D, negated so that the dS warps add them; loads issued before the wait
-        float nl2[4], nd[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int q = q0 + lane + 32 * e;
-          nl2[e] = -INFINITY;
-          nd[e] = 0.f;
-          if (q < a.Nq) {
-            const float lse = a.lse[stat_row + q];
-            nl2[e] = (lse == -INFINITY) ? -INFINITY : -lse * 1.4426950408889634f;
-            nd[e] = -a.delta[stat_row + q];
-          }
+      PipeCursor cur;
+      cur.start(a, n_items);
+      bool ok = true;
+      float nl2[4], nd[4];
+      if (cur.valid) {
+        pipe_load_stats(a, cur, lane, nl2, nd);
+        if (lane == 0) {  // the first item's K and V
+          mbar_arrive_expect_tx(bar_k_full, L::kTileBytes);
+          tma_load_4d(smem + L::kOffK, &tmK, bar_k_full, 0, cur.itm.h, cur.itm.j * 128, cur.itm.b);
+          mbar_arrive_expect_tx(bar_v_full, L::kTileBytes);
+          tma_load_4d(smem + L::kOffV, &tmV, bar_v_full, 0, cur.itm.h, cur.itm.j * 128, cur.itm.b);
         }
-        bool ok = true;
-        if (lane == 0) ok = mbar_wait(bar_q_empty + st, ((it / L::kQStages) & 1) ^ 1, a.timeout_ns) && !*abort_flag;
-        if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) {
-          if (lane == 0) bwd_timeout(a.status, abort_flag);
+      }
+      for (int T = 0; cur.valid && ok; ++T) {
+        const int st = T % L::kQStages;
+        const int q0 = (cur.itm.i_first + cur.t) * 128;
+        PipeCursor nxt = cur;
+        nxt.advance(a, n_items);
+        // the next tile's statistics are loaded while this tile waits for its stage
+        float nl2n[4], ndn[4];
+        if (nxt.valid) pipe_load_stats(a, nxt, lane, nl2n, ndn);
+        bool got = true;
+        if (lane == 0) got = mbar_wait(bar_q_empty + st, ((T / L::kQStages) & 1) ^ 1, a.timeout_ns) && !*abort_flag;
+        if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) {
+          ok = false;
           break;
         }
         if (lane == 0) {
           mbar_arrive_expect_tx(bar_q_full + st, 2 * L::kTileBytes);
-          tma_load_4d(smem + L::kOffQ + st * L::kTileBytes, &tmQ, bar_q_full + st, 0, h, q0, b);
-          tma_load_4d(smem + L::kOffDO + st * L::kTileBytes, &tmDO, bar_q_full + st, 0, h, q0, b);
+          tma_load_4d(smem + L::kOffQ + st * L::kTileBytes, &tmQ, bar_q_full + st, 0, cur.itm.h, q0, cur.itm.b);
+          tma_load_4d(smem + L::kOffDO + st * L::kTileBytes, &tmDO, bar_q_full + st, 0, cur.itm.h, q0, cur.itm.b);
         }
         float* stat = reinterpret_cast<float*>(smem + L::kOffStat) + st * 256;
 #pragma unroll
@@ -708,10 +782,38 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_q_full + st);
+        if (cur.t + 1 == cur.itm.n && nxt.valid) {
+          // the last query tile of item u is staged: load item u + 1's K (into the slot
+          // item u - 1 used) and V (once item u's last dP^T has read it)
+          const int u1 = cur.k + 1;
+          if (lane == 0) {
+            got = (u1 < 2 || mbar_wait(bar_k_free + (u1 & 1), ((u1 >> 1) - 1) & 1, a.timeout_ns)) && !*abort_flag;
+            if (got) {
+              mbar_arrive_expect_tx(bar_k_full + (u1 & 1), L::kTileBytes);
+              tma_load_4d(smem + L::kOffK + (u1 & 1) * L::kTileBytes, &tmK, bar_k_full + (u1 & 1), 0, nxt.itm.h,
+                          nxt.itm.j * 128, nxt.itm.b);
+              got = mbar_wait(bar_v_free, cur.k & 1, a.timeout_ns) && !*abort_flag;
+            }
+            if (got) {
+              mbar_arrive_expect_tx(bar_v_full, L::kTileBytes);
+              tma_load_4d(smem + L::kOffV, &tmV, bar_v_full, 0, nxt.itm.h, nxt.itm.j * 128, nxt.itm.b);
+            }
+          }
+          if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) {
+            ok = false;
+            break;
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          nl2[e] = nl2n[e];
+          nd[e] = ndn[e];
+        }
+        cur = nxt;
       }
+      if (!ok && lane == 0) bwd_timeout(a.status, abort_flag);
     } else if (warp == 1 && lane == 0) {
       // -------------------------------------------------------------- MMA issuer
-      bool ok = mbar_wait(bar_kv_full, 0, a.timeout_ns);
       const SDesc k_kmaj = sdesc_make(sbase + L::kOffK, 16, 1024), v_kmaj = sdesc_make(sbase + L::kOffV, 16, 1024);
       const SDesc k_mn = sdesc_make(sbase + L::kOffK, 16384, 1024);
       const SDesc q_kmaj = sdesc_make(sbase + L::kOffQ, 16, 1024), do_kmaj = sdesc_make(sbase + L::kOffDO, 16, 1024);
@@ -719,67 +821,98 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       const SDesc ds_kmaj = sdesc_make(sbase + L::kOffDS, 16, 1024), ds_mn = sdesc_make(sbase + L::kOffDS, 16384, 1024);
       constexpr uint32_t kTile16 = L::kTileBytes / 16, kDs16 = L::kDsBytes / 16;
       auto at = [](SDesc d, uint32_t off16) { return SDesc{d.lo + off16, d.hi}; };
-      auto issue_sdp = [&](int it) -> bool {
-        const int st = it % L::kQStages;
-        if (!mbar_wait(bar_q_full + st, (it / L::kQStages) & 1, a.timeout_ns) || *abort_flag) return false;
+      // S^T and dP^T of global query tile T with K in slot ks; the item's last
+      // dP^T releases V
+      auto issue_sdp = [&](int T, int ks, bool last_of_item) -> bool {
+        const int st = T % L::kQStages;
+        if (!mbar_wait(bar_q_full + st, (T / L::kQStages) & 1, a.timeout_ns) || *abort_flag) return false;
         tc_fence_after();
-        issue_scores<D, false>(tmem + L::kTmSt, 0u, k_kmaj, at(q_kmaj, st * kTile16));
+        issue_scores<D, false>(tmem + L::kTmSt, 0u, at(k_kmaj, ks * kTile16), at(q_kmaj, st * kTile16));
         issue_scores<D, false>(tmem + L::kTmDPt, 0u, v_kmaj, at(do_kmaj, st * kTile16));
         umma_commit(bar_s_full);
+        if (last_of_item) umma_commit(bar_v_free);
         return true;
       };
-      if (ok) {
-        tc_fence_after();
-        if (n_iters > 0) ok = issue_sdp(0);
-      }
-      for (int it = 0; it < n_iters && ok; ++it) {
-        const int st = it % L::kQStages;
-        const int db = it % L::kDsBufs;
-        // the dS warps hold S^T(it) and dP^T(it) in registers: start the next tile's
-        if (!mbar_wait(bar_s_free, it & 1, a.timeout_ns) || *abort_flag) {
+      bool ok = true;
+      int T = 0, u = 0;
+      for (int w; (w = pipe_item_index(u)) < n_items && ok; ++u) {
+        const PipeItem itm = pipe_item(a, w);
+        const int ks = u & 1;
+        // this item's K and V; its first scores
+        if (!mbar_wait(bar_k_full + ks, (u >> 1) & 1, a.timeout_ns) || !mbar_wait(bar_v_full, u & 1, a.timeout_ns) ||
+            *abort_flag) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (it + 1 < n_iters && !issue_sdp(it + 1)) {
+        if (!issue_sdp(T, ks, itm.n == 1)) {
           ok = false;
           break;
         }
-        if (!mbar_wait(bar_p_full, it & 1, a.timeout_ns) || *abort_flag) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        issue_acc_tmem_linear<D>(tmem + L::kTmDV, tmem + L::kTmPt, at(do_mn, st * kTile16), it == 0);
-        issue_acc<D, false>(tmem + L::kTmDK, 0u, at(ds_kmaj, db * kDs16), at(q_mn, st * kTile16), it == 0);
-        umma_commit(bar_q_empty + st);  // Q and dO of this tile are no longer read
-        umma_commit(bar_pt_free);       // nor is P^T
-        if (it > 0) {                   // the previous dQ tile must have left tensor memory
-          if (!mbar_wait(bar_dq_empty, (it - 1) & 1, a.timeout_ns) || *abort_flag) {
+        for (int t = 0; t < itm.n; ++t, ++T) {
+          const int st = T % L::kQStages;
+          const int db = T % L::kDsBufs;
+          const bool last = (t + 1 == itm.n);
+          // the dS warps hold S^T(T) and dP^T(T) in registers: start the next tile's
+          if (!mbar_wait(bar_s_free, T & 1, a.timeout_ns) || *abort_flag) {
             ok = false;
             break;
           }
           tc_fence_after();
+          if (!last && !issue_sdp(T + 1, ks, t + 2 == itm.n)) {
+            ok = false;
+            break;
+          }
+          if (!mbar_wait(bar_p_full, T & 1, a.timeout_ns) || *abort_flag) {
+            ok = false;
+            break;
+          }
+          // the previous item's dK / dV must have left tensor memory before they restart
+          if (t == 0 && u > 0 && (!mbar_wait(bar_acc_free, (u - 1) & 1, a.timeout_ns) || *abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_acc_tmem_linear<D>(tmem + L::kTmDV, tmem + L::kTmPt, at(do_mn, st * kTile16), t == 0);
+          issue_acc<D, false>(tmem + L::kTmDK, 0u, at(ds_kmaj, db * kDs16), at(q_mn, st * kTile16), t == 0);
+          umma_commit(bar_q_empty + st);  // Q and dO of this tile are no longer read
+          umma_commit(bar_pt_free);       // nor is P^T
+          if (T > 0) {                    // the previous dQ tile must have left tensor memory
+            if (!mbar_wait(bar_dq_empty, (T - 1) & 1, a.timeout_ns) || *abort_flag) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          issue_dq<D>(tmem + L::kTmDQ, at(ds_mn, db * kDs16), at(k_mn, ks * kTile16));
+          umma_commit(bar_dq_full);
+          umma_commit(bar_ds_free + db);
+          if (last) {
+            umma_commit(bar_k_free + ks);  // this K slot may be refilled
+            umma_commit(bar_dkv_done);     // dK and dV of this item are complete
+          }
         }
-        issue_dq<D>(tmem + L::kTmDQ, at(ds_mn, db * kDs16), k_mn);
-        umma_commit(bar_dq_full);
-        umma_commit(bar_ds_free + db);
       }
-      if (!ok) bwd_timeout(a.status, abort_flag);
-      umma_commit(bar_dkv_done);
+      if (!ok) {
+        bwd_timeout(a.status, abort_flag);
+        umma_commit(bar_dkv_done);
+      }
     }
   } else if (warp < 8) {
     regs_dec<kPipeRegsDrain>();
     // ---------------------------------------------------------------- dQ drain (thread = query)
     const uint32_t quarter = warp & 3;
     const uint32_t lane_field = (quarter * 32) << 16;
-    // this warp's 4 KB turn-around buffer: row = lane, 16-byte chunk c at (c ^ (row & 7))
-    const uint32_t scratch = sbase + L::kOffStage + quarter * 4096;
     const int rr_sub = lane >> 3, cc = lane & 7;  // read side: row 4k + rr_sub, chunk cc
     bool ok = true;
-    for (int it = 0; it < n_iters && ok; ++it) {
-      const int q0 = (i_first + it) * 128 + quarter * 32;  // first query row of this warp
-      if (!warp_wait_b(bar_dq_full, it & 1, a.timeout_ns) || *abort_flag) {
+    PipeCursor cur;
+    cur.start(a, n_items);
+    for (int T = 0; cur.valid; ++T, cur.advance(a, n_items)) {
+      const int q0 = (cur.itm.i_first + cur.t) * 128 + quarter * 32;  // first query row of this warp
+      // this warp's 4 KB turn-around buffer in the drained tile's dS buffer:
+      // row = lane, 16-byte chunk c at (c ^ (row & 7))
+      const uint32_t scratch = sbase + L::kOffDS + (T % L::kDsBufs) * L::kDsBytes + quarter * 4096;
+      if (!warp_wait_b(bar_dq_full, T & 1, a.timeout_ns) || *abort_flag) {
         ok = false;
         break;
       }
@@ -803,11 +936,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
           const int row = 4 * k + rr_sub;
           const float4 v = ld_shared_f4(scratch + row * 128 + ((cc ^ (row & 7)) << 4));
           if (q0 + row < a.Nq)
-            red_add_v4(a.dq_acc + (((size_t)b * a.Nq + q0 + row) * a.H + h) * D + half * 32 + cc * 4, v.x, v.y, v.z,
-                       v.w);
+            red_add_v4(a.dq_acc + (((size_t)cur.itm.b * a.Nq + q0 + row) * a.H + cur.itm.h) * D + half * 32 + cc * 4,
+                       v.x, v.y, v.z, v.w);
         }
         __syncwarp();
       }
+      mbar_arrive_warp(bar_ds_free + (T % L::kDsBufs));  // the scratch may be overwritten
     }
     if (!ok && lane == 0) bwd_timeout(a.status, abort_flag);
   } else {
@@ -816,108 +950,105 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     const uint32_t quarter = warp & 3;
     const int grp = (warp - 8) >> 2;  // column group: queries [64 grp, 64 grp + 64) of each tile
     const int r = quarter * 32 + lane;
-    const int key = j * 128 + r;
     const uint32_t lane_field = (quarter * 32) << 16;
-    const bool key_ok = key < a.Nk;
-    const int qmin = a.causal ? key - (a.Nk - a.Nq) : -(1 << 30);
     const int col = 64 * grp;
     bool ok = true;
-    for (int it = 0; it < n_iters && ok; ++it) {
-      const int st = it % L::kQStages;
-      const int db = it % L::kDsBufs;
-      const int q0 = (i_first + it) * 128;
-      if (!warp_wait_b(bar_q_full + st, (it / L::kQStages) & 1, a.timeout_ns) ||
-          !warp_wait_b(bar_s_full, it & 1, a.timeout_ns) || *abort_flag) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t sv0[32], sv1[32], dp0[32], dp1[32];
-      tmem_ld32(tmem + lane_field + L::kTmSt + col, sv0);
-      tmem_ld32(tmem + lane_field + L::kTmSt + col + 32, sv1);
-      tmem_ld32(tmem + lane_field + L::kTmDPt + col, dp0);
-      tmem_ld32(tmem + lane_field + L::kTmDPt + col + 32, dp1);
-      tmem_ld_wait(sv0);
-      reg_pin(sv1);
-      reg_pin(dp0);
-      reg_pin(dp1);
-      tc_fence_before();
-      mbar_arrive_warp(bar_s_free);  // S^T / dP^T may be overwritten
-      const uint32_t stat_u32 = sbase + L::kOffStat + st * 1024 + col * 4;
-      const uint32_t ds_row = sbase + L::kOffDS + db * L::kDsBytes + grp * 16384 + r * 128;
-      const int qs0 = q0 + col, qs1 = q0 + col + 32;
-      const bool key_tail = j * 128 + 128 > a.Nk;
-      const int last_key_qmin = j * 128 + 127 - (a.Nk - a.Nq);
-      uint32_t pk[16], dk2[16];
-      if (key_tail || (a.causal && last_key_qmin > qs0))
-        ds_block<32, true>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk, dk2);
-      else
-        ds_block<32, false>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk, dk2);
-      // P^T may be written once the previous tile's dV has read it
-      if (it > 0 && (!warp_wait_b(bar_pt_free, (it - 1) & 1, a.timeout_ns) || *abort_flag)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      tmem_st16(tmem + lane_field + L::kTmPt + 32 * grp, pk);
-      if (!warp_wait_b(bar_ds_free + db, ((it / L::kDsBufs) & 1) ^ 1, a.timeout_ns) || *abort_flag) {
-        ok = false;
-        break;
-      }
+    int T = 0, u = 0;
+    for (int w; (w = pipe_item_index(u)) < n_items && ok; ++u) {
+      const PipeItem itm = pipe_item(a, w);
+      const int key = itm.j * 128 + r;
+      const bool key_ok = key < a.Nk;
+      const int qmin = a.causal ? key - (a.Nk - a.Nq) : -(1 << 30);
+      const bool key_tail = itm.j * 128 + 128 > a.Nk;
+      const int last_key_qmin = itm.j * 128 + 127 - (a.Nk - a.Nq);
+      for (int t = 0; t < itm.n; ++t, ++T) {
+        const int st = T % L::kQStages;
+        const int db = T % L::kDsBufs;
+        const int q0 = (itm.i_first + t) * 128;
+        if (!warp_wait_b(bar_q_full + st, (T / L::kQStages) & 1, a.timeout_ns) ||
+            !warp_wait_b(bar_s_full, T & 1, a.timeout_ns) || *abort_flag) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t sv0[32], sv1[32], dp0[32], dp1[32];
+        tmem_ld32(tmem + lane_field + L::kTmSt + col, sv0);
+        tmem_ld32(tmem + lane_field + L::kTmSt + col + 32, sv1);
+        tmem_ld32(tmem + lane_field + L::kTmDPt + col, dp0);
+        tmem_ld32(tmem + lane_field + L::kTmDPt + col + 32, dp1);
+        tmem_ld_wait(sv0);
+        reg_pin(sv1);
+        reg_pin(dp0);
+        reg_pin(dp1);
+        tc_fence_before();
+        mbar_arrive_warp(bar_s_free);  // S^T / dP^T may be overwritten
+        const uint32_t stat_u32 = sbase + L::kOffStat + st * 1024 + col * 4;
+        const uint32_t ds_row = sbase + L::kOffDS + db * L::kDsBytes + grp * 16384 + r * 128;
+        const int qs0 = q0 + col, qs1 = q0 + col + 32;
+        uint32_t pk[16], dk2[16];
+        if (key_tail || (a.causal && last_key_qmin > qs0))
+          ds_block<32, true>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk, dk2);
+        else
+          ds_block<32, false>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk, dk2);
+        // P^T may be written once the previous tile's dV has read it
+        if (T > 0 && (!warp_wait_b(bar_pt_free, (T - 1) & 1, a.timeout_ns) || *abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st16(tmem + lane_field + L::kTmPt + 32 * grp, pk);
+        if (!warp_wait_b(bar_ds_free + db, ((T / L::kDsBufs) & 1) ^ 1, a.timeout_ns) || *abort_flag) {
+          ok = false;
+          break;
+        }
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4)
-        st_shared_v4(ds_row + ((c4 ^ (r & 7)) << 4), dk2[4 * c4], dk2[4 * c4 + 1], dk2[4 * c4 + 2], dk2[4 * c4 + 3]);
-      if (key_tail || (a.causal && last_key_qmin > qs1))
-        ds_block<32, true>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk, dk2);
-      else
-        ds_block<32, false>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk, dk2);
-      tmem_st16(tmem + lane_field + L::kTmPt + 32 * grp + 16, pk);
+        for (int c4 = 0; c4 < 4; ++c4)
+          st_shared_v4(ds_row + ((c4 ^ (r & 7)) << 4), dk2[4 * c4], dk2[4 * c4 + 1], dk2[4 * c4 + 2],
+                       dk2[4 * c4 + 3]);
+        if (key_tail || (a.causal && last_key_qmin > qs1))
+          ds_block<32, true>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk, dk2);
+        else
+          ds_block<32, false>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk, dk2);
+        tmem_st16(tmem + lane_field + L::kTmPt + 32 * grp + 16, pk);
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4)
-        st_shared_v4(ds_row + (((4 + c4) ^ (r & 7)) << 4), dk2[4 * c4], dk2[4 * c4 + 1], dk2[4 * c4 + 2],
-                     dk2[4 * c4 + 3]);
-      fence_proxy_async_smem();
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive_warp(bar_p_full);
-    }
-    // ---------------------------------------------------------------- dK / dV epilogue
-    // group 0 stores dK (times scale) through the K tile's smem, group 1 dV through V's
-    if (ok && warp_wait_b(bar_dkv_done, 0, a.timeout_ns) && !*abort_flag) {
+        for (int c4 = 0; c4 < 4; ++c4)
+          st_shared_v4(ds_row + (((4 + c4) ^ (r & 7)) << 4), dk2[4 * c4], dk2[4 * c4 + 1], dk2[4 * c4 + 2],
+                       dk2[4 * c4 + 3]);
+        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive_warp(bar_p_full);
+      }
+      if (!ok) break;
+      // -------------------------------------------------------------- dK / dV of this item
+      // group 0 writes dK (times scale), group 1 dV: one key row per thread, bf16
+      if (!warp_wait_b(bar_dkv_done, u & 1, a.timeout_ns) || *abort_flag) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
+      uint32_t o0[32], o1[32];
       const uint32_t src = tmem + lane_field + (grp == 0 ? L::kTmDK : L::kTmDV);
-      const uint32_t dst = sbase + (grp == 0 ? L::kOffK : L::kOffV);
-      const float mul = grp == 0 ? a.scale : 1.f;
-#pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(src + cc * 32, o);
-        tmem_ld_wait(o);
+      tmem_ld32(src, o0);
+      tmem_ld32(src + 32, o1);
+      tmem_ld_wait(o0);
+      reg_pin(o1);
+      tc_fence_before();
+      mbar_arrive_warp(bar_acc_free);  // the next item may restart dK / dV
+      if (key_ok) {
+        const float mul = grp == 0 ? a.scale : 1.f;
+        uint4* dst = (grp == 0 ? a.dk : a.dv) + (((size_t)itm.b * a.Nk + key) * a.H + itm.h) * (D / 8);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const int chunk = cc * 4 + q4;
-          const uint32_t addr = dst + r * 128 + ((chunk ^ (r & 7)) << 4);
-          const float* f = reinterpret_cast<const float*>(o) + q4 * 8;
-          st_shared_v4(addr, pack_bf16x2(f[0] * mul, f[1] * mul), pack_bf16x2(f[2] * mul, f[3] * mul),
-                       pack_bf16x2(f[4] * mul, f[5] * mul), pack_bf16x2(f[6] * mul, f[7] * mul));
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t* f = (c < 4 ? o0 : o1) + (c & 3) * 8;
+          dst[c] = make_uint4(pack_bf16x2(__uint_as_float(f[0]) * mul, __uint_as_float(f[1]) * mul),
+                              pack_bf16x2(__uint_as_float(f[2]) * mul, __uint_as_float(f[3]) * mul),
+                              pack_bf16x2(__uint_as_float(f[4]) * mul, __uint_as_float(f[5]) * mul),
+                              pack_bf16x2(__uint_as_float(f[6]) * mul, __uint_as_float(f[7]) * mul));
         }
       }
-      fence_proxy_async_smem();
-      mbar_arrive_warp(bar_epi);
-      if (warp == 8 && lane == 0) {
-        if (mbar_wait(bar_epi, 0, a.timeout_ns)) {
-          tma_store_4d(&tmDK, smem + L::kOffK, 0, h, j * 128, b);
-          tma_store_4d(&tmDV, smem + L::kOffV, 0, h, j * 128, b);
-          bulk_commit_group();
-          bulk_wait_group0();
-        } else {
-          bwd_timeout(a.status, abort_flag);
-        }
-      }
-      __syncwarp();
-    } else if (lane == 0) {
-      bwd_timeout(a.status, abort_flag);
     }
+    if (!ok && lane == 0) bwd_timeout(a.status, abort_flag);
   }
 
   tc_fence_before();
@@ -1028,11 +1159,14 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   a.scale_log2 = L0.scale * 1.4426950408889634f;
   a.n_kv_tiles = (L0.Nk + 127) / 128;
   a.timeout_ns = L0.timeout_ns;
+  a.dk = static_cast<uint4*>(L0.dk);
+  a.dv = static_cast<uint4*>(L0.dv);
   const long long grid = (long long)a.n_kv_tiles * L0.B * L0.H;
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   prof_before(stream, kKBwdMain);
   if constexpr (D == 64) {
-    bwd_pipe_kernel<<<(unsigned)grid, kPipeThreads, PipeLayout::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
+    const int pgrid = (int)std::min<long long>(grid, (long long)num_sms());
+    bwd_pipe_kernel<<<pgrid, kPipeThreads, PipeLayout::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
   } else {
     bwd_main_kernel<D><<<(unsigned)grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
   }
