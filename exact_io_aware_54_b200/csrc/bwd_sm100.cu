@@ -551,7 +551,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 // in shared memory so that one vector reduction instruction covers four whole
 // 128-byte rows (reductions of partial rows run at half the L2 rate).
 //
-// Tensor core order per query tile i:   S^T(i+1) dP^T(i+1) | dV(i) dK(i) | dQ(i)
+// Two threads issue MMAs: one the scores S^T(i), dP^T(i) (as soon as the dS warps
+// have released tile i - 1), the other the gradient products dV(i), dK(i), dQ(i)
+// (as soon as tile i's P^T and dS are written).  The two streams use disjoint
+// tensor-memory columns and meet only through the dS warps, so neither waits
+// behind the other's back-pressured issue queue.
 // dS warps:    load S^T(i), dP^T(i) -> release -> P^T(i) to TMEM, dS(i) to smem
 // drain warps: dQ(i) TMEM -> registers -> release -> smem transpose -> red.global.add.v4
 //
@@ -587,7 +591,8 @@ struct PipeLayout {
   static_assert(kScratchBytes <= kDsBytes, "drain scratch");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
-// warps 0-3: TMA producer, MMA issuer, two idle; 4-7: dQ drain; 8-15: dS (two column groups)
+// warps 0-3: TMA producer, score MMA issuer, gradient MMA issuer, idle; 4-7: dQ drain;
+// 8-15: dS (two column groups)
 constexpr int kPipeThreads = 512;
 constexpr uint32_t kPipeRegsCtl = 72, kPipeRegsDrain = 80, kPipeRegsDs = 176;
 static_assert(128 * kPipeRegsCtl + 128 * kPipeRegsDrain + 256 * kPipeRegsDs <= kPipeThreads * 128,
@@ -812,8 +817,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         cur = nxt;
       }
       if (!ok && lane == 0) bwd_timeout(a.status, abort_flag);
-    } else if (warp == 1 && lane == 0) {
-      // -------------------------------------------------------------- MMA issuer
+    } else if ((warp == 1 || warp == 2) && lane == 0) {
       const SDesc k_kmaj = sdesc_make(sbase + L::kOffK, 16, 1024), v_kmaj = sdesc_make(sbase + L::kOffV, 16, 1024);
       const SDesc k_mn = sdesc_make(sbase + L::kOffK, 16384, 1024);
       const SDesc q_kmaj = sdesc_make(sbase + L::kOffQ, 16, 1024), do_kmaj = sdesc_make(sbase + L::kOffDO, 16, 1024);
@@ -821,81 +825,76 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       const SDesc ds_kmaj = sdesc_make(sbase + L::kOffDS, 16, 1024), ds_mn = sdesc_make(sbase + L::kOffDS, 16384, 1024);
       constexpr uint32_t kTile16 = L::kTileBytes / 16, kDs16 = L::kDsBytes / 16;
       auto at = [](SDesc d, uint32_t off16) { return SDesc{d.lo + off16, d.hi}; };
-      // S^T and dP^T of global query tile T with K in slot ks; the item's last
-      // dP^T releases V
-      auto issue_sdp = [&](int T, int ks, bool last_of_item) -> bool {
-        const int st = T % L::kQStages;
-        if (!mbar_wait(bar_q_full + st, (T / L::kQStages) & 1, a.timeout_ns) || *abort_flag) return false;
-        tc_fence_after();
-        issue_scores<D, false>(tmem + L::kTmSt, 0u, at(k_kmaj, ks * kTile16), at(q_kmaj, st * kTile16));
-        issue_scores<D, false>(tmem + L::kTmDPt, 0u, v_kmaj, at(do_kmaj, st * kTile16));
-        umma_commit(bar_s_full);
-        if (last_of_item) umma_commit(bar_v_free);
-        return true;
-      };
       bool ok = true;
       int T = 0, u = 0;
-      for (int w; (w = pipe_item_index(u)) < n_items && ok; ++u) {
-        const PipeItem itm = pipe_item(a, w);
-        const int ks = u & 1;
-        // this item's K and V; its first scores
-        if (!mbar_wait(bar_k_full + ks, (u >> 1) & 1, a.timeout_ns) || !mbar_wait(bar_v_full, u & 1, a.timeout_ns) ||
-            *abort_flag) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (!issue_sdp(T, ks, itm.n == 1)) {
-          ok = false;
-          break;
-        }
-        for (int t = 0; t < itm.n; ++t, ++T) {
-          const int st = T % L::kQStages;
-          const int db = T % L::kDsBufs;
-          const bool last = (t + 1 == itm.n);
-          // the dS warps hold S^T(T) and dP^T(T) in registers: start the next tile's
-          if (!mbar_wait(bar_s_free, T & 1, a.timeout_ns) || *abort_flag) {
+      if (warp == 1) {
+        // ------------------------------------------------------------ score MMAs
+        for (int w; (w = pipe_item_index(u)) < n_items && ok; ++u) {
+          const PipeItem itm = pipe_item(a, w);
+          const int ks = u & 1;
+          if (!mbar_wait(bar_k_full + ks, (u >> 1) & 1, a.timeout_ns) || !mbar_wait(bar_v_full, u & 1, a.timeout_ns) ||
+              *abort_flag) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          if (!last && !issue_sdp(T + 1, ks, t + 2 == itm.n)) {
-            ok = false;
-            break;
-          }
-          if (!mbar_wait(bar_p_full, T & 1, a.timeout_ns) || *abort_flag) {
-            ok = false;
-            break;
-          }
-          // the previous item's dK / dV must have left tensor memory before they restart
-          if (t == 0 && u > 0 && (!mbar_wait(bar_acc_free, (u - 1) & 1, a.timeout_ns) || *abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_acc_tmem_linear<D>(tmem + L::kTmDV, tmem + L::kTmPt, at(do_mn, st * kTile16), t == 0);
-          issue_acc<D, false>(tmem + L::kTmDK, 0u, at(ds_kmaj, db * kDs16), at(q_mn, st * kTile16), t == 0);
-          umma_commit(bar_q_empty + st);  // Q and dO of this tile are no longer read
-          umma_commit(bar_pt_free);       // nor is P^T
-          if (T > 0) {                    // the previous dQ tile must have left tensor memory
-            if (!mbar_wait(bar_dq_empty, (T - 1) & 1, a.timeout_ns) || *abort_flag) {
+          for (int t = 0; t < itm.n; ++t, ++T) {
+            const int st = T % L::kQStages;
+            // this tile's Q and dO; S^T / dP^T free again (the dS warps hold tile T - 1)
+            if (!mbar_wait(bar_q_full + st, (T / L::kQStages) & 1, a.timeout_ns) ||
+                (T > 0 && !mbar_wait(bar_s_free, (T - 1) & 1, a.timeout_ns)) || *abort_flag) {
               ok = false;
               break;
             }
             tc_fence_after();
-          }
-          issue_dq<D>(tmem + L::kTmDQ, at(ds_mn, db * kDs16), at(k_mn, ks * kTile16));
-          umma_commit(bar_dq_full);
-          umma_commit(bar_ds_free + db);
-          if (last) {
-            umma_commit(bar_k_free + ks);  // this K slot may be refilled
-            umma_commit(bar_dkv_done);     // dK and dV of this item are complete
+            issue_scores<D, false>(tmem + L::kTmSt, 0u, at(k_kmaj, ks * kTile16), at(q_kmaj, st * kTile16));
+            issue_scores<D, false>(tmem + L::kTmDPt, 0u, v_kmaj, at(do_kmaj, st * kTile16));
+            umma_commit(bar_s_full);
+            if (t + 1 == itm.n) umma_commit(bar_v_free);  // the item's last dP^T has been issued
           }
         }
-      }
-      if (!ok) {
-        bwd_timeout(a.status, abort_flag);
-        umma_commit(bar_dkv_done);
+        if (!ok) bwd_timeout(a.status, abort_flag);
+      } else {
+        // ------------------------------------------------------------ gradient MMAs
+        for (int w; (w = pipe_item_index(u)) < n_items && ok; ++u) {
+          const PipeItem itm = pipe_item(a, w);
+          const int ks = u & 1;
+          for (int t = 0; t < itm.n; ++t, ++T) {
+            const int st = T % L::kQStages;
+            const int db = T % L::kDsBufs;
+            if (!mbar_wait(bar_p_full, T & 1, a.timeout_ns) || *abort_flag) {
+              ok = false;
+              break;
+            }
+            // the previous item's dK / dV must have left tensor memory before they restart
+            if (t == 0 && u > 0 && (!mbar_wait(bar_acc_free, (u - 1) & 1, a.timeout_ns) || *abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_acc_tmem_linear<D>(tmem + L::kTmDV, tmem + L::kTmPt, at(do_mn, st * kTile16), t == 0);
+            issue_acc<D, false>(tmem + L::kTmDK, 0u, at(ds_kmaj, db * kDs16), at(q_mn, st * kTile16), t == 0);
+            umma_commit(bar_q_empty + st);  // Q and dO of this tile are no longer read
+            umma_commit(bar_pt_free);       // nor is P^T
+            if (T > 0) {                    // the previous dQ tile must have left tensor memory
+              if (!mbar_wait(bar_dq_empty, (T - 1) & 1, a.timeout_ns) || *abort_flag) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+            }
+            issue_dq<D>(tmem + L::kTmDQ, at(ds_mn, db * kDs16), at(k_mn, ks * kTile16));
+            umma_commit(bar_dq_full);
+            umma_commit(bar_ds_free + db);
+            if (t + 1 == itm.n) {
+              umma_commit(bar_k_free + ks);  // this K slot may be refilled
+              umma_commit(bar_dkv_done);     // dK and dV of this item are complete
+            }
+          }
+        }
+        if (!ok) {
+          bwd_timeout(a.status, abort_flag);
+          umma_commit(bar_dkv_done);
+        }
       }
     }
   } else if (warp < 8) {
