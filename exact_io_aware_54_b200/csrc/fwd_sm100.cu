@@ -19,11 +19,16 @@
 //                  its registers to the softmax warpgroups).
 //      warps 4-7   softmax group for query tile 0, warps 8-11 for tile 1; thread
 //                  = query row = TMEM lane.
-//  * Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
-//    O1 [384,384+d).  P (bf16) is written over the first 64 columns of its S
-//    tile and fed to the P.V MMA directly from tensor memory.
-//  * The two query tiles ping-pong: while one softmax group works on its scores
-//    the tensor core runs the other tile's MMAs.
+//  * Tensor memory (512 columns), d = 128: S0 [0,128), S1 [128,256), O0 [256,384),
+//    O1 [384,512); P (bf16) is written over the first 64 columns of its S tile
+//    and fed to the P.V MMA directly from tensor memory.  The two query tiles
+//    ping-pong: while one softmax group works on its scores the tensor core runs
+//    the other tile's MMAs.
+//  * d = 64 has room for separate P columns: S0, S1 [0,256), P0 [256,320),
+//    P1 [320,384), O0 [384,448), O1 [448,512).  A softmax group copies its S tile
+//    into registers and releases it at once, so the next Q K^T of the same query
+//    tile runs while the group works; one thread issues the Q K^T MMAs (warp 1)
+//    and another the P V MMAs (warp 2), each as soon as its operands are ready.
 //  * Online softmax in the log2 domain (x = s * scale * log2 e).  The running
 //    max is only moved when a tile raises it by more than 8 (a factor 256), so
 //    the O rescale (a TMEM round trip) is rare; the result is unchanged because
@@ -54,7 +59,19 @@ static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * 168, "register split exc
 constexpr uint32_t kTmemCols = 512;
 // tensor-memory column of the score tile / O accumulator of query tile t
 __host__ __device__ constexpr uint32_t tm_s(int t) { return t * 128u; }
-__host__ __device__ constexpr uint32_t tm_o(int t) { return 256u + t * 128u; }
+// separate P columns (d = 64): S is released as soon as the softmax has read it
+template <int D>
+__host__ __device__ constexpr bool sep_p() {
+  return D == 64;
+}
+template <int D>
+__host__ __device__ constexpr uint32_t tm_p(int t) {
+  return sep_p<D>() ? 256u + 64u * t : tm_s(t);
+}
+template <int D>
+__host__ __device__ constexpr uint32_t tm_o(int t) {
+  return sep_p<D>() ? 384u + 64u * t : 256u + t * 128u;
+}
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
@@ -66,8 +83,9 @@ struct FwdLayout {
   static constexpr int kOffQ = 0;                  // Q tile 0, Q tile 1
   static constexpr int kOffRing = 2 * kTileBytes;
   static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
-  // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], epi[2]
-  static constexpr int kNumBars = 2 + 2 * kStages + 8;
+  // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], epi[2],
+  // s_free[2], p_free[2]
+  static constexpr int kNumBars = 2 + 2 * kStages + 12;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
 };
@@ -154,6 +172,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_p_full = bar_s_full + 2;
   uint64_t* bar_o_done = bar_s_full + 4;
   uint64_t* bar_epi = bar_s_full + 6;
+  uint64_t* bar_s_free = bar_s_full + 8;  // separate P: the softmax group has read S
+  uint64_t* bar_p_free = bar_s_full + 10;  // separate P: the P V MMA has read P
+  constexpr bool kSepP = sep_p<D>();
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);
 
@@ -173,6 +194,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_p_full + t, 4);  // one arrival per softmax warp
       mbar_init(bar_o_done + t, 1);
       mbar_init(bar_epi + t, 4);
+      mbar_init(bar_s_free + t, 4);  // one arrival per softmax warp
+      mbar_init(bar_p_free + t, 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -228,6 +251,84 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_4d(dst + bx * L::kBoxBytes, kv == 0 ? &tmK : &tmV, bar_kv_full + slot, bx * 64, h, j * 128,
                           b);
           }
+        }
+      }
+    }
+  } else if (kSepP && (warp == 1 || warp == 2)) {
+    // ------------------------------------------------------------------ MMA issuers (separate P)
+    if (lane == 0) {
+      const SDesc q_desc[2] = {sdesc_make(smem_base + L::kOffQ, 16, 1024),
+                               sdesc_make(smem_base + L::kOffQ + L::kTileBytes, 16, 1024)};
+      const SDesc ring_k = sdesc_make(smem_base + L::kOffRing, 16, 1024);     // K tiles, K-major
+      const SDesc ring_v = sdesc_make(smem_base + L::kOffRing, 16384, 1024);  // V tiles, MN-major
+      constexpr uint32_t kSlot16 = L::kTileBytes / 16;
+      bool ok = true;
+      auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) {
+        if (!ok) return false;
+        if (!mbar_wait(bar, parity, a.timeout_ns) || *abort_flag) {
+          record_timeout(a.status, abort_flag);
+          ok = false;
+        }
+        return ok;
+      };
+      // ring slots alternate K, V per KV step: K of step j at g, V at g + 1
+      uint32_t item_iter = 0, g = 0;
+      uint32_t cnt[2] = {0, 0};  // Q K^T (warp 1) or P V (warp 2) MMAs issued per query tile
+      for (int w = blockIdx.x; w < a.n_items && ok; w += gridDim.x, ++item_iter) {
+        int b, h, pair;
+        item_coords(a, w, b, h, pair);
+        const int row0 = pair * 256;
+        const int nt[2] = {tile_kv_count(a, row0), tile_kv_count(a, row0 + 128)};
+        const int nkv = max(nt[0], nt[1]);
+        if (warp == 1) {
+          // S_t = Q_t K_j^T once the group has read its previous S tile
+          if (!wait_or_abort(bar_q_full, item_iter & 1)) break;
+          tc_fence_after();
+          for (int j = 0; j < nkv && ok; ++j, g += 2) {
+            const uint32_t slot_k = g % L::kStages;
+            if (!wait_or_abort(bar_kv_full + slot_k, (g / L::kStages) & 1)) break;
+            tc_fence_after();
+            const SDesc k_desc = SDesc{ring_k.lo + slot_k * kSlot16, ring_k.hi};
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (j < nt[t]) {
+                if (cnt[t] > 0 && !wait_or_abort(bar_s_free + t, (cnt[t] - 1) & 1)) break;
+                tc_fence_after();
+                issue_qk<D>(tmem_base + tm_s(t), q_desc[t], k_desc);
+                umma_commit(bar_s_full + t);
+                ++cnt[t];
+              }
+            }
+            if (!ok) break;
+            umma_commit(bar_kv_empty + slot_k);
+          }
+        } else {
+          // O_t += P_t V_j once the group has written P.  The epilogue stages O
+          // through the Q tiles: o_done must also follow this item's Q load (it
+          // decides alone when a tile sees no key at all).
+          if (!wait_or_abort(bar_q_full, item_iter & 1)) break;
+          for (int j = 0; j < nkv && ok; ++j, g += 2) {
+            const uint32_t slot_v = (g + 1) % L::kStages;
+            if (!wait_or_abort(bar_kv_full + slot_v, ((g + 1) / L::kStages) & 1)) break;
+            tc_fence_after();
+            const SDesc v_desc = SDesc{ring_v.lo + slot_v * kSlot16, ring_v.hi};
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (j < nt[t]) {
+                if (!wait_or_abort(bar_p_full + t, cnt[t] & 1)) break;
+                tc_fence_after();
+                issue_pv<D>(tmem_base + tm_o<D>(t), tmem_base + tm_p<D>(t), v_desc, j > 0);
+                umma_commit(bar_p_free + t);
+                ++cnt[t];
+              }
+            }
+            if (!ok) break;
+            umma_commit(bar_kv_empty + slot_v);
+          }
+          if (!ok) break;
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+            if (nt[t] >= 0) umma_commit(bar_o_done + t);
         }
       }
     }
@@ -289,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (!wait_or_abort(bar_p_full + t, p_cnt[t] & 1)) break;
               tc_fence_after();
               ++p_cnt[t];
-              issue_pv<D>(tmem_base + tm_o(t), tmem_base + tm_s(t), v_desc, j > 0);
+              issue_pv<D>(tmem_base + tm_o<D>(t), tmem_base + tm_s(t), v_desc, j > 0);
             }
             if (t == 0 && more) {
               slot_k = g % L::kStages;
@@ -324,7 +425,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;           // row within the tile
     const uint32_t lane_field = (quarter * 32) << 16;
     const uint32_t tS = tmem_base + lane_field + tm_s(t);
-    const uint32_t tO = tmem_base + lane_field + tm_o(t);
+    const uint32_t tO = tmem_base + lane_field + tm_o<D>(t);
+    const uint32_t tP = tmem_base + lane_field + tm_p<D>(t);
     const int tid_in_group = threadIdx.x - 128 - t * 128;
     uint32_t s_cnt = 0, tile_iter = 0;  // tile_iter counts items in which this tile is present
     uint8_t* q_tile = smem + L::kOffQ + t * L::kTileBytes;
@@ -365,6 +467,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         reg_pin(s[1]);
         reg_pin(s[2]);
         reg_pin(s[3]);
+        if constexpr (kSepP) {  // the next Q K^T of this tile may overwrite S
+          tc_fence_before();
+          mbar_arrive_warp(bar_s_free + t);
+        }
 
         // mask (only tiles that cross the diagonal or the key tail)
         const int kbase = j * 128;
@@ -392,9 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_ref, -m_ref);
         float2 ex0 = make_float2(0.f, 0.f), ex1 = make_float2(0.f, 0.f);  // unrounded sums
         float2 rd0 = make_float2(0.f, 0.f), rd1 = make_float2(0.f, 0.f);  // sums of the bf16 values
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t pk[32];
+        // probabilities of score half hf (64 columns) packed into pk
+        auto exp_half = [&](int hf, uint32_t(&pk)[32]) {
 #pragma unroll
           for (int ii = 0; ii < 2; ++ii) {
 #pragma unroll
@@ -413,14 +518,38 @@ __global__ void __launch_bounds__(kThreads, 1)
               rd1 = fadd2(rd1, make_float2(__uint_as_float(k1 << 16), __uint_as_float(k1 & 0xFFFF0000u)));
             }
           }
-          tmem_st32(tS + hf * 32, pk);
+        };
+        // separate P: both halves wait in registers for the P columns
+        uint32_t pkk[kSepP ? 2 : 1][32];
+        if constexpr (kSepP) {
+          exp_half(0, pkk[0]);
+          exp_half(1, pkk[1]);
+        } else {
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            uint32_t pk[32];
+            exp_half(hf, pk);
+            tmem_st32(tS + hf * 32, pk);
+          }
+        }
+        if constexpr (kSepP) {
+          // the previous P V of this tile has read the P columns (and updated O)
+          if (s_cnt > 0 && !warp_wait(bar_p_free + t, (s_cnt - 1) & 1, a.timeout_ns)) {
+            if (lane == 0) record_timeout(a.status, abort_flag);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          tmem_st32(tP, pkk[0]);
+          tmem_st32(tP + 32, pkk[1]);
         }
         l = l * alpha + ((rd0.x + rd0.y) + (rd1.x + rd1.y));
         le = le * alpha + ((ex0.x + ex0.y) + (ex1.x + ex1.y));
         m2 = m_use;
         // rescale the O accumulator when some row of this warp moved its reference.
-        // The previous P.V of this tile has completed: the scores just read were
-        // issued after it and tcgen05 operations complete in order.
+        // The previous P.V of this tile has completed: with P over S, the scores just
+        // read were issued after it and tcgen05 operations complete in order; with
+        // separate P the wait for the P columns above covered it.
         if (j > 0 && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
