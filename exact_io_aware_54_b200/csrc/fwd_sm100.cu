@@ -73,6 +73,14 @@ __host__ __device__ constexpr uint32_t tm_o(int t) {
   return sep_p<D>() ? 384u + 64u * t : 256u + t * 128u;
 }
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Every kExpFmaEvery-th group of four probabilities computes one pair of its
+// exponentials on the FMA pipes (exp2_fma2) instead of the MUFU unit: a quarter
+// of them at d = 64, an eighth at d = 128 (where the tile has twice the MMA work
+// per exponential).  Measured on B200 against other splits.
+template <int D>
+__host__ __device__ constexpr int exp_fma_every() {
+  return D == 64 ? 2 : 4;
+}
 
 template <int D>
 struct FwdLayout {
@@ -508,7 +516,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float2 x0 = ffma2(make_float2(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2);
               const float2 x1 = ffma2(make_float2(__uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3])), sc2, nm2);
               const float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
-              const float2 p1 = make_float2(ex2(x1.x), ex2(x1.y));
+              // one pair in kExpFmaEvery * 2 goes to the FMA pipes: the MUFU unit
+              // alone (16 per cycle per SM) would bound the tile
+              constexpr int kEvery = exp_fma_every<D>();
+              const float2 p1 =
+                  (((c >> 2) % kEvery) == kEvery - 1) ? exp2_fma2(x1) : make_float2(ex2(x1.x), ex2(x1.y));
               const uint32_t k0 = pack_bf16x2(p0.x, p0.y), k1 = pack_bf16x2(p1.x, p1.y);
               pk[ii * 16 + (c >> 1)] = k0;
               pk[ii * 16 + (c >> 1) + 1] = k1;

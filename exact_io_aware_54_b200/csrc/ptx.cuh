@@ -404,6 +404,40 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   return d;
 }
 
+// 2^x for two values on the FMA and integer pipes, leaving the MUFU unit free
+// (Cody and Waite range reduction, "Software Manual for the Elementary Functions",
+// 1980, with a polynomial fitted here):
+//   x is clamped to >= -127, so results below 2^-126.5 become +0 (as with
+//   ex2.approx.ftz, and exactly 0 for x = -inf);
+//   n = rint(x) is read off the fp32 rounding of x + 1.5 * 2^23 (exact for |x| < 2^22);
+//   f = x - n lies in [-1/2, 1/2] and 2^f = c0 + f (c1 + f (c2 + f (c3 + f c4))),
+//   coefficients fitted for the smallest maximum relative error on that interval
+//   (2.7e-6 in fp32 arithmetic; the unit test re-derives the bound from these
+//   constants);
+//   2^n is assembled in an exponent field: the bit pattern of x + 1.5 * 2^23 shifted
+//   left by 23 is n << 23, and adding the pattern of 1.0f gives (n + 127) << 23,
+//   which is +0 for n = -127.
+constexpr float kExp2C0 = 0.9999992847442627f;
+constexpr float kExp2C1 = 0.6931217908859253f;
+constexpr float kExp2C2 = 0.24024732410907745f;
+constexpr float kExp2C3 = 0.055917903780937195f;
+constexpr float kExp2C4 = 0.009570610709488392f;
+constexpr float kExp2Round = 12582912.0f;  // 1.5 * 2^23
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -127.f);
+  x.y = fmaxf(x.y, -127.f);
+  const float2 t = fadd2(x, make_float2(kExp2Round, kExp2Round));
+  const float2 n = fadd2(t, make_float2(-kExp2Round, -kExp2Round));
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);
+  float2 p = ffma2(make_float2(kExp2C4, kExp2C4), f, make_float2(kExp2C3, kExp2C3));
+  p = ffma2(p, f, make_float2(kExp2C2, kExp2C2));
+  p = ffma2(p, f, make_float2(kExp2C1, kExp2C1));
+  p = ffma2(p, f, make_float2(kExp2C0, kExp2C0));
+  const float2 two_n = make_float2(__uint_as_float((__float_as_uint(t.x) << 23) + 0x3f800000u),
+                                   __uint_as_float((__float_as_uint(t.y) << 23) + 0x3f800000u));
+  return fmul2(p, two_n);
+}
+
 // Three-input maximum (sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
