@@ -299,7 +299,7 @@ def _rotating(make, total_bytes_of_one):
     return [make(i) for i in range(n)]
 
 
-EXTRA_WORKLOADS = ("prefill8k", "decode_single", "decode_batched", "long16k")
+EXTRA_WORKLOADS = ("prefill8k", "decode_single", "decode_batched", "decode_paged", "long16k")
 
 
 def run_extra(args, fa, synth, dev, pk, only=None):
@@ -312,6 +312,8 @@ def run_extra(args, fa, synth, dev, pk, only=None):
         _extra_decode_single(out, iters, fa, synth, dev, pk)
     if want("decode_batched"):
         _extra_decode_batched(out, iters, fa, synth, dev, pk)
+    if want("decode_paged"):
+        _extra_decode_paged(out, iters, fa, synth, dev, pk)
     if want("long16k"):
         _extra_long16k(out, iters, fa, synth, dev, pk)
     return out
@@ -381,6 +383,30 @@ def _extra_decode_batched(out, iters, fa, synth, dev, pk):
                                     "splits": fa.fa_decode_num_splits(64, 32, maxL, 128, 0),
                                     "l2": "no flush: KV cache is 70x the L2"}
     del q, k, v, cu, o, lse
+    torch.cuda.empty_cache()
+
+
+def _extra_decode_paged(out, iters, fa, synth, dev, pk):
+    # the same 64 ragged sequences in a paged cache: pages of 64 keys in seeded random order
+    lengths = synth.ragged_lengths(synth.SEEDS["decode"], 64, 512, 16384)
+    q, kp, vp, table, lens = synth.paged_decode_inputs(synth.SEEDS["decode"], lengths, 32, 128, 64, device=dev)
+    table, lens = table.to(dev), lens.to(dev)
+    maxL = int(lengths.max())
+    o = torch.empty_like(q)
+    lse = torch.empty(64, 32, dtype=torch.float32, device=dev)
+
+    def g3(i):
+        fa.fa_decode_paged(q, kp, vp, table, lens, maxL, out=o, lse=lse)
+    for i in range(3):
+        g3(i)
+    ms = device_time_ms(g3, iters)
+    kv_bytes = 2 * 2 * 32 * 128 * int(lengths.sum())
+    gbs = kv_bytes / (ms * 1e-3) / 1e9
+    out["decode_paged_batched"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
+                                   "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4), "kv_bytes": kv_bytes,
+                                   "page_size": 64, "num_pages": int(kp.shape[0]),
+                                   "l2": "no flush: KV cache is 70x the L2"}
+    del q, kp, vp, table, lens, o, lse
     torch.cuda.empty_cache()
 
 

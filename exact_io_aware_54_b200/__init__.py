@@ -68,7 +68,9 @@ def load():
         lib.fa_bwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _vp, _sz, _vp]
         lib.fa_decode_splitkv.argtypes = [_vp] * 4 + [_i] * 6 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
         lib.fa_decode_splitkv_noalloc.argtypes = [_vp] * 4 + [_i] * 6 + [_f, _i, _vp, _vp, _vp]
-        for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_decode_splitkv, lib.fa_decode_splitkv_noalloc):
+        lib.fa_decode_paged.argtypes = [_vp] * 5 + [_i] * 7 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
+        for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_decode_splitkv, lib.fa_decode_splitkv_noalloc,
+                   lib.fa_decode_paged):
             fn.restype = _i
         lib.fa_fwd_workspace_size.argtypes = [_i] * 5
         lib.fa_fwd_workspace_size.restype = _sz
@@ -240,6 +242,36 @@ def fa_decode_splitkv_noalloc(q, k, v, cu_seqlens_k, max_seqlen_k: int, causal: 
                                        int(max_seqlen_k), d, int(bool(causal)), _scale(softmax_scale),
                                        int(num_splits), out.data_ptr(), lse.data_ptr(), _stream_ptr(q.device))
     _raise("fa_decode_splitkv_noalloc", st)
+    return out, lse
+
+
+def fa_decode_paged(q, k_pages, v_pages, block_table, seqlens_k, max_seqlen_k: int, softmax_scale=None,
+                    num_splits: int = 0, out=None, lse=None, ws=None):
+    """Split-KV decode over a paged cache.  q [B, H, d]; k_pages/v_pages
+    [num_pages, page_size, H, d] bf16; block_table int32 [B, max_pages_per_seq] and
+    seqlens_k int32 [B] on the device.  Returns (o [B, H, d] bf16, lse [B, H] fp32)."""
+    lib = load()
+    B, H, d = q.shape
+    _check_tensor("q", q, torch.bfloat16)
+    _check_tensor("k_pages", k_pages, torch.bfloat16)
+    _check_tensor("v_pages", v_pages, torch.bfloat16, k_pages.shape)
+    if k_pages.dim() != 4 or k_pages.shape[2] != H or k_pages.shape[3] != d:
+        raise ValueError("k_pages/v_pages must be [num_pages, page_size, H, d]")
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be [B, max_pages_per_seq]")
+    _check_tensor("block_table", block_table, torch.int32, tuple(block_table.shape))
+    _check_tensor("seqlens_k", seqlens_k, torch.int32, (B,))
+    num_pages, page_size = int(k_pages.shape[0]), int(k_pages.shape[1])
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    need = lib.fa_decode_workspace_size(B, H, int(max_seqlen_k), d, int(num_splits))
+    if ws is None:
+        ws = workspace(need, q.device, "decode")
+    st = lib.fa_decode_paged(q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), block_table.data_ptr(),
+                             seqlens_k.data_ptr(), B, H, num_pages, page_size, int(block_table.shape[1]),
+                             int(max_seqlen_k), d, _scale(softmax_scale), int(num_splits), out.data_ptr(),
+                             lse.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
+    _raise("fa_decode_paged", st)
     return out, lse
 
 

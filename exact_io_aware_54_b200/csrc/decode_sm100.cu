@@ -25,6 +25,10 @@
 //    atomic ticket -- merges the chunk states and writes o and lse, then resets
 //    the ticket, so tickets are zero between calls.  A sequence with a single chunk skips the
 //    partial-state round trip.
+//  * Paged caches (K and V in pages of page_size keys, a block table per
+//    sequence) only change where the producer reads a key's row from; every page
+//    index is checked against the number of pages (a bad one is recorded in the
+//    status word and read as page 0, so no copy leaves the cache).
 #include "fa_internal.h"
 #include "ptx.cuh"
 
@@ -52,6 +56,9 @@ struct DecArgs {
   const __nv_bfloat16* k;
   const __nv_bfloat16* v;
   const int32_t* cu;
+  const int32_t* block_table;  // paged cache when not null
+  const int32_t* seqlens;
+  int page_size, max_pages, num_pages;
   __nv_bfloat16* o;
   float* lse;
   int* status;
@@ -91,8 +98,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
   const int nh = min(kHeadsPerCta, a.H - h0);
   if (a.check_args && *reinterpret_cast<volatile int*>(a.status) == kStatusBadArg) return;
 
-  const int start = a.cu[b];
-  int len = a.cu[b + 1] - start;
+  const bool paged = a.block_table != nullptr;
+  const int start = paged ? 0 : a.cu[b];
+  int len = paged ? a.seqlens[b] : a.cu[b + 1] - start;
   len = max(0, min(len, a.max_seqlen_k));
   const int nsplit = (len + a.chunk - 1) / a.chunk;
   const uint32_t warp = warp_id(), lane = lane_id();
@@ -151,7 +159,16 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
         const int is_v = lane >= kKeysPerStage;
         const int key = key0 + t;
         if (key < kend) {
-          const __nv_bfloat16* src = (is_v ? a.v : a.k) + ((size_t)start + key) * row_elems + (size_t)h0 * D;
+          size_t row = (size_t)start + key;
+          if (paged) {
+            int page = a.block_table[(size_t)b * a.max_pages + key / a.page_size];
+            if (page < 0 || page >= a.num_pages) {  // never read outside the cache
+              atomicExch(a.status, kStatusBadArg);
+              page = 0;
+            }
+            row = (size_t)page * a.page_size + key % a.page_size;
+          }
+          const __nv_bfloat16* src = (is_v ? a.v : a.k) + row * row_elems + (size_t)h0 * D;
           uint8_t* dst = smem + slot * L::kStageBytes + is_v * kKeysPerStage * L::kRowStride + t * L::kRowStride;
           bulk_load(dst, src, copy_bytes, full + slot);
         }
@@ -426,6 +443,11 @@ static fa_status launch_decode_impl(const DecodeLaunch& L0, cudaStream_t stream)
   a.k = static_cast<const __nv_bfloat16*>(L0.k);
   a.v = static_cast<const __nv_bfloat16*>(L0.v);
   a.cu = L0.cu_seqlens;
+  a.block_table = L0.block_table;
+  a.seqlens = L0.seqlens;
+  a.page_size = L0.page_size;
+  a.max_pages = L0.max_pages;
+  a.num_pages = L0.num_pages;
   a.o = static_cast<__nv_bfloat16*>(L0.o);
   a.lse = L0.lse;
   a.status = L0.status;
@@ -445,7 +467,7 @@ static fa_status launch_decode_impl(const DecodeLaunch& L0, cudaStream_t stream)
     if (cudaMemsetAsync(L0.tickets, 0, sizeof(unsigned) * (size_t)L0.B * L0.H, stream) != cudaSuccess)
       return FA_ERR_CUDA;
   }
-  if (L0.check_args) {
+  if (L0.check_args && !L0.block_table) {
     prof_before(stream, kKDecodeCheck);
     check_cu_seqlens_kernel<<<(L0.B + 256) / 256, 256, 0, stream>>>(L0.cu_seqlens, L0.B, L0.max_seqlen_k,
                                                                       L0.status);

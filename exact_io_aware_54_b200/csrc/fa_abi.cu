@@ -304,6 +304,62 @@ fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, const i
   return launch_decode(a, stream);
 }
 
+fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                          const int32_t* seqlens_k, int B, int H, int num_pages, int page_size, int max_pages_per_seq,
+                          int max_seqlen_k, int d, float softmax_scale, int num_splits, void* o, float* lse,
+                          void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!q || !k_pages || !v_pages || !block_table || !seqlens_k || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || num_pages <= 0 || page_size <= 0 || max_pages_per_seq <= 0 || max_seqlen_k < 0 ||
+      num_splits < 0)
+    return FA_ERR_INVALID_ARG;
+  if ((long long)B * H >= (1LL << 31) || (long long)B * max_pages_per_seq >= (1LL << 31)) return FA_ERR_INVALID_ARG;
+  // every key a sequence may hold must have a block-table entry
+  if ((long long)max_seqlen_k > (long long)max_pages_per_seq * page_size) return FA_ERR_INVALID_ARG;
+  if ((long long)num_pages * page_size * H * (long long)d >= (1LL << 62)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seqlens_k) & 3u))
+    return FA_ERR_ALIGNMENT;
+  const DecodePlan plan = decode_plan(B, H, max_seqlen_k, d, num_splits);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < decode_workspace_bytes(B, H, d, plan))
+    return FA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  DecodeLaunch a;
+  a.q = q;
+  a.k = k_pages;
+  a.v = v_pages;
+  a.cu_seqlens = nullptr;
+  a.block_table = block_table;
+  a.seqlens = seqlens_k;
+  a.page_size = page_size;
+  a.max_pages = max_pages_per_seq;
+  a.num_pages = num_pages;
+  a.o = o;
+  a.lse = lse;
+  a.status = reinterpret_cast<int*>(ws);
+  size_t off = kStatusBytes;
+  a.tickets = reinterpret_cast<unsigned*>(ws + off);
+  a.clear_tickets = 0;
+  off += kDecodeTicketBytes;
+  a.part_ml = reinterpret_cast<float*>(ws + off);
+  off += up256(sizeof(float) * 2 * (size_t)B * H * plan.splits);
+  a.part_u = reinterpret_cast<float*>(ws + off);
+  off += up256(sizeof(float) * (size_t)d * B * H * plan.splits);
+  if ((size_t)B * H > kDecodeFixedTickets) {
+    a.tickets = reinterpret_cast<unsigned*>(ws + off);
+    a.clear_tickets = 1;
+  }
+  a.B = B;
+  a.H = H;
+  a.max_seqlen_k = max_seqlen_k;
+  a.d = d;
+  a.scale = resolve_scale(softmax_scale, d);
+  a.plan = plan;
+  a.check_args = 0;
+  a.timeout_ns = wait_timeout_ns();
+  return launch_decode(a, stream);
+}
+
 fa_status fa_profile_start(void) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
   g_records.clear();

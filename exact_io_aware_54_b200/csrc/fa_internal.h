@@ -88,7 +88,12 @@ struct DecodeLaunch {
   const void* q;
   const void* k;
   const void* v;
-  const int32_t* cu_seqlens;
+  const int32_t* cu_seqlens;  // packed cache: [B + 1] row offsets (nullptr when paged)
+  // paged cache (block_table != nullptr): k, v are [num_pages, page_size, H, d];
+  // key t of sequence b is row t % page_size of page block_table[b * max_pages + t / page_size]
+  const int32_t* block_table = nullptr;
+  const int32_t* seqlens = nullptr;  // [B] keys per sequence
+  int page_size = 0, max_pages = 0, num_pages = 0;
   void* o;
   float* lse;
   int* status;

@@ -64,3 +64,30 @@ def decode_inputs(seed: int, lengths, H: int, d: int, device="cpu"):
     k = _normal((total, H, d), seed + 1, device)
     v = _normal((total, H, d), seed + 2, device)
     return q, k, v, cu
+
+
+def paged_decode_inputs(seed: int, lengths, H: int, d: int, page_size: int, spare_pages: int = 3, device="cpu"):
+    """A paged KV cache holding the given sequence lengths.
+
+    Returns q [B, H, d], k_pages, v_pages [num_pages, page_size, H, d] (bf16), the
+    block table [B, max_pages] and seqlens [B] (int32, CPU).  Pages are handed out
+    in a seeded random order (so a sequence's pages are scattered through the
+    cache), `spare_pages` pages belong to no sequence, and unused block-table
+    entries hold -1.
+    """
+    lengths = torch.as_tensor(lengths, dtype=torch.int64)
+    B = len(lengths)
+    pages_per_seq = [(int(L) + page_size - 1) // page_size for L in lengths]
+    max_pages = max(1, max(pages_per_seq))
+    num_pages = sum(pages_per_seq) + spare_pages
+    g = torch.Generator().manual_seed(seed + 3)
+    order = torch.randperm(num_pages, generator=g)
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    nxt = 0
+    for b, n in enumerate(pages_per_seq):
+        table[b, :n] = order[nxt:nxt + n].to(torch.int32)
+        nxt += n
+    q = _normal((B, H, d), seed + 0, device)
+    k_pages = _normal((num_pages, page_size, H, d), seed + 1, device)
+    v_pages = _normal((num_pages, page_size, H, d), seed + 2, device)
+    return q, k_pages, v_pages, table, lengths.to(torch.int32)

@@ -122,6 +122,32 @@ FA_API fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, 
                             size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Split-KV decode over a paged KV cache (the paging the pages name as the
+ * batched-decode layout question, "FlashAttention saves IO, not N^2 work",
+ * section 6).  Same computation as fa_decode_splitkv; only the cache layout
+ * differs.
+ *   q                : [B, H, d] bf16, one query row per sequence
+ *   k_pages, v_pages : [num_pages, page_size, H, d] bf16 (any page_size >= 1)
+ *   block_table      : device int32 [B, max_pages_per_seq]; key t of sequence b is
+ *                      row t % page_size of page block_table[b][t / page_size].
+ *                      Entries past a sequence's last page are not read.
+ *   seqlens_k        : device int32 [B], keys per sequence; values are clamped to
+ *                      [0, max_seqlen_k]
+ *   max_seqlen_k     : an upper bound of every sequence length; must not exceed
+ *                      max_pages_per_seq * page_size (FA_ERR_INVALID_ARG)
+ *   num_splits, o, lse, workspace: as for fa_decode_splitkv (same workspace size)
+ * A page index outside [0, num_pages) is never dereferenced: the kernel records
+ * it in the workspace status word (fa_check then returns FA_ERR_INVALID_ARG) and
+ * reads page 0 in its place, so that output is meaningless but nothing outside
+ * the cache is touched.  A sequence of length 0 gets O = 0 and LSE = -inf.
+ */
+FA_API fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                 const int32_t* block_table, const int32_t* seqlens_k, int B, int H,
+                                 int num_pages, int page_size, int max_pages_per_seq, int max_seqlen_k,
+                                 int d, float softmax_scale, int num_splits, void* o, float* lse,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * fa_decode_splitkv without a workspace, for callers that cannot allocate
  * device memory -- for example an operator inside a host framework that owns
  * every device allocation and offers it no allocator, or a serving loop that

@@ -156,6 +156,30 @@ def decode(q, k, v, cu_seqlens, scale: float):
     return o, lse
 
 
+def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale: float):
+    """Decode over a paged cache: key t of sequence b is row t % page_size of page
+    block_table[b, t // page_size].  The gathered keys and values of each sequence,
+    in key order, go through `decode` (the paging changes where keys live, not what
+    is computed)."""
+    kp, vp = _f64(k_pages), _f64(v_pages)
+    table = np.asarray(block_table, dtype=np.int64)
+    lens = np.asarray(seqlens, dtype=np.int64)
+    page_size = kp.shape[1]
+    ks, vs = [], []
+    for b, L in enumerate(lens):
+        t = np.arange(int(L))
+        pages = table[b, t // page_size]
+        assert np.all((pages >= 0) & (pages < kp.shape[0])), "page index outside the cache"
+        ks.append(kp[pages, t % page_size])
+        vs.append(vp[pages, t % page_size])
+    H, d = kp.shape[2], kp.shape[3]
+    k = np.concatenate(ks, axis=0) if ks else np.zeros((0, H, d))
+    v = np.concatenate(vs, axis=0) if vs else np.zeros((0, H, d))
+    cu = np.zeros(len(lens) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(lens)
+    return decode(q, k, v, cu, scale)
+
+
 def row_state(scores, values):
     """(m, l, u) of a stream of scores [n] with values [n, dv] (or [n])."""
     s = _f64(scores).reshape(-1)

@@ -111,6 +111,28 @@ def test_decode_argument_validation(lib):
     assert call(wsb=8) == ST["FA_ERR_WORKSPACE"]
 
 
+def test_decode_paged_argument_validation(lib):
+    def call(**kw):
+        a = dict(q=P, k=P, v=P, bt=P, sl=P, B=2, H=4, npg=10, ps=16, mp=4, L=64, d=128, s=0, o=P, lse=P, ws=P,
+                 wsb=1 << 30)
+        a.update(kw)
+        return lib.fa_decode_paged(a["q"], a["k"], a["v"], a["bt"], a["sl"], a["B"], a["H"], a["npg"], a["ps"],
+                                   a["mp"], a["L"], a["d"], 0.0, a["s"], a["o"], a["lse"], a["ws"], a["wsb"], None)
+
+    assert call(bt=None) == ST["FA_ERR_INVALID_ARG"]
+    assert call(sl=None) == ST["FA_ERR_INVALID_ARG"]
+    assert call(npg=0) == ST["FA_ERR_INVALID_ARG"]
+    assert call(ps=0) == ST["FA_ERR_INVALID_ARG"]
+    assert call(mp=0) == ST["FA_ERR_INVALID_ARG"]
+    # 4 pages of 16 keys cannot hold a 65-key sequence
+    assert call(L=65) == ST["FA_ERR_INVALID_ARG"]
+    assert call(d=96) == ST["FA_ERR_UNSUPPORTED"]
+    assert call(k=P + 8) == ST["FA_ERR_ALIGNMENT"]
+    assert call(bt=P + 2) == ST["FA_ERR_ALIGNMENT"]
+    assert call(sl=P + 1) == ST["FA_ERR_ALIGNMENT"]
+    assert call(wsb=8) == ST["FA_ERR_WORKSPACE"]
+
+
 def test_check_rejects_null_workspace(lib):
     assert lib.fa_check(None, None) == ST["FA_ERR_INVALID_ARG"]
 
