@@ -872,9 +872,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             }
             tc_fence_after();
             issue_acc_tmem_linear<D>(tmem + L::kTmDV, tmem + L::kTmPt, at(do_mn, st * kTile16), t == 0);
+            umma_commit(bar_pt_free);  // P^T is no longer read
             issue_acc<D, false>(tmem + L::kTmDK, 0u, at(ds_kmaj, db * kDs16), at(q_mn, st * kTile16), t == 0);
-            umma_commit(bar_q_empty + st);  // Q and dO of this tile are no longer read
-            umma_commit(bar_pt_free);       // nor is P^T
+            umma_commit(bar_q_empty + st);  // nor are Q and dO of this tile
             if (T > 0) {                    // the previous dQ tile must have left tensor memory
               if (!mbar_wait(bar_dq_empty, (T - 1) & 1, a.timeout_ns) || *abort_flag) {
                 ok = false;
@@ -984,35 +984,35 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         const uint32_t stat_u32 = sbase + L::kOffStat + st * 1024 + col * 4;
         const uint32_t ds_row = sbase + L::kOffDS + db * L::kDsBytes + grp * 16384 + r * 128;
         const int qs0 = q0 + col, qs1 = q0 + col + 32;
-        uint32_t pk[16], dk2[16];
+        // both 32-query blocks first: the waits for the P^T columns and the dS buffer
+        // come as late as possible
+        uint32_t pk0[16], dk0[16], pk1[16], dk1[16];
         if (key_tail || (a.causal && last_key_qmin > qs0))
-          ds_block<32, true>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk, dk2);
+          ds_block<32, true>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk0, dk0);
         else
-          ds_block<32, false>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk, dk2);
+          ds_block<32, false>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk0, dk0);
+        if (key_tail || (a.causal && last_key_qmin > qs1))
+          ds_block<32, true>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk1, dk1);
+        else
+          ds_block<32, false>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk1, dk1);
         // P^T may be written once the previous tile's dV has read it
         if (T > 0 && (!warp_wait_b(bar_pt_free, (T - 1) & 1, a.timeout_ns) || *abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        tmem_st16(tmem + lane_field + L::kTmPt + 32 * grp, pk);
+        tmem_st16(tmem + lane_field + L::kTmPt + 32 * grp, pk0);
+        tmem_st16(tmem + lane_field + L::kTmPt + 32 * grp + 16, pk1);
         if (!warp_wait_b(bar_ds_free + db, ((T / L::kDsBufs) & 1) ^ 1, a.timeout_ns) || *abort_flag) {
           ok = false;
           break;
         }
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
-          st_shared_v4(ds_row + ((c4 ^ (r & 7)) << 4), dk2[4 * c4], dk2[4 * c4 + 1], dk2[4 * c4 + 2],
-                       dk2[4 * c4 + 3]);
-        if (key_tail || (a.causal && last_key_qmin > qs1))
-          ds_block<32, true>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk, dk2);
-        else
-          ds_block<32, false>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk, dk2);
-        tmem_st16(tmem + lane_field + L::kTmPt + 32 * grp + 16, pk);
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4)
-          st_shared_v4(ds_row + (((4 + c4) ^ (r & 7)) << 4), dk2[4 * c4], dk2[4 * c4 + 1], dk2[4 * c4 + 2],
-                       dk2[4 * c4 + 3]);
+        for (int c4 = 0; c4 < 4; ++c4) {
+          st_shared_v4(ds_row + ((c4 ^ (r & 7)) << 4), dk0[4 * c4], dk0[4 * c4 + 1], dk0[4 * c4 + 2], dk0[4 * c4 + 3]);
+          st_shared_v4(ds_row + (((4 + c4) ^ (r & 7)) << 4), dk1[4 * c4], dk1[4 * c4 + 1], dk1[4 * c4 + 2],
+                       dk1[4 * c4 + 3]);
+        }
         fence_proxy_async_smem();
         tmem_st_wait();
         tc_fence_before();
