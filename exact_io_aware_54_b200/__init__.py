@@ -69,8 +69,9 @@ def load():
         lib.fa_decode_splitkv.argtypes = [_vp] * 4 + [_i] * 6 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
         lib.fa_decode_splitkv_noalloc.argtypes = [_vp] * 4 + [_i] * 6 + [_f, _i, _vp, _vp, _vp]
         lib.fa_decode_paged.argtypes = [_vp] * 5 + [_i] * 7 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
+        lib.fa_fwd_varlen.argtypes = [_vp] * 7 + [_i] * 8 + [_f, _vp, _sz, _vp]
         for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_decode_splitkv, lib.fa_decode_splitkv_noalloc,
-                   lib.fa_decode_paged):
+                   lib.fa_decode_paged, lib.fa_fwd_varlen):
             fn.restype = _i
         lib.fa_fwd_workspace_size.argtypes = [_i] * 5
         lib.fa_fwd_workspace_size.restype = _sz
@@ -176,6 +177,34 @@ def fa_fwd(q, k, v, causal: bool = False, softmax_scale=None, out=None, lse=None
     st = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Nq, Nk, d,
                     int(bool(causal)), _scale(softmax_scale), ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
     _raise("fa_fwd", st)
+    return out, lse
+
+
+def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int, causal: bool = False,
+                  softmax_scale=None, out=None, lse=None, ws=None):
+    """Forward over packed variable-length sequences.  q [total_q, H, d], k/v
+    [total_k, H, d] bf16; cu_seqlens_q/k int32 [B+1] on the device.
+    Returns (o [total_q, H, d] bf16, lse [H, total_q] fp32)."""
+    lib = load()
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    B = cu_seqlens_q.shape[0] - 1
+    _check_tensor("q", q, torch.bfloat16)
+    _check_tensor("k", k, torch.bfloat16)
+    _check_tensor("v", v, torch.bfloat16, k.shape)
+    _check_tensor("cu_seqlens_q", cu_seqlens_q, torch.int32, (B + 1,))
+    _check_tensor("cu_seqlens_k", cu_seqlens_k, torch.int32, (B + 1,))
+    if k.dim() != 3 or k.shape[1] != H or k.shape[2] != d:
+        raise ValueError("k/v must be [total_k, H, d]")
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device) if lse is None else lse
+    if ws is None:
+        ws = workspace(lib.fa_fwd_workspace_size(1, H, 1, 1, d), q.device, "fwd")
+    st = lib.fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens_q.data_ptr(),
+                           cu_seqlens_k.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, total_q, total_k,
+                           int(max_seqlen_q), int(max_seqlen_k), d, int(bool(causal)), _scale(softmax_scale),
+                           ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
+    _raise("fa_fwd_varlen", st)
     return out, lse
 
 

@@ -222,6 +222,43 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   return launch_fwd(a, stream);
 }
 
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                        const int32_t* cu_seqlens_k, void* o, float* lse, int B, int H, int total_q, int total_k,
+                        int max_seqlen_q, int max_seqlen_k, int d, int causal, float softmax_scale, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
+  if (!q || !k || !v || !cu_seqlens_q || !cu_seqlens_k || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || total_q <= 0 || total_k <= 0 || max_seqlen_q <= 0 || max_seqlen_k <= 0)
+    return FA_ERR_INVALID_ARG;
+  if ((long long)total_q * H * d >= (1LL << 40) || (long long)total_k * H * d >= (1LL << 40) ||
+      (long long)((max_seqlen_q + 255) / 256) * B * H >= (1LL << 31))
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return FA_ERR_ALIGNMENT;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < kStatusBytes) return FA_ERR_WORKSPACE;
+  FwdLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.lse = lse;
+  a.status = static_cast<int*>(workspace);
+  a.cu_q = cu_seqlens_q;
+  a.cu_k = cu_seqlens_k;
+  a.total_q = total_q;
+  a.total_k = total_k;
+  a.B = B;
+  a.H = H;
+  a.Nq = max_seqlen_q;
+  a.Nk = max_seqlen_k;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.scale = resolve_scale(softmax_scale, d);
+  a.timeout_ns = wait_timeout_ns();
+  return launch_fwd(a, stream);
+}
+
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,
                  void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d, int causal,
                  float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {

@@ -50,6 +50,11 @@ struct FwdLaunch {
   void* o;
   float* lse;
   int* status;
+  // variable-length batch (cu_q != nullptr): q, o are [total_q, H, d], k, v
+  // [total_k, H, d], lse [H, total_q]; Nq, Nk are the maximum sequence lengths
+  const int32_t* cu_q = nullptr;
+  const int32_t* cu_k = nullptr;
+  int total_q = 0, total_k = 0;
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;

@@ -41,6 +41,13 @@
 //    adds into the two row sums; the row max uses 3-input max.
 //  * Causal (bottom-right aligned): KV tiles entirely above the diagonal are
 //    never loaded or multiplied; only tiles that cross it are masked.
+//  * Variable-length batches (packed [total, H, d] rows with cu_seqlens): an item
+//    reads its sequence's offsets and lengths; the TMA maps see one long batch,
+//    keys past the sequence's end are masked like the causal triangle, and a
+//    query tile that ends inside its sequence is stored by TMA while the last,
+//    partial tile of a sequence writes its own rows directly, so no store reaches
+//    the next sequence.  Offsets that do not fit the buffers are recorded in the
+//    status word and the sequence is skipped.
 //  * Epilogue: O/l -> bf16 -> swizzled smem (the Q tile's slot) -> TMA store;
 //    lse as coalesced fp32 stores.
 #include "fa_internal.h"
@@ -101,7 +108,11 @@ struct FwdLayout {
 struct FwdArgs {
   float* lse;
   int* status;
-  int B, H, Nq, Nk;
+  __nv_bfloat16* o;  // for the direct stores of partial variable-length tiles
+  const int32_t* cu_q;  // variable-length batch: [B + 1] row offsets (null for a dense batch)
+  const int32_t* cu_k;
+  int total_q, total_k;
+  int B, H, Nq, Nk;  // variable length: Nq, Nk are the maximum sequence lengths
   int causal;
   float scale_log2;
   int n_pairs;
@@ -118,14 +129,41 @@ __device__ __forceinline__ void item_coords(const FwdArgs& a, int w, int& b, int
   h = bh - b * a.H;
 }
 
+// The rows of sequence b: query rows qoff .. qoff + lq - 1 and key rows
+// koff .. koff + lk - 1 of the batch coordinate bc.  A dense batch has lq = Nq,
+// lk = Nk at offset 0 of batch b; a variable-length batch reads cu_seqlens
+// (lq = -1 marks a sequence whose offsets do not fit the buffers).
+struct SeqView {
+  int lq, lk, qoff, koff, bc;
+};
+__device__ __forceinline__ SeqView seq_view(const FwdArgs& a, int b) {
+  SeqView v;
+  if (a.cu_q == nullptr) {
+    v.lq = a.Nq;
+    v.lk = a.Nk;
+    v.qoff = 0;
+    v.koff = 0;
+    v.bc = b;
+    return v;
+  }
+  v.qoff = a.cu_q[b];
+  v.koff = a.cu_k[b];
+  v.lq = min(a.cu_q[b + 1] - v.qoff, a.Nq);
+  v.lk = min(a.cu_k[b + 1] - v.koff, a.Nk);
+  v.bc = 0;
+  if (v.qoff < 0 || v.koff < 0 || v.lq < 0 || v.lk < 0 || v.qoff + v.lq > a.total_q || v.koff + v.lk > a.total_k)
+    v.lq = -1;
+  return v;
+}
+
 // Number of KV tiles query tile starting at row0 needs; -1 when the tile is empty.
-__device__ __forceinline__ int tile_kv_count(const FwdArgs& a, int row0) {
-  if (row0 >= a.Nq) return -1;
-  if (!a.causal) return (a.Nk + 127) >> 7;
-  const int last = min(row0 + 127, a.Nq - 1);
-  long long kend = (long long)last + 1 + a.Nk - a.Nq;
+__device__ __forceinline__ int tile_kv_count(const FwdArgs& a, const SeqView& v, int row0) {
+  if (row0 >= v.lq) return -1;
+  if (!a.causal) return (v.lk + 127) >> 7;
+  const int last = min(row0 + 127, v.lq - 1);
+  long long kend = (long long)last + 1 + v.lk - v.lq;
   if (kend <= 0) return 0;
-  if (kend > a.Nk) kend = a.Nk;
+  if (kend > v.lk) kend = v.lk;
   return (int)((kend + 127) >> 7);
 }
 
@@ -230,13 +268,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t item_iter = 0, g = 0;
-      for (int w = blockIdx.x; w < a.n_items && !*abort_flag; w += gridDim.x, ++item_iter) {
+      for (int w = blockIdx.x; w < a.n_items && !*abort_flag; w += gridDim.x) {
         int b, h, pair;
         item_coords(a, w, b, h, pair);
+        const SeqView sv = seq_view(a, b);
         const int row0 = pair * 256;
-        const int n0 = tile_kv_count(a, row0), n1 = tile_kv_count(a, row0 + 128);
+        const int n0 = tile_kv_count(a, sv, row0), n1 = tile_kv_count(a, sv, row0 + 128);
         const int nkv = max(n0, n1);
-        if (!mbar_wait(bar_q_empty, (item_iter & 1) ^ 1, a.timeout_ns)) {
+        if (n0 < 0) continue;  // no query row of this item exists: every role skips it
+        if (!mbar_wait(bar_q_empty, (item_iter++ & 1) ^ 1, a.timeout_ns)) {
           record_timeout(a.status, abort_flag);
           break;
         }
@@ -244,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = 0; t < 2; ++t)
           for (int bx = 0; bx < L::kBoxes; ++bx)
             tma_load_4d(smem + L::kOffQ + t * L::kTileBytes + bx * L::kBoxBytes, &tmQ, bar_q_full, bx * 64, h,
-                        row0 + t * 128, b);
+                        sv.qoff + row0 + t * 128, sv.bc);
         for (int j = 0; j < nkv; ++j) {
           for (int kv = 0; kv < 2; ++kv, ++g) {
             const uint32_t slot = g % L::kStages, phase = (g / L::kStages) & 1;
@@ -256,8 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(bar_kv_full + slot, L::kTileBytes);
             uint8_t* dst = smem + L::kOffRing + slot * L::kTileBytes;
             for (int bx = 0; bx < L::kBoxes; ++bx)
-              tma_load_4d(dst + bx * L::kBoxBytes, kv == 0 ? &tmK : &tmV, bar_kv_full + slot, bx * 64, h, j * 128,
-                          b);
+              tma_load_4d(dst + bx * L::kBoxBytes, kv == 0 ? &tmK : &tmV, bar_kv_full + slot, bx * 64, h,
+                          sv.koff + j * 128, sv.bc);
           }
         }
       }
@@ -282,15 +322,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ring slots alternate K, V per KV step: K of step j at g, V at g + 1
       uint32_t item_iter = 0, g = 0;
       uint32_t cnt[2] = {0, 0};  // Q K^T (warp 1) or P V (warp 2) MMAs issued per query tile
-      for (int w = blockIdx.x; w < a.n_items && ok; w += gridDim.x, ++item_iter) {
+      for (int w = blockIdx.x; w < a.n_items && ok; w += gridDim.x) {
         int b, h, pair;
         item_coords(a, w, b, h, pair);
+        const SeqView sv = seq_view(a, b);
         const int row0 = pair * 256;
-        const int nt[2] = {tile_kv_count(a, row0), tile_kv_count(a, row0 + 128)};
+        const int nt[2] = {tile_kv_count(a, sv, row0), tile_kv_count(a, sv, row0 + 128)};
         const int nkv = max(nt[0], nt[1]);
+        if (nt[0] < 0) continue;  // no query row of this item exists: every role skips it
+        const uint32_t it_q = item_iter++;  // items processed: q_full phases
         if (warp == 1) {
           // S_t = Q_t K_j^T once the group has read its previous S tile
-          if (!wait_or_abort(bar_q_full, item_iter & 1)) break;
+          if (!wait_or_abort(bar_q_full, it_q & 1)) break;
           tc_fence_after();
           for (int j = 0; j < nkv && ok; ++j, g += 2) {
             const uint32_t slot_k = g % L::kStages;
@@ -314,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // O_t += P_t V_j once the group has written P.  The epilogue stages O
           // through the Q tiles: o_done must also follow this item's Q load (it
           // decides alone when a tile sees no key at all).
-          if (!wait_or_abort(bar_q_full, item_iter & 1)) break;
+          if (!wait_or_abort(bar_q_full, it_q & 1)) break;
           for (int j = 0; j < nkv && ok; ++j, g += 2) {
             const uint32_t slot_v = (g + 1) % L::kStages;
             if (!wait_or_abort(bar_kv_full + slot_v, ((g + 1) / L::kStages) & 1)) break;
@@ -359,13 +402,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return ok;
       };
-      for (int w = blockIdx.x; w < a.n_items && ok; w += gridDim.x, ++item_iter) {
+      for (int w = blockIdx.x; w < a.n_items && ok; w += gridDim.x) {
         int b, h, pair;
         item_coords(a, w, b, h, pair);
+        const SeqView sv = seq_view(a, b);
         const int row0 = pair * 256;
-        const int nt[2] = {tile_kv_count(a, row0), tile_kv_count(a, row0 + 128)};
+        const int nt[2] = {tile_kv_count(a, sv, row0), tile_kv_count(a, sv, row0 + 128)};
         const int nkv = max(nt[0], nt[1]);
-        if (!wait_or_abort(bar_q_full, item_iter & 1)) break;
+        if (nt[0] < 0) continue;  // no query row of this item exists: every role skips it
+        const uint32_t it_q = item_iter++;  // items processed: q_full phases
+        if (!wait_or_abort(bar_q_full, it_q & 1)) break;
         tc_fence_after();
         // K_0 : first scores of both tiles
         uint32_t slot_k = 0;
@@ -437,6 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tP = tmem_base + lane_field + tm_p<D>(t);
     const int tid_in_group = threadIdx.x - 128 - t * 128;
     uint32_t s_cnt = 0, tile_iter = 0;  // tile_iter counts items in which this tile is present
+    uint32_t items_done = 0;            // items with a query row (the producer's q phases)
     uint8_t* q_tile = smem + L::kOffQ + t * L::kTileBytes;
     const uint32_t q_tile_u32 = smem_u32(q_tile);
 
@@ -444,18 +491,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (*abort_flag) break;
       int b, h, pair;
       item_coords(a, w, b, h, pair);
+      const SeqView sv = seq_view(a, b);
+      if (sv.lq < 0 && pair == 0 && t == 0 && tid_in_group == 0) atomicExch(a.status, kStatusBadArg);
       const int row0 = pair * 256 + t * 128;
-      const int nkv = tile_kv_count(a, row0);
-      if (nkv < 0) {  // this query tile lies past Nq: nothing to compute or store
+      const int nkv = tile_kv_count(a, sv, row0);
+      // No query row of this item exists: every role skips it (an arrival here
+      // could complete the producer's q_empty phase before its first wait).
+      if (tile_kv_count(a, sv, pair * 256) < 0) continue;
+      const uint32_t it_q = items_done++;
+      if (nkv < 0) {
+        // This query tile lies past the sequence: nothing to compute or store.  Its
+        // release of the Q pair waits for this item's Q load, so that it can never
+        // count toward the previous item's release (the other group may still be
+        // staging that item's output in its Q tile).
+        if (!warp_wait(bar_q_full, it_q & 1, a.timeout_ns) || *abort_flag) {
+          if (lane == 0) record_timeout(a.status, abort_flag);
+          break;
+        }
         if (tid_in_group == 0) mbar_arrive(bar_q_empty);
         __syncwarp();
         continue;
       }
       const int row = row0 + r;
       // visible keys of this row: [0, lim)
-      int lim = a.Nk;
-      if (a.causal) lim = max(0, min(a.Nk, row + 1 + a.Nk - a.Nq));
-      const int group_first_lim = a.causal ? (row0 + 1 + a.Nk - a.Nq) : a.Nk;  // smallest lim in the tile
+      const int lk = sv.lk;  // only the key count stays live through the KV loop
+      int lim = lk;
+      if (a.causal) lim = max(0, min(lk, row + 1 + lk - sv.lq));
+      const int group_first_lim = a.causal ? (row0 + 1 + lk - sv.lq) : lk;  // smallest lim in the tile
 
       float m2 = -INFINITY;  // running reference max (log2 domain)
       float l = 0.f;         // running sum of the bf16-rounded probabilities (normalises O)
@@ -482,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // mask (only tiles that cross the diagonal or the key tail)
         const int kbase = j * 128;
-        if (kbase + 128 > min(group_first_lim, a.Nk) || kbase + 128 > a.Nk) {
+        if (kbase + 128 > min(group_first_lim, lk) || kbase + 128 > lk) {
 #pragma unroll
           for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -586,6 +648,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const SeqView se = seq_view(a, b);  // read again rather than kept live through the loop
+      // a variable-length tile that runs past its sequence writes its rows itself
+      const bool direct = a.cu_q != nullptr && row0 + 128 > se.lq;
+      uint4* orow = reinterpret_cast<uint4*>(a.o + ((size_t)(se.qoff + row) * a.H + h) * D);
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -602,13 +668,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int chunk = (cc & 1) * 4 + q4;  // 16-byte chunk within the 128-byte row
           const uint32_t addr = q_tile_u32 + box * L::kBoxBytes + r * 128 + ((chunk ^ (r & 7)) << 4);
           const float* f = reinterpret_cast<const float*>(o) + q4 * 8;
-          st_shared_v4(addr, pack_bf16x2(f[0] * inv_l, f[1] * inv_l), pack_bf16x2(f[2] * inv_l, f[3] * inv_l),
-                       pack_bf16x2(f[4] * inv_l, f[5] * inv_l), pack_bf16x2(f[6] * inv_l, f[7] * inv_l));
+          const uint4 packed = make_uint4(pack_bf16x2(f[0] * inv_l, f[1] * inv_l), pack_bf16x2(f[2] * inv_l, f[3] * inv_l),
+                                          pack_bf16x2(f[4] * inv_l, f[5] * inv_l), pack_bf16x2(f[6] * inv_l, f[7] * inv_l));
+          if (!direct)
+            st_shared_v4(addr, packed.x, packed.y, packed.z, packed.w);
+          else if (row < se.lq)
+            orow[cc * 4 + q4] = packed;
         }
       }
-      if (row < a.Nq) {
+      if (row < se.lq) {
         const float lse = (le > 0.f) ? (m2 + __log2f(le)) * 0.69314718055994530942f : -INFINITY;
-        a.lse[((size_t)b * a.H + h) * a.Nq + row] = lse;
+        if (a.cu_q != nullptr)
+          a.lse[(size_t)h * a.total_q + se.qoff + row] = lse;
+        else
+          a.lse[((size_t)b * a.H + h) * a.Nq + row] = lse;
       }
       fence_proxy_async_smem();
       mbar_arrive_warp(bar_epi + t);
@@ -618,10 +691,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           record_timeout(a.status, abort_flag);
           epi_ok = false;
         } else {
-          for (int bx = 0; bx < L::kBoxes; ++bx)
-            tma_store_4d(&tmO, q_tile + bx * L::kBoxBytes, bx * 64, h, row0, b);
-          bulk_commit_group();
-          bulk_wait_group_read0();
+          if (!direct) {
+            for (int bx = 0; bx < L::kBoxes; ++bx)
+              tma_store_4d(&tmO, q_tile + bx * L::kBoxBytes, bx * 64, h, se.qoff + row0, se.bc);
+            bulk_commit_group();
+            bulk_wait_group_read0();
+          }
           mbar_arrive(bar_q_empty);
         }
       }
@@ -654,13 +729,22 @@ static fa_status launch_fwd_impl(const FwdLaunch& L0, cudaStream_t stream) {
       return FA_ERR_CUDA;
     attr_done[dev] = true;
   }
+  // a variable-length batch is one long batch of total rows for the TMA maps
+  const bool varlen = L0.cu_q != nullptr;
+  const int mB = varlen ? 1 : L0.B;
+  const int mNq = varlen ? L0.total_q : L0.Nq, mNk = varlen ? L0.total_k : L0.Nk;
   CUtensorMap tq, tk, tv, to;
-  if (!encode_bshd_map(&tq, L0.q, L0.B, L0.Nq, L0.H, D) || !encode_bshd_map(&tk, L0.k, L0.B, L0.Nk, L0.H, D) ||
-      !encode_bshd_map(&tv, L0.v, L0.B, L0.Nk, L0.H, D) || !encode_bshd_map(&to, L0.o, L0.B, L0.Nq, L0.H, D))
+  if (!encode_bshd_map(&tq, L0.q, mB, mNq, L0.H, D) || !encode_bshd_map(&tk, L0.k, mB, mNk, L0.H, D) ||
+      !encode_bshd_map(&tv, L0.v, mB, mNk, L0.H, D) || !encode_bshd_map(&to, L0.o, mB, mNq, L0.H, D))
     return FA_ERR_CUDA;
   FwdArgs a;
   a.lse = L0.lse;
   a.status = L0.status;
+  a.o = static_cast<__nv_bfloat16*>(L0.o);
+  a.cu_q = L0.cu_q;
+  a.cu_k = L0.cu_k;
+  a.total_q = L0.total_q;
+  a.total_k = L0.total_k;
   a.B = L0.B;
   a.H = L0.H;
   a.Nq = L0.Nq;

@@ -83,6 +83,31 @@ FA_API fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, fl
                  size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Forward pass over a batch of sequences of different lengths, packed without
+ * padding (the variable-length prefill of the paging / padding discussion,
+ * "FlashAttention saves IO, not N^2 work", section 6).  Same computation as
+ * fa_fwd, sequence by sequence; the causal mask is bottom-right aligned within
+ * each sequence.
+ *   q, o        : [total_q, H, d] bf16; sequence b owns rows
+ *                 cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1
+ *   k, v        : [total_k, H, d] bf16, rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1
+ *   cu_seqlens_q, cu_seqlens_k : device int32 [B+1], non-decreasing, starting at 0
+ *   lse         : [H, total_q] fp32 (written)
+ *   max_seqlen_q, max_seqlen_k : upper bounds of the sequence lengths (lengths
+ *                 above them are cut to them)
+ *   workspace   : at least fa_fwd_workspace_size(...) bytes (the status word)
+ * A sequence whose offsets do not fit the buffers is skipped and recorded in
+ * the status word (fa_check then returns FA_ERR_INVALID_ARG); no store leaves
+ * the rows of its own sequence.  Rows of a sequence with no keys get O = 0 and
+ * LSE = -inf.
+ */
+FA_API fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
+                               const int32_t* cu_seqlens_k, void* o, float* lse, int B, int H,
+                               int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d,
+                               int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+
+/*
  * Backward pass (recompute form).
  *   q, o, do_ : [B, Nq, H, d] bf16 ; k, v : [B, Nk, H, d] bf16
  *   lse       : [B, H, Nq] fp32 as written by fa_fwd with the same arguments

@@ -156,6 +156,29 @@ def decode(q, k, v, cu_seqlens, scale: float):
     return o, lse
 
 
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal: bool, scale: float):
+    """Forward over packed variable-length sequences: q [total_q, H, d], k, v
+    [total_k, H, d], row offsets cu_seqlens_* [B+1] -> (o [total_q, H, d],
+    lse [H, total_q]).  Each sequence is one batch element of `attn_fwd` (the
+    causal mask bottom-right aligned within it); packing changes nothing else."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    cq = np.asarray(cu_seqlens_q, dtype=np.int64)
+    ck = np.asarray(cu_seqlens_k, dtype=np.int64)
+    total_q, H, d = q.shape
+    o = np.zeros((total_q, H, d))
+    lse = np.full((H, total_q), -np.inf)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 == q0:
+            continue
+        if k1 == k0:  # no keys: O = 0, lse = -inf
+            continue
+        ob, lb = attn_fwd(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], causal, scale)
+        o[q0:q1] = ob[0]
+        lse[:, q0:q1] = lb[0]
+    return o, lse
+
+
 def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale: float):
     """Decode over a paged cache: key t of sequence b is row t % page_size of page
     block_table[b, t // page_size].  The gathered keys and values of each sequence,

@@ -133,6 +133,24 @@ def test_decode_paged_argument_validation(lib):
     assert call(wsb=8) == ST["FA_ERR_WORKSPACE"]
 
 
+def test_fwd_varlen_argument_validation(lib):
+    def call(**kw):
+        a = dict(q=P, k=P, v=P, cq=P, ck=P, o=P, lse=P, B=3, H=4, tq=300, tk=400, mq=200, mk=300, d=64, ws=P,
+                 wsb=1 << 20)
+        a.update(kw)
+        return lib.fa_fwd_varlen(a["q"], a["k"], a["v"], a["cq"], a["ck"], a["o"], a["lse"], a["B"], a["H"],
+                                 a["tq"], a["tk"], a["mq"], a["mk"], a["d"], 1, 0.0, a["ws"], a["wsb"], None)
+
+    assert call(cq=None) == ST["FA_ERR_INVALID_ARG"]
+    assert call(tk=0) == ST["FA_ERR_INVALID_ARG"]
+    assert call(mq=0) == ST["FA_ERR_INVALID_ARG"]
+    assert call(B=0) == ST["FA_ERR_INVALID_ARG"]
+    assert call(d=80) == ST["FA_ERR_UNSUPPORTED"]
+    assert call(o=P + 4) == ST["FA_ERR_ALIGNMENT"]
+    assert call(ck=P + 2) == ST["FA_ERR_ALIGNMENT"]
+    assert call(ws=None) == ST["FA_ERR_WORKSPACE"]
+
+
 def test_check_rejects_null_workspace(lib):
     assert lib.fa_check(None, None) == ST["FA_ERR_INVALID_ARG"]
 

@@ -54,6 +54,13 @@ def test_many_items_per_cta(d):
     _full_check(4, 512, 512, 48, d, True, 777 + d)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_absent_last_tile_with_many_items_per_cta(causal):
+    """Nq % 256 <= 128 leaves the second query tile of the last pair empty; with
+    B * H above twice the SM count a persistent CTA meets such items back to back."""
+    _full_check(4, 1100, 1100, 80, 64, causal, 888 + causal)
+
+
 def test_explicit_scale():
     _full_check(1, 300, 300, 2, 64, True, 4242, scale=0.37)
 
