@@ -81,6 +81,8 @@ def load():
         lib.fa_decode_workspace_size.restype = _sz
         lib.fa_decode_num_splits.argtypes = [_i] * 5
         lib.fa_decode_num_splits.restype = _i
+        lib.fa_selftest_wait_timeout.argtypes = [_vp, _sz, ctypes.c_uint, _vp]
+        lib.fa_selftest_wait_timeout.restype = _i
         lib.fa_check.argtypes = [_vp, _vp]
         lib.fa_check.restype = _i
         lib.fa_status_string.argtypes = [_i]
@@ -302,6 +304,12 @@ def fa_decode_paged(q, k_pages, v_pages, block_table, seqlens_k, max_seqlen_k: i
                              lse.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
     _raise("fa_decode_paged", st)
     return out, lse
+
+
+def fa_selftest_wait_timeout(ws: torch.Tensor, timeout_us: int = 1000) -> None:
+    """Run the bounded-wait failure path once (see include/fa.h); read the result with fa_check."""
+    _raise("fa_selftest_wait_timeout",
+           load().fa_selftest_wait_timeout(ws.data_ptr(), ws.numel(), int(timeout_us), _stream_ptr(ws.device)))
 
 
 def fa_check(ws: torch.Tensor) -> int:

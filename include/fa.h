@@ -218,6 +218,17 @@ FA_API int fa_decode_num_splits(int B, int H, int max_seqlen_k, int d, int num_s
  */
 FA_API fa_status fa_check(void* workspace, cudaStream_t stream);
 
+/*
+ * Self-test of the failure path (no counterpart in the pages).  Launches one
+ * thread that waits, with the library's bounded wait, on a barrier nothing
+ * arrives on; after `timeout_us` microseconds (1 .. 1000000) the wait gives up
+ * and records FA_ERR_TIMEOUT in the workspace status word, exactly as a stuck
+ * kernel would.  A following fa_check on the same workspace returns
+ * FA_ERR_TIMEOUT and clears the word; the context stays usable.
+ */
+FA_API fa_status fa_selftest_wait_timeout(void* workspace, size_t workspace_bytes, unsigned timeout_us,
+                                          cudaStream_t stream);
+
 /* Human-readable name of a status code (static string). */
 FA_API const char* fa_status_string(fa_status status);
 

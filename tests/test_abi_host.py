@@ -151,6 +151,15 @@ def test_fwd_varlen_argument_validation(lib):
     assert call(ws=None) == ST["FA_ERR_WORKSPACE"]
 
 
+def test_selftest_argument_validation(lib):
+    lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint, ctypes.c_void_p]
+    assert lib.fa_selftest_wait_timeout(None, 256, 100, None) == ST["FA_ERR_WORKSPACE"]
+    assert lib.fa_selftest_wait_timeout(P, 8, 100, None) == ST["FA_ERR_WORKSPACE"]
+    assert lib.fa_selftest_wait_timeout(P + 4, 256, 100, None) == ST["FA_ERR_WORKSPACE"]
+    assert lib.fa_selftest_wait_timeout(P, 256, 0, None) == ST["FA_ERR_INVALID_ARG"]
+    assert lib.fa_selftest_wait_timeout(P, 256, 2000000, None) == ST["FA_ERR_INVALID_ARG"]
+
+
 def test_check_rejects_null_workspace(lib):
     assert lib.fa_check(None, None) == ST["FA_ERR_INVALID_ARG"]
 
