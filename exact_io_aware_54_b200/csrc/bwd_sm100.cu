@@ -9,21 +9,23 @@
 //     dV = P^T dO,   dP = dO V^T,   D_i = dO_i . O_i,   dS = P o (dP - D),
 //     dQ = scale dS K,   dK = scale dS^T Q.
 //
-// Three kernels:
+// Kernels:
 //   1. preprocess: D_i = dO_i . O_i (fp32) and a zeroed fp32 dQ accumulator;
-//   2. main (tcgen05): one CTA per (b, h, 128-key tile); K_j and V_j stay on chip
-//      while the CTA walks the 128-row query tiles that can see them (from the
-//      causal diagonal onward).  Per query tile i:
+//   2. main (tcgen05): K_j and V_j of a 128-key tile stay on chip while the 128-row
+//      query tiles that can see them (from the causal diagonal onward) stream by.
+//      Per query tile i:
 //        S^T = K Q_i^T, dP^T = V dO_i^T       (M = 128 keys, N = 128 queries)
-//        dS warps: P^T and dS^T (bf16) into tensor memory over S^T / dP^T, dS
-//                  into a swizzled shared-memory tile
-//        dV += P^T dO_i, dK += dS^T Q_i        (A operands from tensor memory)
-//        dQ_i = dS K                           (M = 128 queries, A read MN-major)
-//      The tensor core runs dV/dK(i), then S^T/dP^T(i+1), then dQ(i): the dS warps
-//      compute tile i+1 while dQ(i) runs, and drain dQ(i) (fp32 vector reductions
-//      into the accumulator) once their tile i+1 is done.  Every instruction has
-//      N >= 64; tcgen05.mma has a fixed cost of about 44 cycles per instruction,
-//      so the score MMAs use the full N = 128.  dK and dV leave once, through TMA.
+//        dS warps: P^T (bf16) into tensor memory, dS into a swizzled shared-
+//                  memory tile (read K-major for dK and MN-major for dQ)
+//        dV += P^T dO_i (P^T from tensor memory), dK += dS^T Q_i
+//        dQ_i = dS K, added to the fp32 accumulator with vector reductions
+//      tcgen05.mma costs about 44 cycles per instruction for any N <= 64, so the
+//      score MMAs use the full N = 128.
+//      d = 64, bwd_pipe_kernel: persistent, with the score MMAs, the dS warps, the
+//        gradient MMAs and the dQ drain running as concurrent stages (below).
+//      d = 128, bwd_main_kernel: one CTA per (b, h, key tile); the stages of a
+//        query tile run one after another (tensor memory has no room for a second
+//        S^T / dP^T), and the dQ tile reuses the dP^T columns.
 //   3. convert: dQ = bf16(scale * accumulator).
 #include "fa_internal.h"
 #include "ptx.cuh"
@@ -32,16 +34,18 @@ namespace fa {
 
 namespace {
 
-constexpr int kThreads = 320;  // warp 0 TMA + stats, warp 1 MMA, warps 2-9 dS warps (two column groups)
+constexpr int kThreads = 320;  // d = 128 kernel: warp 0 TMA + stats, warp 1 MMA, warps 2-9 dS warps
 constexpr uint32_t kTmemCols = 512;
 
+// Shared and tensor memory of the d = 128 kernel.
 template <int D>
 struct BwdLayout {
+  static_assert(D == 128, "d = 64 uses PipeLayout");
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kBoxes = D / 64;
   static constexpr int kBoxBytes = 16384;
-  static constexpr int kQStages = (D == 64) ? 3 : 2;  // query tiles prefetched ahead
-  static constexpr int kDsBufs = (D == 64) ? 2 : 1;
+  static constexpr int kQStages = 2;  // query tiles prefetched ahead
+  static constexpr int kDsBufs = 1;
   static constexpr int kDsBytes = 2 * 16384;  // [64-query atom][128 keys][64 queries] bf16, 128-byte swizzle
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
@@ -50,22 +54,18 @@ struct BwdLayout {
   static constexpr int kOffDS = kOffDO + kQStages * kTileBytes;
   static constexpr int kOffStat = kOffDS + kDsBufs * kDsBytes;  // per stage: -lse2[128], -D[128]
   static constexpr int kOffBar = kOffStat + kQStages * 2 * 128 * 4;
-  // kv_full, q_full[QS], q_empty[QS], s_full, p_full, ds_free[DSB], dq_full, dq_empty, dkv_done, epi, kv_tmem
-  static constexpr int kNumBars = 1 + 2 * kQStages + 2 + kDsBufs + 5;
+  // kv_full, q_full[QS], q_empty[QS], s_full, p_full, ds_free[DSB], dq_full, dq_empty, dkv_done, epi
+  static constexpr int kNumBars = 1 + 2 * kQStages + 2 + kDsBufs + 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64;
-  // Tensor memory columns.  d = 64 also keeps K and V there (bf16 pairs) as the A
-  // operands of S^T and dP^T, and writes dS^T over dP^T as the A operand of dK;
-  // d = 128 has no room for that, reads K, V and dS^T from shared memory, and
-  // puts the dQ tile over the dP^T columns (drained before the next dP^T).
-  static constexpr bool kKVInTmem = (D == 64);
+  // Tensor memory columns: K, V and dS^T are read from shared memory, and the dQ
+  // tile goes over the dP^T columns (drained before the next dP^T).
   static constexpr uint32_t kTmSt = 0;     // S^T, P^T bf16 over it
-  static constexpr uint32_t kTmDPt = 128;  // dP^T, (d = 64) dS^T bf16 over it
+  static constexpr uint32_t kTmDPt = 128;  // dP^T
   static constexpr uint32_t kTmDV = 256;
   static constexpr uint32_t kTmDK = 256 + D;
-  static constexpr uint32_t kTmDQ = (D == 64) ? 384 : kTmDPt;
-  static constexpr uint32_t kTmK = 448, kTmV = 480;
-  static_assert(kTmDK + D <= kTmemCols && (!kKVInTmem || kTmV + D / 2 <= kTmemCols), "tensor memory budget");
+  static constexpr uint32_t kTmDQ = kTmDPt;
+  static_assert(kTmDK + D <= kTmemCols, "tensor memory budget");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -201,7 +201,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_dq_empty = bar_dq_full + 1;
   uint64_t* bar_dkv_done = bar_dq_empty + 1;
   uint64_t* bar_epi = bar_dkv_done + 1;
-  uint64_t* bar_kv_tmem = bar_epi + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);
 
@@ -231,7 +230,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_dq_empty, 8);
     mbar_init(bar_dkv_done, 1);
     mbar_init(bar_epi, 8);
-    mbar_init(bar_kv_tmem, 8);
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -307,7 +305,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(bar_kv_full, 0, a.timeout_ns);
-      if (ok && L::kKVInTmem) ok = mbar_wait(bar_kv_tmem, 0, a.timeout_ns);
       // operand descriptors, built once; tiles are reached by 32-bit adds (16-byte units)
       const SDesc k_kmaj = sdesc_make(sbase + L::kOffK, 16, 1024), v_kmaj = sdesc_make(sbase + L::kOffV, 16, 1024);
       const SDesc k_mn = sdesc_make(sbase + L::kOffK, 16384, 1024);
@@ -321,8 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int st = it % L::kQStages;
         if (!mbar_wait(bar_q_full + st, (it / L::kQStages) & 1, a.timeout_ns) || *abort_flag) return false;
         tc_fence_after();
-        issue_scores<D, L::kKVInTmem>(tmem + L::kTmSt, tmem + L::kTmK, k_kmaj, at(q_kmaj, st * kTile16));
-        issue_scores<D, L::kKVInTmem>(tmem + L::kTmDPt, tmem + L::kTmV, v_kmaj, at(do_kmaj, st * kTile16));
+        issue_scores<D, false>(tmem + L::kTmSt, 0u, k_kmaj, at(q_kmaj, st * kTile16));
+        issue_scores<D, false>(tmem + L::kTmDPt, 0u, v_kmaj, at(do_kmaj, st * kTile16));
         umma_commit(bar_s_full);
         return true;
       };
@@ -332,8 +329,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const int st = it % L::kQStages;
         issue_acc<D, true>(tmem + L::kTmDV, tmem + L::kTmSt, ds_kmaj, at(do_mn, st * kTile16), it == 0);
-        issue_acc<D, L::kKVInTmem>(tmem + L::kTmDK, tmem + L::kTmDPt, at(ds_kmaj, (it % L::kDsBufs) * kDs16),
-                                   at(q_mn, st * kTile16), it == 0);
+        issue_acc<D, false>(tmem + L::kTmDK, 0u, at(ds_kmaj, (it % L::kDsBufs) * kDs16), at(q_mn, st * kTile16),
+                            it == 0);
         umma_commit(bar_q_empty + st);  // Q and dO of this tile are no longer read
         return true;
       };
@@ -343,28 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma_commit(bar_ds_free + (it % L::kDsBufs));
       };
       if (ok) tc_fence_after();
-      if constexpr (D == 64) {
-        // dV/dK(i), S^T/dP^T(i+1), dQ(i): the dS warps work on tile i+1 while dQ(i) runs
-        if (ok && n_iters > 0) ok = issue_sdp(0);
-        for (int it = 0; it < n_iters && ok; ++it) {
-          if (!issue_dvdk(it)) {
-            ok = false;
-            break;
-          }
-          if (it + 1 < n_iters && !issue_sdp(it + 1)) {
-            ok = false;
-            break;
-          }
-          if (it > 0) {  // the previous dQ tile must have left tensor memory
-            if (!mbar_wait(bar_dq_empty, (it - 1) & 1, a.timeout_ns) || *abort_flag) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-          }
-          issue_dq_tile(it);
-        }
-      } else {
+      {
         // the dQ tile uses the dP^T columns: it is drained before the next dP^T
         for (int it = 0; it < n_iters && ok; ++it) {
           if (it > 0) {
@@ -396,22 +372,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // qmin - qs below must not overflow)
     const int qmin = a.causal ? key - (a.Nk - a.Nq) : -(1 << 30);
     bool ok = true;
-
-    if constexpr (L::kKVInTmem) {
-      // K (group 0) or V (group 1) row of this key into tensor memory as bf16 pairs
-      if (!warp_wait_b(bar_kv_full, 0, a.timeout_ns)) ok = false;
-      if (ok) {
-        const uint32_t src = sbase + (grp == 0 ? L::kOffK : L::kOffV) + r * 128;
-        uint32_t row[32];
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          ld_shared_v4(src + ((c ^ (r & 7)) << 4), row[4 * c], row[4 * c + 1], row[4 * c + 2], row[4 * c + 3]);
-        tmem_st32(tmem + lane_field + (grp == 0 ? L::kTmK : L::kTmV), row);
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive_warp(bar_kv_tmem);
-      }
-    }
 
     // dQ tile of query tile `it`: this group's D/2 columns, fp32 vector reductions
     // into the accumulator
@@ -467,9 +427,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           ds_block<32, true>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2);
         else
           ds_block<32, false>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2);
-        // P^T (and dS^T) as bf16 pairs over the columns of this group already read
+        // P^T as bf16 pairs over the columns of this group already read
         tmem_st16(tmem + lane_field + L::kTmSt + 64 * grp + 16 * ch, pk);
-        if constexpr (L::kKVInTmem) tmem_st16(tmem + lane_field + L::kTmDPt + 64 * grp + 16 * ch, dk2);
         // dS^T row of this key: 4 chunks of 16 bytes, 128-byte swizzle
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
@@ -482,12 +441,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive_warp(bar_p_full);
-      // d = 64: the previous tile's dQ ran while this tile was computed;
-      // d = 128: this tile's dQ follows right after dV / dK
-      if (D == 64 && it > 0) ok = drain_dq(it - 1);
-      if (D == 128) ok = drain_dq(it);
+      // this tile's dQ follows right after dV / dK
+      ok = drain_dq(it);
     }
-    if (D == 64 && ok && n_iters > 0) ok = drain_dq(n_iters - 1);
     // ---------------------------------------------------------------- dK / dV epilogue
     // group 0 stores dK (times scale) through the K tile's smem, group 1 dV through V's
     if (ok && warp_wait_b(bar_dkv_done, 0, a.timeout_ns) && !*abort_flag) {

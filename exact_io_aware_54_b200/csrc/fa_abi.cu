@@ -112,19 +112,6 @@ bool encode_bshd_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int
   return r == CUDA_SUCCESS;
 }
 
-bool encode_bshd_map_f32(CUtensorMap* map, const void* ptr, int B, int N, int H, int D) {
-  EncodeTiledFn fn = get_encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
-  const cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4, (cuuint64_t)N * H * D * 4};
-  const cuuint32_t box[4] = {32, 1, 128, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(ptr), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
-}
-
 static unsigned long long wait_timeout_ns() {
   static unsigned long long v = [] {
     unsigned long long ms = 2000;

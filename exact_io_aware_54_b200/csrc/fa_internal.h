@@ -41,7 +41,6 @@ int num_sms();
 bool encode_bshd_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int D);
 
 // The same for an fp32 tensor [B, N, H, D]: box of 128 rows x 32 columns (128 bytes), 128-byte swizzle.
-bool encode_bshd_map_f32(CUtensorMap* map, const void* ptr, int B, int N, int H, int D);
 
 struct FwdLaunch {
   const void* q;
