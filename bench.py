@@ -299,7 +299,7 @@ def _rotating(make, total_bytes_of_one):
     return [make(i) for i in range(n)]
 
 
-EXTRA_WORKLOADS = ("prefill8k", "decode_single", "decode_batched", "decode_paged", "long16k")
+EXTRA_WORKLOADS = ("prefill8k", "prefill_varlen", "decode_single", "decode_batched", "decode_paged", "long16k")
 
 
 def run_extra(args, fa, synth, dev, pk, only=None):
@@ -308,6 +308,8 @@ def run_extra(args, fa, synth, dev, pk, only=None):
     want = (lambda name: only is None or only == name)
     if want("prefill8k"):
         _extra_prefill(out, iters, fa, synth, dev, pk)
+    if want("prefill_varlen"):
+        _extra_prefill_varlen(out, iters, fa, synth, dev, pk)
     if want("decode_single"):
         _extra_decode_single(out, iters, fa, synth, dev, pk)
     if want("decode_batched"):
@@ -337,6 +339,32 @@ def _extra_prefill(out, iters, fa, synth, dev, pk):
             "ms": round(ms, 4), "TFLOP/s": round(tf, 1), "frac_of_peak": round(tf / pk["bf16_tflops"], 4),
             "l2": f"{len(sets)} rotating input sets"}
     del sets, o, lse
+    torch.cuda.empty_cache()
+
+
+def _extra_prefill_varlen(out, iters, fa, synth, dev, pk):
+    # packed variable-length prefill: 16 causal sequences, lengths U[256, 4096], H=32, d=128
+    lengths = synth.ragged_lengths(synth.SEEDS["prefill8k"], 16, 256, 4096)
+    total = int(lengths.sum())
+    q, k, v = synth.prefill_inputs(synth.SEEDS["prefill8k"], 1, total, total, 32, 128, device=dev)
+    q, k, v = (t.reshape(total, 32, 128) for t in (q, k, v))
+    cu = synth.cu_seqlens_of(lengths).to(dev)
+    maxL = int(lengths.max())
+    o = torch.empty_like(q)
+    lse = torch.empty(32, total, dtype=torch.float32, device=dev)
+
+    def f(i):
+        fa.fa_fwd_varlen(q, k, v, cu, cu, maxL, maxL, causal=True, out=o, lse=lse)
+    for i in range(3):
+        f(i)
+    ms = device_time_ms(f, iters)
+    flops = sum(fwd_flops(1, 32, int(L), int(L), 128, True) for L in lengths)
+    tf = flops / (ms * 1e-3) / 1e12
+    out["prefill_varlen_causal"] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                                    "frac_of_peak": round(tf / pk["bf16_tflops"], 4), "sequences": 16,
+                                    "total_tokens": total, "max_seqlen": maxL,
+                                    "l2": "no flush: Q, K, V together are 779 MB, 6x the L2"}
+    del q, k, v, o, lse, cu
     torch.cuda.empty_cache()
 
 
