@@ -179,6 +179,27 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal: bool, scale: fl
     return o, lse
 
 
+def attn_bwd_varlen(q, k, v, dout, cu_seqlens_q, cu_seqlens_k, causal: bool, scale: float):
+    """Gradients of sum(O * dout) for the packed forward `attn_fwd_varlen`: q, dout
+    [total_q, H, d], k, v [total_k, H, d] -> (dq, dk, dv) of the same shapes, fp64.
+    Each sequence is one batch element of `attn_bwd`; rows outside every sequence,
+    a sequence's queries when it has no keys, and its keys when it has no queries
+    get zero gradient (they take no part in the loss)."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    cq = np.asarray(cu_seqlens_q, dtype=np.int64)
+    ck = np.asarray(cu_seqlens_k, dtype=np.int64)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(len(cq) - 1):
+        q0, q1, k0, k1 = cq[b], cq[b + 1], ck[b], ck[b + 1]
+        if q1 == q0 or k1 == k0:
+            continue
+        g = attn_bwd(q[None, q0:q1], k[None, k0:k1], v[None, k0:k1], dout[None, q0:q1], causal, scale)
+        dq[q0:q1], dk[k0:k1], dv[k0:k1] = g[0][0], g[1][0], g[2][0]
+    return dq, dk, dv
+
+
 def decode_paged(q, k_pages, v_pages, block_table, seqlens, scale: float):
     """Decode over a paged cache: key t of sequence b is row t % page_size of page
     block_table[b, t // page_size].  The gathered keys and values of each sequence,

@@ -77,3 +77,67 @@ def test_empty_sequences():
     o, lse = oracle.attn_fwd_varlen(q, k, v, cq, ck, False, 0.125)
     assert np.all(o[0:4] == 0) and np.all(np.isneginf(lse[:, 0:4]))  # sequence 1 has no keys
     assert np.all(np.isfinite(lse[:, 4:7]))
+
+
+# ---------------------------------------------------------------- backward
+# The gradients of the packed loss sum(O * dO) are pinned by central differences of
+# the packed forward (a gradient that leaked across sequences, dropped a term or
+# mis-aligned the causal mask would miss them), by the softmax identity
+# sum_j dS_ij = 0 (so the keys' dK of one sequence and head sum to zero), and by the
+# rows that take no part in the loss.
+
+
+def _packed_loss(q, k, v, dout, cq, ck, causal, scale):
+    o, _ = oracle.attn_fwd_varlen(q, k, v, cq, ck, causal, scale)
+    return float(np.sum(o * dout))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_finite_differences(causal):
+    rng = np.random.default_rng(86)
+    lq, lk, H, d, scale, h = [2, 0, 3, 4], [3, 2, 1, 2], 2, 3, 0.7, 1e-6
+    q = rng.normal(size=(sum(lq), H, d))
+    k = rng.normal(size=(sum(lk), H, d))
+    v = rng.normal(size=(sum(lk), H, d))
+    dout = rng.normal(size=(sum(lq), H, d))
+    cq = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    ck = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
+    grads = oracle.attn_bwd_varlen(q, k, v, dout, cq, ck, causal, scale)
+    for x, g in zip((q, k, v), grads):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            x0 = x[idx]
+            x[idx] = x0 + h
+            lp = _packed_loss(q, k, v, dout, cq, ck, causal, scale)
+            x[idx] = x0 - h
+            lm = _packed_loss(q, k, v, dout, cq, ck, causal, scale)
+            x[idx] = x0
+            num[idx] = (lp - lm) / (2 * h)
+        assert np.max(np.abs(num - g)) <= 1e-6 * max(1.0, np.max(np.abs(g)))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_dk_sums_to_zero_per_sequence(causal):
+    lq, lk = [7, 20, 1], [9, 20, 5]
+    q, k, v, cq, ck = _pack(87, lq, lk, 2, 16)
+    dout = _f64(synth._normal(q.shape, 90))
+    _, dk, _ = oracle.attn_bwd_varlen(q, k, v, dout, cq, ck, causal, 0.25)
+    for b in range(3):
+        s = dk[ck[b]:ck[b + 1]].sum(axis=0)
+        assert np.max(np.abs(s)) <= 1e-12 * max(1.0, np.max(np.abs(dk)))
+
+
+def test_backward_rows_outside_the_loss_are_zero():
+    # sequence 0 has keys but no queries, sequence 1 queries but no keys, and the
+    # packed buffers end with rows that belong to no sequence
+    lq, lk = [0, 3, 4], [5, 0, 6]
+    q, k, v, cq, ck = _pack(88, lq + [2], lk + [3], 2, 8)
+    cq, ck = cq[:-1], ck[:-1]
+    dout = _f64(synth._normal(q.shape, 91))
+    dq, dk, dv = oracle.attn_bwd_varlen(q, k, v, dout, cq, ck, True, 0.3)
+    assert np.all(dk[0:5] == 0) and np.all(dv[0:5] == 0)
+    assert np.all(dq[0:3] == 0)
+    assert np.all(dq[7:] == 0) and np.all(dk[11:] == 0) and np.all(dv[11:] == 0)
+    assert np.any(dq[3:7] != 0) and np.any(dk[5:11] != 0) and np.any(dv[5:11] != 0)
