@@ -23,8 +23,9 @@ import threading
 import torch
 
 __all__ = [
-    "FAError", "lib_path", "load", "fa_fwd", "fa_bwd", "fa_decode_splitkv", "fa_decode_splitkv_noalloc", "fa_check",
-    "fa_fwd_workspace_size", "fa_bwd_workspace_size", "fa_decode_workspace_size", "fa_decode_num_splits",
+    "FAError", "lib_path", "load", "fa_fwd", "fa_bwd", "fa_fwd_varlen", "fa_bwd_varlen", "fa_decode_splitkv",
+    "fa_decode_splitkv_noalloc", "fa_decode_paged", "fa_check", "fa_fwd_workspace_size", "fa_bwd_workspace_size",
+    "fa_bwd_varlen_workspace_size", "fa_decode_workspace_size", "fa_decode_num_splits",
     "fa_version", "STATUS",
 ]
 
@@ -70,13 +71,16 @@ def load():
         lib.fa_decode_splitkv_noalloc.argtypes = [_vp] * 4 + [_i] * 6 + [_f, _i, _vp, _vp, _vp]
         lib.fa_decode_paged.argtypes = [_vp] * 5 + [_i] * 7 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
         lib.fa_fwd_varlen.argtypes = [_vp] * 7 + [_i] * 8 + [_f, _vp, _sz, _vp]
+        lib.fa_bwd_varlen.argtypes = [_vp] * 11 + [_i] * 8 + [_f, _vp, _sz, _vp]
         for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_decode_splitkv, lib.fa_decode_splitkv_noalloc,
-                   lib.fa_decode_paged, lib.fa_fwd_varlen):
+                   lib.fa_decode_paged, lib.fa_fwd_varlen, lib.fa_bwd_varlen):
             fn.restype = _i
         lib.fa_fwd_workspace_size.argtypes = [_i] * 5
         lib.fa_fwd_workspace_size.restype = _sz
         lib.fa_bwd_workspace_size.argtypes = [_i] * 5
         lib.fa_bwd_workspace_size.restype = _sz
+        lib.fa_bwd_varlen_workspace_size.argtypes = [_i] * 3
+        lib.fa_bwd_varlen_workspace_size.restype = _sz
         lib.fa_decode_workspace_size.argtypes = [_i] * 5
         lib.fa_decode_workspace_size.restype = _sz
         lib.fa_decode_num_splits.argtypes = [_i] * 5
@@ -103,6 +107,10 @@ def fa_fwd_workspace_size(B, H, Nq, Nk, d) -> int:
 
 def fa_bwd_workspace_size(B, H, Nq, Nk, d) -> int:
     return int(load().fa_bwd_workspace_size(B, H, Nq, Nk, d))
+
+
+def fa_bwd_varlen_workspace_size(H, total_q, d) -> int:
+    return int(load().fa_bwd_varlen_workspace_size(H, total_q, d))
 
 
 def fa_decode_workspace_size(B, H, max_seqlen_k, d, num_splits=0) -> int:
@@ -200,6 +208,8 @@ def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_se
         raise ValueError("k/v must be [total_k, H, d]")
     out = torch.empty_like(q) if out is None else out
     lse = torch.empty((H, total_q), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_tensor("out", out, torch.bfloat16, q.shape)
+    _check_tensor("lse", lse, torch.float32, (H, total_q))
     if ws is None:
         ws = workspace(lib.fa_fwd_workspace_size(1, H, 1, 1, d), q.device, "fwd")
     st = lib.fa_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens_q.data_ptr(),
@@ -229,6 +239,37 @@ def fa_bwd(q, k, v, o, dout, lse, causal: bool = False, softmax_scale=None, dq=N
                     dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, Nq, Nk, d, int(bool(causal)),
                     _scale(softmax_scale), ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
     _raise("fa_bwd", st)
+    return dq, dk, dv
+
+
+def fa_bwd_varlen(q, k, v, o, dout, lse, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                  causal: bool = False, softmax_scale=None, dq=None, dk=None, dv=None, ws=None):
+    """Backward over packed variable-length sequences (the inputs and lse of
+    fa_fwd_varlen).  Returns (dq [total_q, H, d], dk, dv [total_k, H, d]) in bf16."""
+    lib = load()
+    total_q, H, d = q.shape
+    total_k = k.shape[0]
+    B = cu_seqlens_q.shape[0] - 1
+    kshape = (total_k, H, d)
+    for name, t, shp in (("q", q, None), ("k", k, kshape), ("v", v, kshape), ("o", o, q.shape),
+                         ("dout", dout, q.shape)):
+        _check_tensor(name, t, torch.bfloat16, shp)
+    _check_tensor("lse", lse, torch.float32, (H, total_q))
+    _check_tensor("cu_seqlens_q", cu_seqlens_q, torch.int32, (B + 1,))
+    _check_tensor("cu_seqlens_k", cu_seqlens_k, torch.int32, (B + 1,))
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t, shp in (("dq", dq, q.shape), ("dk", dk, kshape), ("dv", dv, kshape)):
+        _check_tensor(name, t, torch.bfloat16, shp)
+    if ws is None:
+        ws = workspace(lib.fa_bwd_varlen_workspace_size(H, total_q, d), q.device, "bwd")
+    st = lib.fa_bwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), cu_seqlens_q.data_ptr(),
+                           cu_seqlens_k.data_ptr(), B, H, total_q, total_k, int(max_seqlen_q), int(max_seqlen_k), d,
+                           int(bool(causal)), _scale(softmax_scale), ws.data_ptr(), ws.numel(),
+                           _stream_ptr(q.device))
+    _raise("fa_bwd_varlen", st)
     return dq, dk, dv
 
 

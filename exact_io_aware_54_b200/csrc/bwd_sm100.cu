@@ -82,7 +82,60 @@ struct BwdArgs {
   unsigned long long timeout_ns;
   uint4* dk;  // [B, Nk, H, D] bf16, written directly by the d = 64 kernel
   uint4* dv;
+  // variable-length batch (cu_q != nullptr): the sequences are packed along the
+  // token axis of one batch element ([total, H, D]); Nq, Nk are the longest
+  // sequence's lengths.  stat_n is the row length of lse and D ([B, H, stat_n]:
+  // Nq when dense, total_q when packed).
+  const int32_t* cu_q;
+  const int32_t* cu_k;
+  int total_q, total_k;
+  int stat_n;
 };
+
+// Where sequence b lives.  Dense: batch element b of the [B, N, H, D] tensors.
+// Packed: rows cu[b] .. cu[b + 1] - 1 of batch element 0.  tq / tk are the first
+// query / key row along N, tb the batch coordinate; global token rows are
+// tb * Nq + tq + i (queries) and tb * Nk + tk + j (keys).  lq = -1 marks offsets that
+// do not fit the buffers (the sequence is skipped and the call reports a bad
+// argument).
+struct BwdSeq {
+  int lq, lk, tq, tk, tb;
+};
+__device__ __forceinline__ BwdSeq bwd_seq(const BwdArgs& a, int b) {
+  BwdSeq s;
+  if (a.cu_q == nullptr) {
+    s.lq = a.Nq;
+    s.lk = a.Nk;
+    s.tq = 0;
+    s.tk = 0;
+    s.tb = b;
+    return s;
+  }
+  const long long q0 = a.cu_q[b], q1 = a.cu_q[b + 1], k0 = a.cu_k[b], k1 = a.cu_k[b + 1];
+  const long long lq = min(q1 - q0, (long long)a.Nq), lk = min(k1 - k0, (long long)a.Nk);
+  s.tq = (int)q0;
+  s.tk = (int)k0;
+  s.tb = 0;
+  s.lq = (int)lq;
+  s.lk = (int)lk;
+  if (q0 < 0 || k0 < 0 || lq < 0 || lk < 0 || q0 + lq > a.total_q || k0 + lk > a.total_k) s.lq = -1;
+  return s;
+}
+
+// dK = dV = 0 for the keys of a tile that no query sees (a packed sequence with
+// keys but no queries): threads tid = 0 .. nthreads - 1 of the caller, 16-byte stores.
+template <int D>
+__device__ __forceinline__ void store_zero_dkv(const BwdArgs& a, const BwdSeq& s, int j, int h, int tid,
+                                               int nthreads) {
+  constexpr int kChunks = D / 8;  // 16-byte chunks per row
+  for (int idx = tid; idx < 2 * 128 * kChunks; idx += nthreads) {
+    const int c = idx % kChunks, row = (idx / kChunks) % 128, which = idx / (128 * kChunks);
+    const int key = j * 128 + row;
+    if (key < s.lk)
+      (which == 0 ? a.dk : a.dv)[((size_t)((long long)s.tb * a.Nk + s.tk + key) * a.H + h) * kChunks + c] =
+          make_uint4(0u, 0u, 0u, 0u);
+  }
+}
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
@@ -212,10 +265,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int j = blockIdx.x / bh_count;
   const int bh = blockIdx.x - j * bh_count;
   const int b = bh / a.H, h = bh - (bh / a.H) * a.H;
-  const int n_qtiles = (a.Nq + 127) >> 7;
+  const BwdSeq sq = bwd_seq(a, b);
+  if (sq.lq < 0) {  // block-uniform exits, before any barrier or tensor memory
+    if (threadIdx.x == 0) atomicExch(a.status, kStatusBadArg);
+    return;
+  }
+  if (j * 128 >= sq.lk) return;  // no key of this sequence in the tile
+  const int n_qtiles = (sq.lq + 127) >> 7;
   int i_first = 0;
-  if (a.causal) i_first = max(0, j * 128 - (a.Nk - a.Nq)) >> 7;
-  const int n_iters = n_qtiles - i_first;
+  if (a.causal) i_first = max(0, j * 128 - (sq.lk - sq.lq)) >> 7;
+  const int n_iters = n_qtiles - i_first;  // >= 1 when the sequence has queries
+  if (n_iters <= 0) {
+    store_zero_dkv<D>(a, sq, j, h, threadIdx.x, blockDim.x);
+    return;
+  }
+  // a packed sequence's partial last key tile is stored row by row: a tile store
+  // would run into the next sequence's rows
+  const bool direct_dkv = a.cu_q != nullptr && j * 128 + 128 > sq.lk;
 
   if (threadIdx.x == 0) {
     mbar_init(bar_kv_full, 1);
@@ -248,15 +314,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const size_t stat_row = ((size_t)b * a.H + h) * a.Nq;
+  const size_t stat_row = ((size_t)sq.tb * a.H + h) * a.stat_n + sq.tq;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer: TMA tiles + lse/D
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_kv_full, 2 * L::kTileBytes);
       for (int bx = 0; bx < L::kBoxes; ++bx) {
-        tma_load_4d(smem + L::kOffK + bx * L::kBoxBytes, &tmK, bar_kv_full, bx * 64, h, j * 128, b);
-        tma_load_4d(smem + L::kOffV + bx * L::kBoxBytes, &tmV, bar_kv_full, bx * 64, h, j * 128, b);
+        tma_load_4d(smem + L::kOffK + bx * L::kBoxBytes, &tmK, bar_kv_full, bx * 64, h, sq.tk + j * 128, sq.tb);
+        tma_load_4d(smem + L::kOffV + bx * L::kBoxBytes, &tmV, bar_kv_full, bx * 64, h, sq.tk + j * 128, sq.tb);
       }
     }
     for (int it = 0; it < n_iters; ++it) {
@@ -271,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = q0 + lane + 32 * e;
         nl2[e] = -INFINITY;
         nd[e] = 0.f;
-        if (q < a.Nq) {
+        if (q < sq.lq) {
           const float lse = a.lse[stat_row + q];
           nl2[e] = (lse == -INFINITY) ? -INFINITY : -lse * 1.4426950408889634f;
           nd[e] = -a.delta[stat_row + q];
@@ -287,9 +353,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive_expect_tx(bar_q_full + st, 2 * L::kTileBytes);
         for (int bx = 0; bx < L::kBoxes; ++bx) {
           tma_load_4d(smem + L::kOffQ + st * L::kTileBytes + bx * L::kBoxBytes, &tmQ, bar_q_full + st, bx * 64, h,
-                      q0, b);
+                      sq.tq + q0, sq.tb);
           tma_load_4d(smem + L::kOffDO + st * L::kTileBytes + bx * L::kBoxBytes, &tmDO, bar_q_full + st, bx * 64,
-                      h, q0, b);
+                      h, sq.tq + q0, sq.tb);
         }
       }
       float* stat = reinterpret_cast<float*>(smem + L::kOffStat) + st * 256;
@@ -367,10 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;
     const int key = j * 128 + r;
     const uint32_t lane_field = (quarter * 32) << 16;
-    const bool key_ok = key < a.Nk;
+    const bool key_ok = key < sq.lk;
     // first query that sees this key (a sentinel far below any query when not causal;
     // qmin - qs below must not overflow)
-    const int qmin = a.causal ? key - (a.Nk - a.Nq) : -(1 << 30);
+    const int qmin = a.causal ? key - (sq.lk - sq.lq) : -(1 << 30);
     bool ok = true;
 
     // dQ tile of query tile `it`: this group's D/2 columns, fp32 vector reductions
@@ -387,8 +453,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive_warp(bar_dq_empty);
       const int q = (i_first + it) * 128 + r;
-      if (q < a.Nq) {
-        float* dst = a.dq_acc + (((size_t)b * a.Nq + q) * a.H + h) * D + grp * (D / 2);
+      if (q < sq.lq) {
+        float* dst = a.dq_acc + ((size_t)((long long)sq.tb * a.Nq + sq.tq + q) * a.H + h) * D + grp * (D / 2);
 #pragma unroll
         for (int cc = 0; cc < D / 64; ++cc)
 #pragma unroll
@@ -421,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait(sv);
         reg_pin(dp);
         const uint32_t stat_u32 = sbase + L::kOffStat + st * 1024 + col * 4;
-        const bool tile_mask = (j * 128 + 128 > a.Nk) || (a.causal && (j * 128 + 127 - (a.Nk - a.Nq) > qs));
+        const bool tile_mask = (j * 128 + 128 > sq.lk) || (a.causal && (j * 128 + 127 - (sq.lk - sq.lq) > qs));
         uint32_t pk[16], dk2[16];
         if (tile_mask)
           ds_block<32, true>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2);
@@ -445,11 +511,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = drain_dq(it);
     }
     // ---------------------------------------------------------------- dK / dV epilogue
-    // group 0 stores dK (times scale) through the K tile's smem, group 1 dV through V's
+    // group 0 stores dK (times scale) through the K tile's smem, group 1 dV through V's;
+    // with direct_dkv each thread writes its key row straight to global memory
     if (ok && warp_wait_b(bar_dkv_done, 0, a.timeout_ns) && !*abort_flag) {
       tc_fence_after();
       const uint32_t src = tmem + lane_field + (grp == 0 ? L::kTmDK : L::kTmDV);
       const uint32_t dst = sbase + (grp == 0 ? L::kOffK : L::kOffV);
+      uint4* gdst = (grp == 0 ? a.dk : a.dv) + ((size_t)((long long)sq.tb * a.Nk + sq.tk + key) * a.H + h) * (D / 8);
       const float mul = grp == 0 ? a.scale : 1.f;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -460,27 +528,32 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           const int chunk = (cc & 1) * 4 + q4;
-          const uint32_t addr = dst + box * L::kBoxBytes + r * 128 + ((chunk ^ (r & 7)) << 4);
           const float* f = reinterpret_cast<const float*>(o) + q4 * 8;
-          st_shared_v4(addr, pack_bf16x2(f[0] * mul, f[1] * mul), pack_bf16x2(f[2] * mul, f[3] * mul),
-                       pack_bf16x2(f[4] * mul, f[5] * mul), pack_bf16x2(f[6] * mul, f[7] * mul));
+          const uint4 w = make_uint4(pack_bf16x2(f[0] * mul, f[1] * mul), pack_bf16x2(f[2] * mul, f[3] * mul),
+                                     pack_bf16x2(f[4] * mul, f[5] * mul), pack_bf16x2(f[6] * mul, f[7] * mul));
+          if (!direct_dkv)
+            st_shared_v4(dst + box * L::kBoxBytes + r * 128 + ((chunk ^ (r & 7)) << 4), w.x, w.y, w.z, w.w);
+          else if (key_ok)
+            gdst[cc * 4 + q4] = w;
         }
       }
-      fence_proxy_async_smem();
-      mbar_arrive_warp(bar_epi);
-      if (warp == 2 && lane == 0) {
-        if (mbar_wait(bar_epi, 0, a.timeout_ns)) {
-          for (int bx = 0; bx < L::kBoxes; ++bx) {
-            tma_store_4d(&tmDK, smem + L::kOffK + bx * L::kBoxBytes, bx * 64, h, j * 128, b);
-            tma_store_4d(&tmDV, smem + L::kOffV + bx * L::kBoxBytes, bx * 64, h, j * 128, b);
+      if (!direct_dkv) {
+        fence_proxy_async_smem();
+        mbar_arrive_warp(bar_epi);
+        if (warp == 2 && lane == 0) {
+          if (mbar_wait(bar_epi, 0, a.timeout_ns)) {
+            for (int bx = 0; bx < L::kBoxes; ++bx) {
+              tma_store_4d(&tmDK, smem + L::kOffK + bx * L::kBoxBytes, bx * 64, h, sq.tk + j * 128, sq.tb);
+              tma_store_4d(&tmDV, smem + L::kOffV + bx * L::kBoxBytes, bx * 64, h, sq.tk + j * 128, sq.tb);
+            }
+            bulk_commit_group();
+            bulk_wait_group0();
+          } else {
+            bwd_timeout(a.status, abort_flag);
           }
-          bulk_commit_group();
-          bulk_wait_group0();
-        } else {
-          bwd_timeout(a.status, abort_flag);
         }
+        __syncwarp();
       }
-      __syncwarp();
     } else if (lane == 0) {
       bwd_timeout(a.status, abort_flag);
     }
@@ -550,7 +623,7 @@ struct PipeLayout {
 // warps 0-3: TMA producer, score MMA issuer, gradient MMA issuer, idle; 4-7: dQ drain;
 // 8-15: dS (two column groups)
 constexpr int kPipeThreads = 512;
-constexpr uint32_t kPipeRegsCtl = 72, kPipeRegsDrain = 80, kPipeRegsDs = 176;
+constexpr uint32_t kPipeRegsCtl = 72, kPipeRegsDrain = 88, kPipeRegsDs = 176;
 static_assert(128 * kPipeRegsCtl + 128 * kPipeRegsDrain + 256 * kPipeRegsDs <= kPipeThreads * 128,
               "register split exceeds the launch budget");
 
@@ -572,42 +645,60 @@ __device__ __forceinline__ int pipe_item_index(int k) {
   const int g = gridDim.x;
   return k * g + ((k & 1) ? (g - 1 - (int)blockIdx.x) : (int)blockIdx.x);
 }
+// n = number of query tiles; n = 0 for a tile of keys that no query sees (their dK
+// and dV are zero), n = -1 for a tile past the sequence's last key or a sequence
+// with bad offsets.  Only items with n > 0 take part in the pipeline, and the
+// barrier phases of every role count those items alone.
 struct PipeItem {
-  int j, b, h, i_first, n;
+  int j, h, i_first, n;
+  BwdSeq s;
 };
 __device__ __forceinline__ PipeItem pipe_item(const BwdArgs& a, int w) {
   PipeItem it;
   const int bh_count = a.B * a.H;
   it.j = w / bh_count;
   const int bh = w - it.j * bh_count;
-  it.b = bh / a.H;
-  it.h = bh - it.b * a.H;
-  const int n_qtiles = (a.Nq + 127) >> 7;
-  it.i_first = a.causal ? (max(0, it.j * 128 - (a.Nk - a.Nq)) >> 7) : 0;
+  const int b = bh / a.H;
+  it.h = bh - b * a.H;
+  it.s = bwd_seq(a, b);
+  it.i_first = 0;
+  it.n = -1;
+  if (it.s.lq < 0 || it.j * 128 >= it.s.lk) return it;
+  const int n_qtiles = (it.s.lq + 127) >> 7;
+  it.i_first = a.causal ? (max(0, it.j * 128 - (it.s.lk - it.s.lq)) >> 7) : 0;
   it.n = n_qtiles - it.i_first;
   return it;
 }
 
-// Walks the query tiles of this CTA's items in order.
+// Walks the query tiles of this CTA's items (those with query tiles) in order.
 struct PipeCursor {
-  int k;  // item counter of this CTA
+  int k;  // item index of this CTA (pipe_item_index)
+  int u;  // items with query tiles passed so far
   int t;  // query tile within the item
   bool valid;
   PipeItem itm;
+  // from item k on, the first item with query tiles
+  __device__ __forceinline__ void seek(const BwdArgs& a, int n_items) {
+    for (;; ++k) {
+      const int w = pipe_item_index(k);
+      valid = w < n_items;
+      if (!valid) return;
+      itm = pipe_item(a, w);
+      if (itm.n > 0) return;
+    }
+  }
   __device__ __forceinline__ void start(const BwdArgs& a, int n_items) {
     k = 0;
+    u = 0;
     t = 0;
-    const int w = pipe_item_index(0);
-    valid = w < n_items;
-    if (valid) itm = pipe_item(a, w);
+    seek(a, n_items);
   }
   __device__ __forceinline__ void advance(const BwdArgs& a, int n_items) {
     if (++t < itm.n) return;
     t = 0;
     ++k;
-    const int w = pipe_item_index(k);
-    valid = w < n_items;
-    if (valid) itm = pipe_item(a, w);
+    ++u;
+    seek(a, n_items);
   }
 };
 
@@ -615,14 +706,14 @@ struct PipeCursor {
 // four query rows per lane, negated so that the dS warps add them.
 __device__ __forceinline__ void pipe_load_stats(const BwdArgs& a, const PipeCursor& c, uint32_t lane, float (&nl2)[4],
                                                 float (&nd)[4]) {
-  const size_t stat_row = ((size_t)c.itm.b * a.H + c.itm.h) * a.Nq;
+  const size_t stat_row = ((size_t)c.itm.s.tb * a.H + c.itm.h) * a.stat_n + c.itm.s.tq;
   const int q0 = (c.itm.i_first + c.t) * 128;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     const int q = q0 + lane + 32 * e;
     nl2[e] = -INFINITY;
     nd[e] = 0.f;
-    if (q < a.Nq) {
+    if (q < c.itm.s.lq) {
       const float lse = a.lse[stat_row + q];
       nl2[e] = (lse == -INFINITY) ? -INFINITY : -lse * 1.4426950408889634f;
       nd[e] = -a.delta[stat_row + q];
@@ -711,9 +802,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         pipe_load_stats(a, cur, lane, nl2, nd);
         if (lane == 0) {  // the first item's K and V
           mbar_arrive_expect_tx(bar_k_full, L::kTileBytes);
-          tma_load_4d(smem + L::kOffK, &tmK, bar_k_full, 0, cur.itm.h, cur.itm.j * 128, cur.itm.b);
+          tma_load_4d(smem + L::kOffK, &tmK, bar_k_full, 0, cur.itm.h, cur.itm.s.tk + cur.itm.j * 128, cur.itm.s.tb);
           mbar_arrive_expect_tx(bar_v_full, L::kTileBytes);
-          tma_load_4d(smem + L::kOffV, &tmV, bar_v_full, 0, cur.itm.h, cur.itm.j * 128, cur.itm.b);
+          tma_load_4d(smem + L::kOffV, &tmV, bar_v_full, 0, cur.itm.h, cur.itm.s.tk + cur.itm.j * 128, cur.itm.s.tb);
         }
       }
       for (int T = 0; cur.valid && ok; ++T) {
@@ -732,8 +823,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         }
         if (lane == 0) {
           mbar_arrive_expect_tx(bar_q_full + st, 2 * L::kTileBytes);
-          tma_load_4d(smem + L::kOffQ + st * L::kTileBytes, &tmQ, bar_q_full + st, 0, cur.itm.h, q0, cur.itm.b);
-          tma_load_4d(smem + L::kOffDO + st * L::kTileBytes, &tmDO, bar_q_full + st, 0, cur.itm.h, q0, cur.itm.b);
+          tma_load_4d(smem + L::kOffQ + st * L::kTileBytes, &tmQ, bar_q_full + st, 0, cur.itm.h, cur.itm.s.tq + q0,
+                      cur.itm.s.tb);
+          tma_load_4d(smem + L::kOffDO + st * L::kTileBytes, &tmDO, bar_q_full + st, 0, cur.itm.h,
+                      cur.itm.s.tq + q0, cur.itm.s.tb);
         }
         float* stat = reinterpret_cast<float*>(smem + L::kOffStat) + st * 256;
 #pragma unroll
@@ -746,18 +839,19 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         if (cur.t + 1 == cur.itm.n && nxt.valid) {
           // the last query tile of item u is staged: load item u + 1's K (into the slot
           // item u - 1 used) and V (once item u's last dP^T has read it)
-          const int u1 = cur.k + 1;
+          const int u1 = cur.u + 1;
           if (lane == 0) {
             got = (u1 < 2 || mbar_wait(bar_k_free + (u1 & 1), ((u1 >> 1) - 1) & 1, a.timeout_ns)) && !*abort_flag;
             if (got) {
               mbar_arrive_expect_tx(bar_k_full + (u1 & 1), L::kTileBytes);
               tma_load_4d(smem + L::kOffK + (u1 & 1) * L::kTileBytes, &tmK, bar_k_full + (u1 & 1), 0, nxt.itm.h,
-                          nxt.itm.j * 128, nxt.itm.b);
-              got = mbar_wait(bar_v_free, cur.k & 1, a.timeout_ns) && !*abort_flag;
+                          nxt.itm.s.tk + nxt.itm.j * 128, nxt.itm.s.tb);
+              got = mbar_wait(bar_v_free, cur.u & 1, a.timeout_ns) && !*abort_flag;
             }
             if (got) {
               mbar_arrive_expect_tx(bar_v_full, L::kTileBytes);
-              tma_load_4d(smem + L::kOffV, &tmV, bar_v_full, 0, nxt.itm.h, nxt.itm.j * 128, nxt.itm.b);
+              tma_load_4d(smem + L::kOffV, &tmV, bar_v_full, 0, nxt.itm.h, nxt.itm.s.tk + nxt.itm.j * 128,
+                          nxt.itm.s.tb);
             }
           }
           if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) {
@@ -785,8 +879,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       int T = 0, u = 0;
       if (warp == 1) {
         // ------------------------------------------------------------ score MMAs
-        for (int w; (w = pipe_item_index(u)) < n_items && ok; ++u) {
+        for (int k = 0, w; (w = pipe_item_index(k)) < n_items && ok; ++k) {
           const PipeItem itm = pipe_item(a, w);
+          if (itm.n <= 0) continue;
           const int ks = u & 1;
           if (!mbar_wait(bar_k_full + ks, (u >> 1) & 1, a.timeout_ns) || !mbar_wait(bar_v_full, u & 1, a.timeout_ns) ||
               *abort_flag) {
@@ -807,12 +902,14 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
             umma_commit(bar_s_full);
             if (t + 1 == itm.n) umma_commit(bar_v_free);  // the item's last dP^T has been issued
           }
+          ++u;
         }
         if (!ok) bwd_timeout(a.status, abort_flag);
       } else {
         // ------------------------------------------------------------ gradient MMAs
-        for (int w; (w = pipe_item_index(u)) < n_items && ok; ++u) {
+        for (int k = 0, w; (w = pipe_item_index(k)) < n_items && ok; ++k) {
           const PipeItem itm = pipe_item(a, w);
+          if (itm.n <= 0) continue;
           const int ks = u & 1;
           for (int t = 0; t < itm.n; ++t, ++T) {
             const int st = T % L::kQStages;
@@ -846,6 +943,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
               umma_commit(bar_dkv_done);     // dK and dV of this item are complete
             }
           }
+          ++u;
         }
         if (!ok) {
           bwd_timeout(a.status, abort_flag);
@@ -890,8 +988,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         for (int k = 0; k < 8; ++k) {
           const int row = 4 * k + rr_sub;
           const float4 v = ld_shared_f4(scratch + row * 128 + ((cc ^ (row & 7)) << 4));
-          if (q0 + row < a.Nq)
-            red_add_v4(a.dq_acc + (((size_t)cur.itm.b * a.Nq + q0 + row) * a.H + cur.itm.h) * D + half * 32 + cc * 4,
+          if (q0 + row < cur.itm.s.lq)
+            red_add_v4(a.dq_acc +
+                           ((size_t)((long long)cur.itm.s.tb * a.Nq + cur.itm.s.tq + q0 + row) * a.H + cur.itm.h) * D +
+                           half * 32 + cc * 4,
                        v.x, v.y, v.z, v.w);
         }
         __syncwarp();
@@ -909,13 +1009,21 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     const int col = 64 * grp;
     bool ok = true;
     int T = 0, u = 0;
-    for (int w; (w = pipe_item_index(u)) < n_items && ok; ++u) {
+    for (int k = 0, w; (w = pipe_item_index(k)) < n_items && ok; ++k) {
       const PipeItem itm = pipe_item(a, w);
+      if (itm.n <= 0) {
+        if (itm.s.lq < 0) {
+          if (threadIdx.x == 256) atomicExch(a.status, kStatusBadArg);
+        } else if (itm.n == 0) {
+          store_zero_dkv<D>(a, itm.s, itm.j, itm.h, threadIdx.x - 256, 256);
+        }
+        continue;
+      }
       const int key = itm.j * 128 + r;
-      const bool key_ok = key < a.Nk;
-      const int qmin = a.causal ? key - (a.Nk - a.Nq) : -(1 << 30);
-      const bool key_tail = itm.j * 128 + 128 > a.Nk;
-      const int last_key_qmin = itm.j * 128 + 127 - (a.Nk - a.Nq);
+      const bool key_ok = key < itm.s.lk;
+      const int qmin = a.causal ? key - (itm.s.lk - itm.s.lq) : -(1 << 30);
+      const bool key_tail = itm.j * 128 + 128 > itm.s.lk;
+      const int last_key_qmin = itm.j * 128 + 127 - (itm.s.lk - itm.s.lq);
       for (int t = 0; t < itm.n; ++t, ++T) {
         const int st = T % L::kQStages;
         const int db = T % L::kDsBufs;
@@ -992,7 +1100,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       mbar_arrive_warp(bar_acc_free);  // the next item may restart dK / dV
       if (key_ok) {
         const float mul = grp == 0 ? a.scale : 1.f;
-        uint4* dst = (grp == 0 ? a.dk : a.dv) + (((size_t)itm.b * a.Nk + key) * a.H + itm.h) * (D / 8);
+        uint4* dst =
+            (grp == 0 ? a.dk : a.dv) + ((size_t)((long long)itm.s.tb * a.Nk + itm.s.tk + key) * a.H + itm.h) * (D / 8);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const uint32_t* f = (c < 4 ? o0 : o1) + (c & 3) * 8;
@@ -1002,6 +1111,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
                               pack_bf16x2(__uint_as_float(f[6]) * mul, __uint_as_float(f[7]) * mul));
         }
       }
+      ++u;
     }
     if (!ok && lane == 0) bwd_timeout(a.status, abort_flag);
   }
@@ -1081,24 +1191,29 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
     if (e != cudaSuccess) return FA_ERR_CUDA;
     attr_done[dev] = true;
   }
+  // A packed batch is one batch element of total rows for the tensor maps, the
+  // preprocess and the convert kernels; the main kernels find each sequence's rows.
+  const bool varlen = L0.cu_q != nullptr;
+  const int mB = varlen ? 1 : L0.B;
+  const int mNq = varlen ? L0.total_q : L0.Nq, mNk = varlen ? L0.total_k : L0.Nk;
   // 1. D rows and a zeroed dQ accumulator
   {
-    const long long rows = (long long)L0.B * L0.Nq * L0.H;
+    const long long rows = (long long)mB * mNq * L0.H;
     const long long threads = rows * (D / 8);
     const int grid = (int)((threads + 255) / 256);
     prof_before(stream, kKBwdPre);
     bwd_preprocess_kernel<D><<<grid, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(L0.o),
                                                          static_cast<const __nv_bfloat16*>(L0.dout), L0.delta,
-                                                         L0.dq_acc, L0.B, L0.H, L0.Nq);
+                                                         L0.dq_acc, mB, L0.H, mNq);
     const cudaError_t err = cudaGetLastError();
     prof_after(stream, kKBwdPre);
     if (err != cudaSuccess) return FA_ERR_CUDA;
   }
   // 2. main kernel
   CUtensorMap tq, tk, tv, tdo, tdk, tdv;
-  if (!encode_bshd_map(&tq, L0.q, L0.B, L0.Nq, L0.H, D) || !encode_bshd_map(&tk, L0.k, L0.B, L0.Nk, L0.H, D) ||
-      !encode_bshd_map(&tv, L0.v, L0.B, L0.Nk, L0.H, D) || !encode_bshd_map(&tdo, L0.dout, L0.B, L0.Nq, L0.H, D) ||
-      !encode_bshd_map(&tdk, L0.dk, L0.B, L0.Nk, L0.H, D) || !encode_bshd_map(&tdv, L0.dv, L0.B, L0.Nk, L0.H, D))
+  if (!encode_bshd_map(&tq, L0.q, mB, mNq, L0.H, D) || !encode_bshd_map(&tk, L0.k, mB, mNk, L0.H, D) ||
+      !encode_bshd_map(&tv, L0.v, mB, mNk, L0.H, D) || !encode_bshd_map(&tdo, L0.dout, mB, mNq, L0.H, D) ||
+      !encode_bshd_map(&tdk, L0.dk, mB, mNk, L0.H, D) || !encode_bshd_map(&tdv, L0.dv, mB, mNk, L0.H, D))
     return FA_ERR_CUDA;
   BwdArgs a;
   a.lse = L0.lse;
@@ -1116,6 +1231,11 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   a.timeout_ns = L0.timeout_ns;
   a.dk = static_cast<uint4*>(L0.dk);
   a.dv = static_cast<uint4*>(L0.dv);
+  a.cu_q = L0.cu_q;
+  a.cu_k = L0.cu_k;
+  a.total_q = L0.total_q;
+  a.total_k = L0.total_k;
+  a.stat_n = mNq;
   const long long grid = (long long)a.n_kv_tiles * L0.B * L0.H;
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   prof_before(stream, kKBwdMain);
@@ -1130,7 +1250,7 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   if (err_main != cudaSuccess) return FA_ERR_CUDA;
   // 3. dQ = scale * accumulator in bf16
   {
-    const long long n8 = (long long)L0.B * L0.Nq * L0.H * D / 8;
+    const long long n8 = (long long)mB * mNq * L0.H * D / 8;
     const int grid3 = (int)std::min<long long>((n8 + 255) / 256, (long long)num_sms() * 16);
     prof_before(stream, kKBwdConvert);
     bwd_convert_kernel<<<grid3, 256, 0, stream>>>(L0.dq_acc, static_cast<__nv_bfloat16*>(L0.dq), n8, L0.scale);

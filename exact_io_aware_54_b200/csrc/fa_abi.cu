@@ -173,6 +173,11 @@ size_t fa_bwd_workspace_size(int B, int H, int Nq, int Nk, int d) {
   return kStatusBytes + up256(sizeof(float) * (size_t)B * Nq * H * d) + up256(sizeof(float) * (size_t)B * H * Nq);
 }
 
+size_t fa_bwd_varlen_workspace_size(int H, int total_q, int d) {
+  // a packed batch is one batch element of total_q rows for the workspace arrays
+  return fa_bwd_workspace_size(1, H, total_q, 1, d);
+}
+
 int fa_decode_num_splits(int B, int H, int max_seqlen_k, int d, int num_splits) {
   if (B <= 0 || H <= 0 || max_seqlen_k < 0 || (d != 64 && d != 128) || num_splits < 0) return 0;
   return decode_plan(B, H, max_seqlen_k, d, num_splits).splits;
@@ -275,6 +280,55 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   a.H = H;
   a.Nq = Nq;
   a.Nk = Nk;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.scale = resolve_scale(softmax_scale, d);
+  a.timeout_ns = wait_timeout_ns();
+  return launch_bwd(a, stream);
+}
+
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,
+                        void* dq, void* dk, void* dv, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
+                        int H, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d, int causal,
+                        float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (!q || !k || !v || !o || !do_ || !lse || !dq || !dk || !dv || !cu_seqlens_q || !cu_seqlens_k)
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || max_seqlen_q <= 0 || max_seqlen_k <= 0 || !dims_ok(1, H, total_q, total_k, d))
+    return FA_ERR_INVALID_ARG;
+  // row coordinates of a tile (first row + up to 255) stay in 32 bits; the key-tile
+  // grid fits one launch dimension
+  if ((long long)total_q + 256 >= (1LL << 31) || (long long)total_k + 256 >= (1LL << 31) ||
+      (long long)((max_seqlen_k + 127) / 128) * B * H >= (1LL << 31))
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(do_) || !aligned16(lse) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(cu_seqlens_q) & 3u) ||
+      (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u))
+    return FA_ERR_ALIGNMENT;
+  if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_varlen_workspace_size(H, total_q, d))
+    return FA_ERR_WORKSPACE;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  BwdLaunch a;
+  a.q = q;
+  a.k = k;
+  a.v = v;
+  a.o = o;
+  a.dout = do_;
+  a.lse = lse;
+  a.dq = dq;
+  a.dk = dk;
+  a.dv = dv;
+  a.status = reinterpret_cast<int*>(ws);
+  a.dq_acc = reinterpret_cast<float*>(ws + kStatusBytes);
+  a.delta = reinterpret_cast<float*>(ws + kStatusBytes + up256(sizeof(float) * (size_t)total_q * H * d));
+  a.cu_q = cu_seqlens_q;
+  a.cu_k = cu_seqlens_k;
+  a.total_q = total_q;
+  a.total_k = total_k;
+  a.B = B;
+  a.H = H;
+  a.Nq = max_seqlen_q;
+  a.Nk = max_seqlen_k;
   a.d = d;
   a.causal = causal ? 1 : 0;
   a.scale = resolve_scale(softmax_scale, d);

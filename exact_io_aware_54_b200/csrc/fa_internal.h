@@ -70,9 +70,14 @@ struct BwdLaunch {
   void* dq;
   void* dk;
   void* dv;
-  float* dq_acc;  // [B, Nq, H, d] fp32
-  float* delta;   // [B, H, Nq] fp32
+  float* dq_acc;  // [B, Nq, H, d] fp32 ([total_q, H, d] when packed)
+  float* delta;   // [B, H, Nq] fp32 ([H, total_q] when packed)
   int* status;
+  // variable-length batch (cu_q != nullptr): q, o, dout, dq are [total_q, H, d],
+  // k, v, dk, dv [total_k, H, d], lse [H, total_q]; Nq, Nk are the maximum lengths
+  const int32_t* cu_q = nullptr;
+  const int32_t* cu_k = nullptr;
+  int total_q = 0, total_k = 0;
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;

@@ -127,6 +127,30 @@ FA_API fa_status fa_bwd(const void* q, const void* k, const void* v, const void*
                  cudaStream_t stream);
 
 /*
+ * Backward pass of fa_fwd_varlen: the gradients of sum(O * dO) over a packed
+ * batch, sequence by sequence (the recompute form of fa_bwd; "AI Bible 13",
+ * section 03).
+ *   q, o, do_, dq : [total_q, H, d] bf16 (dq written), rows of sequence b are
+ *                   cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1
+ *   k, v, dk, dv  : [total_k, H, d] bf16 (dk, dv written), rows
+ *                   cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1
+ *   lse           : [H, total_q] fp32 as written by fa_fwd_varlen with the same
+ *                   arguments
+ *   cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k : as fa_fwd_varlen
+ *   workspace     : at least fa_bwd_varlen_workspace_size(H, total_q, d) bytes
+ *                   (fp32 dQ accumulator [total_q, H, d], D [H, total_q], status)
+ * dK and dV of a sequence with no queries are zero, as is dQ of a sequence with
+ * no keys.  dq rows past the last sequence are zero; dk / dv rows past the last
+ * sequence are not written.  Offsets that do not fit the buffers are handled as
+ * in fa_fwd_varlen (skipped, FA_ERR_INVALID_ARG from fa_check).
+ */
+FA_API fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* do_,
+                               const float* lse, void* dq, void* dk, void* dv, const int32_t* cu_seqlens_q,
+                               const int32_t* cu_seqlens_k, int B, int H, int total_q, int total_k,
+                               int max_seqlen_q, int max_seqlen_k, int d, int causal, float softmax_scale,
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Split-KV decode over a ragged, packed KV cache.
  *   q           : [B, H, d] bf16 (one query row per sequence: Nq must be 1)
  *   k, v        : [total_kv, H, d] bf16; sequence b owns rows
@@ -202,6 +226,7 @@ FA_API fa_status fa_decode_splitkv_noalloc(const void* q, const void* k, const v
 /* Workspace sizes in bytes for the calls above (0 when the arguments are invalid). */
 FA_API size_t fa_fwd_workspace_size(int B, int H, int Nq, int Nk, int d);
 FA_API size_t fa_bwd_workspace_size(int B, int H, int Nq, int Nk, int d);
+FA_API size_t fa_bwd_varlen_workspace_size(int H, int total_q, int d);
 FA_API size_t fa_decode_workspace_size(int B, int H, int max_seqlen_k, int d, int num_splits);
 
 /*

@@ -151,6 +151,31 @@ def test_fwd_varlen_argument_validation(lib):
     assert call(ws=None) == ST["FA_ERR_WORKSPACE"]
 
 
+def test_bwd_varlen_argument_validation(lib):
+    def call(**kw):
+        a = dict(q=P, k=P, v=P, o=P, do=P, lse=P, dq=P, dk=P, dv=P, cq=P, ck=P, B=3, H=4, tq=300, tk=400, mq=200,
+                 mk=300, d=64, ws=P, wsb=1 << 30)
+        a.update(kw)
+        return lib.fa_bwd_varlen(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"], a["dv"],
+                                 a["cq"], a["ck"], a["B"], a["H"], a["tq"], a["tk"], a["mq"], a["mk"], a["d"], 1,
+                                 0.0, a["ws"], a["wsb"], None)
+
+    assert call(ck=None) == ST["FA_ERR_INVALID_ARG"]
+    assert call(dk=None) == ST["FA_ERR_INVALID_ARG"]
+    assert call(tq=0) == ST["FA_ERR_INVALID_ARG"]
+    assert call(mk=0) == ST["FA_ERR_INVALID_ARG"]
+    assert call(B=0) == ST["FA_ERR_INVALID_ARG"]
+    assert call(tq=(1 << 31) - 100, H=1) == ST["FA_ERR_INVALID_ARG"]
+    assert call(d=96) == ST["FA_ERR_UNSUPPORTED"]
+    assert call(dv=P + 8) == ST["FA_ERR_ALIGNMENT"]
+    assert call(cq=P + 2) == ST["FA_ERR_ALIGNMENT"]
+    assert call(ws=None) == ST["FA_ERR_WORKSPACE"]
+    need = fa.fa_bwd_varlen_workspace_size(4, 300, 64)
+    assert need >= 4 * 300 * 4 * 64 + 4 * 4 * 300  # fp32 dQ accumulator + D rows
+    assert call(wsb=need - 1) == ST["FA_ERR_WORKSPACE"]
+    assert fa.fa_bwd_varlen_workspace_size(4, 300, 80) == 0
+
+
 def test_selftest_argument_validation(lib):
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint, ctypes.c_void_p]
     assert lib.fa_selftest_wait_timeout(None, 256, 100, None) == ST["FA_ERR_WORKSPACE"]
