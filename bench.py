@@ -364,7 +364,22 @@ def _extra_prefill_varlen(out, iters, fa, synth, dev, pk):
                                     "frac_of_peak": round(tf / pk["bf16_tflops"], 4), "sequences": 16,
                                     "total_tokens": total, "max_seqlen": maxL,
                                     "l2": "no flush: Q, K, V together are 779 MB, 6x the L2"}
-    del q, k, v, o, lse, cu
+    # the backward of the same packed batch (O and lse from the forward above)
+    do = synth.prefill_inputs(synth.SEEDS["prefill8k"] + 1, 1, total, total, 32, 128,
+                              device=dev)[0].reshape(total, 32, 128)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def g(i):
+        fa.fa_bwd_varlen(q, k, v, o, do, lse, cu, cu, maxL, maxL, causal=True, dq=dq, dk=dk, dv=dv)
+    for i in range(3):
+        g(i)
+    ms_b = device_time_ms(g, max(10, iters // 2))
+    tf_b = sum(bwd_flops(1, 32, int(L), int(L), 128, True) for L in lengths) / (ms_b * 1e-3) / 1e12
+    out["prefill_varlen_causal_bwd"] = {"ms": round(ms_b, 4), "TFLOP/s": round(tf_b, 1),
+                                        "frac_of_peak": round(tf_b / pk["bf16_tflops"], 4),
+                                        "kernels": "preprocess + main + dQ convert",
+                                        "l2": "no flush: Q, K, V, O, dO together are 1.3 GB, 10x the L2"}
+    del q, k, v, o, lse, cu, do, dq, dk, dv
     torch.cuda.empty_cache()
 
 
