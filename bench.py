@@ -164,6 +164,26 @@ def committed_traffic(kernel):
         return None
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def shard_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own shard of independent problems (weak scaling)."""
+    return seed + 1000 * rank
+
+
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """The slowest rank's time; every rank takes this collective, in the same order."""
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank_step: float, ms_max: float, scale: float = 1e12) -> float:
+    """Units all ranks processed per second (divided by `scale`), timed by the slowest rank."""
+    return world * units_per_rank_step / (ms_max * 1e-3) / scale
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, local_rank):
@@ -174,7 +194,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     B, H, N, d, causal = (WORKLOAD[k] for k in ("B", "H", "N", "d", "causal"))
     B = args.batch or B
-    q, k, v, do = synth.prefill_inputs(synth.SEEDS["gpt2m"] + 1000 * rank, B, N, N, H, d, with_dout=True,
+    q, k, v, do = synth.prefill_inputs(shard_seed(synth.SEEDS["gpt2m"], rank), B, N, N, H, d, with_dout=True,
                                        device=dev)
     o = torch.empty_like(q)
     lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
@@ -202,12 +222,9 @@ def run_ours(args, rank, world, local_rank):
     clocks = sampler.stop()
     kernels = profile_kernels(fa)
 
-    t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    ms_max = float(t.item())
+    ms_max = max_over_ranks(ms, world, dev)
     step_flops = fwd_flops(B, H, N, N, d, causal) + bwd_flops(B, H, N, N, d, causal)
-    value = world * step_flops / (ms_max * 1e-3) / 1e12
+    value = whole_job_rate(world, step_flops, ms_max)
 
     pk, pk_src = peaks()
     # roofline of the dominant kernel (largest device time in the timed region)
@@ -259,13 +276,11 @@ def run_ours(args, rank, world, local_rank):
         e2e_step()
         n_e2e = max(3, min(args.steps, 10))
         e_ms = device_time_ms(e2e_step, n_e2e)
-        et = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            torch.distributed.all_reduce(et, op=torch.distributed.ReduceOp.MAX)
+        e_max = max_over_ranks(e_ms, world, dev)
         hin = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
         hout = sum(x.numel() * x.element_size() for x in (hdq, hdk, hdv))
-        e2e = {"value": round(world * step_flops / (float(et.item()) * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-               "h2d_bytes_per_step": hin, "d2h_bytes_per_step": hout, "ms_per_step": round(float(et.item()), 4)}
+        e2e = {"value": round(whole_job_rate(world, step_flops, e_max), 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": hin, "d2h_bytes_per_step": hout, "ms_per_step": round(e_max, 4)}
         del hq, hk, hv, hdo, hdq, hdk, hdv, dq2, dk2, dv2, q2, k2, v2, do2
 
     extra = run_extra(args, fa, synth, dev, pk) if (rank == 0 and not args.no_extra) else None
@@ -518,8 +533,9 @@ def cpu_baseline(seconds):
                       f"fp64 fwd + bwd, {el:.1f} s of oracle time"}
 
 
-def run_reference(args, rank):
-    """The oracle as it stands, one bounded sample of the workload per step."""
+def run_reference(args, rank, world=1):
+    """The oracle as it stands, one bounded sample of the workload per step, on rank
+    0's host cores; the other ranks of a multi-GPU launch return without work."""
     if rank != 0:
         return None
     import oracle
@@ -537,7 +553,7 @@ def run_reference(args, rank):
     sample = f"{heads} whole head(s) of one batch element per step ({done} heads in total), fp64 fwd + bwd"
     cpu = {"value": round(value, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
            "sample": sample}
-    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": 1,
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * t_el / args.steps, 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic (seeded N(0,1) bf16, widened to fp64)",
@@ -578,7 +594,7 @@ def main():
         return
 
     if args.impl == "reference":
-        line = run_reference(args, rank)
+        line = run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
         return
