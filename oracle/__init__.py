@@ -14,6 +14,9 @@ definitions and the passages of the pages they follow:
   two block states);
 * the Flash Attention wiki note, "Safe Softmax" (max, sum, normalise);
 * "AI Bible 13", section 03 (the backward keeps O and the row statistics).
+
+``oracle/masked.py`` (numpy, fp64) adds the key-padding mask and dropout with a
+Philox4x32-10 random mask, forward and backward.
 """
 from __future__ import annotations
 
