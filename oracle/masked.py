@@ -13,6 +13,10 @@ module takes the plain textbook reading:
 * key-padding mask: key j of batch element b takes part iff key_mask[b, j]; it is
   excluded like a causally masked key (its score is -inf), on top of the causal
   mask when both are set.  A row with no key left has O = 0 and lse = -inf.
+* block-sparse attention (the block-sparse variant the second page credits with
+  reaching 64K tokens, "AI Bible 13", section 05): a 0/1 matrix over (query
+  block, key block) of block_q x block_k elements; a zero block excludes all its
+  keys from its queries, on top of the other masks.
 * dropout with probability p acts on the normalised probabilities: with the
   statistics m, l and lse of the undropped row,
       O_i = sum_j P_ij z_ij v_j,   z_ij = keep_ij / (1 - p_eff),
@@ -83,14 +87,30 @@ def dropout_scale(p: float, b, h, i, j, seed: int):
     return keep * (65536.0 / (65536.0 - t))
 
 
-def _visible(Nq, Nk, causal, key_mask_b):
+def _visible(Nq, Nk, causal, key_mask_b, block_mask_bh=None, block=(128, 128)):
     """[Nq, Nk] boolean: key j takes part in row i."""
     vis = np.ones((Nq, Nk), dtype=bool)
     if causal:
         vis &= np.arange(Nk)[None, :] <= np.arange(Nq)[:, None] + (Nk - Nq)
     if key_mask_b is not None:
         vis &= np.asarray(key_mask_b, dtype=bool)[None, :]
+    if block_mask_bh is not None:
+        bm = np.asarray(block_mask_bh, dtype=bool)
+        vis &= bm[np.arange(Nq)[:, None] // block[0], np.arange(Nk)[None, :] // block[1]]
     return vis
+
+
+def _block_mask_of(block_mask, b, h):
+    """The [n_qblocks, n_kblocks] mask of head (b, h) from a [nq, nk], [H, nq, nk]
+    or [B, H, nq, nk] array (None: no block mask)."""
+    if block_mask is None:
+        return None
+    bm = np.asarray(block_mask)
+    if bm.ndim == 2:
+        return bm
+    if bm.ndim == 3:
+        return bm[h]
+    return bm[b, h]
 
 
 def _head_probs(qh, kh, scale, vis):
@@ -108,8 +128,11 @@ def _head_probs(qh, kh, scale, vis):
     return p, lse
 
 
-def attn_fwd_masked(q, k, v, causal: bool, scale: float, key_mask=None, dropout_p: float = 0.0, seed: int = 0):
-    """q [B, Nq, H, d], k, v [B, Nk, H, d]; key_mask [B, Nk] bool or None ->
+def attn_fwd_masked(q, k, v, causal: bool, scale: float, key_mask=None, dropout_p: float = 0.0, seed: int = 0,
+                    block_mask=None, block=(128, 128)):
+    """q [B, Nq, H, d], k, v [B, Nk, H, d]; key_mask [B, Nk] bool or None; block_mask
+    over (query block, key block) of `block` = (block_q, block_k) elements, shared
+    ([nq, nk]), per head ([H, nq, nk]) or per (b, h) ([B, H, nq, nk]), or None ->
     (o [B, Nq, H, d], lse [B, H, Nq]) in fp64."""
     q, k, v = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
     B, Nq, H, d = q.shape
@@ -118,8 +141,9 @@ def attn_fwd_masked(q, k, v, causal: bool, scale: float, key_mask=None, dropout_
     lse = np.full((B, H, Nq), -np.inf)
     ii, jj = np.meshgrid(np.arange(Nq), np.arange(Nk), indexing="ij")
     for b in range(B):
-        vis = _visible(Nq, Nk, causal, None if key_mask is None else key_mask[b])
         for h in range(H):
+            vis = _visible(Nq, Nk, causal, None if key_mask is None else key_mask[b],
+                           _block_mask_of(block_mask, b, h), block)
             p, lse[b, h] = _head_probs(q[b, :, h], k[b, :, h], scale, vis)
             z = dropout_scale(dropout_p, b, h, ii, jj, seed)
             o[b, :, h] = (p * z) @ v[b, :, h]
@@ -127,7 +151,7 @@ def attn_fwd_masked(q, k, v, causal: bool, scale: float, key_mask=None, dropout_
 
 
 def attn_bwd_masked(q, k, v, dout, causal: bool, scale: float, key_mask=None, dropout_p: float = 0.0,
-                    seed: int = 0):
+                    seed: int = 0, block_mask=None, block=(128, 128)):
     """Gradients of sum(O * dout) for `attn_fwd_masked`; returns (dq, dk, dv) in fp64."""
     q, k, v, dout = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dout))
     B, Nq, H, d = q.shape
@@ -135,8 +159,9 @@ def attn_bwd_masked(q, k, v, dout, causal: bool, scale: float, key_mask=None, dr
     dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
     ii, jj = np.meshgrid(np.arange(Nq), np.arange(Nk), indexing="ij")
     for b in range(B):
-        vis = _visible(Nq, Nk, causal, None if key_mask is None else key_mask[b])
         for h in range(H):
+            vis = _visible(Nq, Nk, causal, None if key_mask is None else key_mask[b],
+                           _block_mask_of(block_mask, b, h), block)
             p, _ = _head_probs(q[b, :, h], k[b, :, h], scale, vis)
             z = dropout_scale(dropout_p, b, h, ii, jj, seed)
             do = dout[b, :, h]

@@ -187,3 +187,70 @@ def test_row_term_identity_with_dropout():
     dp = z * (dout[0, :, 0] @ v[0, :, 0].T)
     np.testing.assert_allclose((pr * dp).sum(axis=1), (dout[0, :, 0] * o[0, :, 0]).sum(axis=1), rtol=1e-12,
                                atol=1e-12)
+
+
+# ---------------------------------------------------------------- block-sparse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_all_ones_block_mask_changes_nothing(causal):
+    q, k, v, _ = _rng_inputs(10, 2, 20, 20, 2, 8)
+    bm = np.ones((3, 3), dtype=bool)
+    o, lse = masked.attn_fwd_masked(q, k, v, causal, 0.3, block_mask=bm, block=(8, 8))
+    o2, lse2 = masked.attn_fwd_masked(q, k, v, causal, 0.3)
+    assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+
+
+def test_block_diagonal_mask_is_attention_within_each_block():
+    q, k, v, _ = _rng_inputs(11, 1, 24, 24, 2, 8)
+    bm = np.eye(3, dtype=bool)  # blocks of 8: three independent 8-token problems
+    o, lse = masked.attn_fwd_masked(q, k, v, False, 0.5, block_mask=bm, block=(8, 8))
+    for blk in range(3):
+        sl = slice(8 * blk, 8 * blk + 8)
+        ob, lb = oracle.attn_fwd(q[:, sl], k[:, sl], v[:, sl], False, 0.5)
+        np.testing.assert_allclose(o[:, sl], ob, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[:, :, sl], lb, rtol=1e-13, atol=1e-12)
+
+
+def test_column_pattern_equals_the_key_mask():
+    q, k, v, _ = _rng_inputs(12, 1, 12, 16, 3, 4)
+    cols = np.array([True, False, True, True])  # key blocks of 4
+    bm = np.tile(cols, (3, 1))  # 3 query blocks of 4
+    o, lse = masked.attn_fwd_masked(q, k, v, True, 0.6, block_mask=bm, block=(4, 4))
+    o2, lse2 = masked.attn_fwd_masked(q, k, v, True, 0.6, key_mask=np.repeat(cols, 4)[None, :])
+    assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+
+
+def test_per_head_block_masks():
+    q, k, v, _ = _rng_inputs(13, 1, 8, 8, 2, 4)
+    bm = np.array([[[1, 0], [1, 1]], [[1, 1], [0, 1]]], dtype=bool)  # [H, 2, 2], blocks of 4
+    o, _ = masked.attn_fwd_masked(q, k, v, False, 0.5, block_mask=bm, block=(4, 4))
+    for h in range(2):
+        oh, _ = masked.attn_fwd_masked(q[:, :, h:h + 1], k[:, :, h:h + 1], v[:, :, h:h + 1], False, 0.5,
+                                       block_mask=bm[h], block=(4, 4))
+        assert np.array_equal(o[:, :, h], oh[:, :, 0])
+    # head 0, query block 0 sees only key block 0: a 4-key problem
+    ob, _ = oracle.attn_fwd(q[:, :4, :1], k[:, :4, :1], v[:, :4, :1], False, 0.5)
+    np.testing.assert_allclose(o[:, :4, :1], ob, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_sparse_backward_finite_differences(causal):
+    q, k, v, dout = _rng_inputs(14, 1, 6, 6, 1, 3)
+    bm = np.array([[1, 0, 1], [1, 1, 0], [0, 1, 1]], dtype=bool)  # blocks of 2
+    args = dict(block_mask=bm, block=(2, 2), dropout_p=0.25, seed=4)
+    grads = masked.attn_bwd_masked(q, k, v, dout, causal, 0.9, **args)
+    h = 1e-6
+    for x, g in zip((q, k, v), grads):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            x0 = x[idx]
+            x[idx] = x0 + h
+            lp = float(np.sum(masked.attn_fwd_masked(q, k, v, causal, 0.9, **args)[0] * dout))
+            x[idx] = x0 - h
+            lm = float(np.sum(masked.attn_fwd_masked(q, k, v, causal, 0.9, **args)[0] * dout))
+            x[idx] = x0
+            num[idx] = (lp - lm) / (2 * h)
+        assert np.max(np.abs(num - g)) <= 1e-6 * max(1.0, np.max(np.abs(g)))
