@@ -148,11 +148,18 @@ __device__ __forceinline__ SeqView seq_view(const FwdArgs& a, int b) {
   }
   v.qoff = a.cu_q[b];
   v.koff = a.cu_k[b];
-  v.lq = min(a.cu_q[b + 1] - v.qoff, a.Nq);
-  v.lk = min(a.cu_k[b + 1] - v.koff, a.Nk);
+  const int q1 = a.cu_q[b + 1], k1 = a.cu_k[b + 1];
   v.bc = 0;
-  if (v.qoff < 0 || v.koff < 0 || v.lq < 0 || v.lk < 0 || v.qoff + v.lq > a.total_q || v.koff + v.lk > a.total_k)
+  // no expression below can wrap: ends are compared with starts before they are
+  // subtracted, and the fit is checked against total - start (both non-negative)
+  if (v.qoff < 0 || v.koff < 0 || q1 < v.qoff || k1 < v.koff) {
     v.lq = -1;
+    v.lk = 0;
+    return v;
+  }
+  v.lq = min(q1 - v.qoff, a.Nq);
+  v.lk = min(k1 - v.koff, a.Nk);
+  if (v.lq > a.total_q - v.qoff || v.lk > a.total_k - v.koff) v.lq = -1;
   return v;
 }
 

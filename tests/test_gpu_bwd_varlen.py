@@ -139,3 +139,26 @@ def test_offsets_outside_the_buffers_are_reported(d):
     compare_grad(f64(dq[:100]), rq, "dQ[seq 0]")
     compare_grad(f64(dk[:100]), rk, "dK[seq 0]")
     compare_grad(f64(dv[:100]), rv, "dV[seq 0]")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_offsets_that_would_wrap_32_bit_arithmetic_are_reported(d):
+    """Key offsets near 2^31 and a negative end: those sequences are skipped and
+    recorded; dK / dV rows outside sequence 0 keep their fill."""
+    q, k, v, do, cq, ck = _inputs(2100 + d, [100, 50, 50], [100, 50, 50], 2, d)
+    qc, kc, vc, dc = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o, lse = fa_fwd_varlen(qc, kc, vc, cq.cuda(), ck.cuda(), 100, 100, causal=False)
+    torch.cuda.synchronize()
+    ws = workspace(256, torch.device("cuda"), "bwd")
+    assert fa_check(ws) == 0
+    bad_k = torch.tensor([0, 100, 2 ** 31 - 5, -2 ** 31], dtype=torch.int32, device="cuda")
+    dk = torch.full_like(kc, 7.0)
+    dv = torch.full_like(vc, 7.0)
+    dq, dk, dv = fa_bwd_varlen(qc, kc, vc, o, dc, lse, cq.cuda(), bad_k, 100, 150, causal=False, dk=dk, dv=dv)
+    assert fa_check(ws) == FA_ERR_INVALID_ARG
+    assert torch.all(dk[100:] == 7.0) and torch.all(dv[100:] == 7.0)
+    rq, rk, rv = oracle.attn_bwd_varlen(f64(q)[:100], f64(k)[:100], f64(v)[:100], f64(do)[:100], np.array([0, 100]),
+                                        np.array([0, 100]), False, default_scale(d))
+    compare_grad(f64(dq[:100]), rq, "dQ[seq 0]")
+    compare_grad(f64(dk[:100]), rk, "dK[seq 0]")
+    compare_grad(f64(dv[:100]), rv, "dV[seq 0]")

@@ -87,3 +87,21 @@ def test_offsets_outside_the_buffers_are_reported():
                                             np.array([0, 100]), False, default_scale(64))
     compare_o(f64(o)[:100], o_ref)
     compare_lse(f64(lse)[:, :100], lse_ref)
+
+
+def test_offsets_that_would_wrap_32_bit_arithmetic_are_reported():
+    """Sequence 1 ends near 2^31 and sequence 2 starts there and ends at -2^31: both
+    are skipped and recorded, and no row outside sequence 0 is written."""
+    q, k, v, cq, ck = _inputs(1510, [100, 50, 50], [100, 50, 50], 2, 64)
+    bad_q = torch.tensor([0, 100, 2 ** 31 - 5, -2 ** 31], dtype=torch.int32, device="cuda")
+    ws = workspace(256, torch.device("cuda"), "fwd")
+    assert fa_check(ws) == 0
+    o = torch.full((200, 2, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((2, 200), 7.0, dtype=torch.float32, device="cuda")
+    fa_fwd_varlen(q.cuda(), k.cuda(), v.cuda(), bad_q, ck.cuda(), 150, 100, causal=True, out=o, lse=lse)
+    assert fa_check(ws) == FA_ERR_INVALID_ARG
+    assert torch.all(o[100:] == 7.0) and torch.all(lse[:, 100:] == 7.0)
+    o_ref, lse_ref = oracle.attn_fwd_varlen(f64(q)[:100], f64(k)[:100], f64(v)[:100], np.array([0, 100]),
+                                            np.array([0, 100]), True, default_scale(64))
+    compare_o(f64(o)[:100], o_ref)
+    compare_lse(f64(lse)[:, :100], lse_ref)
