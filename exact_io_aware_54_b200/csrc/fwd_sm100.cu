@@ -59,8 +59,8 @@ namespace {
 
 constexpr int kThreads = 384;
 // Register split: launched at 168 per thread (384 x 168 = 64512); the producer /
-// MMA warpgroup drops to 56 and the two softmax warpgroups rise to 224:
-// 128 x 56 + 256 x 224 = 64512.
+// MMA warpgroup drops to 80 and the two softmax warpgroups rise to 208:
+// 128 x 80 + 256 x 208 = 63488.
 constexpr uint32_t kRegsLow = 80, kRegsHigh = 208;
 static_assert(128 * kRegsLow + 256 * kRegsHigh <= 384 * 168, "register split exceeds the launch budget");
 constexpr uint32_t kTmemCols = 512;
