@@ -155,8 +155,11 @@ FA_API fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, cons
  *   q           : [B, H, d] bf16 (one query row per sequence: Nq must be 1)
  *   k, v        : [total_kv, H, d] bf16; sequence b owns rows
  *                 cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1
- *   cu_seqlens_k: device int32 [B+1], non-decreasing, cu_seqlens_k[0] = 0
- *                 (validated on the device only when FA_CHECKS=1)
+ *   cu_seqlens_k: device int32 [B+1], non-decreasing, cu_seqlens_k[0] = 0,
+ *                 cu_seqlens_k[B] <= total_kv.  This is a precondition: the
+ *                 call has no total_kv to check the last bound against, and
+ *                 offsets that break it make the kernel read outside k and v.
+ *                 FA_CHECKS=1 checks the order on the device first.
  *   max_seqlen_k: an upper bound of every sequence length (plays the role of Nk)
  *   num_splits  : chunks per sequence; 0 picks a value from the shape
  *   o           : [B, H, d] bf16 (written);  lse : [B, H] fp32 (written)
@@ -237,9 +240,11 @@ FA_API int fa_decode_num_splits(int B, int H, int max_seqlen_k, int d, int num_s
 
 /*
  * Synchronises `stream` and reads the status word that the kernels of the
- * previous call(s) with this workspace recorded.  Returns FA_OK, FA_ERR_TIMEOUT
- * (a bounded wait ran out), FA_ERR_INVALID_ARG (FA_CHECKS=1 found malformed
- * cu_seqlens) or FA_ERR_CUDA.
+ * previous call(s) with this workspace recorded, then clears it.  Returns FA_OK,
+ * FA_ERR_TIMEOUT (a bounded wait ran out), FA_ERR_INVALID_ARG (an argument the
+ * kernels found bad: variable-length offsets outside the buffers, a paged-decode
+ * page index outside the cache, or, with FA_CHECKS=1, decode cu_seqlens out of
+ * order) or FA_ERR_CUDA.
  */
 FA_API fa_status fa_check(void* workspace, cudaStream_t stream);
 
