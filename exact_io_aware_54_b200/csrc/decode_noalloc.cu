@@ -59,6 +59,7 @@ extern "C" fa_status fa_decode_splitkv_noalloc(const void* q, const void* k, con
                                                const int32_t* cu_seqlens_k, int B, int H, int Nq,
                                                int max_seqlen_k, int d, int causal, float softmax_scale,
                                                int num_splits, void* o, float* lse, cudaStream_t stream) {
+  const NvtxRange range("fa_decode_splitkv_noalloc");
   (void)causal;  // one query row: the bottom-right aligned mask admits every key
   if (!q || !k || !v || !cu_seqlens_k || !o || !lse) return FA_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || Nq != 1 || max_seqlen_k < 0 || num_splits < 0) return FA_ERR_INVALID_ARG;

@@ -191,6 +191,7 @@ size_t fa_decode_workspace_size(int B, int H, int max_seqlen_k, int d, int num_s
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
                  int d, int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
                  cudaStream_t stream) {
+  const NvtxRange range("fa_fwd");
   if (!q || !k || !v || !o || !lse || !dims_ok(B, H, Nq, Nk, d)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
@@ -218,6 +219,7 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, const int32
                         const int32_t* cu_seqlens_k, void* o, float* lse, int B, int H, int total_q, int total_k,
                         int max_seqlen_q, int max_seqlen_k, int d, int causal, float softmax_scale, void* workspace,
                         size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_fwd_varlen");
   if (!q || !k || !v || !cu_seqlens_q || !cu_seqlens_k || !o || !lse) return FA_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || total_q <= 0 || total_k <= 0 || max_seqlen_q <= 0 || max_seqlen_k <= 0)
     return FA_ERR_INVALID_ARG;
@@ -254,6 +256,7 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, const int32
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,
                  void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d, int causal,
                  float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_bwd");
   if (!q || !k || !v || !o || !do_ || !lse || !dq || !dk || !dv || !dims_ok(B, H, Nq, Nk, d))
     return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
@@ -291,6 +294,7 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
                         void* dq, void* dk, void* dv, const int32_t* cu_seqlens_q, const int32_t* cu_seqlens_k, int B,
                         int H, int total_q, int total_k, int max_seqlen_q, int max_seqlen_k, int d, int causal,
                         float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_bwd_varlen");
   if (!q || !k || !v || !o || !do_ || !lse || !dq || !dk || !dv || !cu_seqlens_q || !cu_seqlens_k)
     return FA_ERR_INVALID_ARG;
   if (B <= 0 || max_seqlen_q <= 0 || max_seqlen_k <= 0 || !dims_ok(1, H, total_q, total_k, d))
@@ -339,6 +343,7 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
 fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_k, int B, int H,
                             int Nq, int max_seqlen_k, int d, int causal, float softmax_scale, int num_splits, void* o,
                             float* lse, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_decode_splitkv");
   (void)causal;  // one query row: the bottom-right aligned mask admits every key
   if (!q || !k || !v || !cu_seqlens_k || !o || !lse) return FA_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || Nq != 1 || max_seqlen_k < 0 || num_splits < 0) return FA_ERR_INVALID_ARG;
@@ -386,6 +391,7 @@ fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_page
                           const int32_t* seqlens_k, int B, int H, int num_pages, int page_size, int max_pages_per_seq,
                           int max_seqlen_k, int d, float softmax_scale, int num_splits, void* o, float* lse,
                           void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_decode_paged");
   if (!q || !k_pages || !v_pages || !block_table || !seqlens_k || !o || !lse) return FA_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || num_pages <= 0 || page_size <= 0 || max_pages_per_seq <= 0 || max_seqlen_k < 0 ||
       num_splits < 0)

@@ -8,9 +8,20 @@
 
 #include <algorithm>
 
+#include <nvtx3/nvToolsExt.h>  // header-only NVTX v3: a range costs a pointer check unless a profiler listens
+
 #include "fa.h"  // include/ (on the compiler include path)
 
 namespace fa {
+
+// An NVTX range named after the entry point, open for the duration of the call,
+// so that a profiler's timeline shows which library call launched which kernels.
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Workspace: the first kStatusBytes hold the status word (int32) and padding.
 constexpr size_t kStatusBytes = 256;
