@@ -66,3 +66,49 @@ def rounding_floor(o_ref):
 
 def default_scale(d):
     return 1.0 / math.sqrt(d)
+
+
+class OAccumulator:
+    """O compared over a whole tensor that is checked slice by slice: the maximum and
+    the mean of |o_gpu - o_oracle| are taken over every element of every slice."""
+
+    def __init__(self, what="O"):
+        self.what, self.max, self.sum, self.n = what, 0.0, 0.0, 0
+
+    def add(self, o_gpu, o_ref):
+        o_gpu = np.asarray(o_gpu, dtype=np.float64)
+        o_ref = np.asarray(o_ref, dtype=np.float64)
+        assert o_gpu.shape == o_ref.shape, (o_gpu.shape, o_ref.shape)
+        assert np.all(np.isfinite(o_gpu)), f"{self.what}: non-finite values"
+        err = np.abs(o_gpu - o_ref)
+        self.max = max(self.max, float(err.max(initial=0.0)))
+        self.sum += float(err.sum())
+        self.n += err.size
+
+    def check(self, mean_tol=O_MEAN_ABS, max_tol=O_MAX_ABS):
+        mean = self.sum / max(self.n, 1)
+        assert self.max <= max_tol, f"{self.what}: max abs err {self.max:.3e} > {max_tol}"
+        assert mean <= mean_tol, f"{self.what}: mean abs err {mean:.3e} > {mean_tol}"
+        return self.max, mean
+
+
+class GradAccumulator:
+    """One gradient tensor compared slice by slice: max |g_gpu - g_oracle| over the
+    whole tensor, normalised by max |g_oracle| over the whole tensor."""
+
+    def __init__(self, what):
+        self.what, self.err, self.scale, self.n = what, 0.0, 0.0, 0
+
+    def add(self, g_gpu, g_ref):
+        g_gpu = np.asarray(g_gpu, dtype=np.float64)
+        g_ref = np.asarray(g_ref, dtype=np.float64)
+        assert g_gpu.shape == g_ref.shape, (g_gpu.shape, g_ref.shape)
+        assert np.all(np.isfinite(g_gpu)), f"{self.what}: non-finite values"
+        self.err = max(self.err, float(np.abs(g_gpu - g_ref).max(initial=0.0)))
+        self.scale = max(self.scale, float(np.abs(g_ref).max(initial=0.0)))
+        self.n += g_gpu.size
+
+    def check(self):
+        rel = self.err / max(self.scale, GRAD_FLOOR)
+        assert rel <= GRAD_REL, f"{self.what}: normalised max err {rel:.3e} > {GRAD_REL}"
+        return rel

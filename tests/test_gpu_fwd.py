@@ -1,11 +1,10 @@
 """GPU parity of fa_fwd against the fp64 oracle (through the C ABI binding)."""
-import numpy as np
 import pytest
 import torch
 
 import oracle
 from exact_io_aware_54_b200 import fa_check, fa_fwd, synth, workspace
-from tests._harness import compare_lse, compare_o, default_scale, f64, rounding_floor
+from tests._harness import OAccumulator, compare_lse, compare_o, default_scale, f64, rounding_floor
 
 pytestmark = pytest.mark.gpu
 
@@ -65,35 +64,39 @@ def test_explicit_scale():
     _full_check(1, 300, 300, 2, 64, True, 4242, scale=0.37)
 
 
-def _sampled_rows_check(B, N, H, d, causal, seed, n_heads=6, n_rows=48):
+def _whole_tensor_check(B, N, H, d, causal, seed, batch_chunk=None):
+    """Every element of O and LSE of the workload against the oracle on the same
+    inputs; nothing is subsampled.  The oracle runs on `batch_chunk` batch elements
+    at a time (to bound host memory); O's max and mean errors are taken over the
+    whole tensor."""
     q, k, v = synth.prefill_inputs(seed, B, N, N, H, d, device="cuda")
     o, lse = fa_fwd(q, k, v, causal=causal)
     torch.cuda.synchronize()
     assert fa_check(workspace(256, q.device, "fwd")) == 0
-    g = np.random.default_rng(seed)
-    heads = [(0, 0), (B - 1, H - 1)] + [(int(g.integers(B)), int(g.integers(H))) for _ in range(n_heads - 2)]
-    for b, h in heads:
-        rows = np.unique(np.concatenate([[0, 1, 127, 128, N - 1], g.integers(0, N, n_rows)]))
-        kk, vv = f64(k[b, :, h]), f64(v[b, :, h])
-        o_ref, lse_ref = oracle.attn_fwd_rows(f64(q[b, rows, h]), rows, kk, vv, N, causal, default_scale(d))
-        compare_o(f64(o[b, rows, h]), o_ref, what=f"O[b={b},h={h}]")
-        compare_lse(f64(lse[b, h, rows]), lse_ref, what=f"LSE[b={b},h={h}]")
+    acc = OAccumulator()
+    step = batch_chunk or B
+    for b0 in range(0, B, step):
+        sl = slice(b0, min(B, b0 + step))
+        o_ref, lse_ref = oracle.attn_fwd(f64(q[sl]), f64(k[sl]), f64(v[sl]), causal, default_scale(d))
+        acc.add(f64(o[sl]), o_ref)
+        compare_lse(f64(lse[sl]), lse_ref, what=f"LSE[b={b0}..]")
+    acc.check()
 
 
-def test_gpt2_medium_shape_sampled():
-    """B=64, H=16, N=1024, d=64, causal: sampled rows of sampled heads."""
-    _sampled_rows_check(64, 1024, 16, 64, True, synth.SEEDS["gpt2m"])
+def test_gpt2_medium_shape_whole_tensor():
+    """B=64, H=16, N=1024, d=64, causal (seed 54002): all of O and LSE."""
+    _whole_tensor_check(64, 1024, 16, 64, True, synth.SEEDS["gpt2m"], batch_chunk=8)
 
 
 @pytest.mark.parametrize("causal", [True, False])
-def test_long_prefill_sampled(causal):
-    """B=1, H=32, N=8192, d=128 (causal and non-causal): sampled rows."""
-    _sampled_rows_check(1, 8192, 32, 128, causal, synth.SEEDS["prefill8k"], n_heads=4, n_rows=24)
+def test_long_prefill_whole_tensor(causal):
+    """B=1, H=32, N=8192, d=128, causal and non-causal (seed 54003): all of O and LSE."""
+    _whole_tensor_check(1, 8192, 32, 128, causal, synth.SEEDS["prefill8k"])
 
 
-def test_long_sequence_sampled():
-    """B=1, H=16, N=16384, d=64, causal: sampled rows."""
-    _sampled_rows_check(1, 16384, 16, 64, True, synth.SEEDS["long16k"], n_heads=3, n_rows=16)
+def test_long_sequence_whole_tensor():
+    """B=1, H=16, N=16384, d=64, causal (seed 54005): all of O and LSE."""
+    _whole_tensor_check(1, 16384, 16, 64, True, synth.SEEDS["long16k"])
 
 
 def test_deterministic_and_reentrant():
