@@ -5,8 +5,11 @@ One step = forward + recompute backward of causal multi-head attention at the
 GPT-2-medium attention shape (B=64, H=16, N=1024, d=64, bf16), the workload the
 headline metric is quoted on.  The value is algorithmic TFLOP/s of the whole job:
 (4 + 10) * B * H * d * (causal pairs) per step, summed over ranks, divided by the
-slowest rank's device time.  The other workloads (long prefill, decode, long
-training sequence) are timed once each and reported under "extra".
+slowest rank's device time; the K steps are timed back to back with an event after
+each step (median / p10 / p90 of the step times under "step_time").  The other
+workloads (long prefill, variable-length prefill, decode, long training
+sequence) are timed launch by launch, each launch between its own pair of events
+with L2 flushed before it, and reported under "extra".
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -67,7 +70,7 @@ def peaks():
 
 class ClockSampler:
     """SM clock, power and clock-event (throttle) reasons sampled through NVML every
-    20 ms while active (the data nvidia-smi's clocks query shows)."""
+    5 ms while active (the data nvidia-smi's clocks query shows)."""
 
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4}
@@ -98,7 +101,7 @@ class ClockSampler:
                     self.samples.append((sm, rs, pw))
                 except Exception:
                     pass
-                time.sleep(0.02)
+                time.sleep(0.005)
 
         self._thread = threading.Thread(target=loop, daemon=True)
         self._thread.start()
@@ -119,6 +122,7 @@ class ClockSampler:
 # ----------------------------------------------------------------------------- timing helpers
 
 def device_time_ms(fn, iters, stream=None):
+    """Mean device time of `iters` back-to-back calls, one event pair around the loop."""
     stream = stream or torch.cuda.current_stream()
     s = torch.cuda.Event(enable_timing=True)
     e = torch.cuda.Event(enable_timing=True)
@@ -129,6 +133,60 @@ def device_time_ms(fn, iters, stream=None):
     e.record(stream)
     torch.cuda.synchronize()
     return s.elapsed_time(e) / iters
+
+
+class L2Flush:
+    """Writes a buffer of twice the L2 size, so that the next launch finds none of its
+    inputs in L2.  The write also keeps the GPU busy while the host enqueues the
+    launch that follows, so a launch's start event is not taken while the GPU waits
+    for the host."""
+
+    def __init__(self, device):
+        self.buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
+        self.n = 0
+
+    def __call__(self):
+        self.n += 1
+        self.buf.fill_(self.n & 0xFF)
+
+
+def quantiles(ms):
+    xs = sorted(ms)
+    n = len(xs)
+    return {"median_ms": round(statistics.median(xs), 5), "p10_ms": round(xs[n // 10], 5),
+            "p90_ms": round(xs[min(n - 1, (9 * n) // 10)], 5), "mean_ms": round(sum(xs) / n, 5), "launches": n}
+
+
+def per_launch_ms(fn, n, flush=None, stream=None):
+    """Device time of each of `n` calls, each bracketed by its own pair of events on the
+    launching stream; with `flush`, L2 is flushed before every call (outside the
+    events).  Returns the times in ms, in call order."""
+    stream = stream or torch.cuda.current_stream()
+    evs = []
+    for i in range(n):
+        if flush is not None:
+            flush()
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        fn(i)
+        e.record(stream)
+        evs.append((s, e))
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in evs]
+
+
+def timed_steps(fn, k, stream=None):
+    """K back-to-back steps with an event before the first and after every step: the
+    total (first to last event) and the K per-step times."""
+    stream = stream or torch.cuda.current_stream()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(k + 1)]
+    evs[0].record(stream)
+    for i in range(k):
+        fn(i)
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    return evs[0].elapsed_time(evs[k]), [evs[i].elapsed_time(evs[i + 1]) for i in range(k)]
 
 
 def profile_kernels(fa):
@@ -214,12 +272,27 @@ def run_ours(args, rank, world, local_rank):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
     fa.load().fa_profile_start()
-    ms = device_time_ms(step, args.steps)
+    total_ms, step_ms = timed_steps(step, args.steps)
     fa.load().fa_profile_stop()
+    ms = total_ms / args.steps
     if world > 1:
         torch.distributed.barrier()
+    timed_samples = len(sampler.samples)
+    # The same step keeps running (untimed) until at least one second has passed
+    # since the timed region began, so that the clock record holds enough samples
+    # of this workload even when the timed region itself is short.
+    soak = 0
+    while time.perf_counter() - t_wall0 < 1.0:
+        for _ in range(20):
+            step()
+        soak += 20
+        torch.cuda.synchronize()
     clocks = sampler.stop()
+    if clocks is not None:
+        clocks.update({"timed_region_samples": timed_samples, "soak_steps_after_timed_region": soak,
+                       "window_s": round(time.perf_counter() - t_wall0, 3)})
     kernels = profile_kernels(fa)
 
     ms_max = max_over_ranks(ms, world, dev)
@@ -302,62 +375,77 @@ def run_ours(args, rank, world, local_rank):
                    "frac_of_peak": round(value / world / pk["bf16_tflops"], 4),
                    "l2": "no flush: the inputs of one step (Q, K, V, O, dO: 640 MiB) exceed the 126 MB L2",
                    "parallelism": f"replicas x{world} (independent shards, no collective)"},
+        "step_time": quantiles(step_ms),
         "roofline": roofline, "kernels": per_kernel, "cpu_baseline": cpu_base, "e2e": e2e,
         "gpu_launches": launches, "clocks": clocks, "extra": extra,
     }
     return line
 
 
-def _rotating(make, total_bytes_of_one):
-    """Enough input sets that consecutive iterations never find their inputs in L2."""
-    n = max(2, math.ceil(3 * L2_BYTES / max(1, total_bytes_of_one)))
-    return [make(i) for i in range(n)]
-
-
 EXTRA_WORKLOADS = ("prefill8k", "prefill_varlen", "decode_single", "decode_batched", "decode_paged", "long16k")
 
 
 def run_extra(args, fa, synth, dev, pk, only=None):
+    """The other workloads, each timed launch by launch: L2 flushed before every
+    launch (outside its events), at least `--extra-launches` launches after warm-up,
+    median / p10 / p90 reported; rates use the median."""
     out = {}
-    iters = max(5, min(args.steps, 40))
+    n = max(50, args.extra_launches)
+    flush = L2Flush(dev)
     want = (lambda name: only is None or only == name)
     if want("prefill8k"):
-        _extra_prefill(out, iters, fa, synth, dev, pk)
+        _extra_prefill(out, n, flush, fa, synth, dev, pk)
     if want("prefill_varlen"):
-        _extra_prefill_varlen(out, iters, fa, synth, dev, pk)
+        _extra_prefill_varlen(out, n, flush, fa, synth, dev, pk)
     if want("decode_single"):
-        _extra_decode_single(out, iters, fa, synth, dev, pk)
+        _extra_decode_single(out, n, flush, fa, synth, dev, pk)
     if want("decode_batched"):
-        _extra_decode_batched(out, iters, fa, synth, dev, pk)
+        _extra_decode_batched(out, n, flush, fa, synth, dev, pk)
     if want("decode_paged"):
-        _extra_decode_paged(out, iters, fa, synth, dev, pk)
+        _extra_decode_paged(out, n, flush, fa, synth, dev, pk)
     if want("long16k"):
-        _extra_long16k(out, iters, fa, synth, dev, pk)
+        _extra_long16k(out, n, flush, fa, synth, dev, pk)
+    del flush
+    torch.cuda.empty_cache()
     return out
 
 
-def _extra_prefill(out, iters, fa, synth, dev, pk):
+def _timed(fn, n, flush, warm=3):
+    for i in range(warm):
+        fn(i)
+    return quantiles(per_launch_ms(fn, n, flush))
+
+
+def _tensor_entry(q, flops, pk, extra=None):
+    tf = flops / (q["median_ms"] * 1e-3) / 1e12
+    e = {**q, "TFLOP/s": round(tf, 1), "frac_of_peak": round(tf / pk["bf16_tflops"], 4),
+         "l2": "flushed before every launch"}
+    e.update(extra or {})
+    return e
+
+
+def _hbm_entry(q, nbytes, pk, extra=None):
+    gbs = nbytes / (q["median_ms"] * 1e-3) / 1e9
+    e = {**q, "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4), "kv_bytes": nbytes,
+         "l2": "flushed before every launch"}
+    e.update(extra or {})
+    return e
+
+
+def _extra_prefill(out, n, flush, fa, synth, dev, pk):
     # long prefill forward, B=1 H=32 N=8192 d=128 (causal and not)
-    sets = _rotating(lambda i: synth.prefill_inputs(synth.SEEDS["prefill8k"] + 10 * i, 1, 8192, 8192, 32, 128,
-                                                    device=dev), 3 * 64 * 2 ** 20)
-    o = torch.empty_like(sets[0][0])
+    q, k, v = synth.prefill_inputs(synth.SEEDS["prefill8k"], 1, 8192, 8192, 32, 128, device=dev)
+    o = torch.empty_like(q)
     lse = torch.empty(1, 32, 8192, dtype=torch.float32, device=dev)
     for causal in (True, False):
-        def f(i, causal=causal):
-            q, k, v = sets[i % len(sets)]
+        def f(_i, causal=causal):
             fa.fa_fwd(q, k, v, causal=causal, out=o, lse=lse)
-        for i in range(3):
-            f(i)
-        ms = device_time_ms(f, iters)
-        tf = fwd_flops(1, 32, 8192, 8192, 128, causal) / (ms * 1e-3) / 1e12
-        out["prefill8k_fwd_causal" if causal else "prefill8k_fwd_noncausal"] = {
-            "ms": round(ms, 4), "TFLOP/s": round(tf, 1), "frac_of_peak": round(tf / pk["bf16_tflops"], 4),
-            "l2": f"{len(sets)} rotating input sets"}
-    del sets, o, lse
-    torch.cuda.empty_cache()
+        out["prefill8k_fwd_causal" if causal else "prefill8k_fwd_noncausal"] = _tensor_entry(
+            _timed(f, n, flush), fwd_flops(1, 32, 8192, 8192, 128, causal), pk)
+    del q, k, v, o, lse
 
 
-def _extra_prefill_varlen(out, iters, fa, synth, dev, pk):
+def _extra_prefill_varlen(out, n, flush, fa, synth, dev, pk):
     # packed variable-length prefill: 16 causal sequences, lengths U[256, 4096], H=32, d=128
     lengths = synth.ragged_lengths(synth.SEEDS["prefill8k"], 16, 256, 4096)
     total = int(lengths.sum())
@@ -368,59 +456,40 @@ def _extra_prefill_varlen(out, iters, fa, synth, dev, pk):
     o = torch.empty_like(q)
     lse = torch.empty(32, total, dtype=torch.float32, device=dev)
 
-    def f(i):
+    def f(_i):
         fa.fa_fwd_varlen(q, k, v, cu, cu, maxL, maxL, causal=True, out=o, lse=lse)
-    for i in range(3):
-        f(i)
-    ms = device_time_ms(f, iters)
     flops = sum(fwd_flops(1, 32, int(L), int(L), 128, True) for L in lengths)
-    tf = flops / (ms * 1e-3) / 1e12
-    out["prefill_varlen_causal"] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1),
-                                    "frac_of_peak": round(tf / pk["bf16_tflops"], 4), "sequences": 16,
-                                    "total_tokens": total, "max_seqlen": maxL,
-                                    "l2": "no flush: Q, K, V together are 779 MB, 6x the L2"}
+    out["prefill_varlen_causal"] = _tensor_entry(_timed(f, n, flush), flops, pk,
+                                                 {"sequences": 16, "total_tokens": total, "max_seqlen": maxL})
     # the backward of the same packed batch (O and lse from the forward above)
     do = synth.prefill_inputs(synth.SEEDS["prefill8k"] + 1, 1, total, total, 32, 128,
                               device=dev)[0].reshape(total, 32, 128)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
 
-    def g(i):
+    def g(_i):
         fa.fa_bwd_varlen(q, k, v, o, do, lse, cu, cu, maxL, maxL, causal=True, dq=dq, dk=dk, dv=dv)
-    for i in range(3):
-        g(i)
-    ms_b = device_time_ms(g, max(10, iters // 2))
-    tf_b = sum(bwd_flops(1, 32, int(L), int(L), 128, True) for L in lengths) / (ms_b * 1e-3) / 1e12
-    out["prefill_varlen_causal_bwd"] = {"ms": round(ms_b, 4), "TFLOP/s": round(tf_b, 1),
-                                        "frac_of_peak": round(tf_b / pk["bf16_tflops"], 4),
-                                        "kernels": "preprocess + main + dQ convert",
-                                        "l2": "no flush: Q, K, V, O, dO together are 1.3 GB, 10x the L2"}
+    flops_b = sum(bwd_flops(1, 32, int(L), int(L), 128, True) for L in lengths)
+    out["prefill_varlen_causal_bwd"] = _tensor_entry(_timed(g, n, flush), flops_b, pk,
+                                                     {"kernels": "preprocess + main + dQ convert"})
     del q, k, v, o, lse, cu, do, dq, dk, dv
-    torch.cuda.empty_cache()
 
 
-def _extra_decode_single(out, iters, fa, synth, dev, pk):
+def _extra_decode_single(out, n, flush, fa, synth, dev, pk):
     # decode: single request, L=8192, H=32, d=128
     L = 8192
-    sets = _rotating(lambda i: tuple(t.to(dev) for t in synth.decode_inputs(synth.SEEDS["decode"] + 10 * i, [L], 32,
-                                                                            128, device=dev)), 2 * L * 32 * 128 * 2)
-    o = torch.empty_like(sets[0][0])
+    q, k, v, cu = synth.decode_inputs(synth.SEEDS["decode"], [L], 32, 128, device=dev)
+    cu = cu.to(dev)
+    o = torch.empty_like(q)
     lse = torch.empty(1, 32, dtype=torch.float32, device=dev)
 
-    def g(i):
-        q, k, v, cu = sets[i % len(sets)]
+    def g(_i):
         fa.fa_decode_splitkv(q, k, v, cu, L, out=o, lse=lse)
-    for i in range(3):
-        g(i)
-    ms = device_time_ms(g, max(20, iters))
-    gbs = 2 * 2 * 32 * 128 * L / (ms * 1e-3) / 1e9
-    out["decode_single_8k"] = {"ms": round(ms, 5), "GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4),
-                               "splits": fa.fa_decode_num_splits(1, 32, L, 128, 0),
-                               "l2": f"{len(sets)} rotating KV caches"}
-    del sets, o, lse
-    torch.cuda.empty_cache()
+    out["decode_single_8k"] = _hbm_entry(_timed(g, n, flush), 2 * 2 * 32 * 128 * L, pk,
+                                         {"splits": fa.fa_decode_num_splits(1, 32, L, 128, 0)})
+    del q, k, v, cu, o, lse
 
 
-def _extra_decode_batched(out, iters, fa, synth, dev, pk):
+def _extra_decode_batched(out, n, flush, fa, synth, dev, pk):
     # decode: 64 ragged sequences, lengths U[512, 16384]
     lengths = synth.ragged_lengths(synth.SEEDS["decode"], 64, 512, 16384)
     q, k, v, cu = synth.decode_inputs(synth.SEEDS["decode"], lengths, 32, 128, device=dev)
@@ -429,22 +498,14 @@ def _extra_decode_batched(out, iters, fa, synth, dev, pk):
     o = torch.empty_like(q)
     lse = torch.empty(64, 32, dtype=torch.float32, device=dev)
 
-    def g2(i):
+    def g2(_i):
         fa.fa_decode_splitkv(q, k, v, cu, maxL, out=o, lse=lse)
-    for i in range(3):
-        g2(i)
-    ms = device_time_ms(g2, iters)
-    kv_bytes = 2 * 2 * 32 * 128 * int(lengths.sum())
-    gbs = kv_bytes / (ms * 1e-3) / 1e9
-    out["decode_batched_ragged"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
-                                    "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4), "kv_bytes": kv_bytes,
-                                    "splits": fa.fa_decode_num_splits(64, 32, maxL, 128, 0),
-                                    "l2": "no flush: KV cache is 70x the L2"}
+    out["decode_batched_ragged"] = _hbm_entry(_timed(g2, n, flush), 2 * 2 * 32 * 128 * int(lengths.sum()), pk,
+                                              {"splits": fa.fa_decode_num_splits(64, 32, maxL, 128, 0)})
     del q, k, v, cu, o, lse
-    torch.cuda.empty_cache()
 
 
-def _extra_decode_paged(out, iters, fa, synth, dev, pk):
+def _extra_decode_paged(out, n, flush, fa, synth, dev, pk):
     # the same 64 ragged sequences in a paged cache: pages of 64 keys in seeded random order
     lengths = synth.ragged_lengths(synth.SEEDS["decode"], 64, 512, 16384)
     q, kp, vp, table, lens = synth.paged_decode_inputs(synth.SEEDS["decode"], lengths, 32, 128, 64, device=dev)
@@ -453,22 +514,14 @@ def _extra_decode_paged(out, iters, fa, synth, dev, pk):
     o = torch.empty_like(q)
     lse = torch.empty(64, 32, dtype=torch.float32, device=dev)
 
-    def g3(i):
+    def g3(_i):
         fa.fa_decode_paged(q, kp, vp, table, lens, maxL, out=o, lse=lse)
-    for i in range(3):
-        g3(i)
-    ms = device_time_ms(g3, iters)
-    kv_bytes = 2 * 2 * 32 * 128 * int(lengths.sum())
-    gbs = kv_bytes / (ms * 1e-3) / 1e9
-    out["decode_paged_batched"] = {"ms": round(ms, 4), "GB/s": round(gbs, 1),
-                                   "frac_of_hbm": round(gbs / pk["hbm_gbs"], 4), "kv_bytes": kv_bytes,
-                                   "page_size": 64, "num_pages": int(kp.shape[0]),
-                                   "l2": "no flush: KV cache is 70x the L2"}
+    out["decode_paged_batched"] = _hbm_entry(_timed(g3, n, flush), 2 * 2 * 32 * 128 * int(lengths.sum()), pk,
+                                             {"page_size": 64, "num_pages": int(kp.shape[0])})
     del q, kp, vp, table, lens, o, lse
-    torch.cuda.empty_cache()
 
 
-def _extra_long16k(out, iters, fa, synth, dev, pk):
+def _extra_long16k(out, n, flush, fa, synth, dev, pk):
     # long training sequence, B=1 H=16 N=16384 d=64 causal: fwd + bwd and peak memory
     q, k, v, do = synth.prefill_inputs(synth.SEEDS["long16k"], 1, 16384, 16384, 16, 64, with_dout=True, device=dev)
     o = torch.empty_like(q)
@@ -481,23 +534,23 @@ def _extra_long16k(out, iters, fa, synth, dev, pk):
     torch.cuda.reset_peak_memory_stats(dev)
     free0, _ = torch.cuda.mem_get_info(dev)
 
-    def h(i):
+    def h(_i):
         fa.fa_fwd(q, k, v, causal=True, out=o, lse=lse, ws=ws_f)
         fa.fa_bwd(q, k, v, o, do, lse, causal=True, dq=dq, dk=dk, dv=dv, ws=ws_b)
-    for i in range(2):
-        h(i)
-    ms = device_time_ms(h, max(3, iters // 2))
+    qs = _timed(h, n, None, warm=2)  # no flush: the flush buffer would count as extra memory here
     free1, _ = torch.cuda.mem_get_info(dev)
     peak_extra = torch.cuda.max_memory_allocated(dev) - base
     fl = fwd_flops(1, 16, 16384, 16384, 64, True) + bwd_flops(1, 16, 16384, 16384, 64, True)
-    tf = fl / (ms * 1e-3) / 1e12
-    out["long16k_fwd_bwd"] = {
-        "ms": round(ms, 4), "TFLOP/s": round(tf, 1), "frac_of_peak": round(tf / pk["bf16_tflops"], 4),
-        "peak_alloc_increase_bytes_during_calls": int(peak_extra),
-        "device_free_bytes_change": int(free0 - free1),
-        "workspace_bytes": int(ws_f.numel() + ws_b.numel()),
-        "one_NxN_bf16_matrix_bytes": 16384 * 16384 * 2,
-        "o_n_memory_ok": bool(peak_extra < 16384 * 16384 * 2 and (ws_f.numel() + ws_b.numel()) < 16384 * 16384 * 2)}
+    e = _tensor_entry(qs, fl, pk)
+    e.update({"l2": "no flush: Q, K, V, O, dO and the gradients (256 MiB) exceed the L2",
+              "peak_alloc_increase_bytes_during_calls": int(peak_extra),
+              "device_free_bytes_change": int(free0 - free1),
+              "workspace_bytes": int(ws_f.numel() + ws_b.numel()),
+              "one_NxN_bf16_matrix_bytes": 16384 * 16384 * 2,
+              "o_n_memory_ok": bool(peak_extra < 16384 * 16384 * 2 and
+                                    (ws_f.numel() + ws_b.numel()) < 16384 * 16384 * 2)})
+    out["long16k_fwd_bwd"] = e
+    del q, k, v, do, o, lse, dq, dk, dv
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -576,6 +629,8 @@ def main():
     ap.add_argument("--batch", type=int, default=0,
                     help="override B of the step (small cases for profiler captures; 0 = the workload's B=64)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--extra-launches", type=int, default=50,
+                    help="timed launches per other workload (at least 50)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
