@@ -24,7 +24,7 @@ import torch
 
 __all__ = [
     "FAError", "lib_path", "load", "fa_fwd", "fa_bwd", "fa_fwd_varlen", "fa_bwd_varlen", "fa_decode_splitkv",
-    "fa_decode_splitkv_noalloc", "fa_decode_paged", "fa_check", "fa_fwd_workspace_size", "fa_bwd_workspace_size",
+    "fa_decode_splitkv_noalloc", "fa_decode_splitkv_checked", "fa_decode_paged", "fa_check", "fa_fwd_workspace_size", "fa_bwd_workspace_size",
     "fa_bwd_varlen_workspace_size", "fa_decode_workspace_size", "fa_decode_num_splits",
     "fa_version", "STATUS",
 ]
@@ -69,10 +69,12 @@ def load():
         lib.fa_bwd.argtypes = [_vp] * 9 + [_i] * 6 + [_f, _vp, _sz, _vp]
         lib.fa_decode_splitkv.argtypes = [_vp] * 4 + [_i] * 6 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
         lib.fa_decode_splitkv_noalloc.argtypes = [_vp] * 4 + [_i] * 6 + [_f, _i, _vp, _vp, _vp]
+        lib.fa_decode_splitkv_checked.argtypes = [_vp] * 4 + [_i] * 7 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
         lib.fa_decode_paged.argtypes = [_vp] * 5 + [_i] * 7 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
         lib.fa_fwd_varlen.argtypes = [_vp] * 7 + [_i] * 8 + [_f, _vp, _sz, _vp]
         lib.fa_bwd_varlen.argtypes = [_vp] * 11 + [_i] * 8 + [_f, _vp, _sz, _vp]
         for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_decode_splitkv, lib.fa_decode_splitkv_noalloc,
+                   lib.fa_decode_splitkv_checked,
                    lib.fa_decode_paged, lib.fa_fwd_varlen, lib.fa_bwd_varlen):
             fn.restype = _i
         lib.fa_fwd_workspace_size.argtypes = [_i] * 5
@@ -294,6 +296,34 @@ def fa_decode_splitkv(q, k, v, cu_seqlens_k, max_seqlen_k: int, causal: bool = F
                                int(max_seqlen_k), d, int(bool(causal)), _scale(softmax_scale), int(num_splits),
                                out.data_ptr(), lse.data_ptr(), ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
     _raise("fa_decode_splitkv", st)
+    return out, lse
+
+
+def fa_decode_splitkv_checked(q, k, v, cu_seqlens_k, max_seqlen_k: int, softmax_scale=None, num_splits: int = 0,
+                              out=None, lse=None, ws=None):
+    """fa_decode_splitkv with every sequence's offsets checked on the device against
+    the rows of k and v (k.shape[0]); a sequence outside them is skipped (its o and
+    lse are not written) and fa_check then reports FA_ERR_INVALID_ARG."""
+    lib = load()
+    B, H, d = q.shape
+    _check_tensor("q", q, torch.bfloat16)
+    _check_tensor("k", k, torch.bfloat16)
+    _check_tensor("v", v, torch.bfloat16, k.shape)
+    _check_tensor("cu_seqlens_k", cu_seqlens_k, torch.int32, (B + 1,))
+    if k.dim() != 3 or k.shape[1] != H or k.shape[2] != d:
+        raise ValueError("k/v must be [total, H, d]")
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_tensor("out", out, torch.bfloat16, q.shape)
+    _check_tensor("lse", lse, torch.float32, (B, H))
+    need = lib.fa_decode_workspace_size(B, H, int(max_seqlen_k), d, int(num_splits))
+    if ws is None:
+        ws = workspace(need, q.device, "decode")
+    st = lib.fa_decode_splitkv_checked(q.data_ptr(), k.data_ptr(), v.data_ptr(), cu_seqlens_k.data_ptr(), B, H, 1,
+                                       int(k.shape[0]), int(max_seqlen_k), d, 0, _scale(softmax_scale),
+                                       int(num_splits), out.data_ptr(), lse.data_ptr(), ws.data_ptr(), ws.numel(),
+                                       _stream_ptr(q.device))
+    _raise("fa_decode_splitkv_checked", st)
     return out, lse
 
 

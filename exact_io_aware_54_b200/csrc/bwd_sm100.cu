@@ -1179,18 +1179,17 @@ __global__ void __launch_bounds__(256) bwd_convert_kernel(const float* __restric
 template <int D>
 static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   using L = BwdLayout<D>;
-  static bool attr_done[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
-  if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e;
-    if constexpr (D == 64)
-      e = cudaFuncSetAttribute(bwd_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, PipeLayout::kSmemBytes);
-    else
-      e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
-    if (e != cudaSuccess) return FA_ERR_CUDA;
-    attr_done[dev] = true;
-  }
+  static PerDeviceOnce attr_once;
+  if (!attr_once.run([] {
+        cudaError_t e;
+        if constexpr (D == 64)
+          e = cudaFuncSetAttribute(bwd_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   PipeLayout::kSmemBytes);
+        else
+          e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+        return e == cudaSuccess;
+      }))
+    return FA_ERR_CUDA;
   // A packed batch is one batch element of total rows for the tensor maps, the
   // preprocess and the convert kernels; the main kernels find each sequence's rows.
   const bool varlen = L0.cu_q != nullptr;

@@ -29,7 +29,9 @@ void* g_scratch_addr[64] = {};
 
 size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// Device address of the scratch on the current device; looked up once per device.
+// Device address of the scratch on the current device; looked up once per device
+// and kept for the life of the process (a device reset after that is not
+// supported: the kept address would no longer be valid).
 fa_status scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
@@ -107,7 +109,7 @@ extern "C" fa_status fa_decode_splitkv_noalloc(const void* q, const void* k, con
   a.d = d;
   a.scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)d);
   a.plan = plan;
-  a.check_args = 0;
-  a.timeout_ns = 2000000000ull;
+  a.check_args = checks_enabled() ? 1 : 0;  // FA_CHECKS=1: cu_seqlens order checked first, as in fa_decode_splitkv
+  a.timeout_ns = wait_timeout_ns();
   return launch_decode(a, stream);
 }

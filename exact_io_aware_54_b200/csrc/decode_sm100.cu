@@ -25,6 +25,9 @@
 //    atomic ticket -- merges the chunk states and writes o and lse, then resets
 //    the ticket, so tickets are zero between calls.  A sequence with a single chunk skips the
 //    partial-state round trip.
+//  * Given the number of rows of a packed cache, every sequence's offsets are
+//    checked against it first; a sequence outside the buffers is skipped and
+//    recorded in the status word.
 //  * Paged caches (K and V in pages of page_size keys, a block table per
 //    sequence) only change where the producer reads a key's row from; every page
 //    index is checked against the number of pages (a bad one is recorded in the
@@ -59,6 +62,7 @@ struct DecArgs {
   const int32_t* block_table;  // paged cache when not null
   const int32_t* seqlens;
   int page_size, max_pages, num_pages;
+  int total_kv;  // packed cache rows, checked against the offsets when >= 0
   __nv_bfloat16* o;
   float* lse;
   int* status;
@@ -100,6 +104,15 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
 
   const bool paged = a.block_table != nullptr;
   const int start = paged ? 0 : a.cu[b];
+  if (!paged && a.total_kv >= 0) {
+    // rows start .. end - 1 must lie inside k and v; otherwise every CTA of this
+    // sequence leaves it alone (nothing is read or written for it)
+    const int end = a.cu[b + 1];
+    if (start < 0 || end < start || end > a.total_kv) {
+      if (split == 0 && group == 0 && threadIdx.x == 0) atomicExch(a.status, kStatusBadArg);
+      return;
+    }
+  }
   int len = paged ? a.seqlens[b] : a.cu[b + 1] - start;
   len = max(0, min(len, a.max_seqlen_k));
   const int nsplit = (len + a.chunk - 1) / a.chunk;
@@ -429,15 +442,12 @@ size_t decode_workspace_bytes(int B, int H, int d, const DecodePlan& plan) {
 template <int D>
 static fa_status launch_decode_impl(const DecodeLaunch& L0, cudaStream_t stream) {
   using L = DecLayout<D>;
-  static bool attr_done[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
-  if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes) !=
-        cudaSuccess)
-      return FA_ERR_CUDA;
-    attr_done[dev] = true;
-  }
+  static PerDeviceOnce attr_once;
+  if (!attr_once.run([] {
+        return cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    L::kSmemBytes) == cudaSuccess;
+      }))
+    return FA_ERR_CUDA;
   DecArgs a;
   a.q = static_cast<const __nv_bfloat16*>(L0.q);
   a.k = static_cast<const __nv_bfloat16*>(L0.k);
@@ -448,6 +458,7 @@ static fa_status launch_decode_impl(const DecodeLaunch& L0, cudaStream_t stream)
   a.page_size = L0.page_size;
   a.max_pages = L0.max_pages;
   a.num_pages = L0.num_pages;
+  a.total_kv = L0.total_kv;
   a.o = static_cast<__nv_bfloat16*>(L0.o);
   a.lse = L0.lse;
   a.status = L0.status;

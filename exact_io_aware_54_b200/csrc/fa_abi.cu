@@ -112,7 +112,7 @@ bool encode_bshd_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int
   return r == CUDA_SUCCESS;
 }
 
-static unsigned long long wait_timeout_ns() {
+unsigned long long wait_timeout_ns() {
   static unsigned long long v = [] {
     unsigned long long ms = 2000;
     if (const char* env = getenv("FA_WAIT_TIMEOUT_MS")) {
@@ -124,7 +124,7 @@ static unsigned long long wait_timeout_ns() {
   return v;
 }
 
-static bool checks_enabled() {
+bool checks_enabled() {
   const char* env = getenv("FA_CHECKS");
   return env && env[0] == '1';
 }
@@ -340,11 +340,14 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
   return launch_bwd(a, stream);
 }
 
-fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_k, int B, int H,
-                            int Nq, int max_seqlen_k, int d, int causal, float softmax_scale, int num_splits, void* o,
-                            float* lse, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  const NvtxRange range("fa_decode_splitkv");
-  (void)causal;  // one query row: the bottom-right aligned mask admits every key
+}  // extern "C"
+
+// The packed split-KV decode behind fa_decode_splitkv (total_kv = -1: offsets not
+// checked against the buffers) and fa_decode_splitkv_checked.
+static fa_status decode_packed(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_k, int B,
+                               int H, int Nq, int total_kv, int max_seqlen_k, int d, float softmax_scale,
+                               int num_splits, void* o, float* lse, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream) {
   if (!q || !k || !v || !cu_seqlens_k || !o || !lse) return FA_ERR_INVALID_ARG;
   if (B <= 0 || H <= 0 || Nq != 1 || max_seqlen_k < 0 || num_splits < 0) return FA_ERR_INVALID_ARG;
   if ((long long)B * H >= (1LL << 31)) return FA_ERR_INVALID_ARG;
@@ -361,6 +364,7 @@ fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, const i
   a.k = k;
   a.v = v;
   a.cu_seqlens = cu_seqlens_k;
+  a.total_kv = total_kv;
   a.o = o;
   a.lse = lse;
   a.status = reinterpret_cast<int*>(ws);
@@ -385,6 +389,28 @@ fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, const i
   a.check_args = checks_enabled() ? 1 : 0;
   a.timeout_ns = wait_timeout_ns();
   return launch_decode(a, stream);
+}
+
+extern "C" {
+
+fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_k, int B, int H,
+                            int Nq, int max_seqlen_k, int d, int causal, float softmax_scale, int num_splits, void* o,
+                            float* lse, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_decode_splitkv");
+  (void)causal;  // one query row: the bottom-right aligned mask admits every key
+  return decode_packed(q, k, v, cu_seqlens_k, B, H, Nq, -1, max_seqlen_k, d, softmax_scale, num_splits, o, lse,
+                       workspace, workspace_bytes, stream);
+}
+
+fa_status fa_decode_splitkv_checked(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_k,
+                                    int B, int H, int Nq, int total_kv, int max_seqlen_k, int d, int causal,
+                                    float softmax_scale, int num_splits, void* o, float* lse, void* workspace,
+                                    size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_decode_splitkv_checked");
+  (void)causal;
+  if (total_kv < 0) return FA_ERR_INVALID_ARG;
+  return decode_packed(q, k, v, cu_seqlens_k, B, H, Nq, total_kv, max_seqlen_k, d, softmax_scale, num_splits, o,
+                       lse, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,

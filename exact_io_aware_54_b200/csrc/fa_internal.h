@@ -7,6 +7,8 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
+#include <mutex>
 
 #include <nvtx3/nvToolsExt.h>  // header-only NVTX v3: a range costs a pointer check unless a profiler listens
 
@@ -46,6 +48,41 @@ void prof_after(cudaStream_t s, int kernel_id);
 
 // Number of SMs of the current device (cached per device).
 int num_sms();
+
+// Wall-time limit of every bounded wait inside a kernel: FA_WAIT_TIMEOUT_MS
+// milliseconds when set (and positive), else 2 s.  Read once per process.
+unsigned long long wait_timeout_ns();
+
+// FA_CHECKS=1 turns on the optional device-side argument checks.
+bool checks_enabled();
+
+// One-time, per-device set-up (a kernel attribute, say) that is safe when several
+// host threads make their first call at the same time: the first caller on a
+// device runs `set` under a lock, the others wait for it; after a success later
+// calls only read an atomic flag.  A failed `set` is retried by the next call.
+class PerDeviceOnce {
+ public:
+  template <class F>
+  bool run(F&& set) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return set();  // outside the table: set up on every call
+    if (done_[dev].load(std::memory_order_acquire)) return true;
+    std::lock_guard<std::mutex> lk(mu_);
+    if (done_[dev].load(std::memory_order_relaxed)) return true;
+    if (!set()) return false;
+    done_[dev].store(true, std::memory_order_release);
+    return true;
+  }
+
+ private:
+  static constexpr int kMaxDevices = 64;
+  std::atomic<bool> done_[kMaxDevices]{};
+  std::mutex mu_;
+};
 
 // Encode a TMA descriptor for a bf16 tensor [B, N, H, D] (D innermost), with a
 // box of 128 rows x 64 columns and 128-byte swizzle.  Returns false on failure.
@@ -125,6 +162,9 @@ struct DecodeLaunch {
   float scale;
   DecodePlan plan;
   int check_args;      // validate cu_seqlens on the device first
+  // packed cache: rows in k and v (>= 0: a sequence whose rows do not lie in
+  // [0, total_kv) is skipped and recorded as a bad argument; -1: not checked)
+  int total_kv = -1;
   unsigned long long timeout_ns;
 };
 fa_status launch_decode(const DecodeLaunch& a, cudaStream_t stream);

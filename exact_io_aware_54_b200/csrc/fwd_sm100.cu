@@ -727,15 +727,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 static fa_status launch_fwd_impl(const FwdLaunch& L0, cudaStream_t stream) {
   using L = FwdLayout<D>;
-  static bool attr_done[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
-  if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes) !=
-        cudaSuccess)
-      return FA_ERR_CUDA;
-    attr_done[dev] = true;
-  }
+  static PerDeviceOnce attr_once;
+  if (!attr_once.run([] {
+        return cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes) ==
+               cudaSuccess;
+      }))
+    return FA_ERR_CUDA;
   // a variable-length batch is one long batch of total rows for the TMA maps
   const bool varlen = L0.cu_q != nullptr;
   const int mB = varlen ? 1 : L0.B;

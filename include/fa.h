@@ -159,7 +159,9 @@ FA_API fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, cons
  *                 cu_seqlens_k[B] <= total_kv.  This is a precondition: the
  *                 call has no total_kv to check the last bound against, and
  *                 offsets that break it make the kernel read outside k and v.
- *                 FA_CHECKS=1 checks the order on the device first.
+ *                 FA_CHECKS=1 checks the order on the device first.  Callers
+ *                 whose offsets come from untrusted data use
+ *                 fa_decode_splitkv_checked, which checks them against total_kv.
  *   max_seqlen_k: an upper bound of every sequence length (plays the role of Nk)
  *   num_splits  : chunks per sequence; 0 picks a value from the shape
  *   o           : [B, H, d] bf16 (written);  lse : [B, H] fp32 (written)
@@ -172,6 +174,24 @@ FA_API fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, 
                             int B, int H, int Nq, int max_seqlen_k, int d, int causal,
                             float softmax_scale, int num_splits, void* o, float* lse, void* workspace,
                             size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * fa_decode_splitkv with the number of rows of k and v, so that the offsets can
+ * be checked on the device instead of being a precondition.  Same computation,
+ * layouts and workspace as fa_decode_splitkv.
+ *   total_kv : rows of k and v ([total_kv, H, d]); >= 0, else FA_ERR_INVALID_ARG
+ * A sequence b whose rows cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1 do not lie in
+ * [0, total_kv) (a negative start, an end before its start, or an end past
+ * total_kv) is skipped before any of its rows is read: its o and lse are left
+ * as they were, and the kernel records the fault in the workspace status word
+ * (fa_check then returns FA_ERR_INVALID_ARG).  The other sequences are computed
+ * as usual.
+ */
+FA_API fa_status fa_decode_splitkv_checked(const void* q, const void* k, const void* v,
+                                           const int32_t* cu_seqlens_k, int B, int H, int Nq, int total_kv,
+                                           int max_seqlen_k, int d, int causal, float softmax_scale,
+                                           int num_splits, void* o, float* lse, void* workspace,
+                                           size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * Split-KV decode over a paged KV cache (the paging the pages name as the
@@ -211,7 +231,13 @@ FA_API fa_status fa_decode_paged(const void* q, const void* k_pages, const void*
  * which every GPU that loads the library holds until the process exits.
  *  - The call allocates nothing.  Its first call on a device looks up the
  *    array's device address (cudaGetSymbolAddress, with that device current);
- *    make that first call before any stream capture.
+ *    make that first call before any stream capture.  With lazy module loading
+ *    that first lookup is also when the CUDA runtime loads the library's device
+ *    code and places the array, which may allocate and synchronise: make the
+ *    first call outside any latency-critical loop.  The address is kept for the
+ *    life of the process, so the device must not be reset (cudaDeviceReset)
+ *    after the first call.
+ *  - FA_CHECKS=1 and FA_WAIT_TIMEOUT_MS act as for fa_decode_splitkv.
  *  - Returns FA_ERR_WORKSPACE when the shape needs more than the 16 MiB of
  *    scratch (B * H * splits * (d + 2) * 4 bytes plus small overheads); pass a
  *    smaller num_splits then.
@@ -242,9 +268,9 @@ FA_API int fa_decode_num_splits(int B, int H, int max_seqlen_k, int d, int num_s
  * Synchronises `stream` and reads the status word that the kernels of the
  * previous call(s) with this workspace recorded, then clears it.  Returns FA_OK,
  * FA_ERR_TIMEOUT (a bounded wait ran out), FA_ERR_INVALID_ARG (an argument the
- * kernels found bad: variable-length offsets outside the buffers, a paged-decode
- * page index outside the cache, or, with FA_CHECKS=1, decode cu_seqlens out of
- * order) or FA_ERR_CUDA.
+ * kernels found bad: variable-length or checked-decode offsets outside the
+ * buffers, a paged-decode page index outside the cache, or, with FA_CHECKS=1,
+ * decode cu_seqlens out of order) or FA_ERR_CUDA.
  */
 FA_API fa_status fa_check(void* workspace, cudaStream_t stream);
 

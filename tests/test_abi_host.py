@@ -111,6 +111,22 @@ def test_decode_argument_validation(lib):
     assert call(wsb=8) == ST["FA_ERR_WORKSPACE"]
 
 
+def test_decode_checked_argument_validation(lib):
+    def call(**kw):
+        a = dict(q=P, k=P, v=P, cu=P, B=2, H=4, Nq=1, T=128, L=64, d=128, s=0, o=P, lse=P, ws=P, wsb=1 << 30)
+        a.update(kw)
+        return lib.fa_decode_splitkv_checked(a["q"], a["k"], a["v"], a["cu"], a["B"], a["H"], a["Nq"], a["T"],
+                                             a["L"], a["d"], 0, 0.0, a["s"], a["o"], a["lse"], a["ws"], a["wsb"],
+                                             None)
+
+    assert call(T=-1) == ST["FA_ERR_INVALID_ARG"]
+    assert call(Nq=2) == ST["FA_ERR_INVALID_ARG"]
+    assert call(cu=None) == ST["FA_ERR_INVALID_ARG"]
+    assert call(d=80) == ST["FA_ERR_UNSUPPORTED"]
+    assert call(v=P + 2) == ST["FA_ERR_ALIGNMENT"]
+    assert call(wsb=8) == ST["FA_ERR_WORKSPACE"]
+
+
 def test_decode_paged_argument_validation(lib):
     def call(**kw):
         a = dict(q=P, k=P, v=P, bt=P, sl=P, B=2, H=4, npg=10, ps=16, mp=4, L=64, d=128, s=0, o=P, lse=P, ws=P,
