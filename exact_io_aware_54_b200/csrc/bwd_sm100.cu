@@ -90,7 +90,17 @@ struct BwdArgs {
   const int32_t* cu_k;
   int total_q, total_k;
   int stat_n;
+  // key-padding mask (null: none): [B, km_words] bits, bit j % 32 of word j / 32 set
+  // when key j of the batch element takes part
+  const uint32_t* key_mask;
+  int km_words;
 };
+
+// Whether in-range key `key` of batch element b takes part (always without a mask).
+__device__ __forceinline__ bool key_attended(const BwdArgs& a, int b, int key) {
+  if (a.key_mask == nullptr) return true;
+  return (__ldg(a.key_mask + (size_t)b * a.km_words + (key >> 5)) >> (key & 31)) & 1u;
+}
 
 // Where sequence b lives.  Dense: batch element b of the [B, N, H, D] tensors.
 // Packed: rows cu[b] .. cu[b + 1] - 1 of batch element 0.  tq / tk are the first
@@ -433,7 +443,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;
     const int key = j * 128 + r;
     const uint32_t lane_field = (quarter * 32) << 16;
-    const bool key_ok = key < sq.lk;
+    const bool key_in = key < sq.lk;  // a row of dK / dV to write
+    const bool key_ok = key_in && key_attended(a, b, key);  // and its P is not masked out
     // first query that sees this key (a sentinel far below any query when not causal;
     // qmin - qs below must not overflow)
     const int qmin = a.causal ? key - (sq.lk - sq.lq) : -(1 << 30);
@@ -487,7 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait(sv);
         reg_pin(dp);
         const uint32_t stat_u32 = sbase + L::kOffStat + st * 1024 + col * 4;
-        const bool tile_mask = (j * 128 + 128 > sq.lk) || (a.causal && (j * 128 + 127 - (sq.lk - sq.lq) > qs));
+        const bool tile_mask = a.key_mask != nullptr || (j * 128 + 128 > sq.lk) ||
+                               (a.causal && (j * 128 + 127 - (sq.lk - sq.lq) > qs));
         uint32_t pk[16], dk2[16];
         if (tile_mask)
           ds_block<32, true>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2);
@@ -533,7 +545,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      pack_bf16x2(f[4] * mul, f[5] * mul), pack_bf16x2(f[6] * mul, f[7] * mul));
           if (!direct_dkv)
             st_shared_v4(dst + box * L::kBoxBytes + r * 128 + ((chunk ^ (r & 7)) << 4), w.x, w.y, w.z, w.w);
-          else if (key_ok)
+          else if (key_in)
             gdst[cc * 4 + q4] = w;
         }
       }
@@ -1020,9 +1032,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         continue;
       }
       const int key = itm.j * 128 + r;
-      const bool key_ok = key < itm.s.lk;
+      const bool key_in = key < itm.s.lk;  // a row of dK / dV to write
+      const bool key_ok = key_in && key_attended(a, (w % (a.B * a.H)) / a.H, key);  // P not masked out
       const int qmin = a.causal ? key - (itm.s.lk - itm.s.lq) : -(1 << 30);
-      const bool key_tail = itm.j * 128 + 128 > itm.s.lk;
+      const bool key_tail = a.key_mask != nullptr || itm.j * 128 + 128 > itm.s.lk;  // masked variant
       const int last_key_qmin = itm.j * 128 + 127 - (itm.s.lk - itm.s.lq);
       for (int t = 0; t < itm.n; ++t, ++T) {
         const int st = T % L::kQStages;
@@ -1098,7 +1111,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       reg_pin(o1);
       tc_fence_before();
       mbar_arrive_warp(bar_acc_free);  // the next item may restart dK / dV
-      if (key_ok) {
+      if (key_in) {
         const float mul = grp == 0 ? a.scale : 1.f;
         uint4* dst =
             (grp == 0 ? a.dk : a.dv) + ((size_t)((long long)itm.s.tb * a.Nk + itm.s.tk + key) * a.H + itm.h) * (D / 8);
@@ -1236,6 +1249,8 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   a.total_q = L0.total_q;
   a.total_k = L0.total_k;
   a.stat_n = mNq;
+  a.key_mask = L0.key_mask;
+  a.km_words = (L0.Nk + 31) / 32;
   const long long grid = (long long)a.n_kv_tiles * L0.B * L0.H;
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   prof_before(stream, kKBwdMain);

@@ -65,6 +65,9 @@ struct FwdLaunch {
   const int32_t* cu_q = nullptr;
   const int32_t* cu_k = nullptr;
   int total_q = 0, total_k = 0;
+  // key-padding mask (dense batches): device uint32 [B, ceil(Nk / 32)], bit j % 32
+  // of word j / 32 set when key j takes part; null for none
+  const uint32_t* key_mask = nullptr;
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;
@@ -89,6 +92,7 @@ struct BwdLaunch {
   const int32_t* cu_q = nullptr;
   const int32_t* cu_k = nullptr;
   int total_q = 0, total_k = 0;
+  const uint32_t* key_mask = nullptr;  // as for the forward
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;

@@ -118,7 +118,22 @@ struct FwdArgs {
   int n_pairs;
   int n_items;
   unsigned long long timeout_ns;
+  // key-padding mask (null: none): [B, km_words] bits, bit j % 32 of word j / 32
+  // set when key j of the batch element takes part
+  const uint32_t* key_mask;
+  int km_words;
 };
+
+// The 128 mask bits of KV tile j of batch element b (all set without a mask;
+// words past the row are 0, their keys are past the end anyway).
+__device__ __forceinline__ void tile_mask_words(const FwdArgs& a, int b, int j, uint32_t (&w)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = ~0u;
+  if (a.key_mask == nullptr) return;
+  const uint32_t* row = a.key_mask + (size_t)b * a.km_words;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = (j * 4 + i < a.km_words) ? __ldg(row + j * 4 + i) : 0u;
+}
 
 __device__ __forceinline__ void item_coords(const FwdArgs& a, int w, int& b, int& h, int& pair) {
   const int bh_count = a.B * a.H;
@@ -549,14 +564,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_warp(bar_s_free + t);
         }
 
-        // mask (only tiles that cross the diagonal or the key tail)
+        // mask (only tiles that cross the diagonal or the key tail, or every tile
+        // under a key-padding mask)
         const int kbase = j * 128;
-        if (kbase + 128 > min(group_first_lim, lk) || kbase + 128 > lk) {
+        if (a.key_mask != nullptr || kbase + 128 > min(group_first_lim, lk) || kbase + 128 > lk) {
+          uint32_t kmw[4];
+          tile_mask_words(a, b, j, kmw);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int c = 0; c < 32; ++c)
-              if (kbase + i * 32 + c >= lim) s[i][c] = __float_as_uint(-INFINITY);
+              if (kbase + i * 32 + c >= lim || !((kmw[i] >> c) & 1u)) s[i][c] = __float_as_uint(-INFINITY);
         }
         // row max with four independent 3-input max chains
         float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -761,6 +779,8 @@ static fa_status launch_fwd_impl(const FwdLaunch& L0, cudaStream_t stream) {
   a.n_pairs = (L0.Nq + 255) / 256;
   a.n_items = a.n_pairs * L0.B * L0.H;
   a.timeout_ns = L0.timeout_ns;
+  a.key_mask = L0.key_mask;
+  a.km_words = (L0.Nk + 31) / 32;
   const int grid = std::min(a.n_items, num_sms() * 1);
   prof_before(stream, kKFwd);
   fwd_kernel<D><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);

@@ -151,6 +151,29 @@ FA_API fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, cons
                                void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Forward and backward passes with a key-padding mask (the padding mask the pages
+ * list among the semantics a fused attention kernel has to match, "FlashAttention
+ * saves IO, not N^2 work", section 8; masks applied inside the one kernel, "AI
+ * Bible 13", section 03).  Arguments, layouts and results are those of fa_fwd and
+ * fa_bwd, plus
+ *   key_mask : device uint32 [B, (Nk + 31) / 32], 4-byte aligned; bit j % 32 of
+ *              word j / 32 is set when key j of batch element b takes part.  A
+ *              masked key is excluded like a causally masked one (both apply when
+ *              both are set; the causal alignment still counts all Nk keys).  A
+ *              row left with no key gets O = 0 and LSE = -inf; a masked key gets
+ *              dK = dV = 0.  Bits of words past key Nk - 1 are ignored.
+ * A NULL key_mask makes the calls fa_fwd and fa_bwd.  The backward takes the lse
+ * of the masked forward with the same mask.
+ */
+FA_API fa_status fa_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse,
+                               const uint32_t* key_mask, int B, int H, int Nq, int Nk, int d, int causal,
+                               float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+FA_API fa_status fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, const void* do_,
+                               const float* lse, void* dq, void* dk, void* dv, const uint32_t* key_mask, int B,
+                               int H, int Nq, int Nk, int d, int causal, float softmax_scale, void* workspace,
+                               size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Split-KV decode over a ragged, packed KV cache.
  *   q           : [B, H, d] bf16 (one query row per sequence: Nq must be 1)
  *   k, v        : [total_kv, H, d] bf16; sequence b owns rows
