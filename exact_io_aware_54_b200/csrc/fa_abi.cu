@@ -8,6 +8,8 @@
 #include <mutex>
 #include <vector>
 
+#include <cmath>
+
 #include "fa_internal.h"
 
 namespace fa {
@@ -188,10 +190,21 @@ size_t fa_decode_workspace_size(int B, int H, int max_seqlen_k, int d, int num_s
   return decode_workspace_bytes(B, H, d, decode_plan(B, H, max_seqlen_k, d, num_splits));
 }
 
-// Dense forward, with an optional key-padding mask (4-byte aligned when given).
+// Dropout threshold t = round(65536 p) for 0 <= p < 1; false when p is out of range
+// or so close to 1 that no draw would be kept.
+static bool dropout_threshold(float p, uint32_t* t) {
+  if (!(p >= 0.f && p < 1.f)) return false;
+  const double x = std::floor((double)p * 65536.0 + 0.5);
+  if (x >= 65536.0) return false;
+  *t = (uint32_t)x;
+  return true;
+}
+
+// Dense forward, with an optional key-padding mask (4-byte aligned when given) and
+// dropout (drop_t = 0: none).
 static fa_status fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, const uint32_t* key_mask,
-                           int B, int H, int Nq, int Nk, int d, int causal, float softmax_scale, void* workspace,
-                           size_t workspace_bytes, cudaStream_t stream) {
+                           uint32_t drop_t, unsigned long long seed, int B, int H, int Nq, int Nk, int d, int causal,
+                           float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!q || !k || !v || !o || !lse || !dims_ok(B, H, Nq, Nk, d)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
@@ -207,6 +220,8 @@ static fa_status fwd_dense(const void* q, const void* k, const void* v, void* o,
   a.lse = lse;
   a.status = static_cast<int*>(workspace);
   a.key_mask = key_mask;
+  a.drop_t = drop_t;
+  a.seed = seed;
   a.B = B;
   a.H = H;
   a.Nq = Nq;
@@ -222,16 +237,18 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int d, int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
                  cudaStream_t stream) {
   const NvtxRange range("fa_fwd");
-  return fwd_dense(q, k, v, o, lse, nullptr, B, H, Nq, Nk, d, causal, softmax_scale, workspace, workspace_bytes,
-                   stream);
+  return fwd_dense(q, k, v, o, lse, nullptr, 0u, 0ull, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
+                   workspace_bytes, stream);
 }
 
 fa_status fa_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, const uint32_t* key_mask,
-                        int B, int H, int Nq, int Nk, int d, int causal, float softmax_scale, void* workspace,
-                        size_t workspace_bytes, cudaStream_t stream) {
+                        float dropout_p, unsigned long long seed, int B, int H, int Nq, int Nk, int d, int causal,
+                        float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   const NvtxRange range("fa_fwd_masked");
-  return fwd_dense(q, k, v, o, lse, key_mask, B, H, Nq, Nk, d, causal, softmax_scale, workspace, workspace_bytes,
-                   stream);
+  uint32_t t = 0;
+  if (!dropout_threshold(dropout_p, &t)) return FA_ERR_INVALID_ARG;
+  return fwd_dense(q, k, v, o, lse, key_mask, t, seed, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
+                   workspace_bytes, stream);
 }
 
 fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
@@ -272,11 +289,12 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, const int32
   return launch_fwd(a, stream);
 }
 
-// Dense backward, with an optional key-padding mask (4-byte aligned when given).
+// Dense backward, with an optional key-padding mask (4-byte aligned when given) and
+// the forward's dropout (drop_t = 0: none).
 static fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, const void* do_,
-                           const float* lse, void* dq, void* dk, void* dv, const uint32_t* key_mask, int B, int H,
-                           int Nq, int Nk, int d, int causal, float softmax_scale, void* workspace,
-                           size_t workspace_bytes, cudaStream_t stream) {
+                           const float* lse, void* dq, void* dk, void* dv, const uint32_t* key_mask, uint32_t drop_t,
+                           unsigned long long seed, int B, int H, int Nq, int Nk, int d, int causal,
+                           float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!q || !k || !v || !o || !do_ || !lse || !dq || !dk || !dv || !dims_ok(B, H, Nq, Nk, d))
     return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
@@ -300,6 +318,8 @@ static fa_status bwd_dense(const void* q, const void* k, const void* v, const vo
   a.dq_acc = reinterpret_cast<float*>(ws + kStatusBytes);
   a.delta = reinterpret_cast<float*>(ws + kStatusBytes + up256(sizeof(float) * (size_t)B * Nq * H * d));
   a.key_mask = key_mask;
+  a.drop_t = drop_t;
+  a.seed = seed;
   a.B = B;
   a.H = H;
   a.Nq = Nq;
@@ -315,17 +335,19 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d, int causal,
                  float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   const NvtxRange range("fa_bwd");
-  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, nullptr, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
-                   workspace_bytes, stream);
+  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, nullptr, 0u, 0ull, B, H, Nq, Nk, d, causal, softmax_scale,
+                   workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, const void* do_,
-                        const float* lse, void* dq, void* dk, void* dv, const uint32_t* key_mask, int B, int H,
-                        int Nq, int Nk, int d, int causal, float softmax_scale, void* workspace,
-                        size_t workspace_bytes, cudaStream_t stream) {
+                        const float* lse, void* dq, void* dk, void* dv, const uint32_t* key_mask, float dropout_p,
+                        unsigned long long seed, int B, int H, int Nq, int Nk, int d, int causal,
+                        float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   const NvtxRange range("fa_bwd_masked");
-  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, key_mask, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
-                   workspace_bytes, stream);
+  uint32_t t = 0;
+  if (!dropout_threshold(dropout_p, &t)) return FA_ERR_INVALID_ARG;
+  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, key_mask, t, seed, B, H, Nq, Nk, d, causal, softmax_scale,
+                   workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,
