@@ -314,7 +314,8 @@ def _rotating(make, total_bytes_of_one):
     return [make(i) for i in range(n)]
 
 
-EXTRA_WORKLOADS = ("prefill8k", "prefill_varlen", "decode_single", "decode_batched", "decode_paged", "long16k")
+EXTRA_WORKLOADS = ("prefill8k", "prefill_varlen", "decode_single", "decode_batched", "decode_paged", "long16k",
+                   "dropout_gpt2m")
 
 
 def run_extra(args, fa, synth, dev, pk, only=None):
@@ -333,7 +334,32 @@ def run_extra(args, fa, synth, dev, pk, only=None):
         _extra_decode_paged(out, iters, fa, synth, dev, pk)
     if want("long16k"):
         _extra_long16k(out, iters, fa, synth, dev, pk)
+    if want("dropout_gpt2m"):
+        _extra_dropout_gpt2m(out, iters, fa, synth, dev, pk)
     return out
+
+
+def _extra_dropout_gpt2m(out, iters, fa, synth, dev, pk):
+    # the headline training step (B=64 H=16 N=1024 d=64 causal) with dropout 0.1 and
+    # no key mask: what the regenerated Philox mask costs
+    B, H, N, d = 64, 16, 1024, 64
+    q, k, v, do = synth.prefill_inputs(synth.SEEDS["gpt2m"], B, N, N, H, d, with_dout=True, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def h(i):
+        fa.fa_fwd_masked(q, k, v, None, dropout_p=0.1, seed=1234 + i, causal=True, out=o, lse=lse)
+        fa.fa_bwd_masked(q, k, v, o, do, lse, None, dropout_p=0.1, seed=1234 + i, causal=True, dq=dq, dk=dk, dv=dv)
+    for i in range(3):
+        h(i)
+    ms = device_time_ms(h, max(5, iters // 2))
+    fl = fwd_flops(B, H, N, N, d, True) + bwd_flops(B, H, N, N, d, True)
+    tf = fl / (ms * 1e-3) / 1e12
+    out["dropout_gpt2m_fwd_bwd"] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                                    "frac_of_peak": round(tf / pk["bf16_tflops"], 4), "dropout_p": 0.1}
+    del q, k, v, do, o, lse, dq, dk, dv
+    torch.cuda.empty_cache()
 
 
 def _extra_prefill(out, iters, fa, synth, dev, pk):
