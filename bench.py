@@ -382,7 +382,8 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
-EXTRA_WORKLOADS = ("prefill8k", "prefill_varlen", "decode_single", "decode_batched", "decode_paged", "long16k")
+EXTRA_WORKLOADS = ("prefill8k", "prefill_varlen", "decode_single", "decode_batched", "decode_paged", "long16k",
+                   "dropout_gpt2m")
 
 
 def run_extra(args, fa, synth, dev, pk, only=None):
@@ -405,6 +406,8 @@ def run_extra(args, fa, synth, dev, pk, only=None):
         _extra_decode_paged(out, n, flush, fa, synth, dev, pk)
     if want("long16k"):
         _extra_long16k(out, n, flush, fa, synth, dev, pk)
+    if want("dropout_gpt2m"):
+        _extra_dropout_gpt2m(out, n, flush, fa, synth, dev, pk)
     del flush
     torch.cuda.empty_cache()
     return out
@@ -430,6 +433,24 @@ def _hbm_entry(q, nbytes, pk, extra=None):
          "l2": "flushed before every launch"}
     e.update(extra or {})
     return e
+
+
+def _extra_dropout_gpt2m(out, n, flush, fa, synth, dev, pk):
+    # the headline training step (B=64 H=16 N=1024 d=64 causal) with dropout 0.1 and
+    # no key mask: what the regenerated Philox mask costs
+    B, H, N, d = 64, 16, 1024, 64
+    q, k, v, do = synth.prefill_inputs(synth.SEEDS["gpt2m"], B, N, N, H, d, with_dout=True, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def h(i):
+        fa.fa_fwd_masked(q, k, v, None, dropout_p=0.1, seed=1234 + i, causal=True, out=o, lse=lse)
+        fa.fa_bwd_masked(q, k, v, o, do, lse, None, dropout_p=0.1, seed=1234 + i, causal=True, dq=dq, dk=dk, dv=dv)
+    fl = fwd_flops(B, H, N, N, d, True) + bwd_flops(B, H, N, N, d, True)
+    out["dropout_gpt2m_fwd_bwd"] = _tensor_entry(_timed(h, n, None), fl, pk, {
+        "dropout_p": 0.1, "l2": "no flush: the inputs of one step (640 MiB) exceed the L2"})
+    del q, k, v, do, o, lse, dq, dk, dv
 
 
 def _extra_prefill(out, n, flush, fa, synth, dev, pk):

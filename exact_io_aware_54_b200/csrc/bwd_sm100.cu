@@ -28,6 +28,7 @@
 //        S^T / dP^T), and the dQ tile reuses the dP^T columns.
 //   3. convert: dQ = bf16(scale * accumulator).
 #include "fa_internal.h"
+#include "philox.cuh"
 #include "ptx.cuh"
 
 namespace fa {
@@ -90,7 +91,29 @@ struct BwdArgs {
   const int32_t* cu_k;
   int total_q, total_k;
   int stat_n;
+  // key-padding mask (null: none): [B, km_words] bits, bit j % 32 of word j / 32 set
+  // when key j of the batch element takes part
+  const uint32_t* key_mask;
+  int km_words;
+  // dropout (drop_t = 0: none), the forward's: keep when the 16-bit draw >= drop_t
+  uint32_t drop_t;
+  float drop_scale;
+  uint32_t seed_lo, seed_hi;
 };
+
+// Where one dS block's dropout draws come from: its key, head and batch element.
+struct DropCtx {
+  uint32_t t;
+  float scale;
+  uint32_t seed_lo, seed_hi;
+  int key, h, b;
+};
+
+// Whether in-range key `key` of batch element b takes part (always without a mask).
+__device__ __forceinline__ bool key_attended(const BwdArgs& a, int b, int key) {
+  if (a.key_mask == nullptr) return true;
+  return (__ldg(a.key_mask + (size_t)b * a.km_words + (key >> 5)) >> (key & 31)) & 1u;
+}
 
 // Where sequence b lives.  Dense: batch element b of the [B, N, H, D] tensors.
 // Packed: rows cu[b] .. cu[b + 1] - 1 of batch element 0.  tq / tk are the first
@@ -202,11 +225,13 @@ __device__ __forceinline__ void issue_dq(uint32_t dq_tmem, SDesc ds, SDesc k) {
 // packed to bf16 pairs.  `stat` holds -lse2 (128 floats) then -D (128 floats) of
 // the query tile, already offset to the first query.  With kMask, queries before
 // `qrel_min` (relative to the first query) and all queries of an out-of-range key
-// get p = 0.
-template <int kN, bool kMask>
+// get p = 0.  With kDrop, z = 0 or drop_scale per (query, key) from the dropout
+// draws (philox.cuh), q0 the first query: P^T goes out as p z (the dV operand) and
+// ds = p (z dp - D).
+template <int kN, bool kMask, bool kDrop = false>
 __device__ __forceinline__ void ds_block(const uint32_t (&sv)[kN], const uint32_t (&dp)[kN], uint32_t stat,
                                          float scale_log2, bool key_ok, int qrel_min, uint32_t (&pk)[kN / 2],
-                                         uint32_t (&dsk)[kN / 2]) {
+                                         uint32_t (&dsk)[kN / 2], const DropCtx* drop = nullptr, int q0 = 0) {
   const float2 sc2 = make_float2(scale_log2, scale_log2);
 #pragma unroll
   for (int c = 0; c < kN; c += 4) {
@@ -224,18 +249,40 @@ __device__ __forceinline__ void ds_block(const uint32_t (&sv)[kN], const uint32_
       if (!key_ok || c + 2 < qrel_min) p1.x = 0.f;
       if (!key_ok || c + 3 < qrel_min) p1.y = 0.f;
     }
-    const float2 t0 = fadd2(make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1])), make_float2(nd.x, nd.y));
-    const float2 t1 = fadd2(make_float2(__uint_as_float(dp[c + 2]), __uint_as_float(dp[c + 3])),
-                            make_float2(nd.z, nd.w));
-    const float2 d0 = fmul2(p0, t0), d1 = fmul2(p1, t1);
-    pk[c / 2] = pack_bf16x2(p0.x, p0.y);
-    pk[c / 2 + 1] = pack_bf16x2(p1.x, p1.y);
-    dsk[c / 2] = pack_bf16x2(d0.x, d0.y);
-    dsk[c / 2 + 1] = pack_bf16x2(d1.x, d1.y);
+    const float2 dp0 = make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1]));
+    const float2 dp1 = make_float2(__uint_as_float(dp[c + 2]), __uint_as_float(dp[c + 3]));
+    if constexpr (kDrop) {
+      // queries q0 + c .. q0 + c + 3 are the four words of one call (q0 + c is a
+      // multiple of 4); this key takes the low or high 16 bits of each
+      const uint4 w = philox4x32_10(
+          make_uint4((uint32_t)drop->key >> 1, (uint32_t)(q0 + c) >> 2, (uint32_t)drop->h, (uint32_t)drop->b),
+          drop->seed_lo, drop->seed_hi);
+      const int sh = (drop->key & 1) * 16;
+      const float2 z0 = make_float2(((w.x >> sh) & 0xFFFFu) >= drop->t ? drop->scale : 0.f,
+                                    ((w.y >> sh) & 0xFFFFu) >= drop->t ? drop->scale : 0.f);
+      const float2 z1 = make_float2(((w.z >> sh) & 0xFFFFu) >= drop->t ? drop->scale : 0.f,
+                                    ((w.w >> sh) & 0xFFFFu) >= drop->t ? drop->scale : 0.f);
+      const float2 d0 = fmul2(p0, ffma2(dp0, z0, make_float2(nd.x, nd.y)));
+      const float2 d1 = fmul2(p1, ffma2(dp1, z1, make_float2(nd.z, nd.w)));
+      const float2 pz0 = fmul2(p0, z0), pz1 = fmul2(p1, z1);
+      pk[c / 2] = pack_bf16x2(pz0.x, pz0.y);
+      pk[c / 2 + 1] = pack_bf16x2(pz1.x, pz1.y);
+      dsk[c / 2] = pack_bf16x2(d0.x, d0.y);
+      dsk[c / 2 + 1] = pack_bf16x2(d1.x, d1.y);
+    } else {
+      const float2 t0 = fadd2(dp0, make_float2(nd.x, nd.y));
+      const float2 t1 = fadd2(dp1, make_float2(nd.z, nd.w));
+      const float2 d0 = fmul2(p0, t0), d1 = fmul2(p1, t1);
+      pk[c / 2] = pack_bf16x2(p0.x, p0.y);
+      pk[c / 2 + 1] = pack_bf16x2(p1.x, p1.y);
+      dsk[c / 2] = pack_bf16x2(d0.x, d0.y);
+      dsk[c / 2 + 1] = pack_bf16x2(d1.x, d1.y);
+    }
   }
 }
 
-template <int D>
+// kDrop: dropout (a separate instantiation, so the plain kernel is unchanged)
+template <int D, bool kDrop>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -433,7 +480,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;
     const int key = j * 128 + r;
     const uint32_t lane_field = (quarter * 32) << 16;
-    const bool key_ok = key < sq.lk;
+    const bool key_in = key < sq.lk;  // a row of dK / dV to write
+    const bool key_ok = key_in && key_attended(a, b, key);  // and its P is not masked out
     // first query that sees this key (a sentinel far below any query when not causal;
     // qmin - qs below must not overflow)
     const int qmin = a.causal ? key - (sq.lk - sq.lq) : -(1 << 30);
@@ -487,12 +535,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait(sv);
         reg_pin(dp);
         const uint32_t stat_u32 = sbase + L::kOffStat + st * 1024 + col * 4;
-        const bool tile_mask = (j * 128 + 128 > sq.lk) || (a.causal && (j * 128 + 127 - (sq.lk - sq.lq) > qs));
+        const bool tile_mask = a.key_mask != nullptr || (j * 128 + 128 > sq.lk) ||
+                               (a.causal && (j * 128 + 127 - (sq.lk - sq.lq) > qs));
         uint32_t pk[16], dk2[16];
-        if (tile_mask)
+        if constexpr (kDrop) {
+          const DropCtx dctx{a.drop_t, a.drop_scale, a.seed_lo, a.seed_hi, key, h, b};
+          ds_block<32, true, true>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2, &dctx, qs);
+        } else if (tile_mask) {
           ds_block<32, true>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2);
-        else
+        } else {
           ds_block<32, false>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2);
+        }
         // P^T as bf16 pairs over the columns of this group already read
         tmem_st16(tmem + lane_field + L::kTmSt + 64 * grp + 16 * ch, pk);
         // dS^T row of this key: 4 chunks of 16 bytes, 128-byte swizzle
@@ -533,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      pack_bf16x2(f[4] * mul, f[5] * mul), pack_bf16x2(f[6] * mul, f[7] * mul));
           if (!direct_dkv)
             st_shared_v4(dst + box * L::kBoxBytes + r * 128 + ((chunk ^ (r & 7)) << 4), w.x, w.y, w.z, w.w);
-          else if (key_ok)
+          else if (key_in)
             gdst[cc * 4 + q4] = w;
         }
       }
@@ -721,6 +774,7 @@ __device__ __forceinline__ void pipe_load_stats(const BwdArgs& a, const PipeCurs
   }
 }
 
+template <bool kDrop>
 __global__ void __launch_bounds__(kPipeThreads, 1)
     bwd_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -1020,9 +1074,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         continue;
       }
       const int key = itm.j * 128 + r;
-      const bool key_ok = key < itm.s.lk;
+      const bool key_in = key < itm.s.lk;  // a row of dK / dV to write
+      const bool key_ok = key_in && key_attended(a, (w % (a.B * a.H)) / a.H, key);  // P not masked out
       const int qmin = a.causal ? key - (itm.s.lk - itm.s.lq) : -(1 << 30);
-      const bool key_tail = itm.j * 128 + 128 > itm.s.lk;
+      const bool key_tail = a.key_mask != nullptr || itm.j * 128 + 128 > itm.s.lk;  // masked variant
       const int last_key_qmin = itm.j * 128 + 127 - (itm.s.lk - itm.s.lq);
       for (int t = 0; t < itm.n; ++t, ++T) {
         const int st = T % L::kQStages;
@@ -1051,14 +1106,21 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         // both 32-query blocks first: the waits for the P^T columns and the dS buffer
         // come as late as possible
         uint32_t pk0[16], dk0[16], pk1[16], dk1[16];
-        if (key_tail || (a.causal && last_key_qmin > qs0))
-          ds_block<32, true>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk0, dk0);
-        else
-          ds_block<32, false>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk0, dk0);
-        if (key_tail || (a.causal && last_key_qmin > qs1))
-          ds_block<32, true>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk1, dk1);
-        else
-          ds_block<32, false>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk1, dk1);
+        if constexpr (kDrop) {
+          const DropCtx dctx{a.drop_t, a.drop_scale, a.seed_lo, a.seed_hi, key, itm.h, (w % (a.B * a.H)) / a.H};
+          ds_block<32, true, true>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk0, dk0, &dctx, qs0);
+          ds_block<32, true, true>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk1, dk1, &dctx,
+                                   qs1);
+        } else {
+          if (key_tail || (a.causal && last_key_qmin > qs0))
+            ds_block<32, true>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk0, dk0);
+          else
+            ds_block<32, false>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk0, dk0);
+          if (key_tail || (a.causal && last_key_qmin > qs1))
+            ds_block<32, true>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk1, dk1);
+          else
+            ds_block<32, false>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk1, dk1);
+        }
         // P^T may be written once the previous tile's dV has read it
         if (T > 0 && (!warp_wait_b(bar_pt_free, (T - 1) & 1, a.timeout_ns) || *abort_flag)) {
           ok = false;
@@ -1098,7 +1160,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       reg_pin(o1);
       tc_fence_before();
       mbar_arrive_warp(bar_acc_free);  // the next item may restart dK / dV
-      if (key_ok) {
+      if (key_in) {
         const float mul = grp == 0 ? a.scale : 1.f;
         uint4* dst =
             (grp == 0 ? a.dk : a.dv) + ((size_t)((long long)itm.s.tb * a.Nk + itm.s.tk + key) * a.H + itm.h) * (D / 8);
@@ -1182,11 +1244,19 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   static PerDeviceOnce attr_once;
   if (!attr_once.run([] {
         cudaError_t e;
-        if constexpr (D == 64)
-          e = cudaFuncSetAttribute(bwd_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if constexpr (D == 64) {
+          e = cudaFuncSetAttribute(bwd_pipe_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    PipeLayout::kSmemBytes);
-        else
-          e = cudaFuncSetAttribute(bwd_main_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes);
+          if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(bwd_pipe_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     PipeLayout::kSmemBytes);
+        } else {
+          e = cudaFuncSetAttribute(bwd_main_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   L::kSmemBytes);
+          if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(bwd_main_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     L::kSmemBytes);
+        }
         return e == cudaSuccess;
       }))
     return FA_ERR_CUDA;
@@ -1235,14 +1305,26 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   a.total_q = L0.total_q;
   a.total_k = L0.total_k;
   a.stat_n = mNq;
+  a.key_mask = L0.key_mask;
+  a.km_words = (L0.Nk + 31) / 32;
+  a.drop_t = L0.drop_t;
+  a.drop_scale = L0.drop_t ? (float)(65536.0 / (65536.0 - (double)L0.drop_t)) : 1.f;
+  a.seed_lo = (uint32_t)(L0.seed & 0xFFFFFFFFull);
+  a.seed_hi = (uint32_t)(L0.seed >> 32);
   const long long grid = (long long)a.n_kv_tiles * L0.B * L0.H;
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   prof_before(stream, kKBwdMain);
   if constexpr (D == 64) {
     const int pgrid = (int)std::min<long long>(grid, (long long)num_sms());
-    bwd_pipe_kernel<<<pgrid, kPipeThreads, PipeLayout::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
+    if (a.drop_t != 0u)
+      bwd_pipe_kernel<true><<<pgrid, kPipeThreads, PipeLayout::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
+    else
+      bwd_pipe_kernel<false><<<pgrid, kPipeThreads, PipeLayout::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
   } else {
-    bwd_main_kernel<D><<<(unsigned)grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
+    if (a.drop_t != 0u)
+      bwd_main_kernel<D, true><<<(unsigned)grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
+    else
+      bwd_main_kernel<D, false><<<(unsigned)grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
   }
   const cudaError_t err_main = cudaGetLastError();
   prof_after(stream, kKBwdMain);

@@ -8,6 +8,8 @@
 #include <mutex>
 #include <vector>
 
+#include <cmath>
+
 #include "fa_internal.h"
 
 namespace fa {
@@ -188,13 +190,26 @@ size_t fa_decode_workspace_size(int B, int H, int max_seqlen_k, int d, int num_s
   return decode_workspace_bytes(B, H, d, decode_plan(B, H, max_seqlen_k, d, num_splits));
 }
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
-                 int d, int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
-                 cudaStream_t stream) {
-  const NvtxRange range("fa_fwd");
+// Dropout threshold t = round(65536 p) for 0 <= p < 1; false when p is out of range
+// or so close to 1 that no draw would be kept.
+static bool dropout_threshold(float p, uint32_t* t) {
+  if (!(p >= 0.f && p < 1.f)) return false;
+  const double x = std::floor((double)p * 65536.0 + 0.5);
+  if (x >= 65536.0) return false;
+  *t = (uint32_t)x;
+  return true;
+}
+
+// Dense forward, with an optional key-padding mask (4-byte aligned when given) and
+// dropout (drop_t = 0: none).
+static fa_status fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, const uint32_t* key_mask,
+                           uint32_t drop_t, unsigned long long seed, int B, int H, int Nq, int Nk, int d, int causal,
+                           float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!q || !k || !v || !o || !lse || !dims_ok(B, H, Nq, Nk, d)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+      (reinterpret_cast<uintptr_t>(key_mask) & 3u))
+    return FA_ERR_ALIGNMENT;
   if (!workspace || !aligned16(workspace) || workspace_bytes < fa_fwd_workspace_size(B, H, Nq, Nk, d))
     return FA_ERR_WORKSPACE;
   FwdLaunch a;
@@ -204,6 +219,9 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   a.o = o;
   a.lse = lse;
   a.status = static_cast<int*>(workspace);
+  a.key_mask = key_mask;
+  a.drop_t = drop_t;
+  a.seed = seed;
   a.B = B;
   a.H = H;
   a.Nq = Nq;
@@ -213,6 +231,24 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   a.scale = resolve_scale(softmax_scale, d);
   a.timeout_ns = wait_timeout_ns();
   return launch_fwd(a, stream);
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                 int d, int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
+                 cudaStream_t stream) {
+  const NvtxRange range("fa_fwd");
+  return fwd_dense(q, k, v, o, lse, nullptr, 0u, 0ull, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
+                   workspace_bytes, stream);
+}
+
+fa_status fa_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse, const uint32_t* key_mask,
+                        float dropout_p, unsigned long long seed, int B, int H, int Nq, int Nk, int d, int causal,
+                        float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_fwd_masked");
+  uint32_t t = 0;
+  if (!dropout_threshold(dropout_p, &t)) return FA_ERR_INVALID_ARG;
+  return fwd_dense(q, k, v, o, lse, key_mask, t, seed, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
+                   workspace_bytes, stream);
 }
 
 fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
@@ -253,15 +289,17 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, const int32
   return launch_fwd(a, stream);
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,
-                 void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d, int causal,
-                 float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  const NvtxRange range("fa_bwd");
+// Dense backward, with an optional key-padding mask (4-byte aligned when given) and
+// the forward's dropout (drop_t = 0: none).
+static fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, const void* do_,
+                           const float* lse, void* dq, void* dk, void* dv, const uint32_t* key_mask, uint32_t drop_t,
+                           unsigned long long seed, int B, int H, int Nq, int Nk, int d, int causal,
+                           float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!q || !k || !v || !o || !do_ || !lse || !dq || !dk || !dv || !dims_ok(B, H, Nq, Nk, d))
     return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(do_) || !aligned16(lse) ||
-      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || (reinterpret_cast<uintptr_t>(key_mask) & 3u))
     return FA_ERR_ALIGNMENT;
   if (!workspace || !aligned16(workspace) || workspace_bytes < fa_bwd_workspace_size(B, H, Nq, Nk, d))
     return FA_ERR_WORKSPACE;
@@ -279,6 +317,9 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   a.status = reinterpret_cast<int*>(ws);
   a.dq_acc = reinterpret_cast<float*>(ws + kStatusBytes);
   a.delta = reinterpret_cast<float*>(ws + kStatusBytes + up256(sizeof(float) * (size_t)B * Nq * H * d));
+  a.key_mask = key_mask;
+  a.drop_t = drop_t;
+  a.seed = seed;
   a.B = B;
   a.H = H;
   a.Nq = Nq;
@@ -288,6 +329,25 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   a.scale = resolve_scale(softmax_scale, d);
   a.timeout_ns = wait_timeout_ns();
   return launch_bwd(a, stream);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d, int causal,
+                 float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_bwd");
+  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, nullptr, 0u, 0ull, B, H, Nq, Nk, d, causal, softmax_scale,
+                   workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, const void* do_,
+                        const float* lse, void* dq, void* dk, void* dv, const uint32_t* key_mask, float dropout_p,
+                        unsigned long long seed, int B, int H, int Nq, int Nk, int d, int causal,
+                        float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_bwd_masked");
+  uint32_t t = 0;
+  if (!dropout_threshold(dropout_p, &t)) return FA_ERR_INVALID_ARG;
+  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, key_mask, t, seed, B, H, Nq, Nk, d, causal, softmax_scale,
+                   workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,

@@ -102,6 +102,12 @@ struct FwdLaunch {
   const int32_t* cu_q = nullptr;
   const int32_t* cu_k = nullptr;
   int total_q = 0, total_k = 0;
+  // key-padding mask (dense batches): device uint32 [B, ceil(Nk / 32)], bit j % 32
+  // of word j / 32 set when key j takes part; null for none
+  const uint32_t* key_mask = nullptr;
+  // dropout: drop_t = round(65536 p) (0: none), seed of the Philox draws
+  uint32_t drop_t = 0;
+  unsigned long long seed = 0;
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;
@@ -126,6 +132,9 @@ struct BwdLaunch {
   const int32_t* cu_q = nullptr;
   const int32_t* cu_k = nullptr;
   int total_q = 0, total_k = 0;
+  const uint32_t* key_mask = nullptr;  // as for the forward
+  uint32_t drop_t = 0;                  // as for the forward
+  unsigned long long seed = 0;
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;

@@ -51,6 +51,7 @@
 //  * Epilogue: O/l -> bf16 -> swizzled smem (the Q tile's slot) -> TMA store;
 //    lse as coalesced fp32 stores.
 #include "fa_internal.h"
+#include "philox.cuh"
 #include "ptx.cuh"
 
 namespace fa {
@@ -118,7 +119,27 @@ struct FwdArgs {
   int n_pairs;
   int n_items;
   unsigned long long timeout_ns;
+  // key-padding mask (null: none): [B, km_words] bits, bit j % 32 of word j / 32
+  // set when key j of the batch element takes part
+  const uint32_t* key_mask;
+  int km_words;
+  // dropout (drop_t = 0: none): a probability is kept when its 16-bit draw is at
+  // least drop_t and then scaled by drop_scale (philox.cuh gives the draws)
+  uint32_t drop_t;
+  float drop_scale;
+  uint32_t seed_lo, seed_hi;
 };
+
+// The 128 mask bits of KV tile j of batch element b (all set without a mask;
+// words past the row are 0, their keys are past the end anyway).
+__device__ __forceinline__ void tile_mask_words(const FwdArgs& a, int b, int j, uint32_t (&w)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = ~0u;
+  if (a.key_mask == nullptr) return;
+  const uint32_t* row = a.key_mask + (size_t)b * a.km_words;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = (j * 4 + i < a.km_words) ? __ldg(row + j * 4 + i) : 0u;
+}
 
 __device__ __forceinline__ void item_coords(const FwdArgs& a, int w, int& b, int& h, int& pair) {
   const int bh_count = a.B * a.H;
@@ -208,7 +229,8 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, SDesc
     umma_ts(o_tmem, p_tmem + kk * 8, sdesc_at(v, kk * 128), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
-template <int D>
+// kDrop: dropout on P (a separate instantiation, so the plain kernel is unchanged)
+template <int D, bool kDrop>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -549,14 +571,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive_warp(bar_s_free + t);
         }
 
-        // mask (only tiles that cross the diagonal or the key tail)
+        // mask (only tiles that cross the diagonal or the key tail, or every tile
+        // under a key-padding mask)
         const int kbase = j * 128;
-        if (kbase + 128 > min(group_first_lim, lk) || kbase + 128 > lk) {
+        if (a.key_mask != nullptr || kbase + 128 > min(group_first_lim, lk) || kbase + 128 > lk) {
+          uint32_t kmw[4];
+          tile_mask_words(a, b, j, kmw);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
 #pragma unroll
             for (int c = 0; c < 32; ++c)
-              if (kbase + i * 32 + c >= lim) s[i][c] = __float_as_uint(-INFINITY);
+              if (kbase + i * 32 + c >= lim || !((kmw[i] >> c) & 1u)) s[i][c] = __float_as_uint(-INFINITY);
         }
         // row max with four independent 3-input max chains
         float mxv[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -591,8 +616,21 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float2 p1 =
                   (((c >> 2) % kEvery) == kEvery - 1) ? exp2_fma2(x1) : make_float2(ex2(x1.x), ex2(x1.y));
               const uint32_t k0 = pack_bf16x2(p0.x, p0.y), k1 = pack_bf16x2(p1.x, p1.y);
-              pk[ii * 16 + (c >> 1)] = k0;
-              pk[ii * 16 + (c >> 1) + 1] = k1;
+              uint32_t s0 = k0, s1 = k1;  // P as the P V product takes it
+              if constexpr (kDrop) {
+                // keys key0 .. key0 + 3 of this row: two calls, the row's word of each
+                const uint32_t kb = (uint32_t)(kbase + hf * 64 + ii * 32 + c) >> 1;
+                const uint32_t w0 = dropout_word(kb, row, h, b, a.seed_lo, a.seed_hi);
+                const uint32_t w1 = dropout_word(kb + 1, row, h, b, a.seed_lo, a.seed_hi);
+                const float z0 = (w0 & 0xFFFFu) >= a.drop_t ? a.drop_scale : 0.f;
+                const float z1 = (w0 >> 16) >= a.drop_t ? a.drop_scale : 0.f;
+                const float z2 = (w1 & 0xFFFFu) >= a.drop_t ? a.drop_scale : 0.f;
+                const float z3 = (w1 >> 16) >= a.drop_t ? a.drop_scale : 0.f;
+                s0 = pack_bf16x2(p0.x * z0, p0.y * z1);
+                s1 = pack_bf16x2(p1.x * z2, p1.y * z3);
+              }
+              pk[ii * 16 + (c >> 1)] = s0;
+              pk[ii * 16 + (c >> 1) + 1] = s1;
               ex0 = fadd2(ex0, p0);
               ex1 = fadd2(ex1, p1);
               rd0 = fadd2(rd0, make_float2(__uint_as_float(k0 << 16), __uint_as_float(k0 & 0xFFFF0000u)));
@@ -729,8 +767,10 @@ static fa_status launch_fwd_impl(const FwdLaunch& L0, cudaStream_t stream) {
   using L = FwdLayout<D>;
   static PerDeviceOnce attr_once;
   if (!attr_once.run([] {
-        return cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes) ==
-               cudaSuccess;
+        return cudaFuncSetAttribute(fwd_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    L::kSmemBytes) == cudaSuccess &&
+               cudaFuncSetAttribute(fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    L::kSmemBytes) == cudaSuccess;
       }))
     return FA_ERR_CUDA;
   // a variable-length batch is one long batch of total rows for the TMA maps
@@ -758,9 +798,18 @@ static fa_status launch_fwd_impl(const FwdLaunch& L0, cudaStream_t stream) {
   a.n_pairs = (L0.Nq + 255) / 256;
   a.n_items = a.n_pairs * L0.B * L0.H;
   a.timeout_ns = L0.timeout_ns;
+  a.key_mask = L0.key_mask;
+  a.km_words = (L0.Nk + 31) / 32;
+  a.drop_t = L0.drop_t;
+  a.drop_scale = L0.drop_t ? (float)(65536.0 / (65536.0 - (double)L0.drop_t)) : 1.f;
+  a.seed_lo = (uint32_t)(L0.seed & 0xFFFFFFFFull);
+  a.seed_hi = (uint32_t)(L0.seed >> 32);
   const int grid = std::min(a.n_items, num_sms() * 1);
   prof_before(stream, kKFwd);
-  fwd_kernel<D><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);
+  if (a.drop_t != 0u)
+    fwd_kernel<D, true><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);
+  else
+    fwd_kernel<D, false><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);
   const cudaError_t err = cudaGetLastError();
   prof_after(stream, kKFwd);
   return err == cudaSuccess ? FA_OK : FA_ERR_CUDA;

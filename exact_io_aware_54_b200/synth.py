@@ -91,3 +91,25 @@ def paged_decode_inputs(seed: int, lengths, H: int, d: int, page_size: int, spar
     k_pages = _normal((num_pages, page_size, H, d), seed + 1, device)
     v_pages = _normal((num_pages, page_size, H, d), seed + 2, device)
     return q, k_pages, v_pages, table, lengths.to(torch.int32)
+
+
+def key_mask_inputs(seed: int, B: int, Nk: int, keep: float = 0.6, pad_to=None):
+    """A key-padding mask: [B, Nk] bool (True = the key takes part) and the same bits
+    packed for the library, int32 [B, ceil(Nk / 32)] (bit j % 32 of word j / 32).
+
+    Keys are kept with probability `keep`, drawn from a seeded generator; with
+    `pad_to` = [L_0, ..., L_{B-1}] the mask is instead right padding (keys j < L_b
+    kept).  The packing is the only transformation: layout, not arithmetic."""
+    if pad_to is not None:
+        mask = torch.arange(Nk)[None, :] < torch.as_tensor(pad_to, dtype=torch.int64)[:, None]
+    else:
+        g = torch.Generator(device="cpu")
+        g.manual_seed(int(seed))
+        mask = torch.rand(B, Nk, generator=g) < keep
+    words = (Nk + 31) // 32
+    bits = torch.zeros(B, words * 32, dtype=torch.int64)
+    bits[:, :Nk] = mask.to(torch.int64)
+    weights = (torch.ones(32, dtype=torch.int64) << torch.arange(32, dtype=torch.int64))
+    packed = (bits.view(B, words, 32) * weights).sum(-1)
+    packed = torch.where(packed >= 2 ** 31, packed - 2 ** 32, packed).to(torch.int32)
+    return mask, packed

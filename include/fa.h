@@ -151,6 +151,42 @@ FA_API fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, cons
                                void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Forward and backward passes with a key-padding mask and dropout (the padding
+ * mask and dropout the pages list among the semantics a fused attention kernel has
+ * to match, "FlashAttention saves IO, not N^2 work", section 8; both inside the one
+ * kernel, with dropout's mask generated again in the backward pass rather than
+ * stored, "AI Bible 13", section 03).  Arguments, layouts and results are those of
+ * fa_fwd and fa_bwd, plus
+ *   key_mask  : device uint32 [B, (Nk + 31) / 32], 4-byte aligned, or NULL for no
+ *               mask; bit j % 32 of word j / 32 is set when key j of batch element
+ *               b takes part.  A masked key is excluded like a causally masked one
+ *               (both apply when both are set; the causal alignment still counts
+ *               all Nk keys).  A row left with no key gets O = 0 and LSE = -inf; a
+ *               masked key gets dK = dV = 0.  Bits past key Nk - 1 are ignored.
+ *   dropout_p : probability of dropping each (query, key) probability, 0 <= p < 1
+ *               (rounded to t / 65536 with t = round(65536 p); FA_ERR_INVALID_ARG
+ *               outside that range).  The output is O = (P o Z) V with Z = keep /
+ *               (1 - t / 65536), P the softmax of the unmasked keys; LSE stays that
+ *               of the undropped softmax.
+ *   seed      : 64-bit seed of the dropout draws.  Element (b, h, i, j) uses
+ *               Philox4x32-10 (Salmon et al., SC'11) keyed by the seed (low word
+ *               first) with counter (j / 2, i / 4, h, b): word i % 4, low 16 bits
+ *               for even j, high 16 bits for odd j; kept when those bits >= t.
+ * The backward pass takes the same key_mask, dropout_p and seed as its forward,
+ * and that forward's O and LSE.  NULL key_mask with dropout_p = 0 makes the calls
+ * fa_fwd and fa_bwd.
+ */
+FA_API fa_status fa_fwd_masked(const void* q, const void* k, const void* v, void* o, float* lse,
+                               const uint32_t* key_mask, float dropout_p, unsigned long long seed, int B, int H,
+                               int Nq, int Nk, int d, int causal, float softmax_scale, void* workspace,
+                               size_t workspace_bytes, cudaStream_t stream);
+FA_API fa_status fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, const void* do_,
+                               const float* lse, void* dq, void* dk, void* dv, const uint32_t* key_mask,
+                               float dropout_p, unsigned long long seed, int B, int H, int Nq, int Nk, int d,
+                               int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+
+/*
  * Split-KV decode over a ragged, packed KV cache.
  *   q           : [B, H, d] bf16 (one query row per sequence: Nq must be 1)
  *   k, v        : [total_kv, H, d] bf16; sequence b owns rows

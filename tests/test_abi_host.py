@@ -192,6 +192,36 @@ def test_bwd_varlen_argument_validation(lib):
     assert fa.fa_bwd_varlen_workspace_size(4, 300, 80) == 0
 
 
+def test_masked_argument_validation(lib):
+    def fwd(**kw):
+        a = dict(q=P, k=P, v=P, o=P, lse=P, km=P, p=0.1, B=2, H=4, Nq=64, Nk=70, d=64, ws=P, wsb=1 << 20)
+        a.update(kw)
+        return lib.fa_fwd_masked(a["q"], a["k"], a["v"], a["o"], a["lse"], a["km"], a["p"], 7, a["B"], a["H"],
+                                 a["Nq"], a["Nk"], a["d"], 1, 0.0, a["ws"], a["wsb"], None)
+
+    def bwd(**kw):
+        a = dict(q=P, k=P, v=P, o=P, do=P, lse=P, dq=P, dk=P, dv=P, km=P, p=0.0, B=2, H=4, Nq=64, Nk=70, d=128, ws=P,
+                 wsb=1 << 30)
+        a.update(kw)
+        return lib.fa_bwd_masked(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"], a["dv"],
+                                 a["km"], a["p"], 7, a["B"], a["H"], a["Nq"], a["Nk"], a["d"], 0, 0.0, a["ws"],
+                                 a["wsb"], None)
+
+    assert fwd(q=None) == ST["FA_ERR_INVALID_ARG"]
+    assert fwd(Nk=0) == ST["FA_ERR_INVALID_ARG"]
+    assert fwd(d=96) == ST["FA_ERR_UNSUPPORTED"]
+    assert fwd(km=P + 2) == ST["FA_ERR_ALIGNMENT"]
+    assert fwd(ws=None) == ST["FA_ERR_WORKSPACE"]
+    assert fwd(p=-0.1) == ST["FA_ERR_INVALID_ARG"]
+    assert fwd(p=1.0) == ST["FA_ERR_INVALID_ARG"]
+    assert fwd(p=0.999995) == ST["FA_ERR_INVALID_ARG"]  # rounds to t = 65536: nothing would be kept
+    assert fwd(p=float("nan")) == ST["FA_ERR_INVALID_ARG"]
+    assert bwd(p=1.5) == ST["FA_ERR_INVALID_ARG"]
+    assert bwd(dk=None) == ST["FA_ERR_INVALID_ARG"]
+    assert bwd(km=P + 1) == ST["FA_ERR_ALIGNMENT"]
+    assert bwd(wsb=16) == ST["FA_ERR_WORKSPACE"]
+
+
 def test_selftest_argument_validation(lib):
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint, ctypes.c_void_p]
     assert lib.fa_selftest_wait_timeout(None, 256, 100, None) == ST["FA_ERR_WORKSPACE"]
