@@ -284,7 +284,7 @@ def run_ours(args, rank, world, local_rank):
     # since the timed region began, so that the clock record holds enough samples
     # of this workload even when the timed region itself is short.
     soak = 0
-    while time.perf_counter() - t_wall0 < 1.0:
+    while not args.profile and time.perf_counter() - t_wall0 < 1.0:
         for _ in range(20):
             step()
         soak += 20
@@ -329,7 +329,7 @@ def run_ours(args, rank, world, local_rank):
 
     # end to end through the public API: pinned host inputs in, gradients out, every step
     e2e = None
-    if True:
+    if not args.profile:
         hq, hk, hv, hdo = (x.cpu().pin_memory() for x in (q, k, v, do))
         hdq, hdk, hdv = (torch.empty(x.shape, dtype=x.dtype).pin_memory() for x in (dq, dk, dv))
         dq2, dk2, dv2 = torch.empty_like(dq), torch.empty_like(dk), torch.empty_like(dv)
@@ -356,12 +356,12 @@ def run_ours(args, rank, world, local_rank):
                "h2d_bytes_per_step": hin, "d2h_bytes_per_step": hout, "ms_per_step": round(e_max, 4)}
         del hq, hk, hv, hdo, hdq, hdk, hdv, dq2, dk2, dv2, q2, k2, v2, do2
 
-    extra = run_extra(args, fa, synth, dev, pk) if (rank == 0 and not args.no_extra) else None
+    extra = run_extra(args, fa, synth, dev, pk) if (rank == 0 and not args.no_extra and not args.profile) else None
     del q, k, v, do, o, lse, dq, dk, dv
     torch.cuda.empty_cache()
 
     cpu_base = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile:
         cpu_base = cpu_baseline(args.cpu_seconds)
 
     if rank != 0:
@@ -401,9 +401,9 @@ def run_extra(args, fa, synth, dev, pk, only=None):
     if want("decode_single"):
         _extra_decode_single(out, n, flush, fa, synth, dev, pk)
     if want("decode_batched"):
-        _extra_decode_batched(out, n, flush, fa, synth, dev, pk)
+        _extra_decode_batched(out, n, flush, fa, synth, dev, pk, args.decode_seqs)
     if want("decode_paged"):
-        _extra_decode_paged(out, n, flush, fa, synth, dev, pk)
+        _extra_decode_paged(out, n, flush, fa, synth, dev, pk, args.decode_seqs)
     if want("long16k"):
         _extra_long16k(out, n, flush, fa, synth, dev, pk)
     if want("dropout_gpt2m"):
@@ -510,30 +510,31 @@ def _extra_decode_single(out, n, flush, fa, synth, dev, pk):
     del q, k, v, cu, o, lse
 
 
-def _extra_decode_batched(out, n, flush, fa, synth, dev, pk):
+def _extra_decode_batched(out, n, flush, fa, synth, dev, pk, n_seqs=64):
     # decode: 64 ragged sequences, lengths U[512, 16384]
-    lengths = synth.ragged_lengths(synth.SEEDS["decode"], 64, 512, 16384)
+    lengths = synth.ragged_lengths(synth.SEEDS["decode"], 64, 512, 16384)[:n_seqs]
     q, k, v, cu = synth.decode_inputs(synth.SEEDS["decode"], lengths, 32, 128, device=dev)
     cu = cu.to(dev)
     maxL = int(lengths.max())
     o = torch.empty_like(q)
-    lse = torch.empty(64, 32, dtype=torch.float32, device=dev)
+    lse = torch.empty(len(lengths), 32, dtype=torch.float32, device=dev)
 
     def g2(_i):
         fa.fa_decode_splitkv(q, k, v, cu, maxL, out=o, lse=lse)
     out["decode_batched_ragged"] = _hbm_entry(_timed(g2, n, flush), 2 * 2 * 32 * 128 * int(lengths.sum()), pk,
-                                              {"splits": fa.fa_decode_num_splits(64, 32, maxL, 128, 0)})
+                                              {"splits": fa.fa_decode_num_splits(len(lengths), 32, maxL, 128, 0),
+                                               "sequences": len(lengths)})
     del q, k, v, cu, o, lse
 
 
-def _extra_decode_paged(out, n, flush, fa, synth, dev, pk):
+def _extra_decode_paged(out, n, flush, fa, synth, dev, pk, n_seqs=64):
     # the same 64 ragged sequences in a paged cache: pages of 64 keys in seeded random order
-    lengths = synth.ragged_lengths(synth.SEEDS["decode"], 64, 512, 16384)
+    lengths = synth.ragged_lengths(synth.SEEDS["decode"], 64, 512, 16384)[:n_seqs]
     q, kp, vp, table, lens = synth.paged_decode_inputs(synth.SEEDS["decode"], lengths, 32, 128, 64, device=dev)
     table, lens = table.to(dev), lens.to(dev)
     maxL = int(lengths.max())
     o = torch.empty_like(q)
-    lse = torch.empty(64, 32, dtype=torch.float32, device=dev)
+    lse = torch.empty(len(lengths), 32, dtype=torch.float32, device=dev)
 
     def g3(_i):
         fa.fa_decode_paged(q, kp, vp, table, lens, maxL, out=o, lse=lse)
@@ -650,6 +651,12 @@ def main():
     ap.add_argument("--batch", type=int, default=0,
                     help="override B of the step (small cases for profiler captures; 0 = the workload's B=64)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--profile", action="store_true",
+                    help="time only the K steps (no clock soak, end-to-end leg, other workloads or CPU baseline): "
+                         "the command profiler captures run")
+    ap.add_argument("--decode-seqs", type=int, default=64,
+                    help="sequences of the batched decode workloads (the first ones of the 64 seeded lengths; "
+                         "fewer for profiler captures)")
     ap.add_argument("--extra-launches", type=int, default=50,
                     help="timed launches per other workload (at least 50)")
     args = ap.parse_args()

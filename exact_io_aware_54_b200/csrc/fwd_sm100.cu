@@ -10,7 +10,8 @@
 //
 // B200 design
 //  * Work item = (b, h, pair of 128-row query tiles).  Persistent grid, one CTA
-//    per SM; items are taken round-robin, heaviest (latest causal rows) first.
+//    per SM; items are numbered heaviest (latest causal rows) first and dealt to
+//    the CTAs in a snake order over rounds.
 //  * Warp roles (384 threads, three warpgroups):
 //      warp 0      TMA producer: Q tiles, then K/V tiles through a ring of smem
 //                  slots (mbarrier full/empty pairs).
@@ -81,13 +82,26 @@ __host__ __device__ constexpr uint32_t tm_o(int t) {
   return sep_p<D>() ? 384u + 64u * t : 256u + t * 128u;
 }
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Polls before a sleeping wait: the MMA issuer (one thread, on the tensor core's
+// critical path) and the softmax warps waiting for their scores.
+#ifndef FA_FWD_MMA_SPINS
+#define FA_FWD_MMA_SPINS 0
+#endif
+#ifndef FA_FWD_SOFTMAX_SPINS
+#define FA_FWD_SOFTMAX_SPINS 0
+#endif
+constexpr int kMmaSpins = FA_FWD_MMA_SPINS;
+constexpr int kSoftmaxSpins = FA_FWD_SOFTMAX_SPINS;
 // Every kExpFmaEvery-th group of four probabilities computes one pair of its
 // exponentials on the FMA pipes (exp2_fma2) instead of the MUFU unit: a quarter
 // of them at d = 64, an eighth at d = 128 (where the tile has twice the MMA work
 // per exponential).  Measured on B200 against other splits.
+#ifndef FA_FWD_EXP_FMA_EVERY_128
+#define FA_FWD_EXP_FMA_EVERY_128 4
+#endif
 template <int D>
 __host__ __device__ constexpr int exp_fma_every() {
-  return D == 64 ? 2 : 4;
+  return D == 64 ? 2 : FA_FWD_EXP_FMA_EVERY_128;
 }
 
 template <int D>
@@ -139,6 +153,16 @@ __device__ __forceinline__ void tile_mask_words(const FwdArgs& a, int b, int j, 
   const uint32_t* row = a.key_mask + (size_t)b * a.km_words;
 #pragma unroll
   for (int i = 0; i < 4; ++i) w[i] = (j * 4 + i < a.km_words) ? __ldg(row + j * 4 + i) : 0u;
+}
+
+// The item a CTA takes in round r.  Items are numbered heaviest first; the rounds
+// alternate direction over the CTAs (a snake), so that a CTA that took one of the
+// heaviest items of a round takes one of the lightest of the next.  With causal
+// masking the static round-robin order leaves the busiest CTA about 13% above the
+// mean at B = 1, H = 32, N = 8192; the snake brings that to about 2%.
+__device__ __forceinline__ int item_of_round(int r) {
+  const int g = (int)gridDim.x, c = (int)blockIdx.x;
+  return r * g + ((r & 1) ? (g - 1 - c) : c);
 }
 
 __device__ __forceinline__ void item_coords(const FwdArgs& a, int w, int& b, int& h, int& pair) {
@@ -201,9 +225,10 @@ __device__ __forceinline__ void record_timeout(int* status, volatile int* abort_
 }
 
 // Warp-uniform bounded wait: lane 0 waits, the verdict is broadcast.
+template <int kSpins = 0>
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, unsigned long long timeout_ns) {
   bool ok = true;
-  if (lane_id() == 0) ok = mbar_wait(bar, parity, timeout_ns);
+  if (lane_id() == 0) ok = mbar_wait_spin<kSpins>(bar, parity, timeout_ns);
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
@@ -297,7 +322,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t item_iter = 0, g = 0;
-      for (int w = blockIdx.x; w < a.n_items && !*abort_flag; w += gridDim.x) {
+      for (int r = 0; r * (int)gridDim.x < a.n_items && !*abort_flag; ++r) {
+        const int w = item_of_round(r);
+        if (w >= a.n_items) continue;
         int b, h, pair;
         item_coords(a, w, b, h, pair);
         const SeqView sv = seq_view(a, b);
@@ -342,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) {
         if (!ok) return false;
-        if (!mbar_wait(bar, parity, a.timeout_ns) || *abort_flag) {
+        if (!mbar_wait_spin<kMmaSpins>(bar, parity, a.timeout_ns) || *abort_flag) {
           record_timeout(a.status, abort_flag);
           ok = false;
         }
@@ -351,7 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ring slots alternate K, V per KV step: K of step j at g, V at g + 1
       uint32_t item_iter = 0, g = 0;
       uint32_t cnt[2] = {0, 0};  // Q K^T (warp 1) or P V (warp 2) MMAs issued per query tile
-      for (int w = blockIdx.x; w < a.n_items && ok; w += gridDim.x) {
+      for (int r = 0; r * (int)gridDim.x < a.n_items && ok; ++r) {
+        const int w = item_of_round(r);
+        if (w >= a.n_items) continue;
         int b, h, pair;
         item_coords(a, w, b, h, pair);
         const SeqView sv = seq_view(a, b);
@@ -425,13 +454,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       auto wait_or_abort = [&](uint64_t* bar, uint32_t parity) {
         if (!ok) return false;
-        if (!mbar_wait(bar, parity, a.timeout_ns) || *abort_flag) {
+        if (!mbar_wait_spin<kMmaSpins>(bar, parity, a.timeout_ns) || *abort_flag) {
           record_timeout(a.status, abort_flag);
           ok = false;
         }
         return ok;
       };
-      for (int w = blockIdx.x; w < a.n_items && ok; w += gridDim.x) {
+      for (int r = 0; r * (int)gridDim.x < a.n_items && ok; ++r) {
+        const int w = item_of_round(r);
+        if (w >= a.n_items) continue;
         int b, h, pair;
         item_coords(a, w, b, h, pair);
         const SeqView sv = seq_view(a, b);
@@ -516,7 +547,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* q_tile = smem + L::kOffQ + t * L::kTileBytes;
     const uint32_t q_tile_u32 = smem_u32(q_tile);
 
-    for (int w = blockIdx.x; w < a.n_items; w += gridDim.x) {
+    for (int r = 0; r * (int)gridDim.x < a.n_items; ++r) {
+      const int w = item_of_round(r);
+      if (w >= a.n_items) continue;
       if (*abort_flag) break;
       int b, h, pair;
       item_coords(a, w, b, h, pair);
@@ -553,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float le = 0.f;        // running sum of the unrounded probabilities (gives lse)
       bool ok = true;
       for (int j = 0; j < nkv; ++j, ++s_cnt) {
-        if (!warp_wait(bar_s_full + t, s_cnt & 1, a.timeout_ns) || *abort_flag) {
+        if (!warp_wait<kSoftmaxSpins>(bar_s_full + t, s_cnt & 1, a.timeout_ns) || *abort_flag) {
           if (lane == 0) record_timeout(a.status, abort_flag);
           ok = false;
           break;
