@@ -65,6 +65,9 @@ struct FwdLaunch {
   const int32_t* cu_q = nullptr;
   const int32_t* cu_k = nullptr;
   int total_q = 0, total_k = 0;
+  // block-sparse mask (dense batches): device uint8 [H, ceil(Nq/128), ceil(Nk/128)],
+  // 0 skips the (query tile, KV tile) block; null for dense attention
+  const uint8_t* block_mask = nullptr;
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;
@@ -89,6 +92,7 @@ struct BwdLaunch {
   const int32_t* cu_q = nullptr;
   const int32_t* cu_k = nullptr;
   int total_q = 0, total_k = 0;
+  const uint8_t* block_mask = nullptr;  // as for the forward
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;

@@ -91,3 +91,24 @@ def paged_decode_inputs(seed: int, lengths, H: int, d: int, page_size: int, spar
     k_pages = _normal((num_pages, page_size, H, d), seed + 1, device)
     v_pages = _normal((num_pages, page_size, H, d), seed + 2, device)
     return q, k_pages, v_pages, table, lengths.to(torch.int32)
+
+
+def block_mask_inputs(seed: int, H: int, Nq: int, Nk: int, keep: float = 0.5, pattern: str = "random"):
+    """A block-sparse mask uint8 [H, ceil(Nq / 128), ceil(Nk / 128)] (1 = the block is
+    computed).  "random": blocks kept with probability `keep` (seeded); "local": a
+    band of the diagonal block and its left neighbour; "strided": every other key
+    tile.  Layout only: no attention arithmetic."""
+    nq, nk = (Nq + 127) // 128, (Nk + 127) // 128
+    if pattern == "random":
+        g = torch.Generator(device="cpu")
+        g.manual_seed(int(seed))
+        m = torch.rand(H, nq, nk, generator=g) < keep
+    elif pattern == "local":
+        i = torch.arange(nq)[:, None]
+        j = torch.arange(nk)[None, :]
+        m = ((j == i) | (j == i - 1)).expand(H, nq, nk)
+    elif pattern == "strided":
+        m = (torch.arange(nk)[None, None, :] % 2 == 0).expand(H, nq, nk)
+    else:
+        raise ValueError(pattern)
+    return m.to(torch.uint8).contiguous()
