@@ -314,7 +314,8 @@ def _rotating(make, total_bytes_of_one):
     return [make(i) for i in range(n)]
 
 
-EXTRA_WORKLOADS = ("prefill8k", "prefill_varlen", "decode_single", "decode_batched", "decode_paged", "long16k")
+EXTRA_WORKLOADS = ("prefill8k", "prefill_varlen", "decode_single", "decode_batched", "decode_paged", "long16k",
+                   "blocksparse16k")
 
 
 def run_extra(args, fa, synth, dev, pk, only=None):
@@ -333,7 +334,39 @@ def run_extra(args, fa, synth, dev, pk, only=None):
         _extra_decode_paged(out, iters, fa, synth, dev, pk)
     if want("long16k"):
         _extra_long16k(out, iters, fa, synth, dev, pk)
+    if want("blocksparse16k"):
+        _extra_blocksparse16k(out, iters, fa, synth, dev, pk)
     return out
+
+
+def _extra_blocksparse16k(out, iters, fa, synth, dev, pk):
+    # block-sparse training step, B=1 H=16 N=16384 d=64 causal, local pattern (each
+    # query tile keeps its own and the previous key tile): algorithmic work counts the
+    # kept blocks' pairs only
+    N, H, d = 16384, 16, 64
+    q, k, v, do = synth.prefill_inputs(synth.SEEDS["long16k"], 1, N, N, H, d, with_dout=True, device=dev)
+    bm = synth.block_mask_inputs(0, H, N, N, pattern="local").to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(1, H, N, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def h(i):
+        fa.fa_fwd_blocksparse(q, k, v, bm, causal=True, out=o, lse=lse)
+        fa.fa_bwd_blocksparse(q, k, v, o, do, lse, bm, causal=True, dq=dq, dk=dk, dv=dv)
+    for i in range(3):
+        h(i)
+    ms = device_time_ms(h, max(5, iters // 2))
+    # pairs per head: the diagonal block (causal triangle, 128 * 129 / 2) for every
+    # query tile and a full previous block for all but the first
+    nt = N // 128
+    pairs = nt * 128 * 129 // 2 + (nt - 1) * 128 * 128
+    fl = (4 + 10) * H * d * pairs
+    tf = fl / (ms * 1e-3) / 1e12
+    out["blocksparse16k_fwd_bwd"] = {"ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                                     "frac_of_peak": round(tf / pk["bf16_tflops"], 4),
+                                     "kept_fraction_of_causal_blocks": round((2 * nt - 1) / (nt * (nt + 1) / 2), 4)}
+    del q, k, v, do, o, lse, dq, dk, dv, bm
+    torch.cuda.empty_cache()
 
 
 def _extra_prefill(out, iters, fa, synth, dev, pk):
