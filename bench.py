@@ -383,7 +383,7 @@ def run_ours(args, rank, world, local_rank):
 
 
 EXTRA_WORKLOADS = ("prefill8k", "prefill_varlen", "decode_single", "decode_batched", "decode_paged", "long16k",
-                   "dropout_gpt2m")
+                   "dropout_gpt2m", "blocksparse16k")
 
 
 def run_extra(args, fa, synth, dev, pk, only=None):
@@ -408,6 +408,8 @@ def run_extra(args, fa, synth, dev, pk, only=None):
         _extra_long16k(out, n, flush, fa, synth, dev, pk)
     if want("dropout_gpt2m"):
         _extra_dropout_gpt2m(out, n, flush, fa, synth, dev, pk)
+    if want("blocksparse16k"):
+        _extra_blocksparse16k(out, n, flush, fa, synth, dev, pk)
     del flush
     torch.cuda.empty_cache()
     return out
@@ -451,6 +453,30 @@ def _extra_dropout_gpt2m(out, n, flush, fa, synth, dev, pk):
     out["dropout_gpt2m_fwd_bwd"] = _tensor_entry(_timed(h, n, None), fl, pk, {
         "dropout_p": 0.1, "l2": "no flush: the inputs of one step (640 MiB) exceed the L2"})
     del q, k, v, do, o, lse, dq, dk, dv
+
+
+def _extra_blocksparse16k(out, n, flush, fa, synth, dev, pk):
+    # block-sparse training step, B=1 H=16 N=16384 d=64 causal, local pattern (each
+    # query tile keeps its own and the previous key tile): algorithmic work counts the
+    # kept blocks' pairs only
+    N, H, d = 16384, 16, 64
+    q, k, v, do = synth.prefill_inputs(synth.SEEDS["long16k"], 1, N, N, H, d, with_dout=True, device=dev)
+    bm = synth.block_mask_inputs(0, H, N, N, pattern="local").to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty(1, H, N, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+
+    def h(_i):
+        fa.fa_fwd_blocksparse(q, k, v, bm, causal=True, out=o, lse=lse)
+        fa.fa_bwd_blocksparse(q, k, v, o, do, lse, bm, causal=True, dq=dq, dk=dk, dv=dv)
+    # pairs per head: the diagonal block (causal triangle, 128 * 129 / 2) for every
+    # query tile and a full previous block for all but the first
+    nt = N // 128
+    pairs = nt * 128 * 129 // 2 + (nt - 1) * 128 * 128
+    fl = (4 + 10) * H * d * pairs
+    out["blocksparse16k_fwd_bwd"] = _tensor_entry(_timed(h, n, flush), fl, pk, {
+        "kept_fraction_of_causal_blocks": round((2 * nt - 1) / (nt * (nt + 1) / 2), 4)})
+    del q, k, v, do, o, lse, dq, dk, dv, bm
 
 
 def _extra_prefill(out, n, flush, fa, synth, dev, pk):

@@ -23,9 +23,9 @@ import threading
 import torch
 
 __all__ = [
-    "FAError", "lib_path", "load", "fa_fwd", "fa_bwd", "fa_fwd_masked", "fa_bwd_masked", "fa_fwd_varlen",
-    "fa_bwd_varlen", "fa_decode_splitkv", "fa_decode_splitkv_noalloc", "fa_decode_splitkv_checked",
-    "fa_decode_paged", "fa_check", "fa_fwd_workspace_size", "fa_bwd_workspace_size",
+    "FAError", "lib_path", "load", "fa_fwd", "fa_bwd", "fa_fwd_masked", "fa_bwd_masked", "fa_fwd_blocksparse",
+    "fa_bwd_blocksparse", "fa_fwd_varlen", "fa_bwd_varlen", "fa_decode_splitkv", "fa_decode_splitkv_noalloc",
+    "fa_decode_splitkv_checked", "fa_decode_paged", "fa_check", "fa_fwd_workspace_size", "fa_bwd_workspace_size",
     "fa_bwd_varlen_workspace_size", "fa_decode_workspace_size", "fa_decode_num_splits",
     "fa_version", "STATUS",
 ]
@@ -77,9 +77,11 @@ def load():
         _u64 = ctypes.c_ulonglong
         lib.fa_fwd_masked.argtypes = [_vp] * 6 + [_f, _u64] + [_i] * 6 + [_f, _vp, _sz, _vp]
         lib.fa_bwd_masked.argtypes = [_vp] * 10 + [_f, _u64] + [_i] * 6 + [_f, _vp, _sz, _vp]
+        lib.fa_fwd_blocksparse.argtypes = [_vp] * 6 + [_i] * 6 + [_f, _vp, _sz, _vp]
+        lib.fa_bwd_blocksparse.argtypes = [_vp] * 10 + [_i] * 6 + [_f, _vp, _sz, _vp]
         for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_decode_splitkv, lib.fa_decode_splitkv_noalloc,
                    lib.fa_decode_splitkv_checked, lib.fa_decode_paged, lib.fa_fwd_varlen, lib.fa_bwd_varlen,
-                   lib.fa_fwd_masked, lib.fa_bwd_masked):
+                   lib.fa_fwd_masked, lib.fa_bwd_masked, lib.fa_fwd_blocksparse, lib.fa_bwd_blocksparse):
             fn.restype = _i
         lib.fa_fwd_workspace_size.argtypes = [_i] * 5
         lib.fa_fwd_workspace_size.restype = _sz
@@ -251,6 +253,57 @@ def fa_bwd_masked(q, k, v, o, dout, lse, key_mask=None, dropout_p: float = 0.0, 
                            Nk, d, int(bool(causal)), _scale(softmax_scale), ws.data_ptr(), ws.numel(),
                            _stream_ptr(q.device))
     _raise("fa_bwd_masked", st)
+    return dq, dk, dv
+
+
+def _check_block_mask(block_mask, H, Nq, Nk):
+    _check_tensor("block_mask", block_mask, torch.uint8, (H, (Nq + 127) // 128, (Nk + 127) // 128))
+
+
+def fa_fwd_blocksparse(q, k, v, block_mask, causal: bool = False, softmax_scale=None, out=None, lse=None, ws=None):
+    """Block-sparse forward.  block_mask: uint8 [H, ceil(Nq/128), ceil(Nk/128)] on the
+    device (0 skips the block).  Returns (o, lse) as fa_fwd."""
+    lib = load()
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    _check_tensor("q", q, torch.bfloat16)
+    _check_tensor("k", k, torch.bfloat16, (B, Nk, H, d))
+    _check_tensor("v", v, torch.bfloat16, (B, Nk, H, d))
+    _check_block_mask(block_mask, H, Nq, Nk)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_tensor("out", out, torch.bfloat16, q.shape)
+    _check_tensor("lse", lse, torch.float32, (B, H, Nq))
+    if ws is None:
+        ws = workspace(lib.fa_fwd_workspace_size(B, H, Nq, Nk, d), q.device, "fwd")
+    st = lib.fa_fwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                block_mask.data_ptr(), B, H, Nq, Nk, d, int(bool(causal)), _scale(softmax_scale),
+                                ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
+    _raise("fa_fwd_blocksparse", st)
+    return out, lse
+
+
+def fa_bwd_blocksparse(q, k, v, o, dout, lse, block_mask, causal: bool = False, softmax_scale=None, dq=None,
+                       dk=None, dv=None, ws=None):
+    """Backward of fa_fwd_blocksparse with the same block_mask.  Returns (dq, dk, dv) in bf16."""
+    lib = load()
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    for name, t, shp in (("q", q, None), ("k", k, (B, Nk, H, d)), ("v", v, (B, Nk, H, d)), ("o", o, q.shape),
+                         ("dout", dout, q.shape)):
+        _check_tensor(name, t, torch.bfloat16, shp)
+    _check_tensor("lse", lse, torch.float32, (B, H, Nq))
+    _check_block_mask(block_mask, H, Nq, Nk)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if ws is None:
+        ws = workspace(lib.fa_bwd_workspace_size(B, H, Nq, Nk, d), q.device, "bwd")
+    st = lib.fa_bwd_blocksparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                                lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), block_mask.data_ptr(),
+                                B, H, Nq, Nk, d, int(bool(causal)), _scale(softmax_scale), ws.data_ptr(), ws.numel(),
+                                _stream_ptr(q.device))
+    _raise("fa_bwd_blocksparse", st)
     return dq, dk, dv
 
 

@@ -99,6 +99,10 @@ struct BwdArgs {
   uint32_t drop_t;
   float drop_scale;
   uint32_t seed_lo, seed_hi;
+  // block-sparse mask (null: dense): [H, nqb, nkb] bytes over (128-row query tile,
+  // 128-key tile); 0 skips the block
+  const uint8_t* block_mask;
+  int nqb, nkb;
 };
 
 // Where one dS block's dropout draws come from: its key, head and batch element.
@@ -113,6 +117,24 @@ struct DropCtx {
 __device__ __forceinline__ bool key_attended(const BwdArgs& a, int b, int key) {
   if (a.key_mask == nullptr) return true;
   return (__ldg(a.key_mask + (size_t)b * a.km_words + (key >> 5)) >> (key & 31)) & 1u;
+}
+
+
+// Query tile i and key tile j of head h form a computed block (always in the dense
+// instantiation).
+template <bool kSparse>
+__device__ __forceinline__ bool bwd_block_kept(const BwdArgs& a, int h, int i, int j) {
+  if constexpr (!kSparse) return true;
+  return __ldg(a.block_mask + ((size_t)h * a.nqb + i) * a.nkb + j) != 0;
+}
+// The first query tile >= i that key tile j of head h keeps (end when none; i itself
+// in the dense instantiation).
+template <bool kSparse>
+__device__ __forceinline__ int next_kept_q(const BwdArgs& a, int h, int j, int i, int end) {
+  if constexpr (kSparse) {
+    while (i < end && !bwd_block_kept<true>(a, h, i, j)) ++i;
+  }
+  return i;
 }
 
 // Where sequence b lives.  Dense: batch element b of the [B, N, H, D] tensors.
@@ -281,8 +303,9 @@ __device__ __forceinline__ void ds_block(const uint32_t (&sv)[kN], const uint32_
   }
 }
 
-// kDrop: dropout (a separate instantiation, so the plain kernel is unchanged)
-template <int D, bool kDrop>
+// kDrop: dropout; kSparse: block-sparse (separate instantiations, so the plain
+// kernel is unchanged)
+template <int D, bool kDrop, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -321,7 +344,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_qtiles = (sq.lq + 127) >> 7;
   int i_first = 0;
   if (a.causal) i_first = max(0, j * 128 - (sq.lk - sq.lq)) >> 7;
-  const int n_iters = n_qtiles - i_first;  // >= 1 when the sequence has queries
+  int n_iters = n_qtiles - i_first;  // >= 1 when the sequence has queries
+  if constexpr (kSparse) {  // the kept query tiles only
+    n_iters = 0;
+    for (int i = i_first; i < n_qtiles; ++i) n_iters += bwd_block_kept<true>(a, h, i, j) ? 1 : 0;
+  }
   if (n_iters <= 0) {
     store_zero_dkv<D>(a, sq, j, h, threadIdx.x, blockDim.x);
     return;
@@ -372,9 +399,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_4d(smem + L::kOffV + bx * L::kBoxBytes, &tmV, bar_kv_full, bx * 64, h, sq.tk + j * 128, sq.tb);
       }
     }
-    for (int it = 0; it < n_iters; ++it) {
+    int qi = next_kept_q<kSparse>(a, h, j, i_first, n_qtiles);  // query tile of step it
+    for (int it = 0; it < n_iters; ++it, qi = next_kept_q<kSparse>(a, h, j, qi + 1, n_qtiles)) {
       const int st = it % L::kQStages;
-      const int q0 = (i_first + it) * 128;
+      const int q0 = qi * 128;
       // -lse in log2 units (-inf for rows past Nq or with no visible key: P = 0 there)
       // and -D, negated so that the dS warps use them as addends.  The global loads
       // are issued before waiting for the stage so that their latency overlaps it.
@@ -489,7 +517,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     // dQ tile of query tile `it`: this group's D/2 columns, fp32 vector reductions
     // into the accumulator
-    auto drain_dq = [&](int it) -> bool {
+    auto drain_dq = [&](int it, int q_first) -> bool {
       if (!warp_wait_b(bar_dq_full, it & 1, a.timeout_ns) || *abort_flag) return false;
       tc_fence_after();
       uint32_t g[D / 64][32];
@@ -500,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int cc = 1; cc < D / 64; ++cc) reg_pin(g[cc]);
       tc_fence_before();
       mbar_arrive_warp(bar_dq_empty);
-      const int q = (i_first + it) * 128 + r;
+      const int q = q_first + r;
       if (q < sq.lq) {
         float* dst = a.dq_acc + ((size_t)((long long)sq.tb * a.Nq + sq.tq + q) * a.H + h) * D + grp * (D / 2);
 #pragma unroll
@@ -513,9 +541,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
 
-    for (int it = 0; it < n_iters && ok; ++it) {
+    int qi = next_kept_q<kSparse>(a, h, j, i_first, n_qtiles);  // query tile of step it
+    for (int it = 0; it < n_iters && ok; ++it, qi = next_kept_q<kSparse>(a, h, j, qi + 1, n_qtiles)) {
       const int st = it % L::kQStages;
-      const int q0 = (i_first + it) * 128;
+      const int q0 = qi * 128;
       // the stats of this query tile are staged with it; its dS buffer must be free
       if (!warp_wait_b(bar_q_full + st, (it / L::kQStages) & 1, a.timeout_ns) ||
           !warp_wait_b(bar_ds_free + (it % L::kDsBufs), ((it / L::kDsBufs) & 1) ^ 1, a.timeout_ns) ||
@@ -561,7 +590,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       mbar_arrive_warp(bar_p_full);
       // this tile's dQ follows right after dV / dK
-      ok = drain_dq(it);
+      ok = drain_dq(it, q0);
     }
     // ---------------------------------------------------------------- dK / dV epilogue
     // group 0 stores dK (times scale) through the K tile's smem, group 1 dV through V's;
@@ -706,6 +735,7 @@ struct PipeItem {
   int j, h, i_first, n;
   BwdSeq s;
 };
+template <bool kSparse>
 __device__ __forceinline__ PipeItem pipe_item(const BwdArgs& a, int w) {
   PipeItem it;
   const int bh_count = a.B * a.H;
@@ -720,24 +750,40 @@ __device__ __forceinline__ PipeItem pipe_item(const BwdArgs& a, int w) {
   const int n_qtiles = (it.s.lq + 127) >> 7;
   it.i_first = a.causal ? (max(0, it.j * 128 - (it.s.lk - it.s.lq)) >> 7) : 0;
   it.n = n_qtiles - it.i_first;
+  if constexpr (kSparse) {  // the kept query tiles only
+    it.n = 0;
+    for (int i = it.i_first; i < n_qtiles; ++i) it.n += bwd_block_kept<true>(a, it.h, i, it.j) ? 1 : 0;
+  }
   return it;
 }
 
 // Walks the query tiles of this CTA's items (those with query tiles) in order.
+template <bool kSparse>
 struct PipeCursor {
-  int k;  // item index of this CTA (pipe_item_index)
-  int u;  // items with query tiles passed so far
-  int t;  // query tile within the item
+  int k;   // item index of this CTA (pipe_item_index)
+  int u;   // items with query tiles passed so far
+  int t;   // query tile within the item (counting the item's tiles)
+  int qi;  // that query tile's index (block-sparse instantiation)
   bool valid;
   PipeItem itm;
+  __device__ __forceinline__ int qtile() const {
+    if constexpr (kSparse) return qi;
+    return itm.i_first + t;
+  }
+  __device__ __forceinline__ void first_q(const BwdArgs& a) {
+    if constexpr (kSparse) qi = next_kept_q<true>(a, itm.h, itm.j, itm.i_first, (itm.s.lq + 127) >> 7);
+  }
   // from item k on, the first item with query tiles
   __device__ __forceinline__ void seek(const BwdArgs& a, int n_items) {
     for (;; ++k) {
       const int w = pipe_item_index(k);
       valid = w < n_items;
       if (!valid) return;
-      itm = pipe_item(a, w);
-      if (itm.n > 0) return;
+      itm = pipe_item<kSparse>(a, w);
+      if (itm.n > 0) {
+        first_q(a);
+        return;
+      }
     }
   }
   __device__ __forceinline__ void start(const BwdArgs& a, int n_items) {
@@ -747,7 +793,10 @@ struct PipeCursor {
     seek(a, n_items);
   }
   __device__ __forceinline__ void advance(const BwdArgs& a, int n_items) {
-    if (++t < itm.n) return;
+    if (++t < itm.n) {
+      if constexpr (kSparse) qi = next_kept_q<true>(a, itm.h, itm.j, qi + 1, (itm.s.lq + 127) >> 7);
+      return;
+    }
     t = 0;
     ++k;
     ++u;
@@ -757,10 +806,11 @@ struct PipeCursor {
 
 // -lse in log2 units (-inf for rows past Nq or with no visible key: P = 0) and -D of
 // four query rows per lane, negated so that the dS warps add them.
-__device__ __forceinline__ void pipe_load_stats(const BwdArgs& a, const PipeCursor& c, uint32_t lane, float (&nl2)[4],
-                                                float (&nd)[4]) {
+template <bool kSparse>
+__device__ __forceinline__ void pipe_load_stats(const BwdArgs& a, const PipeCursor<kSparse>& c, uint32_t lane,
+                                                float (&nl2)[4], float (&nd)[4]) {
   const size_t stat_row = ((size_t)c.itm.s.tb * a.H + c.itm.h) * a.stat_n + c.itm.s.tq;
-  const int q0 = (c.itm.i_first + c.t) * 128;
+  const int q0 = c.qtile() * 128;
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     const int q = q0 + lane + 32 * e;
@@ -774,7 +824,9 @@ __device__ __forceinline__ void pipe_load_stats(const BwdArgs& a, const PipeCurs
   }
 }
 
-template <bool kDrop>
+// kDrop: dropout; kSparse: block-sparse (separate instantiations, so the plain
+// kernel is unchanged)
+template <bool kDrop, bool kSparse>
 __global__ void __launch_bounds__(kPipeThreads, 1)
     bwd_pipe_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -848,7 +900,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     regs_dec<kPipeRegsCtl>();
     if (warp == 0) {
       // -------------------------------------------------------------- producer: TMA tiles + lse/D
-      PipeCursor cur;
+      PipeCursor<kSparse> cur;
       cur.start(a, n_items);
       bool ok = true;
       float nl2[4], nd[4];
@@ -863,8 +915,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       }
       for (int T = 0; cur.valid && ok; ++T) {
         const int st = T % L::kQStages;
-        const int q0 = (cur.itm.i_first + cur.t) * 128;
-        PipeCursor nxt = cur;
+        const int q0 = cur.qtile() * 128;
+        PipeCursor<kSparse> nxt = cur;
         nxt.advance(a, n_items);
         // the next tile's statistics are loaded while this tile waits for its stage
         float nl2n[4], ndn[4];
@@ -934,7 +986,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       if (warp == 1) {
         // ------------------------------------------------------------ score MMAs
         for (int k = 0, w; (w = pipe_item_index(k)) < n_items && ok; ++k) {
-          const PipeItem itm = pipe_item(a, w);
+          const PipeItem itm = pipe_item<kSparse>(a, w);
           if (itm.n <= 0) continue;
           const int ks = u & 1;
           if (!mbar_wait(bar_k_full + ks, (u >> 1) & 1, a.timeout_ns) || !mbar_wait(bar_v_full, u & 1, a.timeout_ns) ||
@@ -962,7 +1014,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       } else {
         // ------------------------------------------------------------ gradient MMAs
         for (int k = 0, w; (w = pipe_item_index(k)) < n_items && ok; ++k) {
-          const PipeItem itm = pipe_item(a, w);
+          const PipeItem itm = pipe_item<kSparse>(a, w);
           if (itm.n <= 0) continue;
           const int ks = u & 1;
           for (int t = 0; t < itm.n; ++t, ++T) {
@@ -1012,10 +1064,10 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     const uint32_t lane_field = (quarter * 32) << 16;
     const int rr_sub = lane >> 3, cc = lane & 7;  // read side: row 4k + rr_sub, chunk cc
     bool ok = true;
-    PipeCursor cur;
+    PipeCursor<kSparse> cur;
     cur.start(a, n_items);
     for (int T = 0; cur.valid; ++T, cur.advance(a, n_items)) {
-      const int q0 = (cur.itm.i_first + cur.t) * 128 + quarter * 32;  // first query row of this warp
+      const int q0 = cur.qtile() * 128 + quarter * 32;  // first query row of this warp
       // this warp's 4 KB turn-around buffer in the drained tile's dS buffer:
       // row = lane, 16-byte chunk c at (c ^ (row & 7))
       const uint32_t scratch = sbase + L::kOffDS + (T % L::kDsBufs) * L::kDsBytes + quarter * 4096;
@@ -1064,7 +1116,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     bool ok = true;
     int T = 0, u = 0;
     for (int k = 0, w; (w = pipe_item_index(k)) < n_items && ok; ++k) {
-      const PipeItem itm = pipe_item(a, w);
+      const PipeItem itm = pipe_item<kSparse>(a, w);
       if (itm.n <= 0) {
         if (itm.s.lq < 0) {
           if (threadIdx.x == 256) atomicExch(a.status, kStatusBadArg);
@@ -1079,10 +1131,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       const int qmin = a.causal ? key - (itm.s.lk - itm.s.lq) : -(1 << 30);
       const bool key_tail = a.key_mask != nullptr || itm.j * 128 + 128 > itm.s.lk;  // masked variant
       const int last_key_qmin = itm.j * 128 + 127 - (itm.s.lk - itm.s.lq);
-      for (int t = 0; t < itm.n; ++t, ++T) {
+      const int n_qt = (itm.s.lq + 127) >> 7;
+      int qi = next_kept_q<kSparse>(a, itm.h, itm.j, itm.i_first, n_qt);  // query tile of step t
+      for (int t = 0; t < itm.n; ++t, ++T, qi = next_kept_q<kSparse>(a, itm.h, itm.j, qi + 1, n_qt)) {
         const int st = T % L::kQStages;
         const int db = T % L::kDsBufs;
-        const int q0 = (itm.i_first + t) * 128;
+        const int q0 = (kSparse ? qi : itm.i_first + t) * 128;
         if (!warp_wait_b(bar_q_full + st, (T / L::kQStages) & 1, a.timeout_ns) ||
             !warp_wait_b(bar_s_full, T & 1, a.timeout_ns) || *abort_flag) {
           ok = false;
@@ -1243,21 +1297,17 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   using L = BwdLayout<D>;
   static PerDeviceOnce attr_once;
   if (!attr_once.run([] {
-        cudaError_t e;
-        if constexpr (D == 64) {
-          e = cudaFuncSetAttribute(bwd_pipe_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   PipeLayout::kSmemBytes);
-          if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(bwd_pipe_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     PipeLayout::kSmemBytes);
-        } else {
-          e = cudaFuncSetAttribute(bwd_main_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   L::kSmemBytes);
-          if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(bwd_main_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     L::kSmemBytes);
-        }
-        return e == cudaSuccess;
+        auto set = [](const void* fn, int bytes) {
+          return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+        };
+        if constexpr (D == 64)
+          return set((const void*)bwd_pipe_kernel<false, false>, PipeLayout::kSmemBytes) &&
+                 set((const void*)bwd_pipe_kernel<true, false>, PipeLayout::kSmemBytes) &&
+                 set((const void*)bwd_pipe_kernel<false, true>, PipeLayout::kSmemBytes);
+        else
+          return set((const void*)bwd_main_kernel<D, false, false>, L::kSmemBytes) &&
+                 set((const void*)bwd_main_kernel<D, true, false>, L::kSmemBytes) &&
+                 set((const void*)bwd_main_kernel<D, false, true>, L::kSmemBytes);
       }))
     return FA_ERR_CUDA;
   // A packed batch is one batch element of total rows for the tensor maps, the
@@ -1311,20 +1361,30 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   a.drop_scale = L0.drop_t ? (float)(65536.0 / (65536.0 - (double)L0.drop_t)) : 1.f;
   a.seed_lo = (uint32_t)(L0.seed & 0xFFFFFFFFull);
   a.seed_hi = (uint32_t)(L0.seed >> 32);
+  a.block_mask = L0.block_mask;
+  a.nqb = (L0.Nq + 127) / 128;
+  a.nkb = (L0.Nk + 127) / 128;
   const long long grid = (long long)a.n_kv_tiles * L0.B * L0.H;
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   prof_before(stream, kKBwdMain);
   if constexpr (D == 64) {
     const int pgrid = (int)std::min<long long>(grid, (long long)num_sms());
-    if (a.drop_t != 0u)
-      bwd_pipe_kernel<true><<<pgrid, kPipeThreads, PipeLayout::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
+    if (a.block_mask != nullptr)
+      bwd_pipe_kernel<false, true><<<pgrid, kPipeThreads, PipeLayout::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
+    else if (a.drop_t != 0u)
+      bwd_pipe_kernel<true, false><<<pgrid, kPipeThreads, PipeLayout::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
     else
-      bwd_pipe_kernel<false><<<pgrid, kPipeThreads, PipeLayout::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
+      bwd_pipe_kernel<false, false><<<pgrid, kPipeThreads, PipeLayout::kSmemBytes, stream>>>(tq, tk, tv, tdo, a);
   } else {
-    if (a.drop_t != 0u)
-      bwd_main_kernel<D, true><<<(unsigned)grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
+    if (a.block_mask != nullptr)
+      bwd_main_kernel<D, false, true>
+          <<<(unsigned)grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
+    else if (a.drop_t != 0u)
+      bwd_main_kernel<D, true, false>
+          <<<(unsigned)grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
     else
-      bwd_main_kernel<D, false><<<(unsigned)grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
+      bwd_main_kernel<D, false, false>
+          <<<(unsigned)grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, tdo, tdk, tdv, a);
   }
   const cudaError_t err_main = cudaGetLastError();
   prof_after(stream, kKBwdMain);

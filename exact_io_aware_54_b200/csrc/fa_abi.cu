@@ -200,10 +200,11 @@ static bool dropout_threshold(float p, uint32_t* t) {
   return true;
 }
 
-// Dense forward, with an optional key-padding mask (4-byte aligned when given) and
-// dropout (drop_t = 0: none).
+// Dense forward, with an optional key-padding mask (4-byte aligned when given),
+// dropout (drop_t = 0: none) or block-sparse mask.
 static fa_status fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, const uint32_t* key_mask,
-                           uint32_t drop_t, unsigned long long seed, int B, int H, int Nq, int Nk, int d, int causal,
+                           uint32_t drop_t, unsigned long long seed, const uint8_t* block_mask, int B, int H, int Nq,
+                           int Nk, int d, int causal,
                            float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!q || !k || !v || !o || !lse || !dims_ok(B, H, Nq, Nk, d)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
@@ -222,6 +223,7 @@ static fa_status fwd_dense(const void* q, const void* k, const void* v, void* o,
   a.key_mask = key_mask;
   a.drop_t = drop_t;
   a.seed = seed;
+  a.block_mask = block_mask;
   a.B = B;
   a.H = H;
   a.Nq = Nq;
@@ -237,7 +239,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int d, int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
                  cudaStream_t stream) {
   const NvtxRange range("fa_fwd");
-  return fwd_dense(q, k, v, o, lse, nullptr, 0u, 0ull, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
+  return fwd_dense(q, k, v, o, lse, nullptr, 0u, 0ull, nullptr, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
                    workspace_bytes, stream);
 }
 
@@ -247,7 +249,16 @@ fa_status fa_fwd_masked(const void* q, const void* k, const void* v, void* o, fl
   const NvtxRange range("fa_fwd_masked");
   uint32_t t = 0;
   if (!dropout_threshold(dropout_p, &t)) return FA_ERR_INVALID_ARG;
-  return fwd_dense(q, k, v, o, lse, key_mask, t, seed, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
+  return fwd_dense(q, k, v, o, lse, key_mask, t, seed, nullptr, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
+                   workspace_bytes, stream);
+}
+
+fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                             const uint8_t* block_mask, int B, int H, int Nq, int Nk, int d, int causal,
+                             float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_fwd_blocksparse");
+  if (!block_mask) return FA_ERR_INVALID_ARG;
+  return fwd_dense(q, k, v, o, lse, nullptr, 0u, 0ull, block_mask, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
                    workspace_bytes, stream);
 }
 
@@ -289,12 +300,13 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, const int32
   return launch_fwd(a, stream);
 }
 
-// Dense backward, with an optional key-padding mask (4-byte aligned when given) and
-// the forward's dropout (drop_t = 0: none).
+// Dense backward, with an optional key-padding mask (4-byte aligned when given),
+// the forward's dropout (drop_t = 0: none) or block-sparse mask.
 static fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, const void* do_,
                            const float* lse, void* dq, void* dk, void* dv, const uint32_t* key_mask, uint32_t drop_t,
-                           unsigned long long seed, int B, int H, int Nq, int Nk, int d, int causal,
-                           float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                           unsigned long long seed, const uint8_t* block_mask, int B, int H, int Nq, int Nk, int d,
+                           int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
   if (!q || !k || !v || !o || !do_ || !lse || !dq || !dk || !dv || !dims_ok(B, H, Nq, Nk, d))
     return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
@@ -320,6 +332,7 @@ static fa_status bwd_dense(const void* q, const void* k, const void* v, const vo
   a.key_mask = key_mask;
   a.drop_t = drop_t;
   a.seed = seed;
+  a.block_mask = block_mask;
   a.B = B;
   a.H = H;
   a.Nq = Nq;
@@ -335,8 +348,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d, int causal,
                  float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   const NvtxRange range("fa_bwd");
-  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, nullptr, 0u, 0ull, B, H, Nq, Nk, d, causal, softmax_scale,
-                   workspace, workspace_bytes, stream);
+  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, nullptr, 0u, 0ull, nullptr, B, H, Nq, Nk, d, causal,
+                   softmax_scale, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd_masked(const void* q, const void* k, const void* v, const void* o, const void* do_,
@@ -346,8 +359,18 @@ fa_status fa_bwd_masked(const void* q, const void* k, const void* v, const void*
   const NvtxRange range("fa_bwd_masked");
   uint32_t t = 0;
   if (!dropout_threshold(dropout_p, &t)) return FA_ERR_INVALID_ARG;
-  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, key_mask, t, seed, B, H, Nq, Nk, d, causal, softmax_scale,
-                   workspace, workspace_bytes, stream);
+  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, key_mask, t, seed, nullptr, B, H, Nq, Nk, d, causal,
+                   softmax_scale, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const void* do_,
+                             const float* lse, void* dq, void* dk, void* dv, const uint8_t* block_mask, int B, int H,
+                             int Nq, int Nk, int d, int causal, float softmax_scale, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_bwd_blocksparse");
+  if (!block_mask) return FA_ERR_INVALID_ARG;
+  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, nullptr, 0u, 0ull, block_mask, B, H, Nq, Nk, d, causal,
+                   softmax_scale, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,

@@ -108,6 +108,9 @@ struct FwdLaunch {
   // dropout: drop_t = round(65536 p) (0: none), seed of the Philox draws
   uint32_t drop_t = 0;
   unsigned long long seed = 0;
+  // block-sparse mask (dense batches): device uint8 [H, ceil(Nq/128), ceil(Nk/128)],
+  // 0 skips the (query tile, KV tile) block; null for dense attention
+  const uint8_t* block_mask = nullptr;
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;
@@ -135,6 +138,7 @@ struct BwdLaunch {
   const uint32_t* key_mask = nullptr;  // as for the forward
   uint32_t drop_t = 0;                  // as for the forward
   unsigned long long seed = 0;
+  const uint8_t* block_mask = nullptr;  // as for the forward
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;

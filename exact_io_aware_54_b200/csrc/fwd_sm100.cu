@@ -142,7 +142,19 @@ struct FwdArgs {
   uint32_t drop_t;
   float drop_scale;
   uint32_t seed_lo, seed_hi;
+  // block-sparse mask (null: dense): [H, nqb, nkb] bytes over (128-row query
+  // tile, 128-key KV tile); 0 skips the block
+  const uint8_t* block_mask;
+  int nqb, nkb;
 };
+
+// KV tile j takes part for 128-row query tile qtile of head h (always in the dense
+// instantiation).
+template <bool kSparse>
+__device__ __forceinline__ bool block_kept(const FwdArgs& a, int h, int qtile, int j) {
+  if constexpr (!kSparse) return true;
+  return __ldg(a.block_mask + ((size_t)h * a.nqb + qtile) * a.nkb + j) != 0;
+}
 
 // The 128 mask bits of KV tile j of batch element b (all set without a mask;
 // words past the row are 0, their keys are past the end anyway).
@@ -254,8 +266,9 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, SDesc
     umma_ts(o_tmem, p_tmem + kk * 8, sdesc_at(v, kk * 128), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// kDrop: dropout on P (a separate instantiation, so the plain kernel is unchanged)
-template <int D, bool kDrop>
+// kDrop: dropout on P; kSparse: block-sparse attention (separate instantiations,
+// so the plain kernel is unchanged)
+template <int D, bool kDrop, bool kSparse>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -342,6 +355,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_load_4d(smem + L::kOffQ + t * L::kTileBytes + bx * L::kBoxBytes, &tmQ, bar_q_full, bx * 64, h,
                         sv.qoff + row0 + t * 128, sv.bc);
         for (int j = 0; j < nkv; ++j) {
+          // KV tiles that neither query tile keeps are never loaded
+          if (!((j < n0 && block_kept<kSparse>(a, h, 2 * pair, j)) || (j < n1 && block_kept<kSparse>(a, h, 2 * pair + 1, j))))
+            continue;
           for (int kv = 0; kv < 2; ++kv, ++g) {
             const uint32_t slot = g % L::kStages, phase = (g / L::kStages) & 1;
             if (!mbar_wait(bar_kv_empty + slot, phase ^ 1, a.timeout_ns)) {
@@ -393,14 +409,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           // S_t = Q_t K_j^T once the group has read its previous S tile
           if (!wait_or_abort(bar_q_full, it_q & 1)) break;
           tc_fence_after();
-          for (int j = 0; j < nkv && ok; ++j, g += 2) {
+          for (int j = 0; j < nkv && ok; ++j) {
+            const bool kp[2] = {j < nt[0] && block_kept<kSparse>(a, h, 2 * pair, j),
+                                j < nt[1] && block_kept<kSparse>(a, h, 2 * pair + 1, j)};
+            if (!kp[0] && !kp[1]) continue;  // not in the item's KV stream
             const uint32_t slot_k = g % L::kStages;
             if (!wait_or_abort(bar_kv_full + slot_k, (g / L::kStages) & 1)) break;
             tc_fence_after();
             const SDesc k_desc = SDesc{ring_k.lo + slot_k * kSlot16, ring_k.hi};
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
-              if (j < nt[t]) {
+              if (kp[t]) {
                 if (cnt[t] > 0 && !wait_or_abort(bar_s_free + t, (cnt[t] - 1) & 1)) break;
                 tc_fence_after();
                 issue_qk<D>(tmem_base + tm_s(t), q_desc[t], k_desc);
@@ -410,29 +429,36 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok) break;
             umma_commit(bar_kv_empty + slot_k);
+            g += 2;
           }
         } else {
           // O_t += P_t V_j once the group has written P.  The epilogue stages O
           // through the Q tiles: o_done must also follow this item's Q load (it
           // decides alone when a tile sees no key at all).
           if (!wait_or_abort(bar_q_full, it_q & 1)) break;
-          for (int j = 0; j < nkv && ok; ++j, g += 2) {
+          bool started[2] = {false, false};  // the tile's O holds a product of this item
+          for (int j = 0; j < nkv && ok; ++j) {
+            const bool kp[2] = {j < nt[0] && block_kept<kSparse>(a, h, 2 * pair, j),
+                                j < nt[1] && block_kept<kSparse>(a, h, 2 * pair + 1, j)};
+            if (!kp[0] && !kp[1]) continue;  // not in the item's KV stream
             const uint32_t slot_v = (g + 1) % L::kStages;
             if (!wait_or_abort(bar_kv_full + slot_v, ((g + 1) / L::kStages) & 1)) break;
             tc_fence_after();
             const SDesc v_desc = SDesc{ring_v.lo + slot_v * kSlot16, ring_v.hi};
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
-              if (j < nt[t]) {
+              if (kp[t]) {
                 if (!wait_or_abort(bar_p_full + t, cnt[t] & 1)) break;
                 tc_fence_after();
-                issue_pv<D>(tmem_base + tm_o<D>(t), tmem_base + tm_p<D>(t), v_desc, j > 0);
+                issue_pv<D>(tmem_base + tm_o<D>(t), tmem_base + tm_p<D>(t), v_desc, started[t]);
+                started[t] = true;
                 umma_commit(bar_p_free + t);
                 ++cnt[t];
               }
             }
             if (!ok) break;
             umma_commit(bar_kv_empty + slot_v);
+            g += 2;
           }
           if (!ok) break;
 #pragma unroll
@@ -473,54 +499,120 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t it_q = item_iter++;  // items processed: q_full phases
         if (!wait_or_abort(bar_q_full, it_q & 1)) break;
         tc_fence_after();
-        // K_0 : first scores of both tiles
-        uint32_t slot_k = 0;
-        if (nkv > 0) {
-          slot_k = g % L::kStages;
-          if (!wait_or_abort(bar_kv_full + slot_k, (g / L::kStages) & 1)) break;
-          tc_fence_after();
-          ++g;
-          const SDesc k_desc = SDesc{ring_k.lo + slot_k * kSlot16, ring_k.hi};
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (nt[t] > 0) {
-              issue_qk<D>(tmem_base + tm_s(t), q_desc[t], k_desc);
-              umma_commit(bar_s_full + t);
+        if constexpr (kSparse) {
+          // The item's KV stream: the tiles that at least one query tile keeps, in
+          // order.  A tile's next scores are issued right after its P V (S and P
+          // share columns; tcgen05 operations run in issue order).
+          auto kept_t = [&](int t, int j) { return j < nt[t] && block_kept<kSparse>(a, h, 2 * pair + t, j); };
+          auto next_in_stream = [&](int j) {
+            for (int x = j + 1; x < nkv; ++x)
+              if (kept_t(0, x) || kept_t(1, x)) return x;
+            return nkv;
+          };
+          // first KV tile of the stream: first scores of the tiles that keep it
+          int j = next_in_stream(-1);
+          uint32_t slot_k = 0;
+          if (j < nkv) {
+            slot_k = g % L::kStages;
+            if (!wait_or_abort(bar_kv_full + slot_k, (g / L::kStages) & 1)) break;
+            tc_fence_after();
+            ++g;
+            const SDesc k_desc = SDesc{ring_k.lo + slot_k * kSlot16, ring_k.hi};
+  #pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (kept_t(t, j)) {
+                issue_qk<D>(tmem_base + tm_s(t), q_desc[t], k_desc);
+                umma_commit(bar_s_full + t);
+              }
             }
+            umma_commit(bar_kv_empty + slot_k);
           }
-          umma_commit(bar_kv_empty + slot_k);
-        }
-        for (int j = 0; j < nkv && ok; ++j) {
-          const uint32_t slot_v = g % L::kStages;
-          if (!wait_or_abort(bar_kv_full + slot_v, (g / L::kStages) & 1)) break;
-          tc_fence_after();
-          ++g;
-          const SDesc v_desc = SDesc{ring_v.lo + slot_v * kSlot16, ring_v.hi};
-          const bool more = (j + 1 < nkv);
-          SDesc k_desc = ring_k;
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (j < nt[t]) {
-              if (!wait_or_abort(bar_p_full + t, p_cnt[t] & 1)) break;
-              tc_fence_after();
-              ++p_cnt[t];
-              issue_pv<D>(tmem_base + tm_o<D>(t), tmem_base + tm_s(t), v_desc, j > 0);
+          bool started[2] = {false, false};  // the tile's O holds a product of this item
+          while (j < nkv && ok) {
+            const int jn = next_in_stream(j);
+            const uint32_t slot_v = g % L::kStages;
+            if (!wait_or_abort(bar_kv_full + slot_v, (g / L::kStages) & 1)) break;
+            tc_fence_after();
+            ++g;
+            const SDesc v_desc = SDesc{ring_v.lo + slot_v * kSlot16, ring_v.hi};
+            const bool more = jn < nkv;
+            SDesc k_desc = ring_k;
+  #pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (kept_t(t, j)) {
+                if (!wait_or_abort(bar_p_full + t, p_cnt[t] & 1)) break;
+                tc_fence_after();
+                ++p_cnt[t];
+                issue_pv<D>(tmem_base + tm_o<D>(t), tmem_base + tm_s(t), v_desc, started[t]);
+                started[t] = true;
+              }
+              if (t == 0 && more) {
+                slot_k = g % L::kStages;
+                if (!wait_or_abort(bar_kv_full + slot_k, (g / L::kStages) & 1)) break;
+                tc_fence_after();
+                ++g;
+                k_desc = SDesc{ring_k.lo + slot_k * kSlot16, ring_k.hi};
+              }
+              if (more && kept_t(t, jn)) {
+                issue_qk<D>(tmem_base + tm_s(t), q_desc[t], k_desc);
+                umma_commit(bar_s_full + t);
+              }
             }
-            if (t == 0 && more) {
-              slot_k = g % L::kStages;
-              if (!wait_or_abort(bar_kv_full + slot_k, (g / L::kStages) & 1)) break;
-              tc_fence_after();
-              ++g;
-              k_desc = SDesc{ring_k.lo + slot_k * kSlot16, ring_k.hi};
-            }
-            if (more && j + 1 < nt[t]) {
-              issue_qk<D>(tmem_base + tm_s(t), q_desc[t], k_desc);
-              umma_commit(bar_s_full + t);
-            }
+            if (!ok) break;
+            umma_commit(bar_kv_empty + slot_v);
+            if (more) umma_commit(bar_kv_empty + slot_k);
+            j = jn;
           }
-          if (!ok) break;
-          umma_commit(bar_kv_empty + slot_v);
-          if (more) umma_commit(bar_kv_empty + slot_k);
+        } else {
+          // K_0 : first scores of both tiles
+          uint32_t slot_k = 0;
+          if (nkv > 0) {
+            slot_k = g % L::kStages;
+            if (!wait_or_abort(bar_kv_full + slot_k, (g / L::kStages) & 1)) break;
+            tc_fence_after();
+            ++g;
+            const SDesc k_desc = SDesc{ring_k.lo + slot_k * kSlot16, ring_k.hi};
+  #pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (nt[t] > 0) {
+                issue_qk<D>(tmem_base + tm_s(t), q_desc[t], k_desc);
+                umma_commit(bar_s_full + t);
+              }
+            }
+            umma_commit(bar_kv_empty + slot_k);
+          }
+          for (int j = 0; j < nkv && ok; ++j) {
+            const uint32_t slot_v = g % L::kStages;
+            if (!wait_or_abort(bar_kv_full + slot_v, (g / L::kStages) & 1)) break;
+            tc_fence_after();
+            ++g;
+            const SDesc v_desc = SDesc{ring_v.lo + slot_v * kSlot16, ring_v.hi};
+            const bool more = (j + 1 < nkv);
+            SDesc k_desc = ring_k;
+  #pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (j < nt[t]) {
+                if (!wait_or_abort(bar_p_full + t, p_cnt[t] & 1)) break;
+                tc_fence_after();
+                ++p_cnt[t];
+                issue_pv<D>(tmem_base + tm_o<D>(t), tmem_base + tm_s(t), v_desc, j > 0);
+              }
+              if (t == 0 && more) {
+                slot_k = g % L::kStages;
+                if (!wait_or_abort(bar_kv_full + slot_k, (g / L::kStages) & 1)) break;
+                tc_fence_after();
+                ++g;
+                k_desc = SDesc{ring_k.lo + slot_k * kSlot16, ring_k.hi};
+              }
+              if (more && j + 1 < nt[t]) {
+                issue_qk<D>(tmem_base + tm_s(t), q_desc[t], k_desc);
+                umma_commit(bar_s_full + t);
+              }
+            }
+            if (!ok) break;
+            umma_commit(bar_kv_empty + slot_v);
+            if (more) umma_commit(bar_kv_empty + slot_k);
+          }
         }
         if (!ok) break;
         // one completion per present tile and item: all of this tile's MMAs are done
@@ -585,7 +677,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l = 0.f;         // running sum of the bf16-rounded probabilities (normalises O)
       float le = 0.f;        // running sum of the unrounded probabilities (gives lse)
       bool ok = true;
-      for (int j = 0; j < nkv; ++j, ++s_cnt) {
+      int kept_n = 0;  // KV tiles of this item that this query tile has processed
+      for (int j = 0; j < nkv; ++j) {
+        if (!block_kept<kSparse>(a, h, 2 * pair + t, j)) continue;  // a skipped block: no scores were issued
         if (!warp_wait<kSoftmaxSpins>(bar_s_full + t, s_cnt & 1, a.timeout_ns) || *abort_flag) {
           if (lane == 0) record_timeout(a.status, abort_flag);
           ok = false;
@@ -702,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // The previous P.V of this tile has completed: with P over S, the scores just
         // read were issued after it and tcgen05 operations complete in order; with
         // separate P the wait for the P columns above covered it.
-        if (j > 0 && __any_sync(0xffffffffu, need)) {
+        if ((kSparse ? kept_n > 0 : j > 0) && __any_sync(0xffffffffu, need)) {
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
             uint32_t o[32];
@@ -716,6 +810,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive_warp(bar_p_full + t);
+        ++s_cnt;
+        if constexpr (kSparse) ++kept_n;
       }
       if (!ok) break;
 
@@ -733,7 +829,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
-        if (nkv > 0) {
+        if (kSparse ? kept_n > 0 : nkv > 0) {
           tmem_ld32(tO + cc * 32, o);
           tmem_ld_wait(o);
         } else {
@@ -800,10 +896,13 @@ static fa_status launch_fwd_impl(const FwdLaunch& L0, cudaStream_t stream) {
   using L = FwdLayout<D>;
   static PerDeviceOnce attr_once;
   if (!attr_once.run([] {
-        return cudaFuncSetAttribute(fwd_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    L::kSmemBytes) == cudaSuccess &&
-               cudaFuncSetAttribute(fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    L::kSmemBytes) == cudaSuccess;
+        const int bytes = L::kSmemBytes;
+        return cudaFuncSetAttribute(fwd_kernel<D, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    bytes) == cudaSuccess &&
+               cudaFuncSetAttribute(fwd_kernel<D, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    bytes) == cudaSuccess &&
+               cudaFuncSetAttribute(fwd_kernel<D, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    bytes) == cudaSuccess;
       }))
     return FA_ERR_CUDA;
   // a variable-length batch is one long batch of total rows for the TMA maps
@@ -837,12 +936,18 @@ static fa_status launch_fwd_impl(const FwdLaunch& L0, cudaStream_t stream) {
   a.drop_scale = L0.drop_t ? (float)(65536.0 / (65536.0 - (double)L0.drop_t)) : 1.f;
   a.seed_lo = (uint32_t)(L0.seed & 0xFFFFFFFFull);
   a.seed_hi = (uint32_t)(L0.seed >> 32);
+  a.block_mask = L0.block_mask;
+  a.nqb = (L0.Nq + 127) / 128;
+  a.nkb = (L0.Nk + 127) / 128;
+  if (a.block_mask != nullptr && a.drop_t != 0u) return FA_ERR_UNSUPPORTED;  // no entry point combines them
   const int grid = std::min(a.n_items, num_sms() * 1);
   prof_before(stream, kKFwd);
-  if (a.drop_t != 0u)
-    fwd_kernel<D, true><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);
+  if (a.block_mask != nullptr)
+    fwd_kernel<D, false, true><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);
+  else if (a.drop_t != 0u)
+    fwd_kernel<D, true, false><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);
   else
-    fwd_kernel<D, false><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);
+    fwd_kernel<D, false, false><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);
   const cudaError_t err = cudaGetLastError();
   prof_after(stream, kKFwd);
   return err == cudaSuccess ? FA_OK : FA_ERR_CUDA;

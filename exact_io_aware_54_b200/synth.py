@@ -113,3 +113,24 @@ def key_mask_inputs(seed: int, B: int, Nk: int, keep: float = 0.6, pad_to=None):
     packed = (bits.view(B, words, 32) * weights).sum(-1)
     packed = torch.where(packed >= 2 ** 31, packed - 2 ** 32, packed).to(torch.int32)
     return mask, packed
+
+
+def block_mask_inputs(seed: int, H: int, Nq: int, Nk: int, keep: float = 0.5, pattern: str = "random"):
+    """A block-sparse mask uint8 [H, ceil(Nq / 128), ceil(Nk / 128)] (1 = the block is
+    computed).  "random": blocks kept with probability `keep` (seeded); "local": a
+    band of the diagonal block and its left neighbour; "strided": every other key
+    tile.  Layout only: no attention arithmetic."""
+    nq, nk = (Nq + 127) // 128, (Nk + 127) // 128
+    if pattern == "random":
+        g = torch.Generator(device="cpu")
+        g.manual_seed(int(seed))
+        m = torch.rand(H, nq, nk, generator=g) < keep
+    elif pattern == "local":
+        i = torch.arange(nq)[:, None]
+        j = torch.arange(nk)[None, :]
+        m = ((j == i) | (j == i - 1)).expand(H, nq, nk)
+    elif pattern == "strided":
+        m = (torch.arange(nk)[None, None, :] % 2 == 0).expand(H, nq, nk)
+    else:
+        raise ValueError(pattern)
+    return m.to(torch.uint8).contiguous()

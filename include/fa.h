@@ -187,6 +187,30 @@ FA_API fa_status fa_bwd_masked(const void* q, const void* k, const void* v, cons
                                cudaStream_t stream);
 
 /*
+ * Block-sparse forward and backward passes (the block-sparse variant "AI Bible 13",
+ * section 05, credits with the 64K-token results): attention restricted to the
+ * (query tile, key tile) blocks a mask keeps.  Arguments, layouts and results are
+ * those of fa_fwd and fa_bwd, plus
+ *   block_mask : device uint8 [H, ceil(Nq / 128), ceil(Nk / 128)] (shared by the
+ *                batch), not NULL; block (i, j) of head h covers query rows
+ *                128 i .. 128 i + 127 and keys 128 j .. 128 j + 127, and a 0 removes
+ *                all of its keys from all of its queries (on top of the causal
+ *                mask).  Blocks that are 0 are not computed, and a key tile that no
+ *                query tile of a work item keeps is not loaded.  A row
+ *                left with no key gets O = 0 and LSE = -inf; keys that no kept block
+ *                reaches get dK = dV = 0.
+ * The backward pass takes the same block_mask as its forward.
+ */
+FA_API fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                                    const uint8_t* block_mask, int B, int H, int Nq, int Nk, int d, int causal,
+                                    float softmax_scale, void* workspace, size_t workspace_bytes,
+                                    cudaStream_t stream);
+FA_API fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const void* o, const void* do_,
+                                    const float* lse, void* dq, void* dk, void* dv, const uint8_t* block_mask, int B,
+                                    int H, int Nq, int Nk, int d, int causal, float softmax_scale, void* workspace,
+                                    size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Split-KV decode over a ragged, packed KV cache.
  *   q           : [B, H, d] bf16 (one query row per sequence: Nq must be 1)
  *   k, v        : [total_kv, H, d] bf16; sequence b owns rows

@@ -219,6 +219,30 @@ def test_masked_argument_validation(lib):
     assert bwd(p=1.5) == ST["FA_ERR_INVALID_ARG"]
     assert bwd(dk=None) == ST["FA_ERR_INVALID_ARG"]
     assert bwd(km=P + 1) == ST["FA_ERR_ALIGNMENT"]
+
+
+def test_blocksparse_argument_validation(lib):
+    def fwd(**kw):
+        a = dict(q=P, k=P, v=P, o=P, lse=P, bm=P, B=2, H=4, Nq=300, Nk=520, d=64, ws=P, wsb=1 << 20)
+        a.update(kw)
+        return lib.fa_fwd_blocksparse(a["q"], a["k"], a["v"], a["o"], a["lse"], a["bm"], a["B"], a["H"], a["Nq"],
+                                      a["Nk"], a["d"], 1, 0.0, a["ws"], a["wsb"], None)
+
+    def bwd(**kw):
+        a = dict(q=P, k=P, v=P, o=P, do=P, lse=P, dq=P, dk=P, dv=P, bm=P, B=2, H=4, Nq=300, Nk=520, d=128, ws=P,
+                 wsb=1 << 30)
+        a.update(kw)
+        return lib.fa_bwd_blocksparse(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"], a["dv"],
+                                      a["bm"], a["B"], a["H"], a["Nq"], a["Nk"], a["d"], 0, 0.0, a["ws"], a["wsb"],
+                                      None)
+
+    assert fwd(bm=None) == ST["FA_ERR_INVALID_ARG"]
+    assert fwd(q=None) == ST["FA_ERR_INVALID_ARG"]
+    assert fwd(d=96) == ST["FA_ERR_UNSUPPORTED"]
+    assert fwd(o=P + 4) == ST["FA_ERR_ALIGNMENT"]
+    assert fwd(ws=None) == ST["FA_ERR_WORKSPACE"]
+    assert bwd(bm=None) == ST["FA_ERR_INVALID_ARG"]
+    assert bwd(dq=P + 8) == ST["FA_ERR_ALIGNMENT"]
     assert bwd(wsb=16) == ST["FA_ERR_WORKSPACE"]
 
 
