@@ -136,18 +136,19 @@ def device_time_ms(fn, iters, stream=None):
 
 
 class L2Flush:
-    """Writes a buffer of twice the L2 size, so that the next launch finds none of its
-    inputs in L2.  The write also keeps the GPU busy while the host enqueues the
-    launch that follows, so a launch's start event is not taken while the GPU waits
-    for the host."""
+    """Reads a buffer of twice the L2 size, so that the next launch finds none of its
+    inputs in L2.  It reads rather than writes: a write would leave L2 full of dirty
+    lines, and the timed launch would pay for writing them back to HBM.  The read
+    also keeps the GPU busy while the host enqueues the launch that follows, so a
+    launch's start event is not taken while the GPU waits for the host."""
 
     def __init__(self, device):
-        self.buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
-        self.n = 0
+        self.buf = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+        self.sink = torch.zeros((), dtype=torch.float32, device=device)
+        torch.cuda.synchronize(device)
 
     def __call__(self):
-        self.n += 1
-        self.buf.fill_(self.n & 0xFF)
+        torch.sum(self.buf, dim=0, out=self.sink)
 
 
 def quantiles(ms):

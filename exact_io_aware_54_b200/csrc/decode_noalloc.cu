@@ -72,10 +72,12 @@ extern "C" fa_status fa_decode_splitkv_noalloc(const void* q, const void* k, con
                         reinterpret_cast<uintptr_t>(lse);
   if ((mis & 15u) || (reinterpret_cast<uintptr_t>(cu_seqlens_k) & 3u)) return FA_ERR_ALIGNMENT;
 
-  // scratch layout: status word | tickets [B*H] | chunk (m, l) [B,H,S,2] | chunk u [B,H,S,d]
+  // scratch layout: status word | tickets [B*H] | chunk counters [B*H] | done counters
+  // [B*H] | chunk (m, l) [B,H,S,2] | chunk u [B,H,S,d] (the counters need only B * groups
+  // entries; B*H bounds that)
   const DecodePlan plan = decode_plan(B, H, max_seqlen_k, d, num_splits);
   const size_t off_tickets = kStatusBytes;
-  const size_t off_ml = off_tickets + up256(sizeof(unsigned) * (size_t)B * H);
+  const size_t off_ml = off_tickets + up256(sizeof(unsigned) * 3 * (size_t)B * H);
   const size_t off_u = off_ml + up256(sizeof(float) * 2 * (size_t)B * H * plan.splits);
   const size_t need = off_u + up256(sizeof(float) * (size_t)d * B * H * plan.splits);
   if (need > kNoAllocScratchBytes) return FA_ERR_WORKSPACE;  // beyond the fixed scratch: pass fewer splits
@@ -84,8 +86,8 @@ extern "C" fa_status fa_decode_splitkv_noalloc(const void* q, const void* k, con
   const fa_status st = scratch_address(&base);
   if (st != FA_OK) return st;
   uint8_t* s = static_cast<uint8_t*>(base);
-  // The array keeps whatever the previous call left: clear the status word and
-  // the merge tickets, which must start at zero.
+  // The array keeps whatever the previous call left: clear the status word, the
+  // merge tickets and the chunk counters, which must start at zero.
   if (cudaMemsetAsync(s, 0, off_ml, stream) != cudaSuccess) {
     cudaGetLastError();
     return FA_ERR_CUDA;
@@ -100,7 +102,10 @@ extern "C" fa_status fa_decode_splitkv_noalloc(const void* q, const void* k, con
   a.lse = lse;
   a.status = reinterpret_cast<int*>(s);
   a.tickets = reinterpret_cast<unsigned*>(s + off_tickets);
-  a.clear_tickets = 0;  // cleared above together with the status word
+  a.grab = a.tickets + (size_t)B * H;
+  a.grab_done = a.grab + (size_t)B * H;
+  a.clear_ptr = nullptr;  // cleared above together with the status word
+  a.clear_bytes = 0;
   a.part_ml = reinterpret_cast<float*>(s + off_ml);
   a.part_u = reinterpret_cast<float*>(s + off_u);
   a.B = B;

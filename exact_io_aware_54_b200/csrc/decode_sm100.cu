@@ -10,8 +10,17 @@
 // HBM bandwidth (section 6 of that page: single-request and batched decode).
 //
 // B200 design
-//  * Grid (chunk, head group, sequence).  A head group is up to 8 heads; the
-//    CTA has one warp per head plus one producer warp.
+//  * Grid (split, head group, sequence).  A head group is up to 8 heads; the
+//    CTA has one warp per head plus one producer warp.  The CTAs of one
+//    (sequence, head group) share its keys dynamically: each producer takes the
+//    next chunk of keys from a per-(sequence, group) atomic counter whenever it
+//    has issued the previous one, and its consumers fold every chunk the CTA
+//    takes into one running state (the (m, l, u) state of any set of keys is
+//    order-independent), so each CTA still leaves exactly one partial state.  A
+//    static split of one wave left the CTAs that the memory system served last
+//    streaming alone at the end (per-SM busy time ranged over 3.5x at one
+//    request of 8192 keys, H = 32); with shared chunks every SM stays busy until
+//    the keys run out.
 //  * For every key of its chunk the head group's K and V slices are contiguous
 //    (8 heads x d bf16), so the producer moves them with plain bulk copies
 //    (cp.async.bulk) into a ring of shared-memory stages of 8 keys, completion
@@ -21,10 +30,15 @@
 //    p owns 16-byte chunks p, p+4, ... of the head dimension.  Scores need two
 //    shuffle levels, the stage max three; every lane keeps a partial u over the
 //    keys of its slot, summed across slots once at the end.
-//  * The last warp of each (sequence, head) to finish its chunk -- found with an
-//    atomic ticket -- merges the chunk states and writes o and lse, then resets
-//    the ticket, so tickets are zero between calls.  A sequence with a single chunk skips the
-//    partial-state round trip.
+//  * The producer writes each stage's first key and key count into a header
+//    beside the stage; a header with no keys tells the consumers that the
+//    counter ran out.  The last producer of a (sequence, group) to run out --
+//    found with a second ticket -- resets the counter, so counters are zero
+//    between calls.
+//  * The last warp of each (sequence, head) to finish its CTA's state -- found with
+//    an atomic ticket -- merges the CTAs' states and writes o and lse, then resets
+//    the ticket, so tickets are zero between calls.  A sequence served by a single
+//    CTA skips the partial-state round trip.
 //  * Given the number of rows of a packed cache, every sequence's offsets are
 //    checked against it first; a sequence outside the buffers is skipped and
 //    recorded in the status word.
@@ -42,15 +56,25 @@ namespace {
 constexpr int kHeadsPerCta = 8;
 constexpr int kKeysPerStage = 8;
 constexpr int kThreads = (kHeadsPerCta + 1) * 32;
+// One CTA per SM whose ring holds about 200 KB of copies in flight: per SM the
+// same bytes in flight as two CTAs of half the ring, but half the chunk states
+// per head for the merge to read.
+#ifndef FA_DEC_CTAS_PER_SM
+#define FA_DEC_CTAS_PER_SM 1
+#endif
+constexpr int kCtasPerSm = FA_DEC_CTAS_PER_SM;
+// states the merge loads per round trip (registers allow more with one CTA per SM)
+constexpr int kMergeBatch = kCtasPerSm == 1 ? 32 : 16;
 
 template <int D>
 struct DecLayout {
   static constexpr int kRowBytes = kHeadsPerCta * D * 2;  // one key, all heads of the group
   static constexpr int kRowStride = kRowBytes + 64;       // padded
   static constexpr int kStageBytes = 2 * kKeysPerStage * kRowStride;  // K rows then V rows
-  static constexpr int kStages = (D == 128) ? 3 : 6;
+  static constexpr int kStages = (D == 128 ? 6 : 12) / kCtasPerSm;
   static constexpr int kOffBar = kStages * kStageBytes;
-  static constexpr int kSmemBytes = kOffBar + 2 * kStages * 8 + 64 + 128;
+  static constexpr int kOffHdr = kOffBar + 2 * kStages * 8 + 64;  // int2 (first key, keys) per stage
+  static constexpr int kSmemBytes = kOffHdr + kStages * 8 + 128;
   static constexpr int kChunks = D / 32;  // 16-byte chunks per lane
 };
 
@@ -66,11 +90,13 @@ struct DecArgs {
   __nv_bfloat16* o;
   float* lse;
   int* status;
-  unsigned int* tickets;
+  unsigned int* tickets;      // [B * H] merge tickets
+  unsigned int* grab;         // [B * groups] next chunk of keys to hand out
+  unsigned int* grab_done;    // [B * groups] producers that found no chunk left
   float* part_ml;
   float* part_u;
   int B, H, max_seqlen_k;
-  int chunk, splits, groups;
+  int gchunk, splits, groups;  // keys per chunk handed out, CTAs per (sequence, group), groups
   float scale_log2;
   int check_args;
   unsigned long long timeout_ns;
@@ -88,7 +114,7 @@ __device__ __forceinline__ void bf16x8_to_f32(uint32_t a, uint32_t b, uint32_t c
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
+__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecArgs a) {
   using L = DecLayout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
@@ -115,7 +141,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
   }
   int len = paged ? a.seqlens[b] : a.cu[b + 1] - start;
   len = max(0, min(len, a.max_seqlen_k));
-  const int nsplit = (len + a.chunk - 1) / a.chunk;
+  // CTAs of this (sequence, group) that take part: at most one per chunk
+  const int nsplit = min(a.splits, (len + a.gchunk - 1) / a.gchunk);
   const uint32_t warp = warp_id(), lane = lane_id();
 
   if (len == 0) {
@@ -128,10 +155,8 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
     return;
   }
   if (split >= nsplit) return;
-
-  const int kbeg = split * a.chunk;
-  const int kend = min(len, kbeg + a.chunk);
-  const int nstages = (kend - kbeg + kKeysPerStage - 1) / kKeysPerStage;
+  int2* hdr = reinterpret_cast<int2*>(smem + L::kOffHdr);
+  const size_t bg = (size_t)b * a.groups + group;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
@@ -149,49 +174,77 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
 
   if (warp == kHeadsPerCta) {
     // ------------------------------------------------------------------ producer warp
-    int issued = 0;
-    for (int s = 0; s < nstages; ++s) {
-      const int slot = s % L::kStages;
-      const uint32_t phase = (s / L::kStages) & 1;
-      bool ok = true;
-      if (lane == 0) {
-        ok = mbar_wait(empty + slot, phase ^ 1, a.timeout_ns) && !flags[0];
-        if (ok) {
-          const int nk = min(kKeysPerStage, kend - (kbeg + s * kKeysPerStage));
-          mbar_arrive_expect_tx(full + slot, 2u * nk * copy_bytes);
-        } else {
-          flags[0] = 1;
-          atomicCAS(a.status, 0, kStatusTimeout);
-        }
-      }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      if (!ok) break;
-      const int key0 = kbeg + s * kKeysPerStage;
-      if (lane < 2 * kKeysPerStage) {
-        const int t = lane & (kKeysPerStage - 1);
-        const int is_v = lane >= kKeysPerStage;
-        const int key = key0 + t;
-        if (key < kend) {
-          size_t row = (size_t)start + key;
-          if (paged) {
-            int page = a.block_table[(size_t)b * a.max_pages + key / a.page_size];
-            if (page < 0 || page >= a.num_pages) {  // never read outside the cache
-              atomicExch(a.status, kStatusBadArg);
-              page = 0;
-            }
-            row = (size_t)page * a.page_size + key % a.page_size;
+    // The first chunk of CTA `split` is chunk `split` (there is one per CTA that
+    // takes part), so no counter round trip delays the first copies; later chunks
+    // come from the counter (nsplit + the value taken).  Lane 0 takes the next one
+    // while the current chunk's copies are issued; every chunk taken is issued.
+    unsigned int next = (unsigned)split;
+    int issued = 0;  // stages issued (ring position)
+    bool ok = true;
+    while (ok) {
+      const int c = (int)__shfl_sync(0xffffffffu, next, 0);
+      const bool more = (long long)c * a.gchunk < len;
+      if (more && lane == 0) next = (unsigned)nsplit + atomicAdd(a.grab + bg, 1u);
+      for (int st = 0; ok; ++st) {
+        const int key0 = more ? c * a.gchunk + st * kKeysPerStage : 0;
+        if (more && (st * kKeysPerStage >= a.gchunk || key0 >= len)) break;
+        const int nk = more ? min(kKeysPerStage, len - key0) : -1;  // -1: no chunk left
+        const int slot = issued % L::kStages;
+        const uint32_t phase = (issued / L::kStages) & 1;
+        if (lane == 0) {
+          ok = mbar_wait(empty + slot, phase ^ 1, a.timeout_ns) && !flags[0];
+          if (ok) {
+            hdr[slot] = make_int2(key0, nk);
+            if (more)
+              mbar_arrive_expect_tx(full + slot, 2u * nk * copy_bytes);
+            else
+              mbar_arrive(full + slot);  // the header alone: no copies
+          } else {
+            flags[0] = 1;
+            atomicCAS(a.status, 0, kStatusTimeout);
           }
-          const __nv_bfloat16* src = (is_v ? a.v : a.k) + row * row_elems + (size_t)h0 * D;
-          uint8_t* dst = smem + slot * L::kStageBytes + is_v * kKeysPerStage * L::kRowStride + t * L::kRowStride;
-          bulk_load(dst, src, copy_bytes, full + slot);
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+        ++issued;
+        if (!more) break;
+        if (lane < 2 * kKeysPerStage) {
+          const int t = lane & (kKeysPerStage - 1);
+          const int is_v = lane >= kKeysPerStage;
+          const int key = key0 + t;
+          if (t < nk) {
+            size_t row = (size_t)start + key;
+            if (paged) {
+              int page = a.block_table[(size_t)b * a.max_pages + key / a.page_size];
+              if (page < 0 || page >= a.num_pages) {  // never read outside the cache
+                atomicExch(a.status, kStatusBadArg);
+                page = 0;
+              }
+              row = (size_t)page * a.page_size + key % a.page_size;
+            }
+            const __nv_bfloat16* src = (is_v ? a.v : a.k) + row * row_elems + (size_t)h0 * D;
+            uint8_t* dst = smem + slot * L::kStageBytes + is_v * kKeysPerStage * L::kRowStride + t * L::kRowStride;
+            bulk_load(dst, src, copy_bytes, full + slot);
+          }
         }
       }
-      ++issued;
+      if (!more) break;
     }
-    // on an early exit, let the copies already issued land before the CTA retires
-    if (lane == 0 && flags[0]) {
-      for (int s = max(0, issued - L::kStages); s < issued; ++s)
-        (void)mbar_wait(full + (s % L::kStages), (s / L::kStages) & 1, a.timeout_ns);
+    if (lane == 0) {
+      if (ok) {
+        // this producer takes no more chunks; the last of the (sequence, group) to
+        // get here resets the counter for the next call (every other producer has
+        // made its final take by then: each takes before it counts itself here)
+        __threadfence();
+        if (atomicAdd(a.grab_done + bg, 1u) == (unsigned)(nsplit - 1)) {
+          atomicExch(a.grab + bg, 0u);
+          atomicExch(a.grab_done + bg, 0u);
+        }
+      } else {
+        // on an early exit, let the copies already issued land before the CTA retires
+        for (int s2 = max(0, issued - L::kStages); s2 < issued; ++s2)
+          (void)mbar_wait(full + (s2 % L::kStages), (s2 / L::kStages) & 1, a.timeout_ns);
+      }
     }
     return;
   }
@@ -220,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
   float m = -INFINITY, l = 0.f;
   bool ok = true;
 
-  for (int s = 0; s < nstages; ++s) {
+  for (int s = 0;; ++s) {
     const int slot = s % L::kStages;
     bool got = true;
     if (lane == 0) got = mbar_wait(full + slot, (s / L::kStages) & 1, a.timeout_ns) && !flags[0];
@@ -233,8 +286,9 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
       ok = false;
       break;
     }
-    const int key = kbeg + s * kKeysPerStage + t;
-    const bool valid = head_ok && key < kend;
+    const int nk = hdr[slot].y;
+    if (nk < 0) break;  // no chunk left for this CTA
+    const bool valid = head_ok && t < nk;
     const uint32_t kaddr = smem_u32(smem + slot * L::kStageBytes + t * L::kRowStride + hw * D * 2);
     const uint32_t vaddr = kaddr + kKeysPerStage * L::kRowStride;
     float dot = 0.f;
@@ -327,29 +381,25 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
   if (!last) return;
   __threadfence();
 
-  // ------------------------------------------------------------------ merge (last chunk of b, h)
-  // Pass 1: lanes stride over the chunks for the common reference max.  Pass 2:
-  // batches of 16 chunks issue all their loads before any use, so the chain of
-  // L2 round trips is nsplit / 16 long rather than nsplit.
+  // ------------------------------------------------------------------ merge (last state of b, h)
+  // The states are read kMergeBatch at a time, every load of a batch issued before
+  // any is used, with a running reference max: one L2 round trip per batch.  Lane
+  // i weighs state s0 + i; each lane sums the u of every state over its own kPerLane
+  // columns, with the weights passed round by shuffles.
   constexpr int kPerLane = D / 32;
-  constexpr int kBatch = 16;
   const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + bh * a.splits;
-  float M = -INFINITY;
-  for (int s = lane; s < nsplit; s += 32) M = fmaxf(M, __ldcg(ml + s).x);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  const float M_ref = (M == -INFINITY) ? 0.f : M;
-  float Lsum = 0.f, U[kPerLane];
+  const float* pu = a.part_u + bh * a.splits * D + lane * kPerLane;
+  float M = -INFINITY, Lsum = 0.f, U[kPerLane];
 #pragma unroll
   for (int e = 0; e < kPerLane; ++e) U[e] = 0.f;
-  const float* pu = a.part_u + bh * a.splits * D + lane * kPerLane;
-  for (int s0 = 0; s0 < nsplit; s0 += kBatch) {
-    float2 st[kBatch];
-    float uu[kBatch][kPerLane];
+  for (int s0 = 0; s0 < nsplit; s0 += kMergeBatch) {
+    const int s_own = s0 + (int)(lane % kMergeBatch);
+    const float2 st = (lane < (uint32_t)kMergeBatch && s_own < nsplit) ? __ldcg(ml + s_own)
+                                                                       : make_float2(-INFINITY, 0.f);
+    float uu[kMergeBatch][kPerLane];
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
+    for (int i = 0; i < kMergeBatch; ++i) {
       const int s = min(s0 + i, nsplit - 1);
-      st[i] = __ldcg(ml + s);
       if constexpr (kPerLane == 4) {
         const float4 x = __ldcg(reinterpret_cast<const float4*>(pu + (size_t)s * D));
         uu[i][0] = x.x;
@@ -362,15 +412,27 @@ __global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecArgs a) {
         uu[i][1] = x.y;
       }
     }
+    float mb = st.x;
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      const bool live = (s0 + i) < nsplit;
-      const float w = (!live || st[i].x == -INFINITY) ? 0.f : ex2(st[i].x - M_ref);
-      Lsum = fmaf(w, st[i].y, Lsum);
+    for (int off = 16; off > 0; off >>= 1) mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
+    const float M_new = fmaxf(M, mb);
+    const float M_ref = (M_new == -INFINITY) ? 0.f : M_new;
+    const float keep = (M == -INFINITY) ? 0.f : ex2(M - M_ref);  // rescale what was summed so far
+    Lsum *= keep;
 #pragma unroll
-      for (int e = 0; e < kPerLane; ++e) U[e] = fmaf(w, uu[i][e], U[e]);
+    for (int e = 0; e < kPerLane; ++e) U[e] *= keep;
+    const float w = (st.x == -INFINITY) ? 0.f : ex2(st.x - M_ref);  // 0 past the last state
+    Lsum = fmaf(w, st.y, Lsum);
+#pragma unroll
+    for (int i = 0; i < kMergeBatch; ++i) {
+      const float wi = __shfl_sync(0xffffffffu, w, i);
+#pragma unroll
+      for (int e = 0; e < kPerLane; ++e) U[e] = fmaf(wi, uu[i][e], U[e]);
     }
+    M = M_new;
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, off);
   const float inv = (Lsum > 0.f) ? 1.f / Lsum : 0.f;
   __nv_bfloat16* out = a.o + bh * D + lane * kPerLane;
 #pragma unroll
@@ -409,7 +471,7 @@ DecodePlan decode_plan(int B, int H, int max_seqlen_k, int d, int num_splits) {
     const int s = std::max(1, std::min(num_splits, (maxL + 7) / 8));
     chunk = roundup8((maxL + s - 1) / s);
   } else {
-    const long long slots = (long long)num_sms() * 2;  // two CTAs per SM
+    const long long slots = (long long)num_sms() * kCtasPerSm;
     const long long work = (long long)B * maxL * p.groups;
     chunk = roundup8((work + slots * 16 - 1) / (slots * 16));  // ~16 waves if all sequences are full
     if (chunk < 256) {
@@ -427,16 +489,47 @@ DecodePlan decode_plan(int B, int H, int max_seqlen_k, int d, int num_splits) {
   }
   p.chunk = chunk;
   p.splits = splits;
+  // chunks handed out: about an eighth of a CTA's even share of the keys, so the
+  // CTAs of a (sequence, group) can even out how fast each is served, but at
+  // least two stages (one counter round trip hides behind two stages of copies)
+  p.gchunk = std::min(256, std::max(16, roundup8(chunk / 8)));
   return p;
 }
 
+namespace {
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+}  // namespace
+
 size_t decode_workspace_bytes(int B, int H, int d, const DecodePlan& plan) {
-  auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
-  size_t bytes = kStatusBytes + kDecodeTicketBytes;
-  if ((size_t)B * H > kDecodeFixedTickets) bytes += up(sizeof(unsigned) * (size_t)B * H);
-  bytes += up(sizeof(float) * 2 * (size_t)B * H * plan.splits);
-  bytes += up(sizeof(float) * (size_t)d * B * H * plan.splits);
+  size_t bytes = kStatusBytes + kDecodeSyncBytes;
+  if ((size_t)B * H > kDecodeFixedTickets) bytes += up256(sizeof(unsigned) * 3 * (size_t)B * H);
+  bytes += up256(sizeof(float) * 2 * (size_t)B * H * plan.splits);
+  bytes += up256(sizeof(float) * (size_t)d * B * H * plan.splits);
   return bytes;
+}
+
+void decode_carve(uint8_t* ws, int B, int H, int d, const DecodePlan& plan, DecodeLaunch& a) {
+  a.status = reinterpret_cast<int*>(ws);
+  unsigned* sync = reinterpret_cast<unsigned*>(ws + kStatusBytes);
+  size_t off = kStatusBytes + kDecodeSyncBytes;
+  a.part_ml = reinterpret_cast<float*>(ws + off);
+  off += up256(sizeof(float) * 2 * (size_t)B * H * plan.splits);
+  a.part_u = reinterpret_cast<float*>(ws + off);
+  off += up256(sizeof(float) * (size_t)d * B * H * plan.splits);
+  size_t n = kDecodeFixedTickets;
+  a.clear_ptr = nullptr;
+  a.clear_bytes = 0;
+  if ((size_t)B * H > kDecodeFixedTickets) {
+    // too many (sequence, head) pairs for the fixed region: a region of this call's
+    // own, cleared before the launch
+    sync = reinterpret_cast<unsigned*>(ws + off);
+    n = (size_t)B * H;
+    a.clear_ptr = sync;
+    a.clear_bytes = sizeof(unsigned) * 3 * n;
+  }
+  a.tickets = sync;
+  a.grab = sync + n;
+  a.grab_done = sync + 2 * n;
 }
 
 template <int D>
@@ -463,20 +556,21 @@ static fa_status launch_decode_impl(const DecodeLaunch& L0, cudaStream_t stream)
   a.lse = L0.lse;
   a.status = L0.status;
   a.tickets = L0.tickets;
+  a.grab = L0.grab;
+  a.grab_done = L0.grab_done;
   a.part_ml = L0.part_ml;
   a.part_u = L0.part_u;
   a.B = L0.B;
   a.H = L0.H;
   a.max_seqlen_k = L0.max_seqlen_k;
-  a.chunk = L0.plan.chunk;
+  a.gchunk = L0.plan.gchunk;
   a.splits = L0.plan.splits;
   a.groups = L0.plan.groups;
   a.scale_log2 = L0.scale * 1.4426950408889634f;
   a.check_args = L0.check_args;
   a.timeout_ns = L0.timeout_ns;
-  if (L0.clear_tickets) {
-    if (cudaMemsetAsync(L0.tickets, 0, sizeof(unsigned) * (size_t)L0.B * L0.H, stream) != cudaSuccess)
-      return FA_ERR_CUDA;
+  if (L0.clear_bytes) {
+    if (cudaMemsetAsync(L0.clear_ptr, 0, L0.clear_bytes, stream) != cudaSuccess) return FA_ERR_CUDA;
   }
   if (L0.check_args && !L0.block_table) {
     prof_before(stream, kKDecodeCheck);

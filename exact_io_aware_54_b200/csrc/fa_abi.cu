@@ -450,19 +450,7 @@ static fa_status decode_packed(const void* q, const void* k, const void* v, cons
   a.total_kv = total_kv;
   a.o = o;
   a.lse = lse;
-  a.status = reinterpret_cast<int*>(ws);
-  size_t off = kStatusBytes;
-  a.tickets = reinterpret_cast<unsigned*>(ws + off);
-  a.clear_tickets = 0;
-  off += kDecodeTicketBytes;
-  a.part_ml = reinterpret_cast<float*>(ws + off);
-  off += up256(sizeof(float) * 2 * (size_t)B * H * plan.splits);
-  a.part_u = reinterpret_cast<float*>(ws + off);
-  off += up256(sizeof(float) * (size_t)d * B * H * plan.splits);
-  if ((size_t)B * H > kDecodeFixedTickets) {
-    a.tickets = reinterpret_cast<unsigned*>(ws + off);
-    a.clear_tickets = 1;
-  }
+  decode_carve(ws, B, H, d, plan, a);
   a.B = B;
   a.H = H;
   a.max_seqlen_k = max_seqlen_k;
@@ -529,19 +517,7 @@ fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_page
   a.num_pages = num_pages;
   a.o = o;
   a.lse = lse;
-  a.status = reinterpret_cast<int*>(ws);
-  size_t off = kStatusBytes;
-  a.tickets = reinterpret_cast<unsigned*>(ws + off);
-  a.clear_tickets = 0;
-  off += kDecodeTicketBytes;
-  a.part_ml = reinterpret_cast<float*>(ws + off);
-  off += up256(sizeof(float) * 2 * (size_t)B * H * plan.splits);
-  a.part_u = reinterpret_cast<float*>(ws + off);
-  off += up256(sizeof(float) * (size_t)d * B * H * plan.splits);
-  if ((size_t)B * H > kDecodeFixedTickets) {
-    a.tickets = reinterpret_cast<unsigned*>(ws + off);
-    a.clear_tickets = 1;
-  }
+  decode_carve(ws, B, H, d, plan, a);
   a.B = B;
   a.H = H;
   a.max_seqlen_k = max_seqlen_k;

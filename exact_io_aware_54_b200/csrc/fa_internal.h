@@ -28,13 +28,16 @@ struct NvtxRange {
 // Workspace: the first kStatusBytes hold the status word (int32) and padding.
 constexpr size_t kStatusBytes = 256;
 
-// Decode merge tickets live in a fixed region right after the status word, so
-// they stay at the same place whatever the shape of the call; the last arrival
-// of every (sequence, head) resets its ticket.  Calls with more than
-// kDecodeFixedTickets (sequence, head) pairs use a region after the partial
-// states that is cleared on every call.
+// Decode counters live in a fixed region right after the status word, so they
+// stay at the same place whatever the shape of the call: the merge tickets of
+// every (sequence, head), then the key-chunk counters and the done-counters of
+// every (sequence, head group).  Each resets itself at the end of a call (the
+// last merge of a (sequence, head) clears its ticket, the last producer of a
+// (sequence, group) its two counters).  Calls with more than kDecodeFixedTickets
+// (sequence, head) pairs use a region after the partial states that is cleared
+// on every call.
 constexpr size_t kDecodeFixedTickets = 65536;
-constexpr size_t kDecodeTicketBytes = kDecodeFixedTickets * 4;
+constexpr size_t kDecodeSyncBytes = 3 * kDecodeFixedTickets * 4;
 
 // Status codes recorded by kernels in the workspace status word (fa_status values).
 constexpr int kStatusTimeout = 6;
@@ -147,8 +150,9 @@ fa_status launch_bwd(const BwdLaunch& a, cudaStream_t stream);
 
 // Split-KV decode plan: keys per chunk and chunks per sequence.
 struct DecodePlan {
-  int chunk;       // keys per split (multiple of 8)
-  int splits;      // splits for a sequence of max_seqlen_k keys
+  int chunk;       // keys per CTA if the keys were split evenly (multiple of 8)
+  int splits;      // CTAs (and partial states) per (sequence, head group)
+  int gchunk;      // keys per chunk handed out to a CTA (multiple of 8)
   int groups;      // head groups per sequence
   int heads_per_group;
 };
@@ -167,8 +171,11 @@ struct DecodeLaunch {
   void* o;
   float* lse;
   int* status;
-  unsigned int* tickets;  // [B * H] merge tickets, zero between calls
-  int clear_tickets;      // tickets live outside the fixed region: clear them first
+  unsigned int* tickets;    // [B * H] merge tickets, zero between calls
+  unsigned int* grab;       // [B * groups] key-chunk counters, zero between calls
+  unsigned int* grab_done;  // [B * groups] producers done, zero between calls
+  void* clear_ptr = nullptr;  // counters outside the fixed region: cleared before the launch
+  size_t clear_bytes = 0;
   float* part_ml;      // [B, H, splits, 2]  (m in log2 units, l)
   float* part_u;       // [B, H, splits, d]
   int B, H, max_seqlen_k, d;
@@ -183,5 +190,9 @@ struct DecodeLaunch {
 fa_status launch_decode(const DecodeLaunch& a, cudaStream_t stream);
 
 size_t decode_workspace_bytes(int B, int H, int d, const DecodePlan& plan);
+
+// Points the status word, counters and partial states of `a` into a caller
+// workspace of at least decode_workspace_bytes(B, H, d, plan) bytes.
+void decode_carve(uint8_t* ws, int B, int H, int d, const DecodePlan& plan, DecodeLaunch& a);
 
 }  // namespace fa

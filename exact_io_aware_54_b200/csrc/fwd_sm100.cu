@@ -335,8 +335,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t item_iter = 0, g = 0;
-      for (int r = 0; r * (int)gridDim.x < a.n_items && !*abort_flag; ++r) {
-        const int w = item_of_round(r);
+      for (int rnd = 0; rnd * (int)gridDim.x < a.n_items && !*abort_flag; ++rnd) {
+        const int w = item_of_round(rnd);
         if (w >= a.n_items) continue;
         int b, h, pair;
         item_coords(a, w, b, h, pair);
@@ -394,8 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ring slots alternate K, V per KV step: K of step j at g, V at g + 1
       uint32_t item_iter = 0, g = 0;
       uint32_t cnt[2] = {0, 0};  // Q K^T (warp 1) or P V (warp 2) MMAs issued per query tile
-      for (int r = 0; r * (int)gridDim.x < a.n_items && ok; ++r) {
-        const int w = item_of_round(r);
+      for (int rnd = 0; rnd * (int)gridDim.x < a.n_items && ok; ++rnd) {
+        const int w = item_of_round(rnd);
         if (w >= a.n_items) continue;
         int b, h, pair;
         item_coords(a, w, b, h, pair);
@@ -486,8 +486,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return ok;
       };
-      for (int r = 0; r * (int)gridDim.x < a.n_items && ok; ++r) {
-        const int w = item_of_round(r);
+      for (int rnd = 0; rnd * (int)gridDim.x < a.n_items && ok; ++rnd) {
+        const int w = item_of_round(rnd);
         if (w >= a.n_items) continue;
         int b, h, pair;
         item_coords(a, w, b, h, pair);
@@ -639,8 +639,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* q_tile = smem + L::kOffQ + t * L::kTileBytes;
     const uint32_t q_tile_u32 = smem_u32(q_tile);
 
-    for (int r = 0; r * (int)gridDim.x < a.n_items; ++r) {
-      const int w = item_of_round(r);
+    for (int rnd = 0; rnd * (int)gridDim.x < a.n_items; ++rnd) {
+      const int w = item_of_round(rnd);
       if (w >= a.n_items) continue;
       if (*abort_flag) break;
       int b, h, pair;

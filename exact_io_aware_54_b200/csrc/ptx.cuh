@@ -68,10 +68,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity, ui
   return ok != 0;
 }
 
+// Polls of every bounded wait before it starts to sleep (0: one poll).
+#ifndef FA_WAIT_SPINS
+#define FA_WAIT_SPINS 0
+#endif
+
 // Bounded wait for the phase of `bar` with the given parity to complete.
 // Returns false when `timeout_ns` of wall time passed without completion.  Each
 // try may sleep up to 0.1 ms, so the clock is read rarely.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t timeout_ns) {
+#pragma unroll 1
+  for (int i = 0; i < FA_WAIT_SPINS; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity, 100000u)) {

@@ -6,7 +6,7 @@ import torch
 import oracle
 from exact_io_aware_54_b200 import (fa_check, fa_decode_num_splits, fa_decode_splitkv, fa_decode_splitkv_checked,
                                     fa_decode_workspace_size, synth, workspace)
-from tests._harness import OAccumulator, compare_lse, compare_o, default_scale, f64
+from tests._harness import OAccumulator, compare_lse, compare_o, compare_reordered, default_scale, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -90,15 +90,15 @@ def test_batched_ragged_whole_tensor():
 
 
 def test_checked_equals_unchecked_on_valid_offsets():
-    """fa_decode_splitkv_checked computes exactly what fa_decode_splitkv does when the
-    offsets fit the buffers (bit for bit: same kernel, same plan)."""
+    """fa_decode_splitkv_checked computes what fa_decode_splitkv does when the offsets
+    fit the buffers (same kernel and plan; the sums agree up to their order)."""
     q, k, v, cu = synth.decode_inputs(61, [300, 17, 1024, 0, 513], 12, 128, device="cuda")
     cu = cu.cuda()
     o1, l1 = fa_decode_splitkv(q, k, v, cu, 1024)
     o2, l2 = fa_decode_splitkv_checked(q, k, v, cu, 1024)
     torch.cuda.synchronize()
     assert fa_check(workspace(256, q.device, "decode")) == 0
-    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    compare_reordered(f64(o1), f64(o2), f64(l1), f64(l2))
 
 
 @pytest.mark.parametrize("cu_bad,bad", [([0, 200, 500, 900, 650], {2, 3}),     # end past total, end < start
@@ -112,8 +112,8 @@ def test_checked_skips_sequences_outside_the_buffers(cu_bad, bad):
     could only reach memory this test owns; it must not happen all the same."""
     H, d, T = 8, 128, 650
     B = len(cu_bad) - 1
-    q, k_all, v_all, _ = synth.decode_inputs(71, [T + 512], H, d, device="cuda")
-    q = synth.decode_inputs(72, [1] * B, H, d, device="cuda")[0]
+    _, k_all, v_all, _ = synth.decode_inputs(71, [T + 512], H, d, device="cuda")
+    q = synth.decode_inputs(81, [1] * B, H, d, device="cuda")[0]  # seeds 81.. share no draw with k, v
     k, v = k_all[:T], v_all[:T]
     cu = torch.tensor(cu_bad, dtype=torch.int32, device="cuda")
     o = torch.full((B, H, d), float("nan"), dtype=torch.bfloat16, device="cuda")

@@ -2,8 +2,8 @@
 
 Reference: the fp64 oracle's paged decode (gather each sequence's keys through its
 block table, then the decode definition).  The paged path and the packed path run
-the same kernel arithmetic in the same order for the same split plan, so on the
-same keys they must also agree bit for bit.
+the same kernel arithmetic for the same split plan, so on the same keys they agree
+up to the order of the fp32 sums (key chunks go to CTAs as they become free).
 """
 import numpy as np
 import pytest
@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from exact_io_aware_54_b200 import fa_check, fa_decode_paged, fa_decode_splitkv, synth, workspace
-from tests._harness import compare_lse, compare_o, default_scale, f64
+from tests._harness import compare_lse, compare_o, compare_reordered, default_scale, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -64,8 +64,9 @@ def test_empty_sequences_and_loose_bound():
 
 
 @pytest.mark.parametrize("page_size,d", [(16, 64), (64, 128)])
-def test_bitwise_equal_to_packed_decode(page_size, d):
-    """The same keys, paged and packed, give identical bits (same plan, same order)."""
+def test_matches_packed_decode(page_size, d):
+    """The same keys, paged and packed, give the same result up to the order of the
+    fp32 sums (same plan; chunks go to CTAs as they become free)."""
     lengths = [37, 700, 4096, 1]
     (q, kp, vp, table, lens), o, lse = _run(lengths, 16, d, page_size, 950 + d)
     ks, vs = [], []
@@ -79,8 +80,7 @@ def test_bitwise_equal_to_packed_decode(page_size, d):
     cu[1:] = torch.cumsum(torch.tensor(lengths), 0)
     o2, lse2 = fa_decode_splitkv(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), max(lengths))
     torch.cuda.synchronize()
-    assert torch.equal(o, o2)
-    assert torch.equal(lse, lse2)
+    compare_reordered(f64(o), f64(o2), f64(lse), f64(lse2))
 
 
 def test_bad_page_index_is_reported_not_followed():

@@ -13,7 +13,7 @@ import torch
 
 import oracle
 from exact_io_aware_54_b200 import FAError, fa_decode_num_splits, fa_decode_splitkv, fa_decode_splitkv_noalloc, synth
-from tests._harness import compare_lse, compare_o, default_scale, f64
+from tests._harness import compare_lse, compare_o, compare_reordered, default_scale, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -56,12 +56,13 @@ def test_noalloc_calls_whose_layout_changes():
 
 def test_noalloc_at_the_end_of_its_scratch():
     """A shape whose chunk states fill the array to within a few KiB of its end
-    (B = 2, H = 32, d = 128, 504 chunks: 512 + 504 * 64 * (2 + 128) * 4 bytes), twice,
-    against the oracle and the workspace entry point with the same split."""
+    (B = 2, H = 32, d = 128, 504 chunk states: 1024 bytes of status word and counters,
+    then 504 * 64 * (2 + 128) * 4 bytes of states), twice, against the oracle and the
+    workspace entry point with the same split."""
     B, H, d, S = 2, 32, 128, 504
     lengths = [4032, 3001]
     assert fa_decode_num_splits(B, H, max(lengths), d, S) == S
-    need = 512 + S * B * H * (2 + d) * 4
+    need = 1024 + S * B * H * (2 + d) * 4
     assert SCRATCH_BYTES - 4096 < need <= SCRATCH_BYTES
     for call in range(2):
         q, k, v, cu = synth.decode_inputs(970 + call, lengths, H, d, device="cuda")
@@ -69,7 +70,7 @@ def test_noalloc_at_the_end_of_its_scratch():
         o, lse = fa_decode_splitkv_noalloc(q, k, v, cu, max(lengths), num_splits=S)
         o_ws, lse_ws = fa_decode_splitkv(q, k, v, cu, max(lengths), num_splits=S)
         torch.cuda.synchronize()
-        assert torch.equal(o, o_ws) and torch.equal(lse, lse_ws)
+        compare_reordered(f64(o), f64(o_ws), f64(lse), f64(lse_ws))
         _oracle_check(q, k, v, cu, o, lse, d, f"call {call}")
     # one chunk more no longer fits
     assert fa_decode_num_splits(B, H, 4040, d, S + 1) == S + 1
