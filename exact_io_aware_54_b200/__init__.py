@@ -23,7 +23,8 @@ import threading
 import torch
 
 __all__ = [
-    "FAError", "lib_path", "load", "fa_fwd", "fa_bwd", "fa_fwd_varlen", "fa_bwd_varlen", "fa_decode_splitkv",
+    "FAError", "lib_path", "load", "fa_fwd", "fa_bwd", "fa_merge_partials", "fa_fwd_varlen", "fa_bwd_varlen",
+    "fa_decode_splitkv",
     "fa_decode_splitkv_noalloc", "fa_decode_paged", "fa_check", "fa_fwd_workspace_size", "fa_bwd_workspace_size",
     "fa_bwd_varlen_workspace_size", "fa_decode_workspace_size", "fa_decode_num_splits",
     "fa_version", "STATUS",
@@ -72,8 +73,9 @@ def load():
         lib.fa_decode_paged.argtypes = [_vp] * 5 + [_i] * 7 + [_f, _i, _vp, _vp, _vp, _sz, _vp]
         lib.fa_fwd_varlen.argtypes = [_vp] * 7 + [_i] * 8 + [_f, _vp, _sz, _vp]
         lib.fa_bwd_varlen.argtypes = [_vp] * 11 + [_i] * 8 + [_f, _vp, _sz, _vp]
+        lib.fa_merge_partials.argtypes = [_vp, _vp] + [_i] * 5 + [_vp, _vp, _vp]
         for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_decode_splitkv, lib.fa_decode_splitkv_noalloc,
-                   lib.fa_decode_paged, lib.fa_fwd_varlen, lib.fa_bwd_varlen):
+                   lib.fa_decode_paged, lib.fa_fwd_varlen, lib.fa_bwd_varlen, lib.fa_merge_partials):
             fn.restype = _i
         lib.fa_fwd_workspace_size.argtypes = [_i] * 5
         lib.fa_fwd_workspace_size.restype = _sz
@@ -187,6 +189,23 @@ def fa_fwd(q, k, v, causal: bool = False, softmax_scale=None, out=None, lse=None
     st = lib.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), B, H, Nq, Nk, d,
                     int(bool(causal)), _scale(softmax_scale), ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
     _raise("fa_fwd", st)
+    return out, lse
+
+
+def fa_merge_partials(o_parts, lse_parts, out=None, lse=None):
+    """Merge shard results: o_parts [S, B, Nq, H, d] bf16, lse_parts [S, B, H, Nq] fp32
+    -> (o [B, Nq, H, d], lse [B, H, Nq])."""
+    lib = load()
+    S, B, Nq, H, d = o_parts.shape
+    _check_tensor("o_parts", o_parts, torch.bfloat16)
+    _check_tensor("lse_parts", lse_parts, torch.float32, (S, B, H, Nq))
+    out = torch.empty(o_parts.shape[1:], dtype=torch.bfloat16, device=o_parts.device) if out is None else out
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=o_parts.device) if lse is None else lse
+    _check_tensor("out", out, torch.bfloat16, (B, Nq, H, d))
+    _check_tensor("lse", lse, torch.float32, (B, H, Nq))
+    st = lib.fa_merge_partials(o_parts.data_ptr(), lse_parts.data_ptr(), S, B, H, Nq, d, out.data_ptr(),
+                               lse.data_ptr(), _stream_ptr(o_parts.device))
+    _raise("fa_merge_partials", st)
     return out, lse
 
 

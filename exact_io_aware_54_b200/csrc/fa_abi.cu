@@ -340,6 +340,16 @@ fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void*
   return launch_bwd(a, stream);
 }
 
+fa_status fa_merge_partials(const void* o_parts, const float* lse_parts, int S, int B, int H, int Nq, int d, void* o,
+                            float* lse, cudaStream_t stream) {
+  const NvtxRange range("fa_merge_partials");
+  if (!o_parts || !lse_parts || !o || !lse || S <= 0 || !dims_ok(B, H, Nq, 1, d)) return FA_ERR_INVALID_ARG;
+  if ((long long)S * B * Nq * H >= (1LL << 40)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(o_parts) || !aligned16(o) || !aligned16(lse_parts) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
+  return launch_merge(o_parts, lse_parts, S, B, H, Nq, d, o, lse, stream);
+}
+
 fa_status fa_decode_splitkv(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_k, int B, int H,
                             int Nq, int max_seqlen_k, int d, int causal, float softmax_scale, int num_splits, void* o,
                             float* lse, void* workspace, size_t workspace_bytes, cudaStream_t stream) {

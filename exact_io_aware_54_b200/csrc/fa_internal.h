@@ -95,6 +95,10 @@ struct BwdLaunch {
 };
 fa_status launch_bwd(const BwdLaunch& a, cudaStream_t stream);
 
+// Merge of S partial (o, lse) results over key shards (merge_sm100.cu).
+fa_status launch_merge(const void* o_parts, const float* lse_parts, int S, int B, int H, int Nq, int d, void* o,
+                       float* lse, cudaStream_t stream);
+
 // Split-KV decode plan: keys per chunk and chunks per sequence.
 struct DecodePlan {
   int chunk;       // keys per split (multiple of 8)

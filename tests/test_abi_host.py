@@ -176,6 +176,21 @@ def test_bwd_varlen_argument_validation(lib):
     assert fa.fa_bwd_varlen_workspace_size(4, 300, 80) == 0
 
 
+def test_merge_partials_argument_validation(lib):
+    def call(**kw):
+        a = dict(op=P, lp=P, S=4, B=2, H=3, Nq=300, d=128, o=P, lse=P)
+        a.update(kw)
+        return lib.fa_merge_partials(a["op"], a["lp"], a["S"], a["B"], a["H"], a["Nq"], a["d"], a["o"], a["lse"],
+                                     None)
+
+    assert call(op=None) == ST["FA_ERR_INVALID_ARG"]
+    assert call(S=0) == ST["FA_ERR_INVALID_ARG"]
+    assert call(Nq=0) == ST["FA_ERR_INVALID_ARG"]
+    assert call(d=96) == ST["FA_ERR_UNSUPPORTED"]
+    assert call(o=P + 4) == ST["FA_ERR_ALIGNMENT"]
+    assert call(lp=P + 8) == ST["FA_ERR_ALIGNMENT"]
+
+
 def test_selftest_argument_validation(lib):
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint, ctypes.c_void_p]
     assert lib.fa_selftest_wait_timeout(None, 256, 100, None) == ST["FA_ERR_WORKSPACE"]
