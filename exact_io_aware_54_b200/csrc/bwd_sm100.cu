@@ -90,6 +90,7 @@ struct BwdArgs {
   const int32_t* cu_k;
   int total_q, total_k;
   int stat_n;
+  int causal_delta;  // as for the forward: query i sees key j iff j <= i + (lk - lq) + causal_delta
 };
 
 // Where sequence b lives.  Dense: batch element b of the [B, N, H, D] tensors.
@@ -273,7 +274,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (j * 128 >= sq.lk) return;  // no key of this sequence in the tile
   const int n_qtiles = (sq.lq + 127) >> 7;
   int i_first = 0;
-  if (a.causal) i_first = max(0, j * 128 - (sq.lk - sq.lq)) >> 7;
+  if (a.causal) i_first = max(0, j * 128 - (sq.lk - sq.lq + a.causal_delta)) >> 7;
   const int n_iters = n_qtiles - i_first;  // >= 1 when the sequence has queries
   if (n_iters <= 0) {
     store_zero_dkv<D>(a, sq, j, h, threadIdx.x, blockDim.x);
@@ -436,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool key_ok = key < sq.lk;
     // first query that sees this key (a sentinel far below any query when not causal;
     // qmin - qs below must not overflow)
-    const int qmin = a.causal ? key - (sq.lk - sq.lq) : -(1 << 30);
+    const int qmin = a.causal ? key - (sq.lk - sq.lq + a.causal_delta) : -(1 << 30);
     bool ok = true;
 
     // dQ tile of query tile `it`: this group's D/2 columns, fp32 vector reductions
@@ -487,7 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld_wait(sv);
         reg_pin(dp);
         const uint32_t stat_u32 = sbase + L::kOffStat + st * 1024 + col * 4;
-        const bool tile_mask = (j * 128 + 128 > sq.lk) || (a.causal && (j * 128 + 127 - (sq.lk - sq.lq) > qs));
+        const bool tile_mask =
+            (j * 128 + 128 > sq.lk) || (a.causal && (j * 128 + 127 - (sq.lk - sq.lq + a.causal_delta) > qs));
         uint32_t pk[16], dk2[16];
         if (tile_mask)
           ds_block<32, true>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2);
@@ -665,8 +667,8 @@ __device__ __forceinline__ PipeItem pipe_item(const BwdArgs& a, int w) {
   it.n = -1;
   if (it.s.lq < 0 || it.j * 128 >= it.s.lk) return it;
   const int n_qtiles = (it.s.lq + 127) >> 7;
-  it.i_first = a.causal ? (max(0, it.j * 128 - (it.s.lk - it.s.lq)) >> 7) : 0;
-  it.n = n_qtiles - it.i_first;
+  it.i_first = a.causal ? (max(0, it.j * 128 - (it.s.lk - it.s.lq + a.causal_delta)) >> 7) : 0;
+  it.n = max(0, n_qtiles - it.i_first);  // 0: keys no query sees (dK = dV = 0)
   return it;
 }
 
@@ -1021,9 +1023,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       }
       const int key = itm.j * 128 + r;
       const bool key_ok = key < itm.s.lk;
-      const int qmin = a.causal ? key - (itm.s.lk - itm.s.lq) : -(1 << 30);
+      const int qmin = a.causal ? key - (itm.s.lk - itm.s.lq + a.causal_delta) : -(1 << 30);
       const bool key_tail = itm.j * 128 + 128 > itm.s.lk;
-      const int last_key_qmin = itm.j * 128 + 127 - (itm.s.lk - itm.s.lq);
+      const int last_key_qmin = itm.j * 128 + 127 - (itm.s.lk - itm.s.lq + a.causal_delta);
       for (int t = 0; t < itm.n; ++t, ++T) {
         const int st = T % L::kQStages;
         const int db = T % L::kDsBufs;
@@ -1236,6 +1238,7 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   a.total_q = L0.total_q;
   a.total_k = L0.total_k;
   a.stat_n = mNq;
+  a.causal_delta = L0.causal_delta;
   const long long grid = (long long)a.n_kv_tiles * L0.B * L0.H;
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   prof_before(stream, kKBwdMain);

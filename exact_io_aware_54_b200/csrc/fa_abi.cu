@@ -188,10 +188,10 @@ size_t fa_decode_workspace_size(int B, int H, int max_seqlen_k, int d, int num_s
   return decode_workspace_bytes(B, H, d, decode_plan(B, H, max_seqlen_k, d, num_splits));
 }
 
-fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
-                 int d, int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
-                 cudaStream_t stream) {
-  const NvtxRange range("fa_fwd");
+// Dense forward; causal_delta shifts the causal boundary (key shards).
+static fa_status fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, int causal_delta, int B,
+                           int H, int Nq, int Nk, int d, int causal, float softmax_scale, void* workspace,
+                           size_t workspace_bytes, cudaStream_t stream) {
   if (!q || !k || !v || !o || !lse || !dims_ok(B, H, Nq, Nk, d)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
@@ -204,6 +204,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   a.o = o;
   a.lse = lse;
   a.status = static_cast<int*>(workspace);
+  a.causal_delta = causal_delta;
   a.B = B;
   a.H = H;
   a.Nq = Nq;
@@ -213,6 +214,31 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   a.scale = resolve_scale(softmax_scale, d);
   a.timeout_ns = wait_timeout_ns();
   return launch_fwd(a, stream);
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int Nq, int Nk,
+                 int d, int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
+                 cudaStream_t stream) {
+  const NvtxRange range("fa_fwd");
+  return fwd_dense(q, k, v, o, lse, 0, B, H, Nq, Nk, d, causal, softmax_scale, workspace, workspace_bytes, stream);
+}
+
+// The shard holds keys key_offset .. key_offset + Nk - 1 of Nk_total: query i sees
+// shard key j iff key_offset + j <= i + Nk_total - Nq, i.e. j <= i + (Nk - Nq) + delta
+// with delta = Nk_total - key_offset - Nk.
+static bool shard_delta(int key_offset, int Nk_total, int Nk, int* delta) {
+  if (key_offset < 0 || Nk_total <= 0 || (long long)key_offset + Nk > Nk_total) return false;
+  *delta = Nk_total - key_offset - Nk;
+  return true;
+}
+
+fa_status fa_fwd_shard(const void* q, const void* k, const void* v, void* o, float* lse, int key_offset, int Nk_total,
+                       int B, int H, int Nq, int Nk, int d, float softmax_scale, void* workspace,
+                       size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_fwd_shard");
+  int delta = 0;
+  if (!shard_delta(key_offset, Nk_total, Nk, &delta)) return FA_ERR_INVALID_ARG;
+  return fwd_dense(q, k, v, o, lse, delta, B, H, Nq, Nk, d, 1, softmax_scale, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, const int32_t* cu_seqlens_q,
@@ -253,10 +279,11 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, const int32
   return launch_fwd(a, stream);
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,
-                 void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d, int causal,
-                 float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
-  const NvtxRange range("fa_bwd");
+// Dense backward; causal_delta as for fwd_dense.
+static fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, const void* do_,
+                           const float* lse, void* dq, void* dk, void* dv, int causal_delta, int B, int H, int Nq,
+                           int Nk, int d, int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
+                           cudaStream_t stream) {
   if (!q || !k || !v || !o || !do_ || !lse || !dq || !dk || !dv || !dims_ok(B, H, Nq, Nk, d))
     return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
@@ -279,6 +306,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   a.status = reinterpret_cast<int*>(ws);
   a.dq_acc = reinterpret_cast<float*>(ws + kStatusBytes);
   a.delta = reinterpret_cast<float*>(ws + kStatusBytes + up256(sizeof(float) * (size_t)B * Nq * H * d));
+  a.causal_delta = causal_delta;
   a.B = B;
   a.H = H;
   a.Nq = Nq;
@@ -288,6 +316,24 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   a.scale = resolve_scale(softmax_scale, d);
   a.timeout_ns = wait_timeout_ns();
   return launch_bwd(a, stream);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,
+                 void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d, int causal,
+                 float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_bwd");
+  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, 0, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
+                   workspace_bytes, stream);
+}
+
+fa_status fa_bwd_shard(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,
+                       void* dq, void* dk, void* dv, int key_offset, int Nk_total, int B, int H, int Nq, int Nk, int d,
+                       float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_bwd_shard");
+  int delta = 0;
+  if (!shard_delta(key_offset, Nk_total, Nk, &delta)) return FA_ERR_INVALID_ARG;
+  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, delta, B, H, Nq, Nk, d, 1, softmax_scale, workspace,
+                   workspace_bytes, stream);
 }
 
 fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,

@@ -65,6 +65,9 @@ struct FwdLaunch {
   const int32_t* cu_q = nullptr;
   const int32_t* cu_k = nullptr;
   int total_q = 0, total_k = 0;
+  // causal visibility offset beyond the bottom-right alignment (a key shard: its
+  // keys start later in the sequence)
+  int causal_delta = 0;
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;
@@ -89,6 +92,7 @@ struct BwdLaunch {
   const int32_t* cu_q = nullptr;
   const int32_t* cu_k = nullptr;
   int total_q = 0, total_k = 0;
+  int causal_delta = 0;  // as for the forward
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;

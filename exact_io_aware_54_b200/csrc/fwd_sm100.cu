@@ -118,6 +118,9 @@ struct FwdArgs {
   int n_pairs;
   int n_items;
   unsigned long long timeout_ns;
+  // causal: query i sees key j iff j <= i + (lk - lq) + causal_delta (0 except for a
+  // key shard, whose keys start later in the sequence)
+  int causal_delta;
 };
 
 __device__ __forceinline__ void item_coords(const FwdArgs& a, int w, int& b, int& h, int& pair) {
@@ -164,11 +167,12 @@ __device__ __forceinline__ SeqView seq_view(const FwdArgs& a, int b) {
 }
 
 // Number of KV tiles query tile starting at row0 needs; -1 when the tile is empty.
+template <bool kShard>
 __device__ __forceinline__ int tile_kv_count(const FwdArgs& a, const SeqView& v, int row0) {
   if (row0 >= v.lq) return -1;
   if (!a.causal) return (v.lk + 127) >> 7;
   const int last = min(row0 + 127, v.lq - 1);
-  long long kend = (long long)last + 1 + v.lk - v.lq;
+  long long kend = (long long)last + 1 + v.lk - v.lq + (kShard ? a.causal_delta : 0);
   if (kend <= 0) return 0;
   if (kend > v.lk) kend = v.lk;
   return (int)((kend + 127) >> 7);
@@ -208,7 +212,9 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, SDesc
     umma_ts(o_tmem, p_tmem + kk * 8, sdesc_at(v, kk * 128), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
-template <int D>
+// kShard: a key shard with a shifted causal boundary (a separate instantiation, so
+// the plain kernel is unchanged)
+template <int D, bool kShard>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -280,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         item_coords(a, w, b, h, pair);
         const SeqView sv = seq_view(a, b);
         const int row0 = pair * 256;
-        const int n0 = tile_kv_count(a, sv, row0), n1 = tile_kv_count(a, sv, row0 + 128);
+        const int n0 = tile_kv_count<kShard>(a, sv, row0), n1 = tile_kv_count<kShard>(a, sv, row0 + 128);
         const int nkv = max(n0, n1);
         if (n0 < 0) continue;  // no query row of this item exists: every role skips it
         if (!mbar_wait(bar_q_empty, (item_iter++ & 1) ^ 1, a.timeout_ns)) {
@@ -334,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         item_coords(a, w, b, h, pair);
         const SeqView sv = seq_view(a, b);
         const int row0 = pair * 256;
-        const int nt[2] = {tile_kv_count(a, sv, row0), tile_kv_count(a, sv, row0 + 128)};
+        const int nt[2] = {tile_kv_count<kShard>(a, sv, row0), tile_kv_count<kShard>(a, sv, row0 + 128)};
         const int nkv = max(nt[0], nt[1]);
         if (nt[0] < 0) continue;  // no query row of this item exists: every role skips it
         const uint32_t it_q = item_iter++;  // items processed: q_full phases
@@ -414,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         item_coords(a, w, b, h, pair);
         const SeqView sv = seq_view(a, b);
         const int row0 = pair * 256;
-        const int nt[2] = {tile_kv_count(a, sv, row0), tile_kv_count(a, sv, row0 + 128)};
+        const int nt[2] = {tile_kv_count<kShard>(a, sv, row0), tile_kv_count<kShard>(a, sv, row0 + 128)};
         const int nkv = max(nt[0], nt[1]);
         if (nt[0] < 0) continue;  // no query row of this item exists: every role skips it
         const uint32_t it_q = item_iter++;  // items processed: q_full phases
@@ -501,10 +507,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const SeqView sv = seq_view(a, b);
       if (sv.lq < 0 && pair == 0 && t == 0 && tid_in_group == 0) atomicExch(a.status, kStatusBadArg);
       const int row0 = pair * 256 + t * 128;
-      const int nkv = tile_kv_count(a, sv, row0);
+      const int nkv = tile_kv_count<kShard>(a, sv, row0);
       // No query row of this item exists: every role skips it (an arrival here
       // could complete the producer's q_empty phase before its first wait).
-      if (tile_kv_count(a, sv, pair * 256) < 0) continue;
+      if (tile_kv_count<kShard>(a, sv, pair * 256) < 0) continue;
       const uint32_t it_q = items_done++;
       if (nkv < 0) {
         // This query tile lies past the sequence: nothing to compute or store.  Its
@@ -523,8 +529,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // visible keys of this row: [0, lim)
       const int lk = sv.lk;  // only the key count stays live through the KV loop
       int lim = lk;
-      if (a.causal) lim = max(0, min(lk, row + 1 + lk - sv.lq));
-      const int group_first_lim = a.causal ? (row0 + 1 + lk - sv.lq) : lk;  // smallest lim in the tile
+      const int cdelta = kShard ? a.causal_delta : 0;
+      if (a.causal) lim = max(0, min(lk, row + 1 + lk - sv.lq + cdelta));
+      const int group_first_lim = a.causal ? (row0 + 1 + lk - sv.lq + cdelta) : lk;  // smallest lim in the tile
 
       float m2 = -INFINITY;  // running reference max (log2 domain)
       float l = 0.f;         // running sum of the bf16-rounded probabilities (normalises O)
@@ -731,8 +738,10 @@ static fa_status launch_fwd_impl(const FwdLaunch& L0, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
   if (dev < 64 && !attr_done[dev]) {
-    if (cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(fwd_kernel<D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmemBytes) !=
+            cudaSuccess)
       return FA_ERR_CUDA;
     attr_done[dev] = true;
   }
@@ -761,9 +770,13 @@ static fa_status launch_fwd_impl(const FwdLaunch& L0, cudaStream_t stream) {
   a.n_pairs = (L0.Nq + 255) / 256;
   a.n_items = a.n_pairs * L0.B * L0.H;
   a.timeout_ns = L0.timeout_ns;
+  a.causal_delta = L0.causal_delta;
   const int grid = std::min(a.n_items, num_sms() * 1);
   prof_before(stream, kKFwd);
-  fwd_kernel<D><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);
+  if (a.causal_delta != 0)
+    fwd_kernel<D, true><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);
+  else
+    fwd_kernel<D, false><<<grid, kThreads, L::kSmemBytes, stream>>>(tq, tk, tv, to, a);
   const cudaError_t err = cudaGetLastError();
   prof_after(stream, kKFwd);
   return err == cudaSuccess ? FA_OK : FA_ERR_CUDA;

@@ -151,10 +151,31 @@ FA_API fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, cons
                                void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Causal attention over one shard of the keys, for causal sequence parallelism:
+ * the shard k, v [B, Nk, H, d] holds keys key_offset .. key_offset + Nk - 1 of a
+ * sequence of Nk_total keys, and query i (of Nq, all queries) sees shard key j iff
+ * key_offset + j <= i + (Nk_total - Nq) (the bottom-right alignment of the whole
+ * sequence).  Layouts and results as fa_fwd / fa_bwd with causal = 1; merge the
+ * shards' forward results with fa_merge_partials, and run the backward of each
+ * shard with the merged O and LSE.  A query row that sees no key of the shard gets
+ * O = 0 and LSE = -inf from fa_fwd_shard, and shard keys no query sees get
+ * dK = dV = 0.  FA_ERR_INVALID_ARG unless 0 <= key_offset and
+ * key_offset + Nk <= Nk_total.
+ */
+FA_API fa_status fa_fwd_shard(const void* q, const void* k, const void* v, void* o, float* lse, int key_offset,
+                              int Nk_total, int B, int H, int Nq, int Nk, int d, float softmax_scale, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
+FA_API fa_status fa_bwd_shard(const void* q, const void* k, const void* v, const void* o, const void* do_,
+                              const float* lse, void* dq, void* dk, void* dv, int key_offset, int Nk_total, int B,
+                              int H, int Nq, int Nk, int d, float softmax_scale, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Merge of partial attention results over key shards, for sequence parallelism
  * (the multi-GPU extension the second page wishes for, "AI Bible 13", section 06):
  * when the keys and values are split into S shards and fa_fwd runs over each shard
- * with all queries (not causal), the shard results combine by the block-merge rule
+ * with all queries (not causal; causal shards go through fa_fwd_shard), the shard
+ * results combine by the block-merge rule
  * ("FlashAttention saves IO, not N^2 work", sections 3 and 7):
  *     O = sum_s exp(lse_s - M) o_s / sum_s exp(lse_s - M),  M = max_s lse_s,
  *     lse = M + ln sum_s exp(lse_s - M).

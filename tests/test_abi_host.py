@@ -191,6 +191,26 @@ def test_merge_partials_argument_validation(lib):
     assert call(lp=P + 8) == ST["FA_ERR_ALIGNMENT"]
 
 
+def test_shard_argument_validation(lib):
+    def fwd(**kw):
+        a = dict(off=0, tot=1024, B=2, H=4, Nq=512, Nk=256, d=64)
+        a.update(kw)
+        return lib.fa_fwd_shard(P, P, P, P, P, a["off"], a["tot"], a["B"], a["H"], a["Nq"], a["Nk"], a["d"], 0.0,
+                                P, 1 << 20, None)
+
+    def bwd(**kw):
+        a = dict(off=0, tot=1024, B=2, H=4, Nq=512, Nk=256, d=128)
+        a.update(kw)
+        return lib.fa_bwd_shard(P, P, P, P, P, P, P, P, P, a["off"], a["tot"], a["B"], a["H"], a["Nq"], a["Nk"],
+                                a["d"], 0.0, P, 1 << 30, None)
+
+    assert fwd(off=-1) == ST["FA_ERR_INVALID_ARG"]
+    assert fwd(off=800) == ST["FA_ERR_INVALID_ARG"]   # 800 + 256 > 1024
+    assert fwd(tot=0) == ST["FA_ERR_INVALID_ARG"]
+    assert bwd(off=900) == ST["FA_ERR_INVALID_ARG"]
+    assert bwd(Nk=2000) == ST["FA_ERR_INVALID_ARG"]
+
+
 def test_selftest_argument_validation(lib):
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint, ctypes.c_void_p]
     assert lib.fa_selftest_wait_timeout(None, 256, 100, None) == ST["FA_ERR_WORKSPACE"]

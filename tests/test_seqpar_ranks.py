@@ -1,11 +1,12 @@
 """Sequence-parallel attention's exchange logic on two gloo ranks (CPU).
 
 The library's per-shard attention and merge run on the GPU; here the module's
-forward and backward take CPU stand-ins for them (the oracle's attention and its
-two-block merge rule), so what is tested is the product's exchange: which shards
-each rank holds, the all-gather of partial (O, lse) in rank order, the merge of
-all of them, and the fp32 all-reduce of the partial dQ.  The result must equal
-attention over the whole sequence.
+forward and backward take CPU stand-ins for them (shard attention written out in
+numpy, and the oracle's two-block merge rule), so what is tested is the product's
+exchange: which shard each rank holds and where it sits in the sequence (the
+causal boundary), the all-gather of partial (O, lse) in rank order, the merge of
+all of them, and the all-reduce of the partial dQ.  The result must equal the
+oracle's attention over the whole sequence, causal or not.
 """
 import datetime
 import json
@@ -14,6 +15,7 @@ import os
 import socket
 
 import numpy as np
+import pytest
 import torch
 import torch.multiprocessing as mp
 
@@ -27,9 +29,30 @@ def _free_port() -> int:
         return s.getsockname()[1]
 
 
+def _visible(Nq, Nk, causal, key_offset, nk_total):
+    """[Nq, Nk]: shard key j is visible to query i (bottom-right over the whole sequence)."""
+    if not causal:
+        return np.ones((Nq, Nk), dtype=bool)
+    return (key_offset + np.arange(Nk))[None, :] <= np.arange(Nq)[:, None] + (nk_total - Nq)
+
+
 def _cpu_attn(scale):
-    def attn(q, k, v):
-        o, lse = oracle.attn_fwd(q.double().numpy(), k.double().numpy(), v.double().numpy(), False, scale)
+    """Attention over one key shard (the CPU stand-in for the library's call)."""
+    def attn(q, k, v, causal, key_offset, nk_total):
+        q, k, v = (t.double().numpy() for t in (q, k, v))
+        B, Nq, H, d = q.shape
+        vis = _visible(Nq, k.shape[1], causal, key_offset, nk_total)
+        o, lse = np.zeros_like(q), np.full((B, H, Nq), -np.inf)
+        for b in range(B):
+            for h in range(H):
+                s = np.where(vis, scale * q[b, :, h] @ k[b, :, h].T, -np.inf)
+                for i in range(Nq):
+                    if not vis[i].any():
+                        continue
+                    m = s[i].max()
+                    p = np.exp(s[i] - m)
+                    o[b, i, h] = p @ v[b, :, h] / p.sum()
+                    lse[b, h, i] = m + math.log(p.sum())
         return torch.from_numpy(o), torch.from_numpy(lse)
     return attn
 
@@ -38,30 +61,34 @@ def _cpu_merge(o_all, lse_all):
     """The two-block merge rule applied shard by shard (oracle.merge_state)."""
     S, B, Nq, H, d = o_all.shape
     o = np.zeros((B, Nq, H, d))
-    lse = np.zeros((B, H, Nq))
+    lse = np.full((B, H, Nq), -np.inf)
     for b in range(B):
         for h in range(H):
             for i in range(Nq):
                 m, l, u = -math.inf, 0.0, np.zeros(d)
                 for s in range(S):
                     ls = float(lse_all[s, b, h, i])
+                    if ls == -math.inf:
+                        continue
                     # a shard's normalised output o_s with l_s = 1 and m_s = lse_s
                     m, l, u = oracle.merge_state((m, l, u), (ls, 1.0, o_all[s, b, i, h].double().numpy()))
-                o[b, i, h] = u / l
-                lse[b, h, i] = m + math.log(l)
+                if l > 0:
+                    o[b, i, h] = u / l
+                    lse[b, h, i] = m + math.log(l)
     return torch.from_numpy(o), torch.from_numpy(lse)
 
 
 def _cpu_attn_bwd(scale):
-    def bwd(q, k, v, o, dout, lse):
-        # the backward over this shard with the merged O and lse: P = exp(s - lse)
+    """The backward over one key shard with the merged O and lse (CPU stand-in)."""
+    def bwd(q, k, v, o, dout, lse, causal, key_offset, nk_total):
         q, k, v, o, dout, lse = (t.double().numpy() for t in (q, k, v, o, dout, lse))
         B, Nq, H, d = q.shape
+        vis = _visible(Nq, k.shape[1], causal, key_offset, nk_total)
         dq, dk, dv = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v)
         for b in range(B):
             for h in range(H):
                 s = scale * q[b, :, h] @ k[b, :, h].T
-                p = np.exp(s - lse[b, h][:, None])
+                p = np.where(vis, np.exp(s - lse[b, h][:, None]), 0.0)
                 dv[b, :, h] = p.T @ dout[b, :, h]
                 dp = dout[b, :, h] @ v[b, :, h].T
                 D = (dout[b, :, h] * o[b, :, h]).sum(axis=1)
@@ -72,7 +99,7 @@ def _cpu_attn_bwd(scale):
     return bwd
 
 
-def _rank_main(rank, world, port, out_dir):
+def _rank_main(rank, world, port, out_dir, causal):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     torch.distributed.init_process_group("gloo", rank=rank, world_size=world,
@@ -83,8 +110,9 @@ def _rank_main(rank, world, port, out_dir):
         q, k, v, do = (t.double() for t in synth.prefill_inputs(6000, B, Nq, Nk, H, d, with_dout=True))
         shard = Nk // world
         ks, vs = k[:, rank * shard:(rank + 1) * shard], v[:, rank * shard:(rank + 1) * shard]
-        o, lse = seqpar.sequence_parallel_fwd(q, ks, vs, attn=_cpu_attn(scale), merge=_cpu_merge)
-        dq, dk, dv = seqpar.sequence_parallel_bwd(q, ks, vs, o, do, lse, attn_bwd=_cpu_attn_bwd(scale))
+        o, lse = seqpar.sequence_parallel_fwd(q, ks, vs, causal=causal, attn=_cpu_attn(scale), merge=_cpu_merge)
+        dq, dk, dv = seqpar.sequence_parallel_bwd(q, ks, vs, o, do, lse, causal=causal,
+                                                  attn_bwd=_cpu_attn_bwd(scale))
         np.save(os.path.join(out_dir, f"r{rank}.npy"),
                 np.concatenate([o.numpy().ravel(), lse.numpy().ravel(), dq.numpy().ravel(), dk.numpy().ravel(),
                                 dv.numpy().ravel()]))
@@ -94,13 +122,14 @@ def _rank_main(rank, world, port, out_dir):
         torch.distributed.destroy_process_group()
 
 
-def test_two_ranks_reproduce_whole_sequence_attention(tmp_path):
+@pytest.mark.parametrize("causal", [False, True])
+def test_two_ranks_reproduce_whole_sequence_attention(tmp_path, causal):
     world = 2
-    mp.spawn(_rank_main, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True)
+    mp.spawn(_rank_main, args=(world, _free_port(), str(tmp_path), causal), nprocs=world, join=True)
     B, Nq, Nk, H, d, scale = 1, 6, 8, 2, 4, 0.5
     q, k, v, do = (t.double().numpy() for t in synth.prefill_inputs(6000, B, Nq, Nk, H, d, with_dout=True))
-    o_ref, lse_ref = oracle.attn_fwd(q, k, v, False, scale)
-    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(q, k, v, do, False, scale)
+    o_ref, lse_ref = oracle.attn_fwd(q, k, v, causal, scale)
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(q, k, v, do, causal, scale)
     shard = Nk // world
     for r in range(world):
         flat = np.load(tmp_path / f"r{r}.npy")
