@@ -25,7 +25,8 @@ import torch
 __all__ = [
     "FAError", "lib_path", "load", "fa_fwd", "fa_bwd", "fa_fwd_masked", "fa_bwd_masked", "fa_fwd_blocksparse",
     "fa_bwd_blocksparse", "fa_fwd_varlen", "fa_bwd_varlen", "fa_decode_splitkv", "fa_decode_splitkv_noalloc",
-    "fa_decode_splitkv_checked", "fa_decode_paged", "fa_check", "fa_fwd_workspace_size", "fa_bwd_workspace_size",
+    "fa_decode_splitkv_checked", "fa_decode_paged", "fa_merge_partials", "fa_fwd_shard", "fa_bwd_shard", "fa_check",
+    "fa_fwd_workspace_size", "fa_bwd_workspace_size",
     "fa_bwd_varlen_workspace_size", "fa_decode_workspace_size", "fa_decode_num_splits",
     "fa_version", "STATUS",
 ]
@@ -79,9 +80,13 @@ def load():
         lib.fa_bwd_masked.argtypes = [_vp] * 10 + [_f, _u64] + [_i] * 6 + [_f, _vp, _sz, _vp]
         lib.fa_fwd_blocksparse.argtypes = [_vp] * 6 + [_i] * 6 + [_f, _vp, _sz, _vp]
         lib.fa_bwd_blocksparse.argtypes = [_vp] * 10 + [_i] * 6 + [_f, _vp, _sz, _vp]
+        lib.fa_merge_partials.argtypes = [_vp, _vp] + [_i] * 5 + [_vp, _vp, _vp]
+        lib.fa_fwd_shard.argtypes = [_vp] * 5 + [_i] * 7 + [_f, _vp, _sz, _vp]
+        lib.fa_bwd_shard.argtypes = [_vp] * 9 + [_i] * 7 + [_f, _vp, _sz, _vp]
         for fn in (lib.fa_fwd, lib.fa_bwd, lib.fa_decode_splitkv, lib.fa_decode_splitkv_noalloc,
                    lib.fa_decode_splitkv_checked, lib.fa_decode_paged, lib.fa_fwd_varlen, lib.fa_bwd_varlen,
-                   lib.fa_fwd_masked, lib.fa_bwd_masked, lib.fa_fwd_blocksparse, lib.fa_bwd_blocksparse):
+                   lib.fa_fwd_masked, lib.fa_bwd_masked, lib.fa_fwd_blocksparse, lib.fa_bwd_blocksparse,
+                   lib.fa_merge_partials, lib.fa_fwd_shard, lib.fa_bwd_shard):
             fn.restype = _i
         lib.fa_fwd_workspace_size.argtypes = [_i] * 5
         lib.fa_fwd_workspace_size.restype = _sz
@@ -305,6 +310,69 @@ def fa_bwd_blocksparse(q, k, v, o, dout, lse, block_mask, causal: bool = False, 
                                 _stream_ptr(q.device))
     _raise("fa_bwd_blocksparse", st)
     return dq, dk, dv
+
+
+def fa_fwd_shard(q, k, v, key_offset: int, Nk_total: int, softmax_scale=None, out=None, lse=None, ws=None):
+    """Causal attention of all queries q [B, Nq, H, d] over a key shard k, v
+    [B, Nk, H, d] holding keys key_offset .. key_offset + Nk - 1 of Nk_total.
+    Returns (o, lse) as fa_fwd (rows that see no key of the shard: 0 and -inf)."""
+    lib = load()
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    _check_tensor("q", q, torch.bfloat16)
+    _check_tensor("k", k, torch.bfloat16, (B, Nk, H, d))
+    _check_tensor("v", v, torch.bfloat16, (B, Nk, H, d))
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _check_tensor("out", out, torch.bfloat16, q.shape)
+    _check_tensor("lse", lse, torch.float32, (B, H, Nq))
+    if ws is None:
+        ws = workspace(lib.fa_fwd_workspace_size(B, H, Nq, Nk, d), q.device, "fwd")
+    st = lib.fa_fwd_shard(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(), int(key_offset),
+                          int(Nk_total), B, H, Nq, Nk, d, _scale(softmax_scale), ws.data_ptr(), ws.numel(),
+                          _stream_ptr(q.device))
+    _raise("fa_fwd_shard", st)
+    return out, lse
+
+
+def fa_bwd_shard(q, k, v, o, dout, lse, key_offset: int, Nk_total: int, softmax_scale=None, dq=None, dk=None,
+                 dv=None, ws=None):
+    """Backward of one causal key shard with the merged o and lse of all shards.
+    Returns (partial dq, dk, dv of the shard) in bf16."""
+    lib = load()
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    for name, t, shp in (("q", q, None), ("k", k, (B, Nk, H, d)), ("v", v, (B, Nk, H, d)), ("o", o, q.shape),
+                         ("dout", dout, q.shape)):
+        _check_tensor(name, t, torch.bfloat16, shp)
+    _check_tensor("lse", lse, torch.float32, (B, H, Nq))
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if ws is None:
+        ws = workspace(lib.fa_bwd_workspace_size(B, H, Nq, Nk, d), q.device, "bwd")
+    st = lib.fa_bwd_shard(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(),
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), int(key_offset), int(Nk_total), B, H, Nq, Nk,
+                          d, _scale(softmax_scale), ws.data_ptr(), ws.numel(), _stream_ptr(q.device))
+    _raise("fa_bwd_shard", st)
+    return dq, dk, dv
+
+
+def fa_merge_partials(o_parts, lse_parts, out=None, lse=None):
+    """Merge shard results: o_parts [S, B, Nq, H, d] bf16, lse_parts [S, B, H, Nq] fp32
+    -> (o [B, Nq, H, d], lse [B, H, Nq])."""
+    lib = load()
+    S, B, Nq, H, d = o_parts.shape
+    _check_tensor("o_parts", o_parts, torch.bfloat16)
+    _check_tensor("lse_parts", lse_parts, torch.float32, (S, B, H, Nq))
+    out = torch.empty(o_parts.shape[1:], dtype=torch.bfloat16, device=o_parts.device) if out is None else out
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=o_parts.device) if lse is None else lse
+    _check_tensor("out", out, torch.bfloat16, (B, Nq, H, d))
+    _check_tensor("lse", lse, torch.float32, (B, H, Nq))
+    st = lib.fa_merge_partials(o_parts.data_ptr(), lse_parts.data_ptr(), S, B, H, Nq, d, out.data_ptr(),
+                               lse.data_ptr(), _stream_ptr(o_parts.device))
+    _raise("fa_merge_partials", st)
+    return out, lse
 
 
 def fa_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int, causal: bool = False,

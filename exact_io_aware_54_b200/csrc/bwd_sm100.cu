@@ -103,6 +103,7 @@ struct BwdArgs {
   // 128-key tile); 0 skips the block
   const uint8_t* block_mask;
   int nqb, nkb;
+  int causal_delta;  // as for the forward: query i sees key j iff j <= i + (lk - lq) + causal_delta
 };
 
 // Where one dS block's dropout draws come from: its key, head and batch element.
@@ -343,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (j * 128 >= sq.lk) return;  // no key of this sequence in the tile
   const int n_qtiles = (sq.lq + 127) >> 7;
   int i_first = 0;
-  if (a.causal) i_first = max(0, j * 128 - (sq.lk - sq.lq)) >> 7;
+  if (a.causal) i_first = max(0, j * 128 - (sq.lk - sq.lq + a.causal_delta)) >> 7;
   int n_iters = n_qtiles - i_first;  // >= 1 when the sequence has queries
   if constexpr (kSparse) {  // the kept query tiles only
     n_iters = 0;
@@ -512,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool key_ok = key_in && key_attended(a, b, key);  // and its P is not masked out
     // first query that sees this key (a sentinel far below any query when not causal;
     // qmin - qs below must not overflow)
-    const int qmin = a.causal ? key - (sq.lk - sq.lq) : -(1 << 30);
+    const int qmin = a.causal ? key - (sq.lk - sq.lq + a.causal_delta) : -(1 << 30);
     bool ok = true;
 
     // dQ tile of query tile `it`: this group's D/2 columns, fp32 vector reductions
@@ -565,7 +566,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         reg_pin(dp);
         const uint32_t stat_u32 = sbase + L::kOffStat + st * 1024 + col * 4;
         const bool tile_mask = a.key_mask != nullptr || (j * 128 + 128 > sq.lk) ||
-                               (a.causal && (j * 128 + 127 - (sq.lk - sq.lq) > qs));
+                               (a.causal && (j * 128 + 127 - (sq.lk - sq.lq + a.causal_delta) > qs));
         uint32_t pk[16], dk2[16];
         if constexpr (kDrop) {
           const DropCtx dctx{a.drop_t, a.drop_scale, a.seed_lo, a.seed_hi, key, h, b};
@@ -748,8 +749,8 @@ __device__ __forceinline__ PipeItem pipe_item(const BwdArgs& a, int w) {
   it.n = -1;
   if (it.s.lq < 0 || it.j * 128 >= it.s.lk) return it;
   const int n_qtiles = (it.s.lq + 127) >> 7;
-  it.i_first = a.causal ? (max(0, it.j * 128 - (it.s.lk - it.s.lq)) >> 7) : 0;
-  it.n = n_qtiles - it.i_first;
+  it.i_first = a.causal ? (max(0, it.j * 128 - (it.s.lk - it.s.lq + a.causal_delta)) >> 7) : 0;
+  it.n = max(0, n_qtiles - it.i_first);  // 0: keys no query sees (dK = dV = 0)
   if constexpr (kSparse) {  // the kept query tiles only
     it.n = 0;
     for (int i = it.i_first; i < n_qtiles; ++i) it.n += bwd_block_kept<true>(a, it.h, i, it.j) ? 1 : 0;
@@ -1128,9 +1129,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       const int key = itm.j * 128 + r;
       const bool key_in = key < itm.s.lk;  // a row of dK / dV to write
       const bool key_ok = key_in && key_attended(a, (w % (a.B * a.H)) / a.H, key);  // P not masked out
-      const int qmin = a.causal ? key - (itm.s.lk - itm.s.lq) : -(1 << 30);
+      const int qmin = a.causal ? key - (itm.s.lk - itm.s.lq + a.causal_delta) : -(1 << 30);
       const bool key_tail = a.key_mask != nullptr || itm.j * 128 + 128 > itm.s.lk;  // masked variant
-      const int last_key_qmin = itm.j * 128 + 127 - (itm.s.lk - itm.s.lq);
+      const int last_key_qmin = itm.j * 128 + 127 - (itm.s.lk - itm.s.lq + a.causal_delta);
       const int n_qt = (itm.s.lq + 127) >> 7;
       int qi = next_kept_q<kSparse>(a, itm.h, itm.j, itm.i_first, n_qt);  // query tile of step t
       for (int t = 0; t < itm.n; ++t, ++T, qi = next_kept_q<kSparse>(a, itm.h, itm.j, qi + 1, n_qt)) {
@@ -1364,6 +1365,7 @@ static fa_status launch_bwd_impl(const BwdLaunch& L0, cudaStream_t stream) {
   a.block_mask = L0.block_mask;
   a.nqb = (L0.Nq + 127) / 128;
   a.nkb = (L0.Nk + 127) / 128;
+  a.causal_delta = L0.causal_delta;
   const long long grid = (long long)a.n_kv_tiles * L0.B * L0.H;
   if (grid > 0x7fffffffLL) return FA_ERR_UNSUPPORTED;
   prof_before(stream, kKBwdMain);

@@ -203,8 +203,8 @@ static bool dropout_threshold(float p, uint32_t* t) {
 // Dense forward, with an optional key-padding mask (4-byte aligned when given),
 // dropout (drop_t = 0: none) or block-sparse mask.
 static fa_status fwd_dense(const void* q, const void* k, const void* v, void* o, float* lse, const uint32_t* key_mask,
-                           uint32_t drop_t, unsigned long long seed, const uint8_t* block_mask, int B, int H, int Nq,
-                           int Nk, int d, int causal,
+                           uint32_t drop_t, unsigned long long seed, const uint8_t* block_mask, int causal_delta, int B,
+                           int H, int Nq, int Nk, int d, int causal,
                            float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!q || !k || !v || !o || !lse || !dims_ok(B, H, Nq, Nk, d)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
@@ -224,6 +224,7 @@ static fa_status fwd_dense(const void* q, const void* k, const void* v, void* o,
   a.drop_t = drop_t;
   a.seed = seed;
   a.block_mask = block_mask;
+  a.causal_delta = causal_delta;
   a.B = B;
   a.H = H;
   a.Nq = Nq;
@@ -239,7 +240,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int d, int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
                  cudaStream_t stream) {
   const NvtxRange range("fa_fwd");
-  return fwd_dense(q, k, v, o, lse, nullptr, 0u, 0ull, nullptr, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
+  return fwd_dense(q, k, v, o, lse, nullptr, 0u, 0ull, nullptr, 0, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
                    workspace_bytes, stream);
 }
 
@@ -249,7 +250,7 @@ fa_status fa_fwd_masked(const void* q, const void* k, const void* v, void* o, fl
   const NvtxRange range("fa_fwd_masked");
   uint32_t t = 0;
   if (!dropout_threshold(dropout_p, &t)) return FA_ERR_INVALID_ARG;
-  return fwd_dense(q, k, v, o, lse, key_mask, t, seed, nullptr, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
+  return fwd_dense(q, k, v, o, lse, key_mask, t, seed, nullptr, 0, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
                    workspace_bytes, stream);
 }
 
@@ -258,7 +259,26 @@ fa_status fa_fwd_blocksparse(const void* q, const void* k, const void* v, void* 
                              float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   const NvtxRange range("fa_fwd_blocksparse");
   if (!block_mask) return FA_ERR_INVALID_ARG;
-  return fwd_dense(q, k, v, o, lse, nullptr, 0u, 0ull, block_mask, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
+  return fwd_dense(q, k, v, o, lse, nullptr, 0u, 0ull, block_mask, 0, B, H, Nq, Nk, d, causal, softmax_scale, workspace,
+                   workspace_bytes, stream);
+}
+
+// The shard holds keys key_offset .. key_offset + Nk - 1 of Nk_total: query i sees
+// shard key j iff key_offset + j <= i + Nk_total - Nq, i.e. j <= i + (Nk - Nq) + delta
+// with delta = Nk_total - key_offset - Nk.
+static bool shard_delta(int key_offset, int Nk_total, int Nk, int* delta) {
+  if (key_offset < 0 || Nk_total <= 0 || (long long)key_offset + Nk > Nk_total) return false;
+  *delta = Nk_total - key_offset - Nk;
+  return true;
+}
+
+fa_status fa_fwd_shard(const void* q, const void* k, const void* v, void* o, float* lse, int key_offset, int Nk_total,
+                       int B, int H, int Nq, int Nk, int d, float softmax_scale, void* workspace,
+                       size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_fwd_shard");
+  int delta = 0;
+  if (!shard_delta(key_offset, Nk_total, Nk, &delta)) return FA_ERR_INVALID_ARG;
+  return fwd_dense(q, k, v, o, lse, nullptr, 0u, 0ull, nullptr, delta, B, H, Nq, Nk, d, 1, softmax_scale, workspace,
                    workspace_bytes, stream);
 }
 
@@ -304,8 +324,8 @@ fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, const int32
 // the forward's dropout (drop_t = 0: none) or block-sparse mask.
 static fa_status bwd_dense(const void* q, const void* k, const void* v, const void* o, const void* do_,
                            const float* lse, void* dq, void* dk, void* dv, const uint32_t* key_mask, uint32_t drop_t,
-                           unsigned long long seed, const uint8_t* block_mask, int B, int H, int Nq, int Nk, int d,
-                           int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
+                           unsigned long long seed, const uint8_t* block_mask, int causal_delta, int B, int H, int Nq,
+                           int Nk, int d, int causal, float softmax_scale, void* workspace, size_t workspace_bytes,
                            cudaStream_t stream) {
   if (!q || !k || !v || !o || !do_ || !lse || !dq || !dk || !dv || !dims_ok(B, H, Nq, Nk, d))
     return FA_ERR_INVALID_ARG;
@@ -333,6 +353,7 @@ static fa_status bwd_dense(const void* q, const void* k, const void* v, const vo
   a.drop_t = drop_t;
   a.seed = seed;
   a.block_mask = block_mask;
+  a.causal_delta = causal_delta;
   a.B = B;
   a.H = H;
   a.Nq = Nq;
@@ -348,7 +369,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d, int causal,
                  float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   const NvtxRange range("fa_bwd");
-  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, nullptr, 0u, 0ull, nullptr, B, H, Nq, Nk, d, causal,
+  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, nullptr, 0u, 0ull, nullptr, 0, B, H, Nq, Nk, d, causal,
                    softmax_scale, workspace, workspace_bytes, stream);
 }
 
@@ -359,7 +380,7 @@ fa_status fa_bwd_masked(const void* q, const void* k, const void* v, const void*
   const NvtxRange range("fa_bwd_masked");
   uint32_t t = 0;
   if (!dropout_threshold(dropout_p, &t)) return FA_ERR_INVALID_ARG;
-  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, key_mask, t, seed, nullptr, B, H, Nq, Nk, d, causal,
+  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, key_mask, t, seed, nullptr, 0, B, H, Nq, Nk, d, causal,
                    softmax_scale, workspace, workspace_bytes, stream);
 }
 
@@ -369,8 +390,28 @@ fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v, const 
                              size_t workspace_bytes, cudaStream_t stream) {
   const NvtxRange range("fa_bwd_blocksparse");
   if (!block_mask) return FA_ERR_INVALID_ARG;
-  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, nullptr, 0u, 0ull, block_mask, B, H, Nq, Nk, d, causal,
+  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, nullptr, 0u, 0ull, block_mask, 0, B, H, Nq, Nk, d, causal,
                    softmax_scale, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_shard(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,
+                       void* dq, void* dk, void* dv, int key_offset, int Nk_total, int B, int H, int Nq, int Nk, int d,
+                       float softmax_scale, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  const NvtxRange range("fa_bwd_shard");
+  int delta = 0;
+  if (!shard_delta(key_offset, Nk_total, Nk, &delta)) return FA_ERR_INVALID_ARG;
+  return bwd_dense(q, k, v, o, do_, lse, dq, dk, dv, nullptr, 0u, 0ull, nullptr, delta, B, H, Nq, Nk, d, 1,
+                   softmax_scale, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_merge_partials(const void* o_parts, const float* lse_parts, int S, int B, int H, int Nq, int d, void* o,
+                            float* lse, cudaStream_t stream) {
+  const NvtxRange range("fa_merge_partials");
+  if (!o_parts || !lse_parts || !o || !lse || S <= 0 || !dims_ok(B, H, Nq, 1, d)) return FA_ERR_INVALID_ARG;
+  if ((long long)S * B * Nq * H >= (1LL << 40)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(o_parts) || !aligned16(o) || !aligned16(lse_parts) || !aligned16(lse)) return FA_ERR_ALIGNMENT;
+  return launch_merge(o_parts, lse_parts, S, B, H, Nq, d, o, lse, stream);
 }
 
 fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const void* do_, const float* lse,

@@ -114,6 +114,9 @@ struct FwdLaunch {
   // block-sparse mask (dense batches): device uint8 [H, ceil(Nq/128), ceil(Nk/128)],
   // 0 skips the (query tile, KV tile) block; null for dense attention
   const uint8_t* block_mask = nullptr;
+  // causal visibility offset beyond the bottom-right alignment (a key shard: its
+  // keys start later in the sequence)
+  int causal_delta = 0;
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;
@@ -142,11 +145,16 @@ struct BwdLaunch {
   uint32_t drop_t = 0;                  // as for the forward
   unsigned long long seed = 0;
   const uint8_t* block_mask = nullptr;  // as for the forward
+  int causal_delta = 0;                 // as for the forward
   int B, H, Nq, Nk, d, causal;
   float scale;
   unsigned long long timeout_ns;
 };
 fa_status launch_bwd(const BwdLaunch& a, cudaStream_t stream);
+
+// Merge of S partial (o, lse) results over key shards (merge_sm100.cu).
+fa_status launch_merge(const void* o_parts, const float* lse_parts, int S, int B, int H, int Nq, int d, void* o,
+                       float* lse, cudaStream_t stream);
 
 // Split-KV decode plan: keys per chunk and chunks per sequence.
 struct DecodePlan {

@@ -146,6 +146,9 @@ struct FwdArgs {
   // tile, 128-key KV tile); 0 skips the block
   const uint8_t* block_mask;
   int nqb, nkb;
+  // causal: query i sees key j iff j <= i + (lk - lq) + causal_delta (0 except for a
+  // key shard, whose keys start later in the sequence)
+  int causal_delta;
 };
 
 // KV tile j takes part for 128-row query tile qtile of head h (always in the dense
@@ -225,7 +228,7 @@ __device__ __forceinline__ int tile_kv_count(const FwdArgs& a, const SeqView& v,
   if (row0 >= v.lq) return -1;
   if (!a.causal) return (v.lk + 127) >> 7;
   const int last = min(row0 + 127, v.lq - 1);
-  long long kend = (long long)last + 1 + v.lk - v.lq;
+  long long kend = (long long)last + 1 + v.lk - v.lq + a.causal_delta;
   if (kend <= 0) return 0;
   if (kend > v.lk) kend = v.lk;
   return (int)((kend + 127) >> 7);
@@ -670,8 +673,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // visible keys of this row: [0, lim)
       const int lk = sv.lk;  // only the key count stays live through the KV loop
       int lim = lk;
-      if (a.causal) lim = max(0, min(lk, row + 1 + lk - sv.lq));
-      const int group_first_lim = a.causal ? (row0 + 1 + lk - sv.lq) : lk;  // smallest lim in the tile
+      const int cdelta = a.causal_delta;
+      if (a.causal) lim = max(0, min(lk, row + 1 + lk - sv.lq + cdelta));
+      const int group_first_lim = a.causal ? (row0 + 1 + lk - sv.lq + cdelta) : lk;  // smallest lim in the tile
 
       float m2 = -INFINITY;  // running reference max (log2 domain)
       float l = 0.f;         // running sum of the bf16-rounded probabilities (normalises O)
@@ -939,6 +943,7 @@ static fa_status launch_fwd_impl(const FwdLaunch& L0, cudaStream_t stream) {
   a.block_mask = L0.block_mask;
   a.nqb = (L0.Nq + 127) / 128;
   a.nkb = (L0.Nk + 127) / 128;
+  a.causal_delta = L0.causal_delta;
   if (a.block_mask != nullptr && a.drop_t != 0u) return FA_ERR_UNSUPPORTED;  // no entry point combines them
   const int grid = std::min(a.n_items, num_sms() * 1);
   prof_before(stream, kKFwd);

@@ -211,6 +211,47 @@ FA_API fa_status fa_bwd_blocksparse(const void* q, const void* k, const void* v,
                                     size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Causal attention over one shard of the keys, for causal sequence parallelism:
+ * the shard k, v [B, Nk, H, d] holds keys key_offset .. key_offset + Nk - 1 of a
+ * sequence of Nk_total keys, and query i (of Nq, all queries) sees shard key j iff
+ * key_offset + j <= i + (Nk_total - Nq) (the bottom-right alignment of the whole
+ * sequence).  Layouts and results as fa_fwd / fa_bwd with causal = 1; merge the
+ * shards' forward results with fa_merge_partials, and run the backward of each
+ * shard with the merged O and LSE.  A query row that sees no key of the shard gets
+ * O = 0 and LSE = -inf from fa_fwd_shard, and shard keys no query sees get
+ * dK = dV = 0.  FA_ERR_INVALID_ARG unless 0 <= key_offset and
+ * key_offset + Nk <= Nk_total.
+ */
+FA_API fa_status fa_fwd_shard(const void* q, const void* k, const void* v, void* o, float* lse, int key_offset,
+                              int Nk_total, int B, int H, int Nq, int Nk, int d, float softmax_scale, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
+FA_API fa_status fa_bwd_shard(const void* q, const void* k, const void* v, const void* o, const void* do_,
+                              const float* lse, void* dq, void* dk, void* dv, int key_offset, int Nk_total, int B,
+                              int H, int Nq, int Nk, int d, float softmax_scale, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Merge of partial attention results over key shards, for sequence parallelism
+ * (the multi-GPU extension the second page wishes for, "AI Bible 13", section 06):
+ * when the keys and values are split into S shards and fa_fwd runs over each shard
+ * with all queries (not causal; causal shards go through fa_fwd_shard), the shard
+ * results combine by the block-merge rule
+ * ("FlashAttention saves IO, not N^2 work", sections 3 and 7):
+ *     O = sum_s exp(lse_s - M) o_s / sum_s exp(lse_s - M),  M = max_s lse_s,
+ *     lse = M + ln sum_s exp(lse_s - M).
+ *   o_parts   : [S, B, Nq, H, d] bf16, shard s's fa_fwd output at o_parts + s * B Nq H d
+ *   lse_parts : [S, B, H, Nq] fp32, shard s's lse
+ *   o, lse    : [B, Nq, H, d] bf16 and [B, H, Nq] fp32 (written)
+ * A shard with lse = -inf for a row contributes nothing to it; a row with no key in
+ * any shard gets O = 0 and LSE = -inf.  No workspace; 16-byte aligned pointers.
+ * The backward of sequence-parallel attention needs no merge: fa_bwd over each
+ * shard with the merged O and lse gives that shard's dK and dV exactly and a
+ * partial dQ, and the partial dQ sum over shards is dQ.
+ */
+FA_API fa_status fa_merge_partials(const void* o_parts, const float* lse_parts, int S, int B, int H, int Nq, int d,
+                                   void* o, float* lse, cudaStream_t stream);
+
+/*
  * Split-KV decode over a ragged, packed KV cache.
  *   q           : [B, H, d] bf16 (one query row per sequence: Nq must be 1)
  *   k, v        : [total_kv, H, d] bf16; sequence b owns rows

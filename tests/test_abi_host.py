@@ -246,6 +246,41 @@ def test_blocksparse_argument_validation(lib):
     assert bwd(wsb=16) == ST["FA_ERR_WORKSPACE"]
 
 
+def test_merge_partials_argument_validation(lib):
+    def call(**kw):
+        a = dict(op=P, lp=P, S=4, B=2, H=3, Nq=300, d=128, o=P, lse=P)
+        a.update(kw)
+        return lib.fa_merge_partials(a["op"], a["lp"], a["S"], a["B"], a["H"], a["Nq"], a["d"], a["o"], a["lse"],
+                                     None)
+
+    assert call(op=None) == ST["FA_ERR_INVALID_ARG"]
+    assert call(S=0) == ST["FA_ERR_INVALID_ARG"]
+    assert call(Nq=0) == ST["FA_ERR_INVALID_ARG"]
+    assert call(d=96) == ST["FA_ERR_UNSUPPORTED"]
+    assert call(o=P + 4) == ST["FA_ERR_ALIGNMENT"]
+    assert call(lp=P + 8) == ST["FA_ERR_ALIGNMENT"]
+
+
+def test_shard_argument_validation(lib):
+    def fwd(**kw):
+        a = dict(off=0, tot=1024, B=2, H=4, Nq=512, Nk=256, d=64)
+        a.update(kw)
+        return lib.fa_fwd_shard(P, P, P, P, P, a["off"], a["tot"], a["B"], a["H"], a["Nq"], a["Nk"], a["d"], 0.0,
+                                P, 1 << 20, None)
+
+    def bwd(**kw):
+        a = dict(off=0, tot=1024, B=2, H=4, Nq=512, Nk=256, d=128)
+        a.update(kw)
+        return lib.fa_bwd_shard(P, P, P, P, P, P, P, P, P, a["off"], a["tot"], a["B"], a["H"], a["Nq"], a["Nk"],
+                                a["d"], 0.0, P, 1 << 30, None)
+
+    assert fwd(off=-1) == ST["FA_ERR_INVALID_ARG"]
+    assert fwd(off=800) == ST["FA_ERR_INVALID_ARG"]   # 800 + 256 > 1024
+    assert fwd(tot=0) == ST["FA_ERR_INVALID_ARG"]
+    assert bwd(off=900) == ST["FA_ERR_INVALID_ARG"]
+    assert bwd(Nk=2000) == ST["FA_ERR_INVALID_ARG"]
+
+
 def test_selftest_argument_validation(lib):
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint, ctypes.c_void_p]
     assert lib.fa_selftest_wait_timeout(None, 256, 100, None) == ST["FA_ERR_WORKSPACE"]
