@@ -118,11 +118,12 @@ def compare_reordered(o_a, o_b, lse_a, lse_b, what="O"):
     """Two GPU results of the same attention that differ only in the order of their
     fp32 sums (the split-KV decode hands key chunks to CTAs as they become free, so
     which keys share a partial state changes from call to call): O agrees to one
-    bf16 rounding step (2^-8 relative) and LSE to 1e-5 relative."""
+    bf16 step (a bf16 value in [2^e, 2^(e+1)) has steps of 2^(e-7), at most 2^-7 of
+    its magnitude) and LSE to 1e-5 relative."""
     a = np.asarray(o_a, dtype=np.float64)
     b = np.asarray(o_b, dtype=np.float64)
     assert a.shape == b.shape
-    tol = 2.0 ** -8 * np.maximum(np.abs(a), np.abs(b)) + 1e-6
+    tol = 2.0 ** -7 * np.maximum(np.abs(a), np.abs(b)) + 1e-6
     bad = np.abs(a - b) > tol
     assert not bad.any(), f"{what}: {int(bad.sum())} elements differ by more than one bf16 step"
     la = np.asarray(lse_a, dtype=np.float64)
