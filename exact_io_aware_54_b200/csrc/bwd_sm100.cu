@@ -256,6 +256,30 @@ __device__ __forceinline__ void ds_block(const uint32_t (&sv)[kN], const uint32_
                                          float scale_log2, bool key_ok, int qrel_min, uint32_t (&pk)[kN / 2],
                                          uint32_t (&dsk)[kN / 2], const DropCtx* drop = nullptr, int q0 = 0) {
   const float2 sc2 = make_float2(scale_log2, scale_log2);
+  // Dropout keep bits of this key for queries q0 .. q0 + kN - 1 (bit c).  One Philox
+  // call covers 4 queries x 2 keys and keys 2k, 2k + 1 sit on neighbouring lanes:
+  // each lane makes every other call of the pair and sends its neighbour the bits
+  // of the neighbour's key.
+  uint32_t keep = 0u;
+  if constexpr (kDrop) {
+    const uint32_t odd = (uint32_t)drop->key & 1u;
+    uint32_t mine = 0u, theirs = 0u;
+#pragma unroll
+    for (int g = 0; g < kN / 4; g += 2) {
+      const int gm = g + (int)odd;  // the query group this lane draws
+      const uint4 w = philox4x32_10(
+          make_uint4((uint32_t)drop->key >> 1, (uint32_t)(q0 + 4 * gm) >> 2, (uint32_t)drop->h, (uint32_t)drop->b),
+          drop->seed_lo, drop->seed_hi);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t lo = ws[e] & 0xFFFFu, hi = ws[e] >> 16;  // even key, odd key
+        mine |= ((odd ? hi : lo) >= drop->t ? 1u : 0u) << (4 * gm + e);
+        theirs |= ((odd ? lo : hi) >= drop->t ? 1u : 0u) << (4 * gm + e);
+      }
+    }
+    keep = mine | __shfl_xor_sync(0xffffffffu, theirs, 1);
+  }
 #pragma unroll
   for (int c = 0; c < kN; c += 4) {
     const float4 nl = ld_shared_f4(stat + c * 4);
@@ -275,16 +299,10 @@ __device__ __forceinline__ void ds_block(const uint32_t (&sv)[kN], const uint32_
     const float2 dp0 = make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1]));
     const float2 dp1 = make_float2(__uint_as_float(dp[c + 2]), __uint_as_float(dp[c + 3]));
     if constexpr (kDrop) {
-      // queries q0 + c .. q0 + c + 3 are the four words of one call (q0 + c is a
-      // multiple of 4); this key takes the low or high 16 bits of each
-      const uint4 w = philox4x32_10(
-          make_uint4((uint32_t)drop->key >> 1, (uint32_t)(q0 + c) >> 2, (uint32_t)drop->h, (uint32_t)drop->b),
-          drop->seed_lo, drop->seed_hi);
-      const int sh = (drop->key & 1) * 16;
-      const float2 z0 = make_float2(((w.x >> sh) & 0xFFFFu) >= drop->t ? drop->scale : 0.f,
-                                    ((w.y >> sh) & 0xFFFFu) >= drop->t ? drop->scale : 0.f);
-      const float2 z1 = make_float2(((w.z >> sh) & 0xFFFFu) >= drop->t ? drop->scale : 0.f,
-                                    ((w.w >> sh) & 0xFFFFu) >= drop->t ? drop->scale : 0.f);
+      // queries q0 + c .. q0 + c + 3
+      const uint32_t kq = keep >> c;
+      const float2 z0 = make_float2((kq & 1u) ? drop->scale : 0.f, (kq & 2u) ? drop->scale : 0.f);
+      const float2 z1 = make_float2((kq & 4u) ? drop->scale : 0.f, (kq & 8u) ? drop->scale : 0.f);
       const float2 d0 = fmul2(p0, ffma2(dp0, z0, make_float2(nd.x, nd.y)));
       const float2 d1 = fmul2(p1, ffma2(dp1, z1, make_float2(nd.z, nd.w)));
       const float2 pz0 = fmul2(p0, z0), pz1 = fmul2(p1, z1);
@@ -733,16 +751,18 @@ __device__ __forceinline__ int pipe_item_index(int k) {
 // with bad offsets.  Only items with n > 0 take part in the pipeline, and the
 // barrier phases of every role count those items alone.
 struct PipeItem {
-  int j, h, i_first, n;
+  int j, b, h, i_first, n;
   BwdSeq s;
 };
 template <bool kSparse>
 __device__ __forceinline__ PipeItem pipe_item(const BwdArgs& a, int w) {
   PipeItem it;
   const int bh_count = a.B * a.H;
+  // key tile j of every head, then j + 1: the heaviest causal items first
   it.j = w / bh_count;
   const int bh = w - it.j * bh_count;
   const int b = bh / a.H;
+  it.b = b;
   it.h = bh - b * a.H;
   it.s = bwd_seq(a, b);
   it.i_first = 0;
@@ -1128,7 +1148,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
       }
       const int key = itm.j * 128 + r;
       const bool key_in = key < itm.s.lk;  // a row of dK / dV to write
-      const bool key_ok = key_in && key_attended(a, (w % (a.B * a.H)) / a.H, key);  // P not masked out
+      const bool key_ok = key_in && key_attended(a, itm.b, key);  // P not masked out
       const int qmin = a.causal ? key - (itm.s.lk - itm.s.lq + a.causal_delta) : -(1 << 30);
       const bool key_tail = a.key_mask != nullptr || itm.j * 128 + 128 > itm.s.lk;  // masked variant
       const int last_key_qmin = itm.j * 128 + 127 - (itm.s.lk - itm.s.lq + a.causal_delta);
@@ -1162,7 +1182,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         // come as late as possible
         uint32_t pk0[16], dk0[16], pk1[16], dk1[16];
         if constexpr (kDrop) {
-          const DropCtx dctx{a.drop_t, a.drop_scale, a.seed_lo, a.seed_hi, key, itm.h, (w % (a.B * a.H)) / a.H};
+          const DropCtx dctx{a.drop_t, a.drop_scale, a.seed_lo, a.seed_hi, key, itm.h, itm.b};
           ds_block<32, true, true>(sv0, dp0, stat_u32, a.scale_log2, key_ok, qmin - qs0, pk0, dk0, &dctx, qs0);
           ds_block<32, true, true>(sv1, dp1, stat_u32 + 128, a.scale_log2, key_ok, qmin - qs1, pk1, dk1, &dctx,
                                    qs1);

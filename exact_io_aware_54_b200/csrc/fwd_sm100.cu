@@ -684,6 +684,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       int kept_n = 0;  // KV tiles of this item that this query tile has processed
       for (int j = 0; j < nkv; ++j) {
         if (!block_kept<kSparse>(a, h, 2 * pair + t, j)) continue;  // a skipped block: no scores were issued
+        // Dropout: the keep bits of this row's 128 keys of KV tile j (bit c of word
+        // c / 32 for key 128 j + c), drawn before the scores arrive (they depend on
+        // nothing else).  One Philox call covers 4 rows x 2 keys, and rows 4i .. 4i+3
+        // sit on four neighbouring lanes: each lane makes a quarter of the calls of
+        // its quad and the four words of every call are handed round by shuffles.
+        uint32_t keepw[4] = {~0u, ~0u, ~0u, ~0u};
+        if constexpr (kDrop) {
+          const uint32_t qd = lane & 3u;
+          const uint32_t quad = lane & ~3u;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) keepw[i] = 0u;
+#pragma unroll 2
+          for (int m = 0; m < 16; ++m) {  // key pairs 4m .. 4m + 3 of the tile: keys 8m .. 8m + 7
+            const uint32_t kb = (uint32_t)j * 64u + 4u * m + qd;
+            const uint4 w = philox4x32_10(make_uint4(kb, (uint32_t)row >> 2, (uint32_t)h, (uint32_t)b), a.seed_lo,
+                                          a.seed_hi);
+            uint32_t bits = 0u;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              // lane s hands out the word of row (s - k) & 3; lane qd receives from lane
+              // (qd + k) & 3 the word of its own row in that lane's call
+              const uint32_t give = (qd - k) & 3u;
+              const uint32_t v = give == 0 ? w.x : (give == 1 ? w.y : (give == 2 ? w.z : w.w));
+              const uint32_t src = (qd + k) & 3u;
+              const uint32_t got = __shfl_sync(0xffffffffu, v, (int)(quad | src));
+              const uint32_t keep2 = ((got & 0xFFFFu) >= a.drop_t ? 1u : 0u) | ((got >> 16) >= a.drop_t ? 2u : 0u);
+              bits |= keep2 << (2 * src);
+            }
+            keepw[m >> 2] |= bits << (8 * (m & 3));
+          }
+        }
         if (!warp_wait<kSoftmaxSpins>(bar_s_full + t, s_cnt & 1, a.timeout_ns) || *abort_flag) {
           if (lane == 0) record_timeout(a.status, abort_flag);
           ok = false;
@@ -749,14 +780,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint32_t k0 = pack_bf16x2(p0.x, p0.y), k1 = pack_bf16x2(p1.x, p1.y);
               uint32_t s0 = k0, s1 = k1;  // P as the P V product takes it
               if constexpr (kDrop) {
-                // keys key0 .. key0 + 3 of this row: two calls, the row's word of each
-                const uint32_t kb = (uint32_t)(kbase + hf * 64 + ii * 32 + c) >> 1;
-                const uint32_t w0 = dropout_word(kb, row, h, b, a.seed_lo, a.seed_hi);
-                const uint32_t w1 = dropout_word(kb + 1, row, h, b, a.seed_lo, a.seed_hi);
-                const float z0 = (w0 & 0xFFFFu) >= a.drop_t ? a.drop_scale : 0.f;
-                const float z1 = (w0 >> 16) >= a.drop_t ? a.drop_scale : 0.f;
-                const float z2 = (w1 & 0xFFFFu) >= a.drop_t ? a.drop_scale : 0.f;
-                const float z3 = (w1 >> 16) >= a.drop_t ? a.drop_scale : 0.f;
+                // keys c .. c + 3 of this 32-key word of the tile
+                const uint32_t kw = keepw[hf * 2 + ii] >> c;
+                const float z0 = (kw & 1u) ? a.drop_scale : 0.f;
+                const float z1 = (kw & 2u) ? a.drop_scale : 0.f;
+                const float z2 = (kw & 4u) ? a.drop_scale : 0.f;
+                const float z3 = (kw & 8u) ? a.drop_scale : 0.f;
                 s0 = pack_bf16x2(p0.x * z0, p0.y * z1);
                 s1 = pack_bf16x2(p1.x * z2, p1.y * z3);
               }
