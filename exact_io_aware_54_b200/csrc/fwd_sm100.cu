@@ -112,10 +112,16 @@ struct FwdLayout {
   static constexpr int kStages = (D == 64) ? 8 : 4;
   static constexpr int kOffQ = 0;                  // Q tile 0, Q tile 1
   static constexpr int kOffRing = 2 * kTileBytes;
-  static constexpr int kOffBar = kOffRing + kStages * kTileBytes;
+  // d = 64 has room for an output staging buffer of its own (two tiles), so the Q
+  // pair is released as soon as the item's last Q K^T MMA has read it and the next
+  // item's Q load overlaps this item's last steps and epilogue; d = 128 stages its
+  // output through the Q tiles and releases them after the epilogue.
+  static constexpr bool kEarlyQ = (D == 64);
+  static constexpr int kOffStage = kOffRing + kStages * kTileBytes;
+  static constexpr int kOffBar = kOffStage + (kEarlyQ ? 2 * kTileBytes : 0);
   // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], epi[2],
-  // s_free[2], p_free[2]
-  static constexpr int kNumBars = 2 + 2 * kStages + 12;
+  // s_free[2], p_free[2], stage_free[2]
+  static constexpr int kNumBars = 2 + 2 * kStages + 14;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
 };
@@ -290,7 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_epi = bar_s_full + 6;
   uint64_t* bar_s_free = bar_s_full + 8;  // separate P: the softmax group has read S
   uint64_t* bar_p_free = bar_s_full + 10;  // separate P: the P V MMA has read P
+  uint64_t* bar_stage_free = bar_s_full + 12;  // early Q release: the output staging buffer is free
   constexpr bool kSepP = sep_p<D>();
+  static_assert(L::kEarlyQ == kSepP, "the separate-P issuers are the ones that release Q early");
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);
 
@@ -300,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q_full, 1);
-    mbar_init(bar_q_empty, 2);
+    mbar_init(bar_q_empty, L::kEarlyQ ? 1 : 2);  // the Q K^T issuer, or both epilogues
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(bar_kv_full + s, 1);
       mbar_init(bar_kv_empty + s, 1);
@@ -312,6 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_epi + t, 4);
       mbar_init(bar_s_free + t, 4);  // one arrival per softmax warp
       mbar_init(bar_p_free + t, 1);
+      mbar_init(bar_stage_free + t, 1);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -434,11 +443,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_commit(bar_kv_empty + slot_k);
             g += 2;
           }
+          if (ok) umma_commit(bar_q_empty);  // arrives once every Q K^T of the item has read Q
         } else {
-          // O_t += P_t V_j once the group has written P.  The epilogue stages O
-          // through the Q tiles: o_done must also follow this item's Q load (it
-          // decides alone when a tile sees no key at all).
-          if (!wait_or_abort(bar_q_full, it_q & 1)) break;
+          // O_t += P_t V_j once the group has written P.  (No wait for the item's Q
+          // here: the Q K^T issuer may already have released it and the producer
+          // loaded the next item's, so its phase could have moved twice.)
           bool started[2] = {false, false};  // the tile's O holds a product of this item
           for (int j = 0; j < nkv && ok; ++j) {
             const bool kp[2] = {j < nt[0] && block_kept<kSparse>(a, h, 2 * pair, j),
@@ -639,8 +648,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int tid_in_group = threadIdx.x - 128 - t * 128;
     uint32_t s_cnt = 0, tile_iter = 0;  // tile_iter counts items in which this tile is present
     uint32_t items_done = 0;            // items with a query row (the producer's q phases)
-    uint8_t* q_tile = smem + L::kOffQ + t * L::kTileBytes;
-    const uint32_t q_tile_u32 = smem_u32(q_tile);
+    // where the epilogue stages this tile's output for its TMA store
+    uint8_t* o_stage = smem + (L::kEarlyQ ? L::kOffStage : L::kOffQ) + t * L::kTileBytes;
+    const uint32_t o_stage_u32 = smem_u32(o_stage);
 
     for (int rnd = 0; rnd * (int)gridDim.x < a.n_items; ++rnd) {
       const int w = item_of_round(rnd);
@@ -657,8 +667,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tile_kv_count(a, sv, pair * 256) < 0) continue;
       const uint32_t it_q = items_done++;
       if (nkv < 0) {
-        // This query tile lies past the sequence: nothing to compute or store.  Its
-        // release of the Q pair waits for this item's Q load, so that it can never
+        // This query tile lies past the sequence: nothing to compute or store.
+        if constexpr (L::kEarlyQ) continue;  // the Q K^T issuer releases the Q pair
+        // Its release of the Q pair waits for this item's Q load, so that it can never
         // count toward the previous item's release (the other group may still be
         // staging that item's output in its Q tile).
         if (!warp_wait(bar_q_full, it_q & 1, a.timeout_ns) || *abort_flag) {
@@ -859,6 +870,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       // a variable-length tile that runs past its sequence writes its rows itself
       const bool direct = a.cu_q != nullptr && row0 + 128 > se.lq;
       uint4* orow = reinterpret_cast<uint4*>(a.o + ((size_t)(se.qoff + row) * a.H + h) * D);
+      if constexpr (L::kEarlyQ) {
+        // the staging buffer is free once this group's previous TMA store has read it
+        if (tid_in_group == 0) {
+          bulk_wait_group_read0();
+          mbar_arrive(bar_stage_free + t);
+        }
+        if (!warp_wait(bar_stage_free + t, tile_iter & 1, a.timeout_ns) || *abort_flag) {
+          if (lane == 0) record_timeout(a.status, abort_flag);
+          break;
+        }
+      }
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -873,7 +895,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           const int chunk = (cc & 1) * 4 + q4;  // 16-byte chunk within the 128-byte row
-          const uint32_t addr = q_tile_u32 + box * L::kBoxBytes + r * 128 + ((chunk ^ (r & 7)) << 4);
+          const uint32_t addr = o_stage_u32 + box * L::kBoxBytes + r * 128 + ((chunk ^ (r & 7)) << 4);
           const float* f = reinterpret_cast<const float*>(o) + q4 * 8;
           const uint4 packed = make_uint4(pack_bf16x2(f[0] * inv_l, f[1] * inv_l), pack_bf16x2(f[2] * inv_l, f[3] * inv_l),
                                           pack_bf16x2(f[4] * inv_l, f[5] * inv_l), pack_bf16x2(f[6] * inv_l, f[7] * inv_l));
@@ -900,11 +922,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
           if (!direct) {
             for (int bx = 0; bx < L::kBoxes; ++bx)
-              tma_store_4d(&tmO, q_tile + bx * L::kBoxBytes, bx * 64, h, se.qoff + row0, se.bc);
+              tma_store_4d(&tmO, o_stage + bx * L::kBoxBytes, bx * 64, h, se.qoff + row0, se.bc);
             bulk_commit_group();
-            bulk_wait_group_read0();
+            if constexpr (!L::kEarlyQ) bulk_wait_group_read0();  // the Q tile is reloaded next
           }
-          mbar_arrive(bar_q_empty);
+          if constexpr (!L::kEarlyQ) mbar_arrive(bar_q_empty);
         }
       }
       // keep the warp converged before its next tcgen05 instruction
