@@ -10,33 +10,39 @@
 // HBM bandwidth (section 6 of that page: single-request and batched decode).
 //
 // B200 design
-//  * Grid (split, head group, sequence).  A head group is up to 8 heads; the
-//    CTA has one warp per head plus one producer warp.  The CTAs of one
-//    (sequence, head group) share its keys dynamically: each producer takes the
-//    next chunk of keys from a per-(sequence, group) atomic counter whenever it
-//    has issued the previous one, and its consumers fold every chunk the CTA
-//    takes into one running state (the (m, l, u) state of any set of keys is
-//    order-independent), so each CTA still leaves exactly one partial state.  A
-//    static split of one wave left the CTAs that the memory system served last
-//    streaming alone at the end (per-SM busy time ranged over 3.5x at one
-//    request of 8192 keys, H = 32); with shared chunks every SM stays busy until
-//    the keys run out.
-//  * For every key of its chunk the head group's K and V slices are contiguous
-//    (8 heads x d bf16), so the producer moves them with plain bulk copies
-//    (cp.async.bulk) into a ring of shared-memory stages of 8 keys, completion
-//    counted on mbarriers.  Rows are padded by 64 bytes so the consumer reads are
-//    free of bank conflicts.
-//  * Consumer warp = head.  Lane = (key slot t in 0..7) x (part p in 0..3); part
-//    p owns 16-byte chunks p, p+4, ... of the head dimension.  Scores need two
-//    shuffle levels, the stage max three; every lane keeps a partial u over the
-//    keys of its slot, summed across slots once at the end.
+//  * Grid (split, head group, sequence).  A head group is the heads whose slices
+//    of one key row make 256 contiguous bytes: one head of d = 128, two of
+//    d = 64.  Eight consumer warps share the group's keys (each takes 8 keys of
+//    every stage), plus one producer warp.  Few heads per CTA keep the number of
+//    partial states per head small -- one per CTA that serves it, about ten at one
+//    request of 8192 keys, H = 32 -- so the last arrival merges them in one L2
+//    round trip.  (Eight heads per CTA left 74 states per head and a merge of five
+//    dependent round trips at the end of every call.)
+//  * The CTAs of one (sequence, head group) share its keys dynamically: each
+//    producer takes the next chunk of keys from a per-(sequence, group) atomic
+//    counter whenever it has issued the previous one, and its consumers fold every
+//    chunk the CTA takes into one running state (the (m, l, u) state of any set of
+//    keys is order-independent), so each CTA still leaves exactly one partial
+//    state.  A static split of one wave left the CTAs that the memory system
+//    served last streaming alone at the end; with shared chunks every SM stays
+//    busy until the keys run out.
+//  * For every key the group's K and V slices are contiguous, so the producer
+//    moves them with plain bulk copies (cp.async.bulk) into a ring of
+//    shared-memory stages, completion counted on mbarriers.  Rows are padded by 16
+//    bytes: the eight rows that a quarter-warp reads then start four banks apart,
+//    so the consumer reads are free of bank conflicts.
+//  * Consumer warp = (head, 8 keys of the stage).  Lane = (part p in 0..3) x (key
+//    slot t in 0..7); part p owns 16-byte chunks p, p+4, ... of the head
+//    dimension.  Scores need two shuffle levels, the stage max three; every lane
+//    keeps a partial u over the keys of its slot, summed across slots at the end,
+//    and the warps of one head combine their states through shared memory.
 //  * The producer writes each stage's first key and key count into a header
 //    beside the stage; a header with no keys tells the consumers that the
 //    counter ran out.  The last producer of a (sequence, group) to run out --
 //    found with a second ticket -- resets the counter, so counters are zero
 //    between calls.
-//  * The last warp of each (sequence, head) to finish its CTA's state -- found with
-//    an atomic ticket -- merges the CTAs' states and writes o and lse, then resets
+//  * The last CTA of each (sequence, head) to finish its state -- found with an
+//    atomic ticket -- merges the CTAs' states and writes o and lse, then resets
 //    the ticket, so tickets are zero between calls.  A sequence served by a single
 //    CTA skips the partial-state round trip.
 //  * Given the number of rows of a packed cache, every sequence's offsets are
@@ -53,9 +59,8 @@ namespace fa {
 
 namespace {
 
-constexpr int kHeadsPerCta = 8;
-constexpr int kKeysPerStage = 8;
-constexpr int kThreads = (kHeadsPerCta + 1) * 32;
+constexpr int kConsumers = 8;  // consumer warps per CTA
+constexpr int kThreads = (kConsumers + 1) * 32;
 // Two CTAs per SM, each with a ring of about 100 KB of copies in flight.  (One CTA
 // per SM with a ring twice as deep halves the chunk states the merge reads, but
 // eight consumer warps per SM then fall behind: measured 17% slower at one request
@@ -67,16 +72,41 @@ constexpr int kCtasPerSm = FA_DEC_CTAS_PER_SM;
 // states the merge loads per round trip (registers allow more with one CTA per SM)
 constexpr int kMergeBatch = kCtasPerSm == 1 ? 32 : 16;
 
-template <int D>
+// Two ways to move the keys.  Packed caches (kTiled): TMA tensor tiles, one box of
+// 64 columns x kKeysPerStage keys per (head, half of a head's 128-byte column
+// blocks), 128-byte swizzled in shared memory, with one head (d = 128) or two
+// (d = 64) per CTA.  Paged caches, whose pages may hold any number of keys: one
+// bulk copy per key of the contiguous slice of eight heads, into padded rows (a
+// copy has a fixed cost of tens of cycles, so slices of 256 bytes would leave the
+// copy engine, not HBM, as the bound: measured 2.5x slower).
+template <int D, bool kTiled>
 struct DecLayout {
-  static constexpr int kRowBytes = kHeadsPerCta * D * 2;  // one key, all heads of the group
-  static constexpr int kRowStride = kRowBytes + 64;       // padded
+  static constexpr int kHeads = kTiled ? 256 / (2 * D) : 8;    // heads per CTA
+  static constexpr int kWarpsPerHead = kConsumers / kHeads;    // consumer warps sharing one head's keys
+  static constexpr int kKeysPerStage = 8 * kWarpsPerHead;      // 8 keys per consumer warp and stage
+  static constexpr int kRowBytes = kHeads * D * 2;             // one key, all heads of the group
+  // bulk copies: rows padded by 16 bytes, so the eight rows a quarter-warp reads
+  // start four banks apart; tiles: dense 128-byte rows, swizzled
+  static constexpr int kRowStride = kTiled ? kRowBytes : kRowBytes + 16;
+  static constexpr int kBoxBytes = kKeysPerStage * 128;        // tiles: one (head, 64-column) box
   static constexpr int kStageBytes = 2 * kKeysPerStage * kRowStride;  // K rows then V rows
   static constexpr int kStages = (D == 128 ? 6 : 12) / kCtasPerSm;
   static constexpr int kOffBar = kStages * kStageBytes;
-  static constexpr int kOffHdr = kOffBar + 2 * kStages * 8 + 64;  // int2 (first key, keys) per stage
-  static constexpr int kSmemBytes = kOffHdr + kStages * 8 + 128;
+  static constexpr int kOffHdr = kOffBar + 2 * kStages * 8 + 64;  // int4 (first key, keys, first row) per stage
+  static constexpr int kOffComb = kOffHdr + kStages * 16;
+  static constexpr int kCombFloats = D + 4;                       // per consumer warp: m, l, -, -, u[D]
+  static constexpr int kSmemBytes = kOffComb + kConsumers * kCombFloats * 4 + 1024;  // + alignment slack
   static constexpr int kChunks = D / 32;  // 16-byte chunks per lane
+  static_assert(!kTiled || (kStageBytes % 1024 == 0 && kBoxBytes % 1024 == 0),
+                "swizzled boxes start on 1024-byte boundaries");
+  // byte offset of 16-byte chunk c of head hw's slice of key row `row`, from the
+  // start of the stage's K (or V) rows
+  __device__ static __forceinline__ uint32_t chunk_off(int row, int hw, int c) {
+    if constexpr (kTiled)
+      return (hw * (D / 64) + (c >> 3)) * kBoxBytes + row * 128 + (((c & 7) ^ (row & 7)) << 4);
+    else
+      return row * kRowStride + hw * D * 2 + c * 16;
+  }
 };
 
 struct DecArgs {
@@ -114,19 +144,21 @@ __device__ __forceinline__ void bf16x8_to_f32(uint32_t a, uint32_t b, uint32_t c
   f[7] = __uint_as_float(d & 0xFFFF0000u);
 }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecArgs a) {
-  using L = DecLayout<D>;
+// tmK / tmV: the packed cache as [rows, H, D] tensors (kTiled only).
+template <int D, bool kTiled>
+__global__ void __launch_bounds__(kThreads, kCtasPerSm)
+    decode_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV, const DecArgs a) {
+  using L = DecLayout<D, kTiled>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
   uint64_t* empty = full + L::kStages;
   volatile int* flags = reinterpret_cast<volatile int*>(smem + L::kOffBar + 2 * L::kStages * 8);
   // flags[0]: abort
 
   const int split = blockIdx.x, group = blockIdx.y, b = blockIdx.z;
-  const int h0 = group * kHeadsPerCta;
-  const int nh = min(kHeadsPerCta, a.H - h0);
+  const int h0 = group * L::kHeads;
+  const int nh = min(L::kHeads, a.H - h0);
   if (a.check_args && *reinterpret_cast<volatile int*>(a.status) == kStatusBadArg) return;
 
   const bool paged = a.block_table != nullptr;
@@ -156,15 +188,19 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecA
     return;
   }
   if (split >= nsplit) return;
-  int2* hdr = reinterpret_cast<int2*>(smem + L::kOffHdr);
+  int4* hdr = reinterpret_cast<int4*>(smem + L::kOffHdr);
   const size_t bg = (size_t)b * a.groups + group;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(full + s, 1);
-      mbar_init(empty + s, kHeadsPerCta);
+      mbar_init(empty + s, kConsumers);
     }
     flags[0] = 0;
+    if constexpr (kTiled) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+    }
     fence_mbar_init();
     fence_proxy_async_smem();
   }
@@ -173,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecA
   const size_t row_elems = (size_t)a.H * D;          // elements per key row of k / v
   const uint32_t copy_bytes = (uint32_t)nh * D * 2;  // this group's slice of one key row
 
-  if (warp == kHeadsPerCta) {
+  if (warp == kConsumers) {
     // ------------------------------------------------------------------ producer warp
     // The first chunk of CTA `split` is chunk `split` (there is one per CTA that
     // takes part), so no counter round trip delays the first copies; later chunks
@@ -187,19 +223,34 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecA
       const bool more = (long long)c * a.gchunk < len;
       if (more && lane == 0) next = (unsigned)nsplit + atomicAdd(a.grab + bg, 1u);
       for (int st = 0; ok; ++st) {
-        const int key0 = more ? c * a.gchunk + st * kKeysPerStage : 0;
-        if (more && (st * kKeysPerStage >= a.gchunk || key0 >= len)) break;
-        const int nk = more ? min(kKeysPerStage, len - key0) : -1;  // -1: no chunk left
+        const int key0 = more ? c * a.gchunk + st * L::kKeysPerStage : 0;
+        if (more && (st * L::kKeysPerStage >= a.gchunk || key0 >= len)) break;
+        const int nk = more ? min(L::kKeysPerStage, len - key0) : -1;  // -1: no chunk left
         const int slot = issued % L::kStages;
         const uint32_t phase = (issued / L::kStages) & 1;
         if (lane == 0) {
           ok = mbar_wait(empty + slot, phase ^ 1, a.timeout_ns) && !flags[0];
           if (ok) {
-            hdr[slot] = make_int2(key0, nk);
-            if (more)
-              mbar_arrive_expect_tx(full + slot, 2u * nk * copy_bytes);
-            else
+            // tiles: the stage's box rows end at its last key, so they never reach
+            // past the sequence (rows before it belong to earlier sequences or, below
+            // row 0, are filled with zeros); the keys are the last nk rows
+            const int lo = kTiled && more ? L::kKeysPerStage - nk : 0;
+            hdr[slot] = make_int4(key0, nk, lo, 0);
+            if (!more) {
               mbar_arrive(full + slot);  // the header alone: no copies
+            } else if constexpr (kTiled) {
+              const int y = start + key0 + nk - L::kKeysPerStage;
+              mbar_arrive_expect_tx(full + slot, 2u * nh * (D / 64) * L::kBoxBytes);
+              uint8_t* dst = smem + slot * L::kStageBytes;
+              for (int hh = 0; hh < nh; ++hh)
+                for (int half = 0; half < D / 64; ++half) {
+                  uint8_t* box = dst + (hh * (D / 64) + half) * L::kBoxBytes;
+                  tma_load_3d(box, &tmK, full + slot, half * 64, h0 + hh, y);
+                  tma_load_3d(box + L::kKeysPerStage * L::kRowBytes, &tmV, full + slot, half * 64, h0 + hh, y);
+                }
+            } else {
+              mbar_arrive_expect_tx(full + slot, 2u * nk * copy_bytes);
+            }
           } else {
             flags[0] = 1;
             atomicCAS(a.status, 0, kStatusTimeout);
@@ -209,23 +260,26 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecA
         if (!ok) break;
         ++issued;
         if (!more) break;
-        if (lane < 2 * kKeysPerStage) {
-          const int t = lane & (kKeysPerStage - 1);
-          const int is_v = lane >= kKeysPerStage;
-          const int key = key0 + t;
-          if (t < nk) {
-            size_t row = (size_t)start + key;
-            if (paged) {
-              int page = a.block_table[(size_t)b * a.max_pages + key / a.page_size];
-              if (page < 0 || page >= a.num_pages) {  // never read outside the cache
-                atomicExch(a.status, kStatusBadArg);
-                page = 0;
+        if constexpr (!kTiled) {  // (tiles: lane 0 issued the stage above)
+          // copy ci < kKeysPerStage: K row of key key0 + ci, then the V rows
+          for (int ci = lane; ci < 2 * L::kKeysPerStage; ci += 32) {
+            const int is_v = ci >= L::kKeysPerStage;
+            const int t = ci - is_v * L::kKeysPerStage;
+            const int key = key0 + t;
+            if (t < nk) {
+              size_t row = (size_t)start + key;
+              if (paged) {
+                int page = a.block_table[(size_t)b * a.max_pages + key / a.page_size];
+                if (page < 0 || page >= a.num_pages) {  // never read outside the cache
+                  atomicExch(a.status, kStatusBadArg);
+                  page = 0;
+                }
+                row = (size_t)page * a.page_size + key % a.page_size;
               }
-              row = (size_t)page * a.page_size + key % a.page_size;
+              const __nv_bfloat16* src = (is_v ? a.v : a.k) + row * row_elems + (size_t)h0 * D;
+              uint8_t* dst = smem + slot * L::kStageBytes + (is_v * L::kKeysPerStage + t) * L::kRowStride;
+              bulk_load(dst, src, copy_bytes, full + slot);
             }
-            const __nv_bfloat16* src = (is_v ? a.v : a.k) + row * row_elems + (size_t)h0 * D;
-            uint8_t* dst = smem + slot * L::kStageBytes + is_v * kKeysPerStage * L::kRowStride + t * L::kRowStride;
-            bulk_load(dst, src, copy_bytes, full + slot);
           }
         }
       }
@@ -251,10 +305,11 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecA
   }
 
   // -------------------------------------------------------------------- consumer warps
-  const int hw = warp;  // head within the group
+  const int hw = warp / L::kWarpsPerHead;  // head within the group
+  const int ks = warp % L::kWarpsPerHead;  // this warp's 8 keys of every stage: ks * 8 ..
   const bool head_ok = hw < nh;
   const int h = h0 + hw;
-  const int t = lane >> 2, p = lane & 3;
+  const int t = lane & 7, p = lane >> 3;
 
   // q chunks owned by this lane, pre-scaled into the log2 domain
   float qf[L::kChunks][8];
@@ -272,7 +327,6 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecA
 #pragma unroll
     for (int e = 0; e < 8; ++e) u[i][e] = 0.f;
   float m = -INFINITY, l = 0.f;
-  bool ok = true;
 
   for (int s = 0;; ++s) {
     const int slot = s % L::kStages;
@@ -284,30 +338,31 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecA
         flags[0] = 1;
         atomicCAS(a.status, 0, kStatusTimeout);
       }
-      ok = false;
       break;
     }
-    const int nk = hdr[slot].y;
+    const int4 hd = hdr[slot];
+    const int nk = hd.y;
     if (nk < 0) break;  // no chunk left for this CTA
-    const bool valid = head_ok && t < nk;
-    const uint32_t kaddr = smem_u32(smem + slot * L::kStageBytes + t * L::kRowStride + hw * D * 2);
-    const uint32_t vaddr = kaddr + kKeysPerStage * L::kRowStride;
+    const int row = ks * 8 + t;
+    const bool valid = head_ok && row >= hd.z && row < hd.z + nk;
+    const uint32_t kaddr = smem_u32(smem + slot * L::kStageBytes);
+    const uint32_t vaddr = kaddr + L::kKeysPerStage * L::kRowStride;
     float dot = 0.f;
 #pragma unroll
     for (int i = 0; i < L::kChunks; ++i) {
       uint32_t r0, r1, r2, r3;
-      ld_shared_v4(kaddr + (p + 4 * i) * 16, r0, r1, r2, r3);
+      ld_shared_v4(kaddr + L::chunk_off(row, hw, p + 4 * i), r0, r1, r2, r3);
       float kf[8];
       bf16x8_to_f32(r0, r1, r2, r3, kf);
 #pragma unroll
       for (int e = 0; e < 8; ++e) dot = fmaf(qf[i][e], kf[e], dot);
     }
-    dot += __shfl_xor_sync(0xffffffffu, dot, 1);
-    dot += __shfl_xor_sync(0xffffffffu, dot, 2);
+    dot += __shfl_xor_sync(0xffffffffu, dot, 8);
+    dot += __shfl_xor_sync(0xffffffffu, dot, 16);
     const float x = valid ? dot : -INFINITY;
-    float mx = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 4));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+    float mx = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
     const float m_new = fmaxf(m, mx);
     const float m_ref = (m_new == -INFINITY) ? 0.f : m_new;
     const float alpha = (m == -INFINITY) ? 0.f : ex2(m - m_ref);
@@ -316,7 +371,7 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecA
 #pragma unroll
     for (int i = 0; i < L::kChunks; ++i) {
       uint32_t r0, r1, r2, r3;
-      ld_shared_v4(vaddr + (p + 4 * i) * 16, r0, r1, r2, r3);
+      ld_shared_v4(vaddr + L::chunk_off(row, hw, p + 4 * i), r0, r1, r2, r3);
       float vf[8];
       bf16x8_to_f32(r0, r1, r2, r3, vf);
 #pragma unroll
@@ -328,51 +383,82 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecA
   }
 
   // combine the 8 key slots: every lane ends with the sums for its own chunks
+  l += __shfl_xor_sync(0xffffffffu, l, 1);
+  l += __shfl_xor_sync(0xffffffffu, l, 2);
   l += __shfl_xor_sync(0xffffffffu, l, 4);
-  l += __shfl_xor_sync(0xffffffffu, l, 8);
-  l += __shfl_xor_sync(0xffffffffu, l, 16);
 #pragma unroll
   for (int i = 0; i < L::kChunks; ++i)
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       float x = u[i][e];
+      x += __shfl_xor_sync(0xffffffffu, x, 1);
+      x += __shfl_xor_sync(0xffffffffu, x, 2);
       x += __shfl_xor_sync(0xffffffffu, x, 4);
-      x += __shfl_xor_sync(0xffffffffu, x, 8);
-      x += __shfl_xor_sync(0xffffffffu, x, 16);
       u[i][e] = x;
     }
-  if (!ok) return;
+
+  // combine the warps of one head through shared memory; from here on lane i holds
+  // columns i * kPerLane .. of the CTA's state (M, Lsum, U)
+  constexpr int kPerLane = D / 32;
+  float* comb = reinterpret_cast<float*>(smem + L::kOffComb);
+  float* mine = comb + warp * L::kCombFloats;
+  if (t == 0) {
+#pragma unroll
+    for (int i = 0; i < L::kChunks; ++i) {
+      float4* dst = reinterpret_cast<float4*>(mine + 4 + (p + 4 * i) * 8);
+      dst[0] = make_float4(u[i][0], u[i][1], u[i][2], u[i][3]);
+      dst[1] = make_float4(u[i][4], u[i][5], u[i][6], u[i][7]);
+    }
+    if (p == 0) {
+      mine[0] = m;
+      mine[1] = l;
+    }
+  }
+  static_assert(L::kWarpsPerHead == 1 || L::kHeads <= 2, "one named barrier per head of the group");
+  if constexpr (L::kWarpsPerHead == 1)
+    __syncwarp();
+  else if (hw == 0)
+    asm volatile("bar.sync 1, %0;" ::"n"(L::kWarpsPerHead * 32) : "memory");
+  else
+    asm volatile("bar.sync 2, %0;" ::"n"(L::kWarpsPerHead * 32) : "memory");
+  if (flags[0] || ks != 0 || !head_ok) return;  // a wait gave up, or another warp finishes this head
+  float M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < L::kWarpsPerHead; ++w) M = fmaxf(M, comb[(warp + w) * L::kCombFloats]);
+  const float M_ref0 = (M == -INFINITY) ? 0.f : M;
+  float Lsum = 0.f, U[kPerLane];
+#pragma unroll
+  for (int e = 0; e < kPerLane; ++e) U[e] = 0.f;
+#pragma unroll
+  for (int w = 0; w < L::kWarpsPerHead; ++w) {
+    const float* st = comb + (warp + w) * L::kCombFloats;
+    const float mw = st[0];
+    const float wt = (mw == -INFINITY) ? 0.f : ex2(mw - M_ref0);
+    Lsum = fmaf(wt, st[1], Lsum);
+#pragma unroll
+    for (int e = 0; e < kPerLane; ++e) U[e] = fmaf(wt, st[4 + lane * kPerLane + e], U[e]);
+  }
 
   const size_t bh = (size_t)b * a.H + h;
   if (nsplit == 1) {
     // the whole history was one chunk: finish here
-    if (head_ok && t == 0) {
-      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    const float inv = (Lsum > 0.f) ? 1.f / Lsum : 0.f;
+    __nv_bfloat16* out = a.o + bh * D + lane * kPerLane;
 #pragma unroll
-      for (int i = 0; i < L::kChunks; ++i) {
-        uint4 w;
-        w.x = pack_bf16x2(u[i][0] * inv, u[i][1] * inv);
-        w.y = pack_bf16x2(u[i][2] * inv, u[i][3] * inv);
-        w.z = pack_bf16x2(u[i][4] * inv, u[i][5] * inv);
-        w.w = pack_bf16x2(u[i][6] * inv, u[i][7] * inv);
-        *reinterpret_cast<uint4*>(a.o + bh * D + (p + 4 * i) * 8) = w;
-      }
-      if (p == 0) a.lse[bh] = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994530942f : -INFINITY;
-    }
+    for (int e = 0; e < kPerLane; e += 2)
+      *reinterpret_cast<uint32_t*>(out + e) = pack_bf16x2(U[e] * inv, U[e + 1] * inv);
+    if (lane == 0) a.lse[bh] = (Lsum > 0.f) ? (M + __log2f(Lsum)) * 0.69314718055994530942f : -INFINITY;
     return;
   }
 
-  // write this chunk's state; the last chunk of (b, h) to finish merges them all
-  if (!head_ok) return;
-  if (t == 0) {
-    float* pu = a.part_u + (bh * a.splits + split) * D;
-#pragma unroll
-    for (int i = 0; i < L::kChunks; ++i) {
-      float4* dst = reinterpret_cast<float4*>(pu + (p + 4 * i) * 8);
-      __stcg(dst, make_float4(u[i][0], u[i][1], u[i][2], u[i][3]));
-      __stcg(dst + 1, make_float4(u[i][4], u[i][5], u[i][6], u[i][7]));
-    }
-    if (p == 0) __stcg(reinterpret_cast<float2*>(a.part_ml) + bh * a.splits + split, make_float2(m, l));
+  // write this CTA's state; the last CTA of (b, h) to finish merges them all
+  {
+    float* pu = a.part_u + (bh * a.splits + split) * D + lane * kPerLane;
+    if constexpr (kPerLane == 4)
+      __stcg(reinterpret_cast<float4*>(pu), make_float4(U[0], U[1], U[2], U[3]));
+    else
+      __stcg(reinterpret_cast<float2*>(pu), make_float2(U[0], U[1]));
+    if (lane == 0) __stcg(reinterpret_cast<float2*>(a.part_ml) + bh * a.splits + split, make_float2(M, Lsum));
   }
   __threadfence();
   __syncwarp();
@@ -387,10 +473,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm) decode_kernel(const DecA
   // any is used, with a running reference max: one L2 round trip per batch.  Lane
   // i weighs state s0 + i; each lane sums the u of every state over its own kPerLane
   // columns, with the weights passed round by shuffles.
-  constexpr int kPerLane = D / 32;
   const float2* ml = reinterpret_cast<const float2*>(a.part_ml) + bh * a.splits;
   const float* pu = a.part_u + bh * a.splits * D + lane * kPerLane;
-  float M = -INFINITY, Lsum = 0.f, U[kPerLane];
+  M = -INFINITY;
+  Lsum = 0.f;
 #pragma unroll
   for (int e = 0; e < kPerLane; ++e) U[e] = 0.f;
   for (int s0 = 0; s0 < nsplit; s0 += kMergeBatch) {
@@ -460,11 +546,17 @@ __global__ void check_cu_seqlens_kernel(const int32_t* cu, int B, int max_seqlen
 
 }  // namespace
 
-DecodePlan decode_plan(int B, int H, int max_seqlen_k, int d, int num_splits) {
-  (void)d;
+DecodePlan decode_plan(int B, int H, int max_seqlen_k, int d, int num_splits, bool paged) {
   DecodePlan p;
-  p.heads_per_group = std::min(H, kHeadsPerCta);
-  p.groups = (H + kHeadsPerCta - 1) / kHeadsPerCta;
+  const int heads = paged ? DecLayout<128, false>::kHeads
+                          : (d == 64 ? DecLayout<64, true>::kHeads : DecLayout<128, true>::kHeads);
+  const int stage_keys = paged ? DecLayout<128, false>::kKeysPerStage
+                               : (d == 64 ? DecLayout<64, true>::kKeysPerStage : DecLayout<128, true>::kKeysPerStage);
+  static_assert(DecLayout<64, false>::kHeads == DecLayout<128, false>::kHeads &&
+                    DecLayout<64, false>::kKeysPerStage == DecLayout<128, false>::kKeysPerStage,
+                "the bulk-copy layout has the same head groups and stages for both d");
+  p.heads_per_group = std::min(H, heads);
+  p.groups = (H + heads - 1) / heads;
   const int maxL = std::max(max_seqlen_k, 1);
   auto roundup8 = [](long long x) { return (int)(((x + 7) / 8) * 8); };
   int chunk;
@@ -476,9 +568,10 @@ DecodePlan decode_plan(int B, int H, int max_seqlen_k, int d, int num_splits) {
     const long long work = (long long)B * maxL * p.groups;
     chunk = roundup8((work + slots * 16 - 1) / (slots * 16));  // ~16 waves if all sequences are full
     if (chunk < 256) {
-      // a small problem: spread it over one wave of CTAs
+      // a small problem: spread it over one wave of CTAs (a CTA of a second wave
+      // would start its first chunk only when one of the first wave retires)
       const long long units = (long long)B * p.groups;
-      const long long s = std::max(1LL, (slots + units - 1) / units);
+      const long long s = std::max(1LL, slots / units);
       chunk = roundup8((maxL + s - 1) / s);
     }
   }
@@ -490,10 +583,12 @@ DecodePlan decode_plan(int B, int H, int max_seqlen_k, int d, int num_splits) {
   }
   p.chunk = chunk;
   p.splits = splits;
-  // chunks handed out: about an eighth of a CTA's even share of the keys, so the
-  // CTAs of a (sequence, group) can even out how fast each is served, but at
-  // least two stages (one counter round trip hides behind two stages of copies)
-  p.gchunk = std::min(256, std::max(16, roundup8(chunk / 8)));
+  // chunks handed out: whole stages, about an eighth of a CTA's even share of the
+  // keys, so the CTAs of a (sequence, group) can even out how fast each is served,
+  // but at least two stages (one counter round trip hides behind two stages of
+  // copies) and at most 256 keys
+  const int per = (chunk / 8 + stage_keys - 1) / stage_keys * stage_keys;
+  p.gchunk = std::min(std::max(256, 2 * stage_keys), std::max(2 * stage_keys, per));
   return p;
 }
 
@@ -533,15 +628,28 @@ void decode_carve(uint8_t* ws, int B, int H, int d, const DecodePlan& plan, Deco
   a.grab_done = sync + 2 * n;
 }
 
-template <int D>
+template <int D, bool kTiled>
 static fa_status launch_decode_impl(const DecodeLaunch& L0, cudaStream_t stream) {
-  using L = DecLayout<D>;
+  using L = DecLayout<D, kTiled>;
   static PerDeviceOnce attr_once;
   if (!attr_once.run([] {
-        return cudaFuncSetAttribute(decode_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        return cudaFuncSetAttribute(decode_kernel<D, kTiled>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     L::kSmemBytes) == cudaSuccess;
       }))
     return FA_ERR_CUDA;
+  CUtensorMap tmK, tmV;
+  memset(&tmK, 0, sizeof(tmK));
+  memset(&tmV, 0, sizeof(tmV));
+  if constexpr (kTiled) {
+    // rows of the packed cache: the given count, else the most that B sequences of
+    // at most max_seqlen_k keys can hold (the boxes never pass a sequence's end, so
+    // this only bounds the map)
+    const long long rows = L0.total_kv >= 0 ? (long long)L0.total_kv : (long long)L0.B * L0.max_seqlen_k;
+    const int r = (int)std::max(1LL, std::min(rows, 0x7fffffffLL));
+    if (!encode_rows_map(&tmK, L0.k, r, L0.H, D, L::kKeysPerStage) ||
+        !encode_rows_map(&tmV, L0.v, r, L0.H, D, L::kKeysPerStage))
+      return FA_ERR_CUDA;
+  }
   DecArgs a;
   a.q = static_cast<const __nv_bfloat16*>(L0.q);
   a.k = static_cast<const __nv_bfloat16*>(L0.k);
@@ -583,15 +691,17 @@ static fa_status launch_decode_impl(const DecodeLaunch& L0, cudaStream_t stream)
   }
   dim3 grid(L0.plan.splits, L0.plan.groups, L0.B);
   prof_before(stream, kKDecode);
-  decode_kernel<D><<<grid, kThreads, L::kSmemBytes, stream>>>(a);
+  decode_kernel<D, kTiled><<<grid, kThreads, L::kSmemBytes, stream>>>(tmK, tmV, a);
   const cudaError_t err = cudaGetLastError();
   prof_after(stream, kKDecode);
   return err == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status launch_decode(const DecodeLaunch& L0, cudaStream_t stream) {
-  if (L0.d == 64) return launch_decode_impl<64>(L0, stream);
-  if (L0.d == 128) return launch_decode_impl<128>(L0, stream);
+  const bool paged = L0.block_table != nullptr;
+  if (L0.d == 64) return paged ? launch_decode_impl<64, false>(L0, stream) : launch_decode_impl<64, true>(L0, stream);
+  if (L0.d == 128)
+    return paged ? launch_decode_impl<128, false>(L0, stream) : launch_decode_impl<128, true>(L0, stream);
   return FA_ERR_UNSUPPORTED;
 }
 

@@ -114,6 +114,19 @@ bool encode_bshd_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int
   return r == CUDA_SUCCESS;
 }
 
+bool encode_rows_map(CUtensorMap* map, const void* ptr, int rows, int H, int D, int box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn || rows <= 0 || box_rows <= 0 || box_rows > 256) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows};
+  const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+  const cuuint32_t box[3] = {64, 1, (cuuint32_t)box_rows};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 unsigned long long wait_timeout_ns() {
   static unsigned long long v = [] {
     unsigned long long ms = 2000;
@@ -187,7 +200,9 @@ int fa_decode_num_splits(int B, int H, int max_seqlen_k, int d, int num_splits) 
 
 size_t fa_decode_workspace_size(int B, int H, int max_seqlen_k, int d, int num_splits) {
   if (B <= 0 || H <= 0 || max_seqlen_k < 0 || (d != 64 && d != 128) || num_splits < 0) return 0;
-  return decode_workspace_bytes(B, H, d, decode_plan(B, H, max_seqlen_k, d, num_splits));
+  // one size serves the packed and the paged decode
+  return std::max(decode_workspace_bytes(B, H, d, decode_plan(B, H, max_seqlen_k, d, num_splits, false)),
+                  decode_workspace_bytes(B, H, d, decode_plan(B, H, max_seqlen_k, d, num_splits, true)));
 }
 
 // Dropout threshold t = round(65536 p) for 0 <= p < 1; false when p is out of range
@@ -542,7 +557,7 @@ fa_status fa_decode_paged(const void* q, const void* k_pages, const void* v_page
   if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) || !aligned16(lse) ||
       (reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seqlens_k) & 3u))
     return FA_ERR_ALIGNMENT;
-  const DecodePlan plan = decode_plan(B, H, max_seqlen_k, d, num_splits);
+  const DecodePlan plan = decode_plan(B, H, max_seqlen_k, d, num_splits, true);
   if (!workspace || !aligned16(workspace) || workspace_bytes < decode_workspace_bytes(B, H, d, plan))
     return FA_ERR_WORKSPACE;
   uint8_t* ws = static_cast<uint8_t*>(workspace);

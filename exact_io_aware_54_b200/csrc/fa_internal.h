@@ -90,6 +90,9 @@ class PerDeviceOnce {
 // Encode a TMA descriptor for a bf16 tensor [B, N, H, D] (D innermost), with a
 // box of 128 rows x 64 columns and 128-byte swizzle.  Returns false on failure.
 bool encode_bshd_map(CUtensorMap* map, const void* ptr, int B, int N, int H, int D);
+// Map of a packed [rows, H, D] bf16 tensor with boxes of 64 columns x one head x
+// box_rows rows, 128-byte swizzled (zeros outside the tensor).
+bool encode_rows_map(CUtensorMap* map, const void* ptr, int rows, int H, int D, int box_rows);
 
 // The same for an fp32 tensor [B, N, H, D]: box of 128 rows x 32 columns (128 bytes), 128-byte swizzle.
 
@@ -160,11 +163,12 @@ fa_status launch_merge(const void* o_parts, const float* lse_parts, int S, int B
 struct DecodePlan {
   int chunk;       // keys per CTA if the keys were split evenly (multiple of 8)
   int splits;      // CTAs (and partial states) per (sequence, head group)
-  int gchunk;      // keys per chunk handed out to a CTA (multiple of 8)
+  int gchunk;      // keys per chunk handed out to a CTA (whole stages of the decode ring)
   int groups;      // head groups per sequence
   int heads_per_group;
 };
-DecodePlan decode_plan(int B, int H, int max_seqlen_k, int d, int num_splits);
+// paged: the plan of the paged-cache kernel (other head groups and stages)
+DecodePlan decode_plan(int B, int H, int max_seqlen_k, int d, int num_splits, bool paged = false);
 
 struct DecodeLaunch {
   const void* q;
