@@ -93,15 +93,18 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr int kMmaSpins = FA_FWD_MMA_SPINS;
 constexpr int kSoftmaxSpins = FA_FWD_SOFTMAX_SPINS;
 // Every kExpFmaEvery-th group of four probabilities computes one pair of its
-// exponentials on the FMA pipes (exp2_fma2) instead of the MUFU unit: a quarter
-// of them at d = 64, an eighth at d = 128 (where the tile has twice the MMA work
-// per exponential).  Measured on B200 against other splits.
+// exponentials on the FMA pipes (exp2_fma2) instead of the MUFU unit: an eighth of
+// them.  Measured on B200 against other splits (at d = 64 a quarter was 5% slower,
+// a sixteenth within 1%).
 #ifndef FA_FWD_EXP_FMA_EVERY_128
 #define FA_FWD_EXP_FMA_EVERY_128 4
 #endif
+#ifndef FA_FWD_EXP_FMA_EVERY_64
+#define FA_FWD_EXP_FMA_EVERY_64 4
+#endif
 template <int D>
 __host__ __device__ constexpr int exp_fma_every() {
-  return D == 64 ? 2 : FA_FWD_EXP_FMA_EVERY_128;
+  return D == 64 ? FA_FWD_EXP_FMA_EVERY_64 : FA_FWD_EXP_FMA_EVERY_128;
 }
 
 template <int D>
@@ -473,6 +476,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             g += 2;
           }
           if (!ok) break;
+          // both tiles' O are released together: releasing each right after its own
+          // last P V measured 2% slower (its epilogue then competes with the other
+          // tile's last step)
 #pragma unroll
           for (int t = 0; t < 2; ++t)
             if (nt[t] >= 0) umma_commit(bar_o_done + t);
