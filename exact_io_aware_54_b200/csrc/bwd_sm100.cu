@@ -693,8 +693,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 // heaviest first.  Every role counts query tiles over all its items, so the
 // per-tile barriers run on one stream of phases.  K has two slots and the next
 // item's K is loaded a whole item ahead; V has one slot, released after the item's
-// last dP^T, so the next V loads while the last query tile is finished.  The dS
-// warps write dK and dV straight from registers to global memory.
+// last dP^T, so the next V loads while the last query tile is finished.  The dQ
+// drain warps also write each item's dK and dV (tensor memory -> registers ->
+// global memory), so the dS warps go straight on to the next item's first query
+// tile (when the dS warps wrote them, they waited on the item's last gradient
+// MMAs: 12% of their time, and the kernel was 3% slower).
 struct PipeLayout {
   static constexpr int D = 64;
   static constexpr int kTileBytes = 128 * D * 2;  // 16 KB
@@ -724,7 +727,7 @@ struct PipeLayout {
 // warps 0-3: TMA producer, score MMA issuer, gradient MMA issuer, idle; 4-7: dQ drain;
 // 8-15: dS (two column groups)
 constexpr int kPipeThreads = 512;
-constexpr uint32_t kPipeRegsCtl = 72, kPipeRegsDrain = 88, kPipeRegsDs = 176;
+constexpr uint32_t kPipeRegsCtl = 72, kPipeRegsDrain = 104, kPipeRegsDs = 168;
 static_assert(128 * kPipeRegsCtl + 128 * kPipeRegsDrain + 256 * kPipeRegsDs <= kPipeThreads * 128,
               "register split exceeds the launch budget");
 
@@ -897,7 +900,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     mbar_init(bar_dq_full, 1);
     mbar_init(bar_dq_empty, 4);  // one arrival per drain warp
     mbar_init(bar_dkv_done, 1);
-    mbar_init(bar_acc_free, 8);
+    mbar_init(bar_acc_free, 4);  // one arrival per drain warp
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -1124,6 +1127,40 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         __syncwarp();
       }
       mbar_arrive_warp(bar_ds_free + (T % L::kDsBufs));  // the scratch may be overwritten
+      if (cur.t + 1 < cur.itm.n) continue;
+      // ------------------------------------------------------------ dK / dV of this item
+      // (the drain warps write them, so that the dS warps go straight on to the next
+      // item's first query tile): one key row per thread, 32 columns at a time
+      if (!warp_wait_b(bar_dkv_done, cur.u & 1, a.timeout_ns) || *abort_flag) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int key = cur.itm.j * 128 + (int)(quarter * 32 + lane);
+      const bool key_in = key < cur.itm.s.lk;
+      const size_t row = ((size_t)((long long)cur.itm.s.tb * a.Nk + cur.itm.s.tk + key) * a.H + cur.itm.h) * (D / 8);
+#pragma unroll 1
+      for (int part = 0; part < 4; ++part) {  // dK columns 0-31, 32-63, then dV
+        uint32_t g[32];
+        tmem_ld32(tmem + lane_field + (part < 2 ? L::kTmDK : L::kTmDV) + (part & 1) * 32, g);
+        tmem_ld_wait(g);
+        if (part == 3) {  // dK and dV are out of tensor memory: the next item may restart them
+          tc_fence_before();
+          mbar_arrive_warp(bar_acc_free);
+        }
+        if (key_in) {
+          const float mul = part < 2 ? a.scale : 1.f;
+          uint4* dst = (part < 2 ? a.dk : a.dv) + row + (part & 1) * 4;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint32_t* f = g + 8 * c;
+            dst[c] = make_uint4(pack_bf16x2(__uint_as_float(f[0]) * mul, __uint_as_float(f[1]) * mul),
+                                pack_bf16x2(__uint_as_float(f[2]) * mul, __uint_as_float(f[3]) * mul),
+                                pack_bf16x2(__uint_as_float(f[4]) * mul, __uint_as_float(f[5]) * mul),
+                                pack_bf16x2(__uint_as_float(f[6]) * mul, __uint_as_float(f[7]) * mul));
+          }
+        }
+      }
     }
     if (!ok && lane == 0) bwd_timeout(a.status, abort_flag);
   } else {
@@ -1135,7 +1172,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
     const uint32_t lane_field = (quarter * 32) << 16;
     const int col = 64 * grp;
     bool ok = true;
-    int T = 0, u = 0;
+    int T = 0;
     for (int k = 0, w; (w = pipe_item_index(k)) < n_items && ok; ++k) {
       const PipeItem itm = pipe_item<kSparse>(a, w);
       if (itm.n <= 0) {
@@ -1147,8 +1184,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         continue;
       }
       const int key = itm.j * 128 + r;
-      const bool key_in = key < itm.s.lk;  // a row of dK / dV to write
-      const bool key_ok = key_in && key_attended(a, itm.b, key);  // P not masked out
+      const bool key_ok = key < itm.s.lk && key_attended(a, itm.b, key);  // P not masked out
       const int qmin = a.causal ? key - (itm.s.lk - itm.s.lq + a.causal_delta) : -(1 << 30);
       const bool key_tail = a.key_mask != nullptr || itm.j * 128 + 128 > itm.s.lk;  // masked variant
       const int last_key_qmin = itm.j * 128 + 127 - (itm.s.lk - itm.s.lq + a.causal_delta);
@@ -1179,7 +1215,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         const uint32_t ds_row = sbase + L::kOffDS + db * L::kDsBytes + grp * 16384 + r * 128;
         const int qs0 = q0 + col, qs1 = q0 + col + 32;
         // both 32-query blocks first: the waits for the P^T columns and the dS buffer
-        // come as late as possible
+        // come as late as possible (storing the first block's P^T and dS while the
+        // second is computed measured 1% slower)
         uint32_t pk0[16], dk0[16], pk1[16], dk1[16];
         if constexpr (kDrop) {
           const DropCtx dctx{a.drop_t, a.drop_scale, a.seed_lo, a.seed_hi, key, itm.h, itm.b};
@@ -1220,35 +1257,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1)
         mbar_arrive_warp(bar_p_full);
       }
       if (!ok) break;
-      // -------------------------------------------------------------- dK / dV of this item
-      // group 0 writes dK (times scale), group 1 dV: one key row per thread, bf16
-      if (!warp_wait_b(bar_dkv_done, u & 1, a.timeout_ns) || *abort_flag) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t o0[32], o1[32];
-      const uint32_t src = tmem + lane_field + (grp == 0 ? L::kTmDK : L::kTmDV);
-      tmem_ld32(src, o0);
-      tmem_ld32(src + 32, o1);
-      tmem_ld_wait(o0);
-      reg_pin(o1);
-      tc_fence_before();
-      mbar_arrive_warp(bar_acc_free);  // the next item may restart dK / dV
-      if (key_in) {
-        const float mul = grp == 0 ? a.scale : 1.f;
-        uint4* dst =
-            (grp == 0 ? a.dk : a.dv) + ((size_t)((long long)itm.s.tb * a.Nk + itm.s.tk + key) * a.H + itm.h) * (D / 8);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t* f = (c < 4 ? o0 : o1) + (c & 3) * 8;
-          dst[c] = make_uint4(pack_bf16x2(__uint_as_float(f[0]) * mul, __uint_as_float(f[1]) * mul),
-                              pack_bf16x2(__uint_as_float(f[2]) * mul, __uint_as_float(f[3]) * mul),
-                              pack_bf16x2(__uint_as_float(f[4]) * mul, __uint_as_float(f[5]) * mul),
-                              pack_bf16x2(__uint_as_float(f[6]) * mul, __uint_as_float(f[7]) * mul));
-        }
-      }
-      ++u;
+      // dK and dV of this item are written by the drain warps
     }
     if (!ok && lane == 0) bwd_timeout(a.status, abort_flag);
   }
