@@ -10,7 +10,7 @@
 // HBM bandwidth (section 6 of that page: single-request and batched decode).
 //
 // B200 design
-//  * Grid (split, head group, sequence).  A head group is the heads whose slices
+//  * Grid (head group, split, sequence).  A head group is the heads whose slices
 //    of one key row make 256 contiguous bytes: one head of d = 128, two of
 //    d = 64.  Eight consumer warps share the group's keys (each takes 8 keys of
 //    every stage), plus one producer warp.  Few heads per CTA keep the number of
@@ -156,7 +156,10 @@ __global__ void __launch_bounds__(kThreads, kCtasPerSm)
   volatile int* flags = reinterpret_cast<volatile int*>(smem + L::kOffBar + 2 * L::kStages * 8);
   // flags[0]: abort
 
-  const int split = blockIdx.x, group = blockIdx.y, b = blockIdx.z;
+  // grid (group, split, sequence): consecutive CTAs serve different head groups, so
+  // the CTAs of one group spread over the whole GPU instead of sitting side by side
+  // (measured: one request of 8192 keys 32.8 -> 30.9 us, the 64-request batch 1%)
+  const int group = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
   const int h0 = group * L::kHeads;
   const int nh = min(L::kHeads, a.H - h0);
   if (a.check_args && *reinterpret_cast<volatile int*>(a.status) == kStatusBadArg) return;
@@ -689,7 +692,7 @@ static fa_status launch_decode_impl(const DecodeLaunch& L0, cudaStream_t stream)
     prof_after(stream, kKDecodeCheck);
     if (err != cudaSuccess) return FA_ERR_CUDA;
   }
-  dim3 grid(L0.plan.splits, L0.plan.groups, L0.B);
+  const dim3 grid(L0.plan.groups, L0.plan.splits, L0.B);
   prof_before(stream, kKDecode);
   decode_kernel<D, kTiled><<<grid, kThreads, L::kSmemBytes, stream>>>(tmK, tmV, a);
   const cudaError_t err = cudaGetLastError();
