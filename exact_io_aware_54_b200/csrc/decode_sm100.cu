@@ -586,12 +586,13 @@ DecodePlan decode_plan(int B, int H, int max_seqlen_k, int d, int num_splits, bo
   }
   p.chunk = chunk;
   p.splits = splits;
-  // chunks handed out: whole stages, about an eighth of a CTA's even share of the
-  // keys, so the CTAs of a (sequence, group) can even out how fast each is served,
-  // but at least two stages (one counter round trip hides behind two stages of
-  // copies) and at most 256 keys
-  const int per = (chunk / 8 + stage_keys - 1) / stage_keys * stage_keys;
-  p.gchunk = std::min(std::max(256, 2 * stage_keys), std::max(2 * stage_keys, per));
+  // chunks handed out: whole stages, about a sixteenth of a CTA's even share of the
+  // keys and at most 256 keys, so the CTAs of a (sequence, group) can even out how
+  // fast each is served: when the counter runs out, the CTAs still streaming hold at
+  // most one chunk each (one request of 8192 keys, H = 32: chunks of one stage, 1
+  // us faster than chunks of two)
+  const int per = (chunk / 16 + stage_keys - 1) / stage_keys * stage_keys;
+  p.gchunk = std::min(std::max(256, stage_keys), std::max(stage_keys, per));
   return p;
 }
 
