@@ -33,10 +33,12 @@ def test_ragged_small(d, num_splits):
     _check([1, 7, 8, 9, 130, 513, 1000, 2048], 8, d, 91 + d, num_splits=num_splits)
 
 
+@pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("H", [1, 5, 8, 12, 40])
-def test_head_groups(H):
-    """Head counts that are not a multiple of the 8-head group."""
-    _check([300, 17, 1024], H, 128, 300 + H)
+def test_head_groups(H, d):
+    """Head counts of every residue: at d = 64 a CTA serves two heads, so odd H leaves
+    a group of one."""
+    _check([300, 17, 1024], H, d, 300 + H + d)
 
 
 def test_empty_and_short_sequences():

@@ -44,6 +44,13 @@ def test_ragged_pages(page_size, d):
     _check([1, 7, 16, 17, 300, 1000, 2049], 8, d, page_size, 700 + page_size + d)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("H", [1, 5, 12])
+def test_head_groups(H, d):
+    """Head counts that are not a multiple of the paged kernel's 8-head group."""
+    _check([5, 300, 1100], H, d, 16, 900 + H + d)
+
+
 def test_single_request_8k_pages_of_64():
     """The single-request decode shape (L=8192, H=32, d=128) through 128 scattered pages."""
     _check([8192], 32, 128, 64, synth.SEEDS["decode"])
