@@ -534,28 +534,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qmin = a.causal ? key - (sq.lk - sq.lq + a.causal_delta) : -(1 << 30);
     bool ok = true;
 
-    // dQ tile of query tile `it`: this group's D/2 columns, fp32 vector reductions
-    // into the accumulator
+    // dQ tile of query tile `it`: this group's D/2 columns, 32 at a time, turned
+    // around in this warp's 4 KB of the dS buffer (free once the dQ product has
+    // completed; the next dS is written by this same warp) so that one vector
+    // reduction covers four whole 128-byte rows: reductions of partial rows run at
+    // about half the L2 rate
+    const int rr_sub = lane >> 3, cc = lane & 7;  // read side: row 4k + rr_sub, chunk cc
+    const uint32_t scratch = sbase + L::kOffDS + grp * 16384 + quarter * 4096;
     auto drain_dq = [&](int it, int q_first) -> bool {
       if (!warp_wait_b(bar_dq_full, it & 1, a.timeout_ns) || *abort_flag) return false;
       tc_fence_after();
-      uint32_t g[D / 64][32];
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        uint32_t g[32];
+        tmem_ld32(tmem + lane_field + L::kTmDQ + grp * (D / 2) + pass * 32, g);
+        tmem_ld_wait(g);
+        if (pass == 1) {  // the dQ tile is out of tensor memory
+          tc_fence_before();
+          mbar_arrive_warp(bar_dq_empty);
+        }
 #pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) tmem_ld32(tmem + lane_field + L::kTmDQ + grp * (D / 2) + cc * 32, g[cc]);
-      tmem_ld_wait(g[0]);
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(scratch + lane * 128 + ((c ^ (lane & 7)) << 4), g[4 * c], g[4 * c + 1], g[4 * c + 2],
+                       g[4 * c + 3]);
+        __syncwarp();
 #pragma unroll
-      for (int cc = 1; cc < D / 64; ++cc) reg_pin(g[cc]);
-      tc_fence_before();
-      mbar_arrive_warp(bar_dq_empty);
-      const int q = q_first + r;
-      if (q < sq.lq) {
-        float* dst = a.dq_acc + ((size_t)((long long)sq.tb * a.Nq + sq.tq + q) * a.H + h) * D + grp * (D / 2);
-#pragma unroll
-        for (int cc = 0; cc < D / 64; ++cc)
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            red_add_v4(dst + cc * 32 + e, __uint_as_float(g[cc][e]), __uint_as_float(g[cc][e + 1]),
-                       __uint_as_float(g[cc][e + 2]), __uint_as_float(g[cc][e + 3]));
+        for (int k = 0; k < 8; ++k) {
+          const int row = 4 * k + rr_sub;
+          const int q = q_first + (int)quarter * 32 + row;
+          const float4 v4 = ld_shared_f4(scratch + row * 128 + ((cc ^ (row & 7)) << 4));
+          if (q < sq.lq)
+            red_add_v4(a.dq_acc + ((size_t)((long long)sq.tb * a.Nq + sq.tq + q) * a.H + h) * D + grp * (D / 2) +
+                           pass * 32 + cc * 4,
+                       v4.x, v4.y, v4.z, v4.w);
+        }
+        __syncwarp();
       }
       return true;
     };
