@@ -25,7 +25,8 @@ struct NvtxRange {
   NvtxRange& operator=(const NvtxRange&) = delete;
 };
 
-// Workspace: the first kStatusBytes hold the status word (int32) and padding.
+// Workspace: the first kStatusBytes hold the status word (int32) and padding; the
+// forward's item counters use bytes 128 .. 135 of the padding (zero between calls).
 constexpr size_t kStatusBytes = 256;
 
 // Decode counters live in a fixed region right after the status word, so they

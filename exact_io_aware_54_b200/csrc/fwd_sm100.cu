@@ -10,8 +10,12 @@
 //
 // B200 design
 //  * Work item = (b, h, pair of 128-row query tiles).  Persistent grid, one CTA
-//    per SM; items are numbered heaviest (latest causal rows) first and dealt to
-//    the CTAs in a snake order over rounds.
+//    per SM; items are numbered heaviest (latest causal rows) first and handed out
+//    in that order by a counter in the workspace: the producer warp takes the next
+//    one whenever it starts an item and publishes it to the other roles through a
+//    small ring in shared memory, so a CTA that drew light items simply takes more
+//    (a static order left the busiest SM 10% above the mean at the GPT-2-medium
+//    shape; sequences of different lengths leave some items empty).
 //  * Warp roles (384 threads, three warpgroups):
 //      warp 0      TMA producer: Q tiles, then K/V tiles through a ring of smem
 //                  slots (mbarrier full/empty pairs).
@@ -123,10 +127,12 @@ struct FwdLayout {
   static constexpr int kOffStage = kOffRing + kStages * kTileBytes;
   static constexpr int kOffBar = kOffStage + (kEarlyQ ? 2 * kTileBytes : 0);
   // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], epi[2],
-  // s_free[2], p_free[2], stage_free[2]
-  static constexpr int kNumBars = 2 + 2 * kStages + 14;
+  // s_free[2], p_free[2], stage_free[2], item_full[R], item_empty[R]
+  static constexpr int kItemRing = 4;  // items the producer may publish ahead of the other roles
+  static constexpr int kNumBars = 2 + 2 * kStages + 14 + 2 * kItemRing;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
+  static constexpr int kOffItems = kOffMisc + 64;  // the item ring: int per slot
+  static constexpr int kSmemBytes = kOffItems + 4 * kItemRing + 1024;  // + alignment slack
 };
 
 struct FwdArgs {
@@ -141,6 +147,10 @@ struct FwdArgs {
   float scale_log2;
   int n_pairs;
   int n_items;
+  // items are handed out in order (heaviest first) by a counter in the workspace;
+  // the last CTA to finish resets it and the exit count for the next call
+  unsigned int* item_ctr;
+  unsigned int* done_ctr;
   unsigned long long timeout_ns;
   // key-padding mask (null: none): [B, km_words] bits, bit j % 32 of word j / 32
   // set when key j of the batch element takes part
@@ -179,15 +189,6 @@ __device__ __forceinline__ void tile_mask_words(const FwdArgs& a, int b, int j, 
   for (int i = 0; i < 4; ++i) w[i] = (j * 4 + i < a.km_words) ? __ldg(row + j * 4 + i) : 0u;
 }
 
-// The item a CTA takes in round r.  Items are numbered heaviest first; the rounds
-// alternate direction over the CTAs (a snake), so that a CTA that took one of the
-// heaviest items of a round takes one of the lightest of the next.  With causal
-// masking the static round-robin order leaves the busiest CTA about 13% above the
-// mean at B = 1, H = 32, N = 8192; the snake brings that to about 2%.
-__device__ __forceinline__ int item_of_round(int r) {
-  const int g = (int)gridDim.x, c = (int)blockIdx.x;
-  return r * g + ((r & 1) ? (g - 1 - c) : c);
-}
 
 __device__ __forceinline__ void item_coords(const FwdArgs& a, int w, int& b, int& h, int& pair) {
   const int bh_count = a.B * a.H;
@@ -300,6 +301,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_s_free = bar_s_full + 8;  // separate P: the softmax group has read S
   uint64_t* bar_p_free = bar_s_full + 10;  // separate P: the P V MMA has read P
   uint64_t* bar_stage_free = bar_s_full + 12;  // early Q release: the output staging buffer is free
+  uint64_t* bar_item_full = bar_s_full + 14;                // [kItemRing]: the producer published an item
+  uint64_t* bar_item_empty = bar_item_full + L::kItemRing;  // [kItemRing]: every other role has read it
+  volatile int* item_ring = reinterpret_cast<volatile int*>(smem + L::kOffItems);
+  // roles that read the item ring: the MMA issuer warp(s) and the eight softmax warps
+  constexpr uint32_t kItemReaders = (sep_p<D>() ? 2 : 1) + 8;
   constexpr bool kSepP = sep_p<D>();
   static_assert(L::kEarlyQ == kSepP, "the separate-P issuers are the ones that release Q early");
   uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
@@ -324,6 +330,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar_s_free + t, 4);  // one arrival per softmax warp
       mbar_init(bar_p_free + t, 1);
       mbar_init(bar_stage_free + t, 1);
+    }
+    for (int r2 = 0; r2 < L::kItemRing; ++r2) {
+      mbar_init(bar_item_full + r2, 1);
+      mbar_init(bar_item_empty + r2, kItemReaders);
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -350,9 +360,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       uint32_t item_iter = 0, g = 0;
-      for (int rnd = 0; rnd * (int)gridDim.x < a.n_items && !*abort_flag; ++rnd) {
-        const int w = item_of_round(rnd);
-        if (w >= a.n_items) continue;
+      for (int n = 0; !*abort_flag; ++n) {
+        // take the next item and publish it to the other roles (-1: none left)
+        const int slot_i = n % L::kItemRing;
+        if (!mbar_wait(bar_item_empty + slot_i, ((n / L::kItemRing) & 1) ^ 1, a.timeout_ns)) {
+          record_timeout(a.status, abort_flag);
+          break;
+        }
+        const unsigned int taken = atomicAdd(a.item_ctr, 1u);
+        const int w = taken < (unsigned)a.n_items ? (int)taken : -1;
+        item_ring[slot_i] = w;
+        mbar_arrive(bar_item_full + slot_i);
+        if (w < 0) break;
         int b, h, pair;
         item_coords(a, w, b, h, pair);
         const SeqView sv = seq_view(a, b);
@@ -406,12 +425,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return ok;
       };
+      // the next item from the producer's ring
+      auto read_item = [&](int n, int& w) {
+        const int slot_i = n % L::kItemRing;
+        if (!wait_or_abort(bar_item_full + slot_i, (n / L::kItemRing) & 1)) return false;
+        w = item_ring[slot_i];
+        mbar_arrive(bar_item_empty + slot_i);
+        return true;
+      };
       // ring slots alternate K, V per KV step: K of step j at g, V at g + 1
       uint32_t item_iter = 0, g = 0;
       uint32_t cnt[2] = {0, 0};  // Q K^T (warp 1) or P V (warp 2) MMAs issued per query tile
-      for (int rnd = 0; rnd * (int)gridDim.x < a.n_items && ok; ++rnd) {
-        const int w = item_of_round(rnd);
-        if (w >= a.n_items) continue;
+      for (int n = 0; ok; ++n) {
+        int w = -1;
+        if (!read_item(n, w)) break;
+        if (w < 0) break;
         int b, h, pair;
         item_coords(a, w, b, h, pair);
         const SeqView sv = seq_view(a, b);
@@ -504,9 +532,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         return ok;
       };
-      for (int rnd = 0; rnd * (int)gridDim.x < a.n_items && ok; ++rnd) {
-        const int w = item_of_round(rnd);
-        if (w >= a.n_items) continue;
+      // the next item from the producer's ring
+      auto read_item = [&](int n, int& w) {
+        const int slot_i = n % L::kItemRing;
+        if (!wait_or_abort(bar_item_full + slot_i, (n / L::kItemRing) & 1)) return false;
+        w = item_ring[slot_i];
+        mbar_arrive(bar_item_empty + slot_i);
+        return true;
+      };
+      for (int n = 0; ok; ++n) {
+        int w = -1;
+        if (!read_item(n, w)) break;
+        if (w < 0) break;
         int b, h, pair;
         item_coords(a, w, b, h, pair);
         const SeqView sv = seq_view(a, b);
@@ -658,9 +695,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* o_stage = smem + (L::kEarlyQ ? L::kOffStage : L::kOffQ) + t * L::kTileBytes;
     const uint32_t o_stage_u32 = smem_u32(o_stage);
 
-    for (int rnd = 0; rnd * (int)gridDim.x < a.n_items; ++rnd) {
-      const int w = item_of_round(rnd);
-      if (w >= a.n_items) continue;
+    for (int n = 0;; ++n) {
+      int w = -1;
+      {
+        // the next item from the producer's ring (every lane gets the index)
+        const int slot_i = n % L::kItemRing;
+        if (!warp_wait(bar_item_full + slot_i, (n / L::kItemRing) & 1, a.timeout_ns)) {
+          if (lane == 0) record_timeout(a.status, abort_flag);
+          break;
+        }
+        w = item_ring[slot_i];
+        mbar_arrive_warp(bar_item_empty + slot_i);
+      }
+      if (w < 0) break;
       if (*abort_flag) break;
       int b, h, pair;
       item_coords(a, w, b, h, pair);
@@ -948,6 +995,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem_base, kTmemCols);
   }
+  if (threadIdx.x == 0) {
+    // this CTA takes no more items; the last CTA to finish leaves the counters at
+    // zero for the next call
+    __threadfence();
+    if (atomicAdd(a.done_ctr, 1u) == gridDim.x - 1) {
+      atomicExch(a.item_ctr, 0u);
+      atomicExch(a.done_ctr, 0u);
+    }
+  }
 }
 
 }  // namespace
@@ -977,6 +1033,9 @@ static fa_status launch_fwd_impl(const FwdLaunch& L0, cudaStream_t stream) {
   FwdArgs a;
   a.lse = L0.lse;
   a.status = L0.status;
+  // the item counters sit in the status block's padding (bytes 128 .. 135)
+  a.item_ctr = reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(L0.status) + 128);
+  a.done_ctr = a.item_ctr + 1;
   a.o = static_cast<__nv_bfloat16*>(L0.o);
   a.cu_q = L0.cu_q;
   a.cu_k = L0.cu_k;
