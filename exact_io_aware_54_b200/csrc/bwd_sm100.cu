@@ -55,8 +55,9 @@ struct BwdLayout {
   static constexpr int kOffDS = kOffDO + kQStages * kTileBytes;
   static constexpr int kOffStat = kOffDS + kDsBufs * kDsBytes;  // per stage: -lse2[128], -D[128]
   static constexpr int kOffBar = kOffStat + kQStages * 2 * 128 * 4;
-  // kv_full, q_full[QS], q_empty[QS], s_full, p_full, ds_free[DSB], dq_full, dq_empty, dkv_done, epi
-  static constexpr int kNumBars = 1 + 2 * kQStages + 2 + kDsBufs + 4;
+  // kv_full, q_full[QS], q_empty[QS], s_full, p_full, ds_free[DSB], dq_full, dq_empty, dkv_done, epi,
+  // dp_full, ds_full
+  static constexpr int kNumBars = 1 + 2 * kQStages + 2 + kDsBufs + 4 + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64;
   // Tensor memory columns: K, V and dS^T are read from shared memory, and the dQ
@@ -322,6 +323,95 @@ __device__ __forceinline__ void ds_block(const uint32_t (&sv)[kN], const uint32_
   }
 }
 
+// The same work as ds_block in two halves, for the d = 128 kernel, whose dP^T comes
+// after the next tile's scores.  p_block: P for one key row and kN queries, left
+// in `v` as fp32 (the S^T bits are overwritten), packed to bf16 pairs in pk (p z
+// with dropout, the keep bits in `keep`).
+template <int kN, bool kMask, bool kDrop = false>
+__device__ __forceinline__ void p_block(uint32_t (&v)[kN], uint32_t stat, float scale_log2, bool key_ok,
+                                        int qrel_min, uint32_t (&pk)[kN / 2], uint32_t& keep,
+                                        const DropCtx* drop = nullptr, int q0 = 0) {
+  const float2 sc2 = make_float2(scale_log2, scale_log2);
+  keep = 0u;
+  if constexpr (kDrop) {
+    const uint32_t odd = (uint32_t)drop->key & 1u;
+    uint32_t mine = 0u, theirs = 0u;
+#pragma unroll
+    for (int g = 0; g < kN / 4; g += 2) {
+      const int gm = g + (int)odd;
+      const uint4 w = philox4x32_10(
+          make_uint4((uint32_t)drop->key >> 1, (uint32_t)(q0 + 4 * gm) >> 2, (uint32_t)drop->h, (uint32_t)drop->b),
+          drop->seed_lo, drop->seed_hi);
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t lo = ws[e] & 0xFFFFu, hi = ws[e] >> 16;
+        mine |= ((odd ? hi : lo) >= drop->t ? 1u : 0u) << (4 * gm + e);
+        theirs |= ((odd ? lo : hi) >= drop->t ? 1u : 0u) << (4 * gm + e);
+      }
+    }
+    keep = mine | __shfl_xor_sync(0xffffffffu, theirs, 1);
+  }
+#pragma unroll
+  for (int c = 0; c < kN; c += 4) {
+    const float4 nl = ld_shared_f4(stat + c * 4);
+    const float2 x0 = ffma2(make_float2(__uint_as_float(v[c]), __uint_as_float(v[c + 1])), sc2,
+                            make_float2(nl.x, nl.y));
+    const float2 x1 = ffma2(make_float2(__uint_as_float(v[c + 2]), __uint_as_float(v[c + 3])), sc2,
+                            make_float2(nl.z, nl.w));
+    float2 p0 = make_float2(ex2(x0.x), ex2(x0.y));
+    float2 p1 = make_float2(ex2(x1.x), ex2(x1.y));
+    if (kMask) {
+      if (!key_ok || c + 0 < qrel_min) p0.x = 0.f;
+      if (!key_ok || c + 1 < qrel_min) p0.y = 0.f;
+      if (!key_ok || c + 2 < qrel_min) p1.x = 0.f;
+      if (!key_ok || c + 3 < qrel_min) p1.y = 0.f;
+    }
+    v[c] = __float_as_uint(p0.x);
+    v[c + 1] = __float_as_uint(p0.y);
+    v[c + 2] = __float_as_uint(p1.x);
+    v[c + 3] = __float_as_uint(p1.y);
+    if constexpr (kDrop) {
+      const uint32_t kq = keep >> c;
+      const float z0 = (kq & 1u) ? drop->scale : 0.f, z1 = (kq & 2u) ? drop->scale : 0.f;
+      const float z2 = (kq & 4u) ? drop->scale : 0.f, z3 = (kq & 8u) ? drop->scale : 0.f;
+      pk[c / 2] = pack_bf16x2(p0.x * z0, p0.y * z1);
+      pk[c / 2 + 1] = pack_bf16x2(p1.x * z2, p1.y * z3);
+    } else {
+      pk[c / 2] = pack_bf16x2(p0.x, p0.y);
+      pk[c / 2 + 1] = pack_bf16x2(p1.x, p1.y);
+    }
+  }
+}
+
+// ds = p (dp - D), or p (z dp - D) with dropout, from p_block's fp32 p; `stat` as for
+// p_block (-D sits 512 bytes after -lse2).
+template <int kN, bool kDrop = false>
+__device__ __forceinline__ void ds_from_p(const uint32_t (&pv)[kN], const uint32_t (&dp)[kN], uint32_t stat,
+                                          uint32_t keep, float drop_scale, uint32_t (&dsk)[kN / 2]) {
+#pragma unroll
+  for (int c = 0; c < kN; c += 4) {
+    const float4 nd = ld_shared_f4(stat + 512 + c * 4);
+    const float2 p0 = make_float2(__uint_as_float(pv[c]), __uint_as_float(pv[c + 1]));
+    const float2 p1 = make_float2(__uint_as_float(pv[c + 2]), __uint_as_float(pv[c + 3]));
+    const float2 dp0 = make_float2(__uint_as_float(dp[c]), __uint_as_float(dp[c + 1]));
+    const float2 dp1 = make_float2(__uint_as_float(dp[c + 2]), __uint_as_float(dp[c + 3]));
+    float2 d0, d1;
+    if constexpr (kDrop) {
+      const uint32_t kq = keep >> c;
+      const float2 z0 = make_float2((kq & 1u) ? drop_scale : 0.f, (kq & 2u) ? drop_scale : 0.f);
+      const float2 z1 = make_float2((kq & 4u) ? drop_scale : 0.f, (kq & 8u) ? drop_scale : 0.f);
+      d0 = fmul2(p0, ffma2(dp0, z0, make_float2(nd.x, nd.y)));
+      d1 = fmul2(p1, ffma2(dp1, z1, make_float2(nd.z, nd.w)));
+    } else {
+      d0 = fmul2(p0, fadd2(dp0, make_float2(nd.x, nd.y)));
+      d1 = fmul2(p1, fadd2(dp1, make_float2(nd.z, nd.w)));
+    }
+    dsk[c / 2] = pack_bf16x2(d0.x, d0.y);
+    dsk[c / 2 + 1] = pack_bf16x2(d1.x, d1.y);
+  }
+}
+
 // kDrop: dropout; kSparse: block-sparse (separate instantiations, so the plain
 // kernel is unchanged)
 template <int D, bool kDrop, bool kSparse>
@@ -343,6 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_dq_empty = bar_dq_full + 1;
   uint64_t* bar_dkv_done = bar_dq_empty + 1;
   uint64_t* bar_epi = bar_dkv_done + 1;
+  // s_full: S^T of a tile is ready; p_full: its P^T is in tensor memory (dV may run);
+  // dp_full: its dP^T is ready; ds_full: its dS is in shared memory (dK, dQ may run)
+  uint64_t* bar_dp_full = bar_epi + 1;
+  uint64_t* bar_ds_full = bar_dp_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);
 
@@ -389,6 +483,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(bar_dq_empty, 8);
     mbar_init(bar_dkv_done, 1);
     mbar_init(bar_epi, 8);
+    mbar_init(bar_dp_full, 1);
+    mbar_init(bar_ds_full, 8);
     *abort_flag = 0;
     fence_mbar_init();
     fence_proxy_async_smem();
@@ -473,49 +569,45 @@ __global__ void __launch_bounds__(kThreads, 1)
       const SDesc ds_kmaj = sdesc_make(sbase + L::kOffDS, 16, 1024), ds_mn = sdesc_make(sbase + L::kOffDS, 16384, 1024);
       constexpr uint32_t kTile16 = L::kTileBytes / 16, kDs16 = L::kDsBytes / 16;
       auto at = [](SDesc d, uint32_t off16) { return SDesc{d.lo + off16, d.hi}; };
-      // S^T and dP^T of query tile `it`
-      auto issue_sdp = [&](int it) -> bool {
-        const int st = it % L::kQStages;
-        if (!mbar_wait(bar_q_full + st, (it / L::kQStages) & 1, a.timeout_ns) || *abort_flag) return false;
-        tc_fence_after();
-        issue_scores<D, false>(tmem + L::kTmSt, 0u, k_kmaj, at(q_kmaj, st * kTile16));
-        issue_scores<D, false>(tmem + L::kTmDPt, 0u, v_kmaj, at(do_kmaj, st * kTile16));
-        umma_commit(bar_s_full);
-        return true;
+      auto wait_ok = [&](uint64_t* bar, uint32_t parity) {
+        return mbar_wait(bar, parity, a.timeout_ns) && !*abort_flag;
       };
-      // dV and dK of query tile `it` (after the dS warps released it)
-      auto issue_dvdk = [&](int it) -> bool {
-        if (!mbar_wait(bar_p_full, it & 1, a.timeout_ns) || *abort_flag) return false;
+      // Per query tile `it`: dP^T (after the previous dQ has left the dP^T columns),
+      // dV once P^T is written, then the next tile's S^T (it reuses the S^T columns
+      // after dV has read P^T: tcgen05 operations run in issue order), and dK and dQ
+      // once dS is written.  The dS warps compute the next tile's P while dK and dQ
+      // run.
+      if (ok && (ok = wait_ok(bar_q_full, 0))) {
         tc_fence_after();
+        issue_scores<D, false>(tmem + L::kTmSt, 0u, k_kmaj, q_kmaj);
+        umma_commit(bar_s_full);
+      }
+      for (int it = 0; it < n_iters && ok; ++it) {
         const int st = it % L::kQStages;
+        if (it > 0) {
+          if (!(ok = wait_ok(bar_dq_empty, (it - 1) & 1))) break;
+          tc_fence_after();
+        }
+        issue_scores<D, false>(tmem + L::kTmDPt, 0u, v_kmaj, at(do_kmaj, st * kTile16));
+        umma_commit(bar_dp_full);
+        if (!(ok = wait_ok(bar_p_full, it & 1))) break;
+        tc_fence_after();
         issue_acc<D, true>(tmem + L::kTmDV, tmem + L::kTmSt, ds_kmaj, at(do_mn, st * kTile16), it == 0);
+        if (it + 1 < n_iters) {
+          const int sn = (it + 1) % L::kQStages;
+          if (!(ok = wait_ok(bar_q_full + sn, ((it + 1) / L::kQStages) & 1))) break;
+          tc_fence_after();
+          issue_scores<D, false>(tmem + L::kTmSt, 0u, k_kmaj, at(q_kmaj, sn * kTile16));
+          umma_commit(bar_s_full);
+        }
+        if (!(ok = wait_ok(bar_ds_full, it & 1))) break;
+        tc_fence_after();
         issue_acc<D, false>(tmem + L::kTmDK, 0u, at(ds_kmaj, (it % L::kDsBufs) * kDs16), at(q_mn, st * kTile16),
                             it == 0);
         umma_commit(bar_q_empty + st);  // Q and dO of this tile are no longer read
-        return true;
-      };
-      auto issue_dq_tile = [&](int it) {
         issue_dq<D>(tmem + L::kTmDQ, at(ds_mn, (it % L::kDsBufs) * kDs16), k_mn);
         umma_commit(bar_dq_full);
         umma_commit(bar_ds_free + (it % L::kDsBufs));
-      };
-      if (ok) tc_fence_after();
-      {
-        // the dQ tile uses the dP^T columns: it is drained before the next dP^T
-        for (int it = 0; it < n_iters && ok; ++it) {
-          if (it > 0) {
-            if (!mbar_wait(bar_dq_empty, (it - 1) & 1, a.timeout_ns) || *abort_flag) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-          }
-          if (!issue_sdp(it) || !issue_dvdk(it)) {
-            ok = false;
-            break;
-          }
-          issue_dq_tile(it);
-        }
       }
       if (!ok) bwd_timeout(a.status, abort_flag);
       umma_commit(bar_dkv_done);
@@ -544,19 +636,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto drain_dq = [&](int it, int q_first) -> bool {
       if (!warp_wait_b(bar_dq_full, it & 1, a.timeout_ns) || *abort_flag) return false;
       tc_fence_after();
-#pragma unroll 1
+      // both halves out of tensor memory first, so the next dP^T can start at once
+      uint32_t g[2][32];
+      tmem_ld32(tmem + lane_field + L::kTmDQ + grp * (D / 2), g[0]);
+      tmem_ld32(tmem + lane_field + L::kTmDQ + grp * (D / 2) + 32, g[1]);
+      tmem_ld_wait(g[0]);
+      reg_pin(g[1]);
+      tc_fence_before();
+      mbar_arrive_warp(bar_dq_empty);
+#pragma unroll
       for (int pass = 0; pass < 2; ++pass) {
-        uint32_t g[32];
-        tmem_ld32(tmem + lane_field + L::kTmDQ + grp * (D / 2) + pass * 32, g);
-        tmem_ld_wait(g);
-        if (pass == 1) {  // the dQ tile is out of tensor memory
-          tc_fence_before();
-          mbar_arrive_warp(bar_dq_empty);
-        }
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-          st_shared_v4(scratch + lane * 128 + ((c ^ (lane & 7)) << 4), g[4 * c], g[4 * c + 1], g[4 * c + 2],
-                       g[4 * c + 3]);
+          st_shared_v4(scratch + lane * 128 + ((c ^ (lane & 7)) << 4), g[pass][4 * c], g[pass][4 * c + 1],
+                       g[pass][4 * c + 2], g[pass][4 * c + 3]);
         __syncwarp();
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
@@ -573,43 +666,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       return true;
     };
 
-    int qi = next_kept_q<kSparse>(a, h, j, i_first, n_qtiles);  // query tile of step it
-    for (int it = 0; it < n_iters && ok; ++it, qi = next_kept_q<kSparse>(a, h, j, qi + 1, n_qtiles)) {
+    // P of query tile `it` (stage st, first query q0): the group's 64 queries in two
+    // chunks of 32, fp32 p kept in pv for the dS that follows, P^T (bf16) over the
+    // S^T columns already read
+    uint32_t pv[2][32];
+    uint32_t keep[2] = {0u, 0u};
+    auto p_phase = [&](int it, int q0) -> bool {
       const int st = it % L::kQStages;
-      const int q0 = qi * 128;
-      // the stats of this query tile are staged with it; its dS buffer must be free
       if (!warp_wait_b(bar_q_full + st, (it / L::kQStages) & 1, a.timeout_ns) ||
-          !warp_wait_b(bar_ds_free + (it % L::kDsBufs), ((it / L::kDsBufs) & 1) ^ 1, a.timeout_ns) ||
-          !warp_wait_b(bar_s_full, it & 1, a.timeout_ns) || *abort_flag) {
-        ok = false;
-        break;
-      }
+          !warp_wait_b(bar_s_full, it & 1, a.timeout_ns) || *abort_flag)
+        return false;
       tc_fence_after();
-      const uint32_t ds_row = sbase + L::kOffDS + (it % L::kDsBufs) * L::kDsBytes + grp * 16384 + r * 128;
-#pragma unroll 1
+      tmem_ld32(tmem + lane_field + L::kTmSt + 64 * grp, pv[0]);
+      tmem_ld32(tmem + lane_field + L::kTmSt + 64 * grp + 32, pv[1]);
+      tmem_ld_wait(pv[0]);
+      reg_pin(pv[1]);
+#pragma unroll
       for (int ch = 0; ch < 2; ++ch) {
-        const int col = 64 * grp + 32 * ch;  // first query of this chunk within the tile
+        const int col = 64 * grp + 32 * ch;
         const int qs = q0 + col;
-        uint32_t sv[32], dp[32];
-        tmem_ld32(tmem + lane_field + L::kTmSt + col, sv);
-        tmem_ld32(tmem + lane_field + L::kTmDPt + col, dp);
-        tmem_ld_wait(sv);
-        reg_pin(dp);
         const uint32_t stat_u32 = sbase + L::kOffStat + st * 1024 + col * 4;
         const bool tile_mask = a.key_mask != nullptr || (j * 128 + 128 > sq.lk) ||
                                (a.causal && (j * 128 + 127 - (sq.lk - sq.lq + a.causal_delta) > qs));
-        uint32_t pk[16], dk2[16];
+        uint32_t pk[16];
         if constexpr (kDrop) {
           const DropCtx dctx{a.drop_t, a.drop_scale, a.seed_lo, a.seed_hi, key, h, b};
-          ds_block<32, true, true>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2, &dctx, qs);
+          p_block<32, true, true>(pv[ch], stat_u32, a.scale_log2, key_ok, qmin - qs, pk, keep[ch], &dctx, qs);
         } else if (tile_mask) {
-          ds_block<32, true>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2);
+          p_block<32, true>(pv[ch], stat_u32, a.scale_log2, key_ok, qmin - qs, pk, keep[ch]);
         } else {
-          ds_block<32, false>(sv, dp, stat_u32, a.scale_log2, key_ok, qmin - qs, pk, dk2);
+          p_block<32, false>(pv[ch], stat_u32, a.scale_log2, key_ok, qmin - qs, pk, keep[ch]);
         }
-        // P^T as bf16 pairs over the columns of this group already read
         tmem_st16(tmem + lane_field + L::kTmSt + 64 * grp + 16 * ch, pk);
-        // dS^T row of this key: 4 chunks of 16 bytes, 128-byte swizzle
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive_warp(bar_p_full);  // dV may read P^T
+      return true;
+    };
+
+    // dS of query tile `it` from pv and dP^T, into the dS buffer (128-byte swizzle)
+    auto ds_phase = [&](int it) -> bool {
+      const int st = it % L::kQStages;
+      if (!warp_wait_b(bar_ds_free + (it % L::kDsBufs), ((it / L::kDsBufs) & 1) ^ 1, a.timeout_ns) ||
+          !warp_wait_b(bar_dp_full, it & 1, a.timeout_ns) || *abort_flag)
+        return false;
+      tc_fence_after();
+      const uint32_t ds_row = sbase + L::kOffDS + (it % L::kDsBufs) * L::kDsBytes + grp * 16384 + r * 128;
+#pragma unroll
+      for (int ch = 0; ch < 2; ++ch) {
+        const int col = 64 * grp + 32 * ch;
+        uint32_t dp[32];
+        tmem_ld32(tmem + lane_field + L::kTmDPt + col, dp);
+        tmem_ld_wait(dp);
+        uint32_t dk2[16];
+        ds_from_p<32, kDrop>(pv[ch], dp, sbase + L::kOffStat + st * 1024 + col * 4, keep[ch], a.drop_scale, dk2);
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
           const int chunk = 4 * ch + c4;
@@ -618,11 +729,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       fence_proxy_async_smem();
-      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive_warp(bar_p_full);
-      // this tile's dQ follows right after dV / dK
+      mbar_arrive_warp(bar_ds_full);  // dK and dQ may read dS
+      return true;
+    };
+
+    int qi = next_kept_q<kSparse>(a, h, j, i_first, n_qtiles);  // query tile of step it
+    ok = p_phase(0, qi * 128);
+    for (int it = 0; it < n_iters && ok; ++it) {
+      const int q0 = qi * 128;
+      if (!(ok = ds_phase(it))) break;
+      // the next tile's P while dK and dQ of this one run
+      const int qn = next_kept_q<kSparse>(a, h, j, qi + 1, n_qtiles);
+      if (it + 1 < n_iters && !(ok = p_phase(it + 1, qn * 128))) break;
       ok = drain_dq(it, q0);
+      qi = qn;
     }
     // ---------------------------------------------------------------- dK / dV epilogue
     // group 0 stores dK (times scale) through the K tile's smem, group 1 dV through V's;
