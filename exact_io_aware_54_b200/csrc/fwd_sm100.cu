@@ -857,8 +857,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               pk[ii * 16 + (c >> 1) + 1] = s1;
               ex0 = fadd2(ex0, p0);
               ex1 = fadd2(ex1, p1);
-              rd0 = fadd2(rd0, make_float2(__uint_as_float(k0 << 16), __uint_as_float(k0 & 0xFFFF0000u)));
-              rd1 = fadd2(rd1, make_float2(__uint_as_float(k1 << 16), __uint_as_float(k1 & 0xFFFF0000u)));
+              if constexpr (D == 128) {
+                // bf16 halves added to fp32 sums directly (sm_100's mixed-precision
+                // add; the same sums bit for bit): 1.7% faster at d = 128, 2.7%
+                // slower at d = 64, which keeps the unpack-and-add pair
+                acc_bf16x2(rd0, k0);
+                acc_bf16x2(rd1, k1);
+              } else {
+                rd0 = fadd2(rd0, make_float2(__uint_as_float(k0 << 16), __uint_as_float(k0 & 0xFFFF0000u)));
+                rd1 = fadd2(rd1, make_float2(__uint_as_float(k1 << 16), __uint_as_float(k1 & 0xFFFF0000u)));
+              }
             }
           }
         };

@@ -468,6 +468,15 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
 }
 
 // Three-input maximum (sm_100).
+// acc.x += the low bf16 of w, acc.y += the high one: each half widened exactly to
+// fp32 and added with one rounding (the mixed-precision add of sm_100), so the
+// sums equal those of unpacking the halves and adding them in fp32.
+__device__ __forceinline__ void acc_bf16x2(float2& acc, uint32_t w) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\tadd.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+      : "+f"(acc.x), "+f"(acc.y)
+      : "r"(w));
+}
+
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
