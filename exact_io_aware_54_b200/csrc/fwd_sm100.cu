@@ -279,6 +279,17 @@ __device__ __forceinline__ void issue_pv(uint32_t o_tmem, uint32_t p_tmem, SDesc
     umma_ts(o_tmem, p_tmem + kk * 8, sdesc_at(v, kk * 128), idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
+// One half of issue_pv: keys 64 half .. 64 half + 63.
+template <int D>
+__device__ __forceinline__ void issue_pv_half(uint32_t o_tmem, uint32_t p_tmem, SDesc v, bool accumulate, int half) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, D, false, true);
+#pragma unroll
+  for (int k4 = 0; k4 < 4; ++k4) {
+    const int kk = 4 * half + k4;
+    umma_ts(o_tmem, p_tmem + kk * 8, sdesc_at(v, kk * 128), idesc, (accumulate || kk > 0) ? 1u : 0u);
+  }
+}
+
 // kDrop: dropout on P; kSparse: block-sparse attention (separate instantiations,
 // so the plain kernel is unchanged)
 template <int D, bool kDrop, bool kSparse>
@@ -299,6 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bar_o_done = bar_s_full + 4;
   uint64_t* bar_epi = bar_s_full + 6;
   uint64_t* bar_s_free = bar_s_full + 8;  // separate P: the softmax group has read S
+  // P over S (d = 128), which has no use for s_free: the P of the tile's first 64
+  // keys is in tensor memory (one arrival per softmax warp), so that their P V
+  // runs while the softmax computes the other half
+  uint64_t* bar_p_half = bar_s_full + 8;
   uint64_t* bar_p_free = bar_s_full + 10;  // separate P: the P V MMA has read P
   uint64_t* bar_stage_free = bar_s_full + 12;  // early Q release: the output staging buffer is free
   uint64_t* bar_item_full = bar_s_full + 14;                // [kItemRing]: the producer published an item
@@ -595,10 +610,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   #pragma unroll
             for (int t = 0; t < 2; ++t) {
               if (kept_t(t, j)) {
+                if (!wait_or_abort(bar_p_half + t, p_cnt[t] & 1)) break;
+                tc_fence_after();
+                issue_pv_half<D>(tmem_base + tm_o<D>(t), tmem_base + tm_s(t), v_desc, started[t], 0);
                 if (!wait_or_abort(bar_p_full + t, p_cnt[t] & 1)) break;
                 tc_fence_after();
                 ++p_cnt[t];
-                issue_pv<D>(tmem_base + tm_o<D>(t), tmem_base + tm_s(t), v_desc, started[t]);
+                issue_pv_half<D>(tmem_base + tm_o<D>(t), tmem_base + tm_s(t), v_desc, true, 1);
                 started[t] = true;
               }
               if (t == 0 && more) {
@@ -647,10 +665,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   #pragma unroll
             for (int t = 0; t < 2; ++t) {
               if (j < nt[t]) {
+                // the first 64 keys' P V as soon as their P is written
+                if (!wait_or_abort(bar_p_half + t, p_cnt[t] & 1)) break;
+                tc_fence_after();
+                issue_pv_half<D>(tmem_base + tm_o<D>(t), tmem_base + tm_s(t), v_desc, j > 0, 0);
                 if (!wait_or_abort(bar_p_full + t, p_cnt[t] & 1)) break;
                 tc_fence_after();
                 ++p_cnt[t];
-                issue_pv<D>(tmem_base + tm_o<D>(t), tmem_base + tm_s(t), v_desc, j > 0);
+                issue_pv_half<D>(tmem_base + tm_o<D>(t), tmem_base + tm_s(t), v_desc, true, 1);
               }
               if (t == 0 && more) {
                 slot_k = g % L::kStages;
@@ -870,18 +892,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         };
+        // rescale the O accumulator when some row of this warp moved its reference.
+        // The previous P.V of this tile has completed: with P over S, the scores just
+        // read were issued after it and tcgen05 operations complete in order; with
+        // separate P the wait for the P columns below covers it.
+        const bool rescale = (kSparse ? kept_n > 0 : j > 0) && __any_sync(0xffffffffu, need);
+        auto rescale_o = [&]() {
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc * 32, o);
+            tmem_ld_wait(o);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st32(tO + cc * 32, o);
+          }
+        };
         // separate P: both halves wait in registers for the P columns
         uint32_t pkk[kSepP ? 2 : 1][32];
         if constexpr (kSepP) {
           exp_half(0, pkk[0]);
           exp_half(1, pkk[1]);
         } else {
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            uint32_t pk[32];
-            exp_half(hf, pk);
-            tmem_st32(tS + hf * 32, pk);
-          }
+          // P over S in two halves: the first 64 keys' P V runs while the second
+          // half's exponentials do (O is rescaled before it)
+          if (rescale) rescale_o();
+          exp_half(0, pkk[0]);
+          tmem_st32(tS, pkk[0]);
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive_warp(bar_p_half + t);
+          exp_half(1, pkk[0]);
+          tmem_st32(tS + 32, pkk[0]);
         }
         if constexpr (kSepP) {
           // the previous P V of this tile has read the P columns (and updated O)
@@ -897,20 +939,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         l = l * alpha + ((rd0.x + rd0.y) + (rd1.x + rd1.y));
         le = le * alpha + ((ex0.x + ex0.y) + (ex1.x + ex1.y));
         m2 = m_use;
-        // rescale the O accumulator when some row of this warp moved its reference.
-        // The previous P.V of this tile has completed: with P over S, the scores just
-        // read were issued after it and tcgen05 operations complete in order; with
-        // separate P the wait for the P columns above covered it.
-        if ((kSparse ? kept_n > 0 : j > 0) && __any_sync(0xffffffffu, need)) {
-#pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            tmem_ld32(tO + cc * 32, o);
-            tmem_ld_wait(o);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(tO + cc * 32, o);
-          }
+        if constexpr (kSepP) {
+          if (rescale) rescale_o();
         }
         tmem_st_wait();
         tc_fence_before();
