@@ -98,10 +98,12 @@ constexpr int kMmaSpins = FA_FWD_MMA_SPINS;
 constexpr int kSoftmaxSpins = FA_FWD_SOFTMAX_SPINS;
 // Every kExpFmaEvery-th group of four probabilities computes one pair of its
 // exponentials on the FMA pipes (exp2_fma2) instead of the MUFU unit: an eighth of
-// them.  Measured on B200 against other splits (at d = 64 a quarter was 5% slower,
-// a sixteenth within 1%).
+// them at d = 64, a sixteenth at d = 128.  Measured on B200 against other splits
+// (at d = 64 a quarter was 5% slower, a sixteenth within 1%; at d = 128, with the
+// P V in two halves, a sixteenth 0.7% faster than an eighth and a quarter 3%
+// slower).
 #ifndef FA_FWD_EXP_FMA_EVERY_128
-#define FA_FWD_EXP_FMA_EVERY_128 4
+#define FA_FWD_EXP_FMA_EVERY_128 8
 #endif
 #ifndef FA_FWD_EXP_FMA_EVERY_64
 #define FA_FWD_EXP_FMA_EVERY_64 4
