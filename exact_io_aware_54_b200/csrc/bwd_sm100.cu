@@ -171,6 +171,9 @@ __device__ __forceinline__ BwdSeq bwd_seq(const BwdArgs& a, int b) {
 
 // dK = dV = 0 for the keys of a tile that no query sees (a packed sequence with
 // keys but no queries): threads tid = 0 .. nthreads - 1 of the caller, 16-byte stores.
+// Heads whose key tiles the d = 128 kernel runs together (its grid order).
+constexpr int kHeadGroup = 16;
+
 template <int D>
 __device__ __forceinline__ void store_zero_dkv(const BwdArgs& a, const BwdSeq& s, int j, int h, int tid,
                                                int nthreads) {
@@ -443,10 +446,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t warp = warp_id(), lane = lane_id();
   const uint32_t sbase = smem_u32(smem);
 
-  // work: key tile j of head (b, h); heavy (early) key tiles first under the causal mask
+  // work: key tile j of head (b, h).  Heads go in groups of kHeadGroup, and the key
+  // tiles of one group's heads run together, heavy (early) key tiles first under the
+  // causal mask: the fp32 dQ rows that a head's key tiles add to then stay in L2
+  // between them, where with every head's key tile j before any key tile j + 1 they
+  // were evicted in between (long sequences moved 6.6x the ideal DRAM bytes)
   const int bh_count = a.B * a.H;
-  const int j = blockIdx.x / bh_count;
-  const int bh = blockIdx.x - j * bh_count;
+  const int gi = blockIdx.x / (a.n_kv_tiles * kHeadGroup);
+  const int g0 = gi * kHeadGroup;
+  const int gsz = min(kHeadGroup, bh_count - g0);
+  const int in_group = blockIdx.x - gi * (a.n_kv_tiles * kHeadGroup);
+  const int j = in_group / gsz;
+  const int bh = g0 + (in_group - j * gsz);
   const int b = bh / a.H, h = bh - (bh / a.H) * a.H;
   const BwdSeq sq = bwd_seq(a, b);
   if (sq.lq < 0) {  // block-uniform exits, before any barrier or tensor memory
