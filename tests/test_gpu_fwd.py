@@ -41,6 +41,23 @@ def test_tiny_config_q_times_40():
 
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
+def test_running_max_moves_across_key_tiles(d, causal):
+    """Q x 40 over four key tiles: scores with a spread of about 58 in log2 units, so
+    a row's reference max moves by more than the lazy-rescale threshold on later key
+    tiles and the O accumulator is rescaled in tensor memory (at d = 128 before the
+    first half of that tile's P V).  V is scaled by 1/4 (exact in bf16): with nearly
+    one-hot rows O is close to single rows of V, and for |O| >= 4 storing O in bf16
+    alone can miss the O bound by half a unit in the last place (1.6e-2)."""
+    q, k, v = synth.prefill_inputs(6100 + d + int(causal), 1, 512, 512, 2, d, q_mult=40.0)
+    v = v * 0.25
+    o, lse = _run(q, k, v, causal)
+    o_ref, lse_ref = oracle.attn_fwd(f64(q), f64(k), f64(v), causal, default_scale(d))
+    compare_o(f64(o), o_ref)
+    compare_lse(f64(lse), lse_ref)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("Nq,Nk", [(1, 1), (1, 300), (129, 129), (200, 200), (256, 640), (383, 257), (513, 130),
                                    (640, 1000)])
 def test_edge_shapes(d, causal, Nq, Nk):
